@@ -1,0 +1,383 @@
+"""Pins for the CPU oracle: each test checks it against something other than itself.
+
+- torch's own bf16 and float8_e4m3fn decoders (library routines), all codes;
+- numpy brute force of the block score (dense unpaged copy, reshape to blocks, max);
+- exhaustive subset search for the selection, hand-worked selection cases
+  (tests/golden/select_worked_examples.json) and the selection invariants stated on the
+  ferrox-core 'Module block_sparse' page;
+- torch.nn.functional.scaled_dot_product_attention in fp64 with an explicit mask (library
+  routine) when every block is selected, and closed forms of attention (q = 0, constant K,
+  first prefill token, hand-worked logits in tests/golden/attention_worked_examples.json).
+"""
+import itertools
+import json
+import math
+import os
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from block_sparse_paged_scores_b200 import workload as wl
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+BLOCK = 128
+
+
+# ----------------------------------------------------------------------------- decoders
+def test_bf16_decoder_matches_torch_on_every_code():
+    codes = np.arange(1 << 16, dtype=np.uint16)
+    ref = torch.from_numpy(codes.view(np.int16).copy()).view(torch.bfloat16).double().numpy()
+    got = np.array([oracle.bf16_value(int(c)) for c in codes])
+    nan = np.isnan(ref)
+    assert np.array_equal(np.isnan(got), nan)
+    assert np.array_equal(got[~nan], ref[~nan])
+
+
+def test_e4m3_decoder_matches_torch_on_every_code():
+    codes = np.arange(256, dtype=np.uint8)
+    ref = torch.from_numpy(codes.copy()).view(torch.float8_e4m3fn).double().numpy()
+    got = np.array([oracle.e4m3_value(int(c)) for c in codes])
+    nan = np.isnan(ref)
+    assert nan.sum() == 2  # 0x7F and 0xFF only: the fn variant has no infinities
+    assert np.array_equal(np.isnan(got), nan)
+    assert np.array_equal(got[~nan], ref[~nan])
+
+
+# ----------------------------------------------------------------------------- helpers
+def _small(name, **kw):
+    base = wl.WORKLOADS[name]
+    return wl.generate(base.scaled(**kw), seed=wl.SEEDS[name] + 100)
+
+
+def _dense_rows(cache, table_row, L, head):
+    """Positions 0..L-1 of one sequence gathered from the paged cache, as fp64 (numpy)."""
+    x = cache[table_row[: (L + BLOCK - 1) // BLOCK].long(), head].double()   # [nb,128,128]
+    return x.reshape(-1, x.shape[-1])[:L].numpy()
+
+
+def _positions(ids_row, count, p):
+    pos = []
+    for j in ids_row[:count]:
+        pos.extend(x for x in range(int(j) * BLOCK, int(j) * BLOCK + BLOCK) if x <= p)
+    return pos
+
+
+SCORE_CASES = [
+    ("tiny_decode", {}),
+    ("spec_decode", dict(batch=3, kv_len=(700, 1500))),
+    ("ragged_prefill", dict(batch=2, q_len=(150, 300), prior_len=(0, 400))),
+    ("bf16_decode", dict(batch=2, kv_len=(300, 900), H_idxk=8)),
+]
+
+
+# ----------------------------------------------------------------------------- scores
+@pytest.mark.parametrize("name,kw", SCORE_CASES)
+def test_scores_equal_numpy_brute_force(name, kw):
+    p = _small(name, **kw)
+    sc = oracle.index_scores(p["row_off"], p["cache_len"], p["table"], p["q_idx"], p["k_idx"],
+                             p["max_blocks"])
+    ro, cl = p["row_off"].tolist(), p["cache_len"].tolist()
+    for b in range(p["batch"]):
+        L = p["kv_lens"][b]
+        for g in range(p["H_kv"]):
+            K = _dense_rows(p["k_idx"], p["table"][b], L, g % p["H_idxk"])     # [L,128]
+            Q = p["q_idx"][ro[b]:ro[b + 1], g].double().numpy()               # [q_len,128]
+            dots = Q @ K.T                                                    # [q_len, L]
+            nbl = p["max_blocks"]
+            full = np.full((Q.shape[0], nbl * BLOCK), -np.inf)
+            full[:, :L] = dots
+            pos_q = cl[b] + np.arange(Q.shape[0])
+            full[np.arange(nbl * BLOCK)[None, :] > pos_q[:, None]] = -np.inf
+            ref = full.reshape(Q.shape[0], nbl, BLOCK).max(axis=2)
+            got = sc[ro[b]:ro[b + 1], g]
+            assert np.array_equal(np.isinf(got), np.isinf(ref))
+            fin = np.isfinite(ref)
+            np.testing.assert_allclose(got[fin], ref[fin], rtol=1e-12, atol=1e-11)
+
+
+def test_block_score_is_max_not_mean():
+    """A single planted key aligned with q_idx puts its block in the selection even though
+    every other position of that block is N(0,1) noise (max over the block, not the mean)."""
+    p = _small("bf16_decode", batch=1, kv_len=2000)
+    b, g, jstar = 0, 3, 6
+    qv = p["q_idx"][0, g].float()
+    spike = (50.0 * qv / qv.norm()).to(torch.bfloat16)
+    page = int(p["table"][b, jstar])
+    p["k_idx"][page, 0, 77] = spike
+    sc = oracle.index_scores(p["row_off"], p["cache_len"], p["table"], p["q_idx"], p["k_idx"],
+                             p["max_blocks"])
+    expect = float((qv.double() * spike.double()).sum())
+    assert sc[0, g, jstar] == pytest.approx(expect, rel=1e-12)
+    ids, cnt = oracle.select_blocks(p["row_off"], p["cache_len"], sc, top_k=1, init_blocks=1,
+                                    local_blocks=1)
+    assert jstar in ids[0, g, :cnt[0, g]].tolist()
+
+
+# ----------------------------------------------------------------------------- selection
+def _select_one(scores, p, init, local, top_k):
+    sc = np.full((1, 1, len(scores)), -np.inf)
+    sc[0, 0, :] = scores
+    ids, cnt = oracle.select_blocks(np.array([0, 1]), np.array([p]), sc, top_k, init, local)
+    return ids[0, 0, :cnt[0, 0]].tolist(), ids[0, 0]
+
+
+def test_select_hand_worked_cases():
+    cases = json.load(open(os.path.join(GOLDEN, "select_worked_examples.json")))["cases"]
+    for c in cases:
+        got, padded = _select_one(c["scores"], c["p"], c["init"], c["local"], c["top_k"])
+        assert got == c["expected"], c["name"]
+        assert all(x == -1 for x in padded[len(got):])
+
+
+def _brute_force_select(scores, nb, init, local, top_k):
+    forced = {j for j in range(nb) if j < init or j >= nb - local}
+    cand = [j for j in range(nb) if j not in forced]
+    k = min(top_k, len(cand))
+    winners = []
+    for subset in itertools.combinations(cand, k):
+        rest = [j for j in cand if j not in subset]
+        # every kept block beats every dropped one: higher score, or equal score and lower id
+        if all(scores[a] > scores[r] or (scores[a] == scores[r] and a < r)
+               for a in subset for r in rest):
+            winners.append(set(subset))
+    assert len(winners) == 1
+    return sorted(forced | winners[0])
+
+
+@pytest.mark.parametrize("seed", range(40))
+def test_select_matches_exhaustive_search(seed):
+    rng = np.random.default_rng(seed)
+    nb = int(rng.integers(1, 11))
+    init, local, top_k = (int(x) for x in rng.integers(0, 3, size=3))
+    top_k += int(rng.integers(0, 3))
+    if init + local + top_k == 0:
+        top_k = 1
+    # integer-valued scores make ties frequent
+    scores = rng.integers(-3, 4, size=nb).astype(np.float64)
+    p = (nb - 1) * BLOCK + int(rng.integers(0, BLOCK))
+    got, _ = _select_one(scores, p, init, local, top_k)
+    assert got == _brute_force_select(scores, nb, init, local, top_k)
+
+
+def _check_selection_invariants(p, sc, ids, cnt):
+    ro, cl = p["row_off"].tolist(), p["cache_len"].tolist()
+    init, local, top_k = p["init_blocks"], p["local_blocks"], p["top_k"]
+    for b in range(p["batch"]):
+        for i in range(ro[b + 1] - ro[b]):
+            t = ro[b] + i
+            nb = (cl[b] + i) // BLOCK + 1
+            for g in range(p["H_kv"]):
+                sel = ids[t, g, :cnt[t, g]].tolist()
+                assert len(sel) >= 1                                   # never empty
+                assert sel == sorted(set(sel))                         # ascending, unique
+                assert all(0 <= j < nb for j in sel)
+                assert all(x == -1 for x in ids[t, g, cnt[t, g]:])
+                forced = {j for j in range(nb) if j < init or j >= nb - local}
+                assert forced <= set(sel)
+                cand = [j for j in range(nb) if j not in forced]
+                assert len(sel) == len(forced) + min(top_k, len(cand))
+                kept = [sc[t, g, j] for j in cand if j in sel]
+                dropped = [sc[t, g, j] for j in cand if j not in sel]
+                if kept and dropped:
+                    assert min(kept) >= max(dropped)
+
+
+@pytest.mark.parametrize("name,kw", SCORE_CASES)
+def test_selection_invariants(name, kw):
+    p = _small(name, **kw)
+    sc = oracle.index_scores(p["row_off"], p["cache_len"], p["table"], p["q_idx"], p["k_idx"],
+                             p["max_blocks"])
+    ids, cnt = oracle.select_blocks(p["row_off"], p["cache_len"], sc, p["top_k"],
+                                    p["init_blocks"], p["local_blocks"])
+    _check_selection_invariants(p, sc, ids, cnt)
+
+
+@pytest.mark.parametrize("factor", [2.0, 0.5, 4.0])
+def test_selection_is_scale_free(factor):
+    """Scaling every index query by a positive power of two (exact in bf16) changes no id:
+    only the order of the scores is consumed (ferrox-core 'Four rules': no softmax scale)."""
+    p = _small("spec_decode", batch=2, kv_len=(2000, 3000))
+    args = (p["top_k"], p["init_blocks"], p["local_blocks"])
+    sc = oracle.index_scores(p["row_off"], p["cache_len"], p["table"], p["q_idx"], p["k_idx"],
+                             p["max_blocks"])
+    ids, cnt = oracle.select_blocks(p["row_off"], p["cache_len"], sc, *args)
+    q2 = (p["q_idx"].float() * factor).to(torch.bfloat16)
+    assert torch.equal(q2.float(), p["q_idx"].float() * factor)
+    sc2 = oracle.index_scores(p["row_off"], p["cache_len"], p["table"], q2, p["k_idx"],
+                              p["max_blocks"])
+    ids2, cnt2 = oracle.select_blocks(p["row_off"], p["cache_len"], sc2, *args)
+    assert np.array_equal(ids, ids2) and np.array_equal(cnt, cnt2)
+
+
+def test_selection_is_per_kv_head():
+    """Head g's selection depends on head g's index query only (no cross-head reduction)."""
+    p = _small("bf16_decode", batch=2, kv_len=(5000, 8000))
+    args = (p["top_k"], p["init_blocks"], p["local_blocks"])
+    sc = oracle.index_scores(p["row_off"], p["cache_len"], p["table"], p["q_idx"], p["k_idx"],
+                             p["max_blocks"])
+    ids, cnt = oracle.select_blocks(p["row_off"], p["cache_len"], sc, *args)
+    g = 5
+    q2 = p["q_idx"].clone()
+    others = [h for h in range(p["H_kv"]) if h != g]
+    q2[:, others] = torch.flip(q2[:, others], dims=[2]) * -1
+    sc2 = oracle.index_scores(p["row_off"], p["cache_len"], p["table"], q2, p["k_idx"],
+                              p["max_blocks"])
+    ids2, cnt2 = oracle.select_blocks(p["row_off"], p["cache_len"], sc2, *args)
+    assert np.array_equal(ids[:, g], ids2[:, g])
+    assert not np.array_equal(ids[:, others], ids2[:, others])
+
+
+# ----------------------------------------------------------------------------- attention
+def _all_blocks(p):
+    """Selection with every visible block (top_k >= nb): ids [total_q,H_kv,S] and counts."""
+    ro, cl = p["row_off"].tolist(), p["cache_len"].tolist()
+    S = p["max_blocks"]
+    ids = np.full((p["total_q"], p["H_kv"], S), -1, dtype=np.int32)
+    cnt = np.zeros((p["total_q"], p["H_kv"]), dtype=np.int32)
+    for b in range(p["batch"]):
+        for i in range(ro[b + 1] - ro[b]):
+            nb = (cl[b] + i) // BLOCK + 1
+            ids[ro[b] + i, :, :nb] = np.arange(nb)
+            cnt[ro[b] + i] = nb
+    return ids, cnt
+
+
+def _kv_float(t):
+    return t.double()
+
+
+ATTN_CASES = [
+    ("tiny_decode", {}),
+    ("spec_decode", dict(batch=2, kv_len=(300, 700), G=3)),
+    ("ragged_prefill", dict(batch=2, q_len=(130, 260), prior_len=(0, 300), H_kv=2, G=2)),
+    ("fp8_long_decode", dict(batch=2, kv_len=(400, 600), H_kv=2)),
+]
+
+
+@pytest.mark.parametrize("name,kw", ATTN_CASES)
+def test_attention_with_every_block_equals_dense_causal_sdpa(name, kw):
+    p = _small(name, **kw)
+    ids, cnt = _all_blocks(p)
+    out = oracle.attention(p["row_off"], p["cache_len"], p["table"], p["q"], p["k"], p["v"],
+                           p["kv_fp8"], ids, cnt, p["scale"])
+    ro, cl = p["row_off"].tolist(), p["cache_len"].tolist()
+    G = p["H_q"] // p["H_kv"]
+    for b in range(p["batch"]):
+        L = p["kv_lens"][b]
+        for g in range(p["H_kv"]):
+            K = torch.from_numpy(_dense_rows(p["k"], p["table"][b], L, g))
+            V = torch.from_numpy(_dense_rows(p["v"], p["table"][b], L, g))
+            Q = p["q"][ro[b]:ro[b + 1], g * G:(g + 1) * G].double().transpose(0, 1)
+            pos_q = torch.arange(cl[b], cl[b] + Q.shape[1])
+            mask = torch.arange(L)[None, :] <= pos_q[:, None]
+            ref = torch.nn.functional.scaled_dot_product_attention(
+                Q[None], K[None, None].expand(1, G, L, 128), V[None, None].expand(1, G, L, 128),
+                attn_mask=mask[None, None], scale=p["scale"])[0].transpose(0, 1)
+            got = out[ro[b]:ro[b + 1], g * G:(g + 1) * G]
+            np.testing.assert_allclose(got, ref.numpy(), rtol=1e-10, atol=1e-12)
+
+
+def _oracle_selection(p):
+    sc = oracle.index_scores(p["row_off"], p["cache_len"], p["table"], p["q_idx"], p["k_idx"],
+                             p["max_blocks"])
+    return oracle.select_blocks(p["row_off"], p["cache_len"], sc, p["top_k"], p["init_blocks"],
+                                p["local_blocks"])
+
+
+def _mean_v_over_selection(p, ids, cnt):
+    ro, cl = p["row_off"].tolist(), p["cache_len"].tolist()
+    G = p["H_q"] // p["H_kv"]
+    ref = np.zeros((p["total_q"], p["H_q"], 128))
+    for b in range(p["batch"]):
+        V_all = {g: _dense_rows(p["v"], p["table"][b], p["kv_lens"][b], g)
+                 for g in range(p["H_kv"])}
+        for i in range(ro[b + 1] - ro[b]):
+            t = ro[b] + i
+            for h in range(p["H_q"]):
+                pos = _positions(ids[t, h // G], cnt[t, h // G], cl[b] + i)
+                ref[t, h] = V_all[h // G][pos].mean(axis=0)
+    return ref
+
+
+@pytest.mark.parametrize("name,kw", ATTN_CASES[1:])
+def test_attention_with_zero_query_is_mean_of_selected_values(name, kw):
+    p = _small(name, **kw)
+    ids, cnt = _oracle_selection(p)
+    p["q"] = torch.zeros_like(p["q"])
+    out = oracle.attention(p["row_off"], p["cache_len"], p["table"], p["q"], p["k"], p["v"],
+                           p["kv_fp8"], ids, cnt, p["scale"])
+    np.testing.assert_allclose(out, _mean_v_over_selection(p, ids, cnt), rtol=1e-10,
+                               atol=1e-12)
+
+
+def test_attention_with_constant_keys_is_mean_of_selected_values():
+    p = _small("spec_decode", batch=2, kv_len=(500, 900))
+    ids, cnt = _oracle_selection(p)
+    row = torch.randn(128, generator=torch.Generator().manual_seed(9)).to(torch.bfloat16)
+    p["k"] = row.expand_as(p["k"]).contiguous()
+    out = oracle.attention(p["row_off"], p["cache_len"], p["table"], p["q"], p["k"], p["v"],
+                           p["kv_fp8"], ids, cnt, p["scale"])
+    np.testing.assert_allclose(out, _mean_v_over_selection(p, ids, cnt), rtol=1e-9, atol=1e-11)
+
+
+def test_attention_is_a_convex_combination_of_selected_values():
+    p = _small("ragged_prefill", batch=1, q_len=200, prior_len=100, H_kv=2, G=2)
+    ids, cnt = _oracle_selection(p)
+    out = oracle.attention(p["row_off"], p["cache_len"], p["table"], p["q"], p["k"], p["v"],
+                           p["kv_fp8"], ids, cnt, p["scale"])
+    cl = p["cache_len"].tolist()
+    V = {g: _dense_rows(p["v"], p["table"][0], p["kv_lens"][0], g) for g in range(2)}
+    for i in range(0, 200, 7):
+        for h in range(4):
+            pos = _positions(ids[i, h // 2], cnt[i, h // 2], cl[0] + i)
+            lo, hi = V[h // 2][pos].min(axis=0), V[h // 2][pos].max(axis=0)
+            assert np.all(out[i, h] >= lo - 1e-12) and np.all(out[i, h] <= hi + 1e-12)
+
+
+def test_first_prefill_token_attends_only_to_itself():
+    p = _small("ragged_prefill", batch=2, q_len=(129, 140), prior_len=0, H_kv=2, G=2)
+    ids, cnt = _oracle_selection(p)
+    out = oracle.attention(p["row_off"], p["cache_len"], p["table"], p["q"], p["k"], p["v"],
+                           p["kv_fp8"], ids, cnt, p["scale"])
+    ro = p["row_off"].tolist()
+    for b in range(2):
+        page = int(p["table"][b, 0])
+        for h in range(4):
+            np.testing.assert_array_equal(out[ro[b], h], p["v"][page, h // 2, 0].double().numpy())
+
+
+def _golden_problem(c):
+    L = c["cache_len"] + c["q_len"]
+    nb = (L + BLOCK - 1) // BLOCK
+    z = lambda *s: torch.zeros(*s, dtype=torch.bfloat16)
+    q = z(c["q_len"], 1, 128)
+    q[:, 0, 0] = c["q"]["dim0"]
+    k, v = z(nb, 1, BLOCK, 128), z(nb, 1, BLOCK, 128)
+    for r in c["k_rows"]:
+        k[r["pos"] // BLOCK, 0, r["pos"] % BLOCK, 0] = r["dim0"]
+    for r in c["v_rows"]:
+        for key in ("dim0", "dim1"):
+            if key in r:
+                v[r["pos"] // BLOCK, 0, r["pos"] % BLOCK, int(key[3:])] = r[key]
+    ids = np.full((c["q_len"], 1, nb), -1, dtype=np.int32)
+    cnt = np.zeros((c["q_len"], 1), dtype=np.int32)
+    for i in range(c["q_len"]):
+        n = (c["cache_len"] + i) // BLOCK + 1
+        ids[i, 0, :n] = np.arange(n)
+        cnt[i, 0] = n
+    table = np.arange(nb, dtype=np.int32)[None]
+    out = oracle.attention(np.array([0, c["q_len"]]), np.array([c["cache_len"]]), table, q, k, v,
+                           False, ids, cnt, c["scale"])
+    return out
+
+
+def test_attention_hand_worked_cases():
+    cases = json.load(open(os.path.join(GOLDEN, "attention_worked_examples.json")))["cases"]
+    env = {"e": math.e}
+    for c in cases:
+        out = _golden_problem(c)
+        exp = c.get("expected") or c.get("expected_token0")
+        for key, formula in exp.items():
+            assert out[0, 0, int(key[3:])] == pytest.approx(eval(formula, env), rel=1e-14), c["name"]
