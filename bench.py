@@ -1,0 +1,439 @@
+"""Benchmark of the block-sparse paged attention hot path on B200.
+
+One step = one pass of the whole path over one batch: block scores -> selection -> sparse
+paged attention (split-K + combine), through the C ABI, on the BF16-decode workload (batch 32,
+1 query token, 8 KV heads x 8 query heads, head dim 128, context U[16384, 65536], page 128,
+top_k 16, init 1, local 2) unless --workload says otherwise.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+
+Under torchrun every rank runs an independent replica (the path does not shard: no
+collective), timed on the device between barriers, and rank 0 prints one JSON line whose
+value is the query tokens of all ranks divided by the slowest rank's time.
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import torch  # noqa: E402
+
+METRIC = "sparse-attn query-tokens/s and achieved HBM GB/s (% of roofline) at 1 B200"
+UNIT = "query-tokens/s"
+L2_BYTES = 126 * 1024 * 1024
+FALLBACK_HBM_GBS = 6650.0
+FALLBACK_BF16_TFLOPS = 1590.0
+
+
+# ------------------------------------------------------------------ distributed plumbing
+def dist_env():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return ws, rank, local
+
+
+def init_dist(backend: str):
+    ws, rank, _ = dist_env()
+    if ws > 1 and not torch.distributed.is_initialized():
+        torch.distributed.init_process_group(backend=backend,
+                                             timeout=datetime.timedelta(seconds=120))
+    return ws, rank
+
+
+def barrier(ws: int, device=None):
+    if ws > 1:
+        if device is not None and torch.distributed.get_backend() == "nccl":
+            torch.distributed.barrier(device_ids=[device.index])
+        else:
+            torch.distributed.barrier()
+
+
+def max_over_ranks(x: float, ws: int, device) -> float:
+    """The largest value of x over all ranks (every rank calls it, in the same order)."""
+    if ws == 1:
+        return float(x)
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def sum_over_ranks(x: float, ws: int, device) -> float:
+    if ws == 1:
+        return float(x)
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.SUM)
+    return float(t.item())
+
+
+# ------------------------------------------------------------------ peaks and clocks
+def measured_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        d = json.load(open(path))
+        return float(d["hbm_gbs"]), float(d["bf16_tflops"]), float(
+            d.get("bf16_tflops_sustained", d["bf16_tflops"])), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, FALLBACK_BF16_TFLOPS, 1400.0, "fallback"
+
+
+class ClockSampler:
+    """nvidia-smi samples (SM clock, throttle reasons) while the timed region runs."""
+    QUERY = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index, self.rows, self.proc, self.thread = index, [], None, None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.QUERY}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+            return self
+        self.thread = threading.Thread(target=self._read, daemon=True)
+        self.thread.start()
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.rows.append((time.time(), [x.strip() for x in line.split(",")]))
+
+    def mark(self):
+        return time.time()
+
+    def stop(self):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+
+    def summary(self, t0: float, t1: float):
+        rows = [r for (t, r) in self.rows if t0 - 0.15 <= t <= t1 + 0.15] or \
+            [r for (_, r) in self.rows]
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        sm, mx, reasons = [], [], set()
+        for r in rows:
+            try:
+                sm.append(float(r[0]))
+                mx.append(float(r[1]))
+            except ValueError:
+                continue
+            for n, v in zip(names, r[4:8]):
+                if v.strip().lower() == "active":
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(mx) if mx else None, "reasons": sorted(reasons),
+                "samples": len(rows)}
+
+
+# ------------------------------------------------------------------ algorithmic work
+def algorithmic_bytes(prob, block_ids, num_selected):
+    """HBM bytes the method itself must move per step (implementation traffic excluded):
+    index: every visible index-K position of every sequence (+ q_idx); attention: K and V of
+    every valid position of each (sequence, KV head)'s union of selected blocks (+ q, out)."""
+    import numpy as np
+    BLOCK, D = 128, 128
+    kv_elem = 1 if prob["kv_fp8"] else 2
+    ro = prob["row_off"].cpu().tolist()
+    L = prob["kv_lens"]
+    ids = block_ids.cpu().numpy()
+    cnt = num_selected.cpu().numpy()
+    idx_bytes = sum(L[b] for b in range(prob["batch"]) if ro[b + 1] > ro[b]) * \
+        prob["H_idxk"] * D * 2 + prob["total_q"] * prob["H_kv"] * D * 2
+    kv_bytes = 0
+    for b in range(prob["batch"]):
+        if ro[b + 1] == ro[b]:
+            continue
+        for g in range(prob["H_kv"]):
+            blocks = set()
+            for t in range(ro[b], ro[b + 1]):
+                blocks.update(ids[t, g, :cnt[t, g]].tolist())
+            for j in blocks:
+                kv_bytes += min(BLOCK, L[b] - j * BLOCK) * D * kv_elem * 2
+    qo_bytes = prob["total_q"] * prob["H_q"] * D * 2 * 2
+    return idx_bytes, kv_bytes + qo_bytes
+
+
+def source_digest(*names):
+    h = hashlib.sha256()
+    for n in names:
+        with open(os.path.join(ROOT, "block_sparse_paged_scores_b200", "csrc", n), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def profiled_traffic(kernel: str, workload: str, digest: str):
+    """DRAM bytes per launch from a committed ncu summary, when it was taken on this exact
+    kernel source; None otherwise."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        d = json.load(open(path))
+        e = d[f"{kernel}/{workload}"]
+        return float(e["dram_bytes_per_launch"]) if e.get("source_digest") == digest else None
+    except Exception:
+        return None
+
+
+# ------------------------------------------------------------------ CPU oracle sample
+def oracle_sample(workload: str, n_seq: int, seed: int):
+    from block_sparse_paged_scores_b200 import workload as wl
+    spec = wl.WORKLOADS[workload]
+    return wl.generate(spec.scaled(batch=min(n_seq, spec.batch)), seed=seed)
+
+
+def time_oracle(prob, min_seconds: float, max_seconds: float):
+    import oracle
+    oracle.build()
+    tokens, t0, reps = 0, time.perf_counter(), 0
+    while True:
+        oracle.forward(prob, prob["top_k"], prob["init_blocks"], prob["local_blocks"],
+                       prob["scale"], prob["max_blocks"])
+        tokens += prob["total_q"]
+        reps += 1
+        el = time.perf_counter() - t0
+        if el >= min_seconds or el * (reps + 1) / reps > max_seconds:
+            return tokens / el, el, reps
+
+
+def cpu_threads():
+    n = os.environ.get("OMP_NUM_THREADS")
+    return int(n) if n else len(os.sched_getaffinity(0))
+
+
+# ------------------------------------------------------------------ arms
+def run_reference(args):
+    """The CPU oracle as the reference arm: each step is the whole path on a bounded sample
+    of the workload (a few of its sequences, same distributions)."""
+    ws, rank, _ = dist_env()
+    if rank != 0:
+        return 0
+    prob = oracle_sample(args.workload, args.cpu_sample_seqs, seed=7)
+    import oracle
+    oracle.build()
+    fwd = lambda: oracle.forward(prob, prob["top_k"], prob["init_blocks"], prob["local_blocks"],
+                                 prob["scale"], prob["max_blocks"])
+    for _ in range(args.warmup):
+        fwd()
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        fwd()
+    el = time.perf_counter() - t0
+    value = prob["total_q"] * args.steps / el
+    cores = cpu_threads()
+    sample = (f"{prob['batch']} of {wl_batch(args.workload)} sequences of {args.workload} "
+              f"(seed 7) per step")
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT,
+            "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": el * 1e3 / args.steps, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": args.workload},
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def wl_batch(name):
+    from block_sparse_paged_scores_b200 import workload as wl
+    return wl.WORKLOADS[name].batch
+
+
+def run_ours(args):
+    from block_sparse_paged_scores_b200 import build as msa_build
+    from block_sparse_paged_scores_b200 import msa
+    from block_sparse_paged_scores_b200 import workload as wl
+
+    ws, rank = init_dist("nccl")
+    _, _, local = dist_env()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if rank == 0:
+        msa_build.build()
+    barrier(ws, dev)
+    msa.load()
+
+    spec = wl.WORKLOADS[args.workload]
+    seed = wl.SEEDS[args.workload] + 1000 * rank
+    prob = wl.generate(spec, seed=seed, device=dev)
+    path = msa.Path(prob, num_splits=args.splits)
+    stream = torch.cuda.current_stream(dev)
+    fp8 = prob["kv_fp8"]
+    kernels_per_step = 3 + (1 if prob["max_q_len"] > 1 else 0)
+    splits_used = 1 if prob["max_q_len"] > 8 else (args.splits or msa.msa_default_num_splits(
+        prob["batch"], prob["max_q_len"], prob["H_kv"], prob["S"],
+        torch.cuda.get_device_properties(dev).multi_processor_count))
+    if splits_used > 1:
+        kernels_per_step += 1
+
+    for _ in range(args.warmup):
+        path.run(stream)
+    torch.cuda.synchronize(dev)
+    assert int(path.dev_err.item()) == 0, "device error flag set during warm-up"
+
+    sampler = ClockSampler(local).start() if rank == 0 else None
+    time.sleep(0.3 if sampler else 0)
+    # ---- device-timed region: exactly K steps between barriers
+    barrier(ws, dev)
+    torch.cuda.synchronize(dev)
+    t_wall0 = time.time()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        path.run(stream)
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    barrier(ws, dev)
+    t_wall1 = time.time()
+    ms_local = e0.elapsed_time(e1)
+    ms = max_over_ranks(ms_local, ws, dev)
+
+    # ---- per-stage durations (separate K-step pass, events between the stages)
+    n_ev = 4
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(n_ev)] for _ in range(args.steps)]
+    for k in range(args.steps):
+        evs[k][0].record(stream)
+        path.index_scores(stream)
+        evs[k][1].record(stream)
+        path.select(stream=stream)
+        evs[k][2].record(stream)
+        path.attend(stream=stream)
+        evs[k][3].record(stream)
+    torch.cuda.synchronize(dev)
+    stage_ms = [sum(evs[k][i].elapsed_time(evs[k][i + 1]) for k in range(args.steps)) /
+                args.steps for i in range(3)]
+    if sampler:
+        sampler.stop()
+    clocks = sampler.summary(t_wall0, t_wall1) if sampler else None
+
+    # ---- end to end through the public API with host buffers
+    host = {k: prob[k].cpu().pin_memory() for k in ("q", "q_idx", "row_off", "cache_len", "table")}
+    out_host = torch.empty(path.out.shape, dtype=path.out.dtype).pin_memory()
+    h2d = sum(v.numel() * v.element_size() for v in host.values())
+    d2h = out_host.numel() * out_host.element_size()
+    for _ in range(max(1, args.warmup)):
+        for k_, v_ in host.items():
+            prob[k_].copy_(v_, non_blocking=True)
+        path.run(stream)
+        out_host.copy_(path.out, non_blocking=True)
+    torch.cuda.synchronize(dev)
+    barrier(ws, dev)
+    x0, x1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    x0.record(stream)
+    for _ in range(args.steps):
+        for k_, v_ in host.items():
+            prob[k_].copy_(v_, non_blocking=True)
+        path.run(stream)
+        out_host.copy_(path.out, non_blocking=True)
+    x1.record(stream)
+    torch.cuda.synchronize(dev)
+    e2e_ms = max_over_ranks(x0.elapsed_time(x1), ws, dev)
+
+    # ---- the realised work of this step, for the roofline
+    idx_bytes, attn_bytes = algorithmic_bytes(prob, path.block_ids, path.num_selected)
+    tokens_total = sum_over_ranks(prob["total_q"], ws, dev) * args.steps
+    assert int(path.dev_err.item()) == 0, "device error flag set"
+
+    cpu = None
+    if rank == 0 and ws == 1 and not args.no_cpu_baseline:
+        sample = oracle_sample(args.workload, args.cpu_sample_seqs, seed=7)
+        v, el, reps = time_oracle(sample, args.cpu_min_s, args.cpu_max_s)
+        cpu = {"value": v, "unit": UNIT, "cores": cpu_threads(), "kind": "oracle",
+               "sample": f"{sample['batch']} of {spec.batch} sequences of {args.workload} "
+                         f"(same distributions, seed 7), {reps} pass(es), {el:.1f} s"}
+
+    if rank != 0:
+        return 0
+    hbm, bf16, bf16_sus, peak_src = measured_peaks()
+    kinds = {"index_scores": (stage_ms[0], idx_bytes, "indexer.cu"),
+             "attention": (stage_ms[2], attn_bytes, "attention.cu")}
+    dom = max(kinds, key=lambda k: kinds[k][0])
+    d_ms, d_bytes, d_src = kinds[dom]
+    achieved = d_bytes / (d_ms * 1e-3) / 1e9
+    digest = source_digest(d_src)
+    line = {
+        "metric": METRIC, "value": tokens_total / (ms * 1e-3), "unit": UNIT, "n_gpus": ws,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "fp8-e4m3 kv / bf16" if fp8 else "bf16", "data": "synthetic",
+        "config": {"workload": args.workload, "batch": prob["batch"],
+                   "q_tokens_per_step": prob["total_q"], "H_kv": prob["H_kv"],
+                   "H_q": prob["H_q"], "head_dim": 128, "page_size": 128,
+                   "top_k": prob["top_k"], "init_blocks": prob["init_blocks"],
+                   "local_blocks": prob["local_blocks"], "kv_lens": f"{spec.kv_len}",
+                   "num_splits": splits_used, "parallelism": f"replicas x{ws}",
+                   "l2": f"inputs larger than L2: {(idx_bytes + attn_bytes) / 1e6:.0f} MB "
+                         f"touched per step vs {L2_BYTES / 1e6:.0f} MB L2"},
+        "roofline": {"bound": "hbm", "kernel": dom, "achieved": achieved, "peak": hbm,
+                     "unit": "GB/s", "frac": achieved / hbm, "peak_source": peak_src,
+                     "traffic": profiled_traffic(dom, args.workload, digest),
+                     "algorithmic_bytes_per_launch": d_bytes},
+        "step_hbm": {"algorithmic_bytes": idx_bytes + attn_bytes,
+                     "achieved_GBps": (idx_bytes + attn_bytes) / (ms / args.steps * 1e-3) / 1e9,
+                     "frac_of_measured": (idx_bytes + attn_bytes) / (ms / args.steps * 1e-3)
+                     / 1e9 / hbm,
+                     "frac_of_8TBps": (idx_bytes + attn_bytes) / (ms / args.steps * 1e-3)
+                     / 8e12},
+        "stages_ms": {"index_scores": stage_ms[0], "select": stage_ms[1],
+                      "attention_incl_plan_and_combine": stage_ms[2]},
+        "gpu_launches": kernels_per_step * args.steps,
+        "clocks": clocks,
+        "e2e": {"value": tokens_total / (e2e_ms * 1e-3), "unit": UNIT,
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                "note": "per-step inputs (q, q_idx, row offsets, cache lengths, page table) "
+                        "copied from pinned host memory and the output read back; the paged "
+                        "caches stay resident"},
+        "cpu_baseline": cpu,
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="bf16_decode")
+    ap.add_argument("--splits", type=int, default=0, help="split-K partitions (0 = heuristic)")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-sample-seqs", type=int, default=4)
+    ap.add_argument("--cpu-min-s", type=float, default=10.0)
+    ap.add_argument("--cpu-max-s", type=float, default=30.0)
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    if args.impl == "reference":
+        return run_reference(args)
+    rc = run_ours(args)
+    ws, _, _ = dist_env()
+    if ws > 1 and torch.distributed.is_initialized():
+        torch.distributed.destroy_process_group()
+    return rc
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,401 @@
+// api.cu — the C ABI of libmsa.so (declared in include/msa.h): argument validation, route
+// selection, split-K sizing, workspace layout, tensor-map encoding and kernel launches.
+//
+// Mojo module "msa": both ops take the same arguments for every step and pick the kernel at
+// run time from the largest number of new query tokens in the batch (1: decode, 2..8:
+// speculative decode, more: prefill); decode splits the selected blocks over SM-filling
+// split-K partitions.  The library owns no device memory: every buffer, the workspace
+// included, comes from the caller, and every call only enqueues work on the caller's stream.
+#include <math.h>
+#include <string.h>
+
+#include <mutex>
+
+#include "internal.h"
+
+namespace msa {
+
+namespace {
+
+// ---- tensor maps: the runtime hands out the driver's encoder, no link against libcuda
+using EncodeTiledFn = CUresult (*)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
+                                   const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
+                                   const cuuint32_t *, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void *p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+// A paged cache [tiles = num_pages * heads][128 tokens][128 dims] as a 3-D tensor map whose
+// box is one (page, head) tile: 128 tokens x 64 bf16 (two loads per tile) or 128 x 128 e4m3,
+// written to shared memory with the 128-byte swizzle.
+bool page_tensor_map(CUtensorMap *map, const void *base, long long tiles, bool fp8) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  const cuuint64_t esz = fp8 ? 1 : 2;
+  const cuuint64_t dims[3] = {static_cast<cuuint64_t>(kHeadDim), static_cast<cuuint64_t>(kBlock),
+                              static_cast<cuuint64_t>(tiles)};
+  const cuuint64_t strides[2] = {kHeadDim * esz, kHeadDim * kBlock * esz};
+  const cuuint32_t box[3] = {fp8 ? 128u : 64u, static_cast<cuuint32_t>(kBlock), 1u};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  memset(map, 0, sizeof(*map));
+  const CUresult r = fn(map, fp8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16,
+                        3, const_cast<void *>(base), dims, strides, box, estr,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+int current_device() {
+  int d = 0;
+  if (cudaGetDevice(&d) != cudaSuccess) return 0;
+  return d;
+}
+
+int num_sms_of_current_device() {
+  static int cache[64] = {0};
+  const int d = current_device();
+  if (d < 0 || d >= 64) return 148;
+  if (!cache[d]) {
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, d) != cudaSuccess || n <= 0)
+      n = 148;
+    cache[d] = n;
+  }
+  return cache[d];
+}
+
+inline bool aligned(const void *p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+inline size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+bool ragged_ok(const msa_ragged_paged_t *rp) {
+  return rp && rp->input_row_offsets && rp->cache_lengths && rp->kv_lookup_table &&
+         rp->batch >= 1 && rp->total_q >= 0 && rp->max_q_len >= 1 &&
+         rp->max_pages_per_seq >= 1 && rp->num_pages >= 1;
+}
+
+// ---- attention route: tiles, row groups, partitions and the workspace layout
+struct Route {
+  bool plan;      // speculative / prefill: per-tile union in the workspace
+  int qt, tiles;  // query tokens per tile, tiles per sequence
+  int rg;         // 16-row groups per CTA
+  int splits;
+  int cap;        // union capacity per item
+  size_t off_o, off_lse, off_list, off_masks, off_counts, bytes;
+};
+
+constexpr int kMaxRows = 64;     // rows (tokens x group heads) per attention CTA
+constexpr int kMaxSplits = 256;
+
+int default_splits(int batch, int max_q_len, int H_kv, int S, int num_sms) {
+  if (max_q_len > MSA_MAX_SPEC_DRAFT) return 1;
+  const long long units = static_cast<long long>(batch) * H_kv;
+  long long ns = (2LL * num_sms + units - 1) / (units > 0 ? units : 1);
+  const int cap = S / 2 > 1 ? S / 2 : 1;
+  if (ns > cap) ns = cap;
+  if (ns < 1) ns = 1;
+  return static_cast<int>(ns);
+}
+
+bool make_route(const msa_ragged_paged_t *rp, int S, int H_q, int H_kv, int max_blocks,
+                int num_splits, int num_sms, Route *r) {
+  const int G = H_q / H_kv;
+  r->plan = rp->max_q_len > 1;
+  if (!r->plan) {
+    r->qt = 1;
+  } else {
+    int qt = kMaxRows / G;
+    if (qt > 32) qt = 32;  // token masks are 32-bit
+    if (qt > rp->max_q_len) qt = rp->max_q_len;
+    r->qt = qt < 1 ? 1 : qt;
+  }
+  r->tiles = (rp->max_q_len + r->qt - 1) / r->qt;
+  r->rg = (r->qt * G + 15) / 16;
+  if (r->rg < 1 || r->rg > 4) return false;
+  if (rp->max_q_len > MSA_MAX_SPEC_DRAFT)
+    r->splits = 1;
+  else
+    r->splits = num_splits > 0 ? num_splits
+                               : default_splits(rp->batch, rp->max_q_len, H_kv, S, num_sms);
+  const long long cap = static_cast<long long>(r->qt) * S;
+  r->cap = static_cast<int>(cap < max_blocks ? cap : max_blocks);
+  const size_t rows = static_cast<size_t>(rp->total_q) * H_q;
+  const size_t items = static_cast<size_t>(rp->batch) * r->tiles * H_kv;
+  size_t off = 0;
+  r->off_o = off;
+  if (r->splits > 1) off = round_up(off + rows * kHeadDim * sizeof(float) * r->splits, 256);
+  r->off_lse = off;
+  if (r->splits > 1) off = round_up(off + rows * sizeof(float) * r->splits, 256);
+  r->off_list = off;
+  if (r->plan) off = round_up(off + items * r->cap * sizeof(int32_t), 256);
+  r->off_masks = off;
+  if (r->plan) off = round_up(off + items * r->cap * sizeof(uint32_t), 256);
+  r->off_counts = off;
+  if (r->plan) off = round_up(off + items * sizeof(int32_t), 256);
+  r->bytes = off;
+  return true;
+}
+
+}  // namespace
+
+// One cudaFuncSetAttribute per (kernel, device) for the dynamic shared-memory opt-in.
+cudaError_t ensure_smem_limit(const void *func, int bytes) {
+  struct Entry {
+    const void *func;
+    int device;
+    int bytes;
+  };
+  static Entry table[256];
+  static int n = 0;
+  static std::mutex mu;
+  const int dev = current_device();
+  std::lock_guard<std::mutex> lock(mu);
+  for (int i = 0; i < n; ++i)
+    if (table[i].func == func && table[i].device == dev && table[i].bytes >= bytes)
+      return cudaSuccess;
+  cudaError_t e = cudaFuncSetAttribute(func, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (e != cudaSuccess) return e;
+  if (n < 256) table[n++] = Entry{func, dev, bytes};
+  return cudaSuccess;
+}
+
+}  // namespace msa
+
+using namespace msa;
+
+extern "C" {
+
+const char *msa_status_string(msa_status_t status) {
+  switch (status) {
+    case MSA_OK: return "MSA_OK";
+    case MSA_ERR_INVALID_ARG: return "MSA_ERR_INVALID_ARG";
+    case MSA_ERR_UNSUPPORTED: return "MSA_ERR_UNSUPPORTED";
+    case MSA_ERR_CUDA: return "MSA_ERR_CUDA";
+  }
+  return "MSA_ERR_UNKNOWN";
+}
+
+int32_t msa_default_num_splits(int32_t batch, int32_t max_q_len, int32_t num_kv_heads, int32_t S,
+                               int32_t num_sms) {
+  if (batch < 1 || max_q_len < 1 || num_kv_heads < 1 || S < 1 || num_sms < 1) return 1;
+  return default_splits(batch, max_q_len, num_kv_heads, S, num_sms);
+}
+
+size_t msa_attn_workspace_bytes(const msa_ragged_paged_t *rp, int32_t S, int32_t num_q_heads,
+                                int32_t num_kv_heads, int32_t max_blocks, int32_t num_splits) {
+  if (!rp || rp->batch < 1 || rp->max_q_len < 1 || S < 1 || num_kv_heads < 1 ||
+      num_q_heads < num_kv_heads || num_q_heads % num_kv_heads || max_blocks < 1 ||
+      num_splits < 0)
+    return 0;
+  Route r;
+  const int sms = num_splits > 0 ? 1 : num_sms_of_current_device();
+  if (!make_route(rp, S, num_q_heads, num_kv_heads, max_blocks, num_splits, sms, &r)) return 0;
+  return r.bytes;
+}
+
+msa_status_t msa_index_scores(const msa_ragged_paged_t *rp, const void *q_idx,
+                              const void *k_idx_cache, int32_t num_kv_heads,
+                              int32_t num_idx_k_heads, int32_t max_blocks, float *scores,
+                              int32_t *dev_err, struct CUstream_st *stream) {
+  if (ragged_ok(rp) && rp->total_q == 0) return MSA_OK;  // nothing to score
+  if (!ragged_ok(rp) || !q_idx || !k_idx_cache || !scores || num_kv_heads < 1 ||
+      !(num_idx_k_heads == 1 || num_idx_k_heads == num_kv_heads) || max_blocks < 1 ||
+      max_blocks > rp->max_pages_per_seq || !aligned(k_idx_cache, 16) || !aligned(q_idx, 4))
+    return MSA_ERR_INVALID_ARG;
+  const int Hg = num_kv_heads / num_idx_k_heads;
+  if (Hg > 32) return MSA_ERR_UNSUPPORTED;
+  if (static_cast<long long>(rp->num_pages) * num_idx_k_heads >= (1LL << 31))
+    return MSA_ERR_UNSUPPORTED;
+
+  IndexerArgs a;
+  a.row_off = rp->input_row_offsets;
+  a.cache_len = rp->cache_lengths;
+  a.table = rp->kv_lookup_table;
+  a.q_idx = static_cast<const uint16_t *>(q_idx);
+  a.scores = scores;
+  a.dev_err = dev_err;
+  a.batch = rp->batch;
+  a.max_q_len = rp->max_q_len;
+  a.max_pages = rp->max_pages_per_seq;
+  a.num_pages = rp->num_pages;
+  a.H_kv = num_kv_heads;
+  a.H_idxk = num_idx_k_heads;
+  a.max_blocks = max_blocks;
+  a.qt = rp->max_q_len * Hg <= 32 ? rp->max_q_len : (32 / Hg > 0 ? 32 / Hg : 1);
+  a.tiles = (rp->max_q_len + a.qt - 1) / a.qt;
+  const int mt = a.qt * Hg <= 16 ? 1 : 2;
+  // pages per CTA: about eight CTAs per SM over the launch, at least 4 pages each
+  const long long units = static_cast<long long>(rp->batch) * a.tiles * num_idx_k_heads;
+  if (units > 0x7fffffffLL) return MSA_ERR_UNSUPPORTED;
+  const long long want = (8LL * num_sms_of_current_device() + units - 1) / units;
+  long long chunk = (max_blocks + want - 1) / want;
+  if (chunk < 4) chunk = 4;
+  long long chunks = (max_blocks + chunk - 1) / chunk;
+  if (chunks > 65535) {
+    chunks = 65535;
+    chunk = (max_blocks + chunks - 1) / chunks;
+  }
+  a.chunk = static_cast<int>(chunk);
+
+  CUtensorMap kmap;
+  if (!page_tensor_map(&kmap, k_idx_cache, static_cast<long long>(rp->num_pages) * num_idx_k_heads,
+                       false))
+    return MSA_ERR_CUDA;
+  return launch_index_scores(kmap, a, mt, static_cast<int>(chunks),
+                             reinterpret_cast<cudaStream_t>(stream)) == cudaSuccess
+             ? MSA_OK
+             : MSA_ERR_CUDA;
+}
+
+msa_status_t msa_select_blocks(const msa_ragged_paged_t *rp, const float *scores,
+                               int32_t num_kv_heads, int32_t max_blocks, int32_t top_k,
+                               int32_t init_blocks, int32_t local_blocks, int32_t *block_ids,
+                               int32_t *num_selected, int32_t *dev_err,
+                               struct CUstream_st *stream) {
+  const long long S = static_cast<long long>(top_k) + init_blocks + local_blocks;
+  if (!ragged_ok(rp) || num_kv_heads < 1 || max_blocks < 1 || top_k < 0 || init_blocks < 0 ||
+      local_blocks < 0 || S < 1 || S > (1 << 20))
+    return MSA_ERR_INVALID_ARG;
+  if (rp->total_q == 0) return MSA_OK;
+  if (!scores || !block_ids || !num_selected) return MSA_ERR_INVALID_ARG;
+  SelectArgs a;
+  a.row_off = rp->input_row_offsets;
+  a.cache_len = rp->cache_lengths;
+  a.scores = scores;
+  a.block_ids = block_ids;
+  a.num_selected = num_selected;
+  a.dev_err = dev_err;
+  a.batch = rp->batch;
+  a.total_q = rp->total_q;
+  a.H_kv = num_kv_heads;
+  a.max_blocks = max_blocks;
+  a.top_k = top_k;
+  a.init_blocks = init_blocks;
+  a.local_blocks = local_blocks;
+  a.S = static_cast<int>(S);
+  return launch_select(a, reinterpret_cast<cudaStream_t>(stream)) == cudaSuccess ? MSA_OK
+                                                                                 : MSA_ERR_CUDA;
+}
+
+msa_status_t msa_splitk_combine(const float *partial_o, const float *partial_lse,
+                                int32_t num_splits, int32_t total_q, int32_t num_q_heads,
+                                void *out, struct CUstream_st *stream) {
+  if (num_splits < 1 || total_q < 0 || num_q_heads < 1) return MSA_ERR_INVALID_ARG;
+  if (total_q == 0) return MSA_OK;
+  if (!partial_o || !partial_lse || !out || !aligned(partial_o, 16) || !aligned(out, 8))
+    return MSA_ERR_INVALID_ARG;
+  return launch_combine(partial_o, partial_lse, num_splits, total_q, num_q_heads,
+                        static_cast<uint16_t *>(out),
+                        reinterpret_cast<cudaStream_t>(stream)) == cudaSuccess
+             ? MSA_OK
+             : MSA_ERR_CUDA;
+}
+
+msa_status_t msa_sparse_attn_paged(const msa_ragged_paged_t *rp, const void *q,
+                                   const void *k_cache, const void *v_cache,
+                                   msa_kv_dtype_t kv_dtype, const int32_t *block_ids,
+                                   const int32_t *num_selected, int32_t S, int32_t num_q_heads,
+                                   int32_t num_kv_heads, int32_t max_blocks, float scale,
+                                   int32_t num_splits, void *workspace, size_t workspace_bytes,
+                                   void *out, int32_t *dev_err, struct CUstream_st *stream) {
+  if (ragged_ok(rp) && rp->total_q == 0 && S >= 1) return MSA_OK;  // nothing to attend
+  if (!ragged_ok(rp) || !q || !k_cache || !v_cache || !block_ids || !num_selected || !out ||
+      S < 1 || num_kv_heads < 1 || num_q_heads < num_kv_heads ||
+      num_q_heads % num_kv_heads != 0 || max_blocks < 1 || max_blocks > rp->max_pages_per_seq ||
+      !(scale > 0.f) || !isfinite(scale) || num_splits < 0 || num_splits > kMaxSplits ||
+      !(kv_dtype == MSA_KV_BF16 || kv_dtype == MSA_KV_FP8_E4M3) || !aligned(q, 16) ||
+      !aligned(k_cache, 16) || !aligned(v_cache, 16) || !aligned(out, 8))
+    return MSA_ERR_INVALID_ARG;
+  const int G = num_q_heads / num_kv_heads;
+  if (G > kMaxRows) return MSA_ERR_UNSUPPORTED;
+  if (static_cast<long long>(rp->num_pages) * num_kv_heads >= (1LL << 31))
+    return MSA_ERR_UNSUPPORTED;
+  Route r;
+  if (!make_route(rp, S, num_q_heads, num_kv_heads, max_blocks, num_splits,
+                  num_sms_of_current_device(), &r))
+    return MSA_ERR_UNSUPPORTED;
+  if (r.plan && (2 * ((max_blocks + 31) / 32) + r.cap) * 4 > 200 * 1024)
+    return MSA_ERR_UNSUPPORTED;
+  if (static_cast<long long>(rp->batch) * r.tiles > 0x7fffffffLL) return MSA_ERR_UNSUPPORTED;
+  if (r.bytes > 0 && (!workspace || workspace_bytes < r.bytes || !aligned(workspace, 256)))
+    return MSA_ERR_INVALID_ARG;
+
+  uint8_t *ws = static_cast<uint8_t *>(workspace);
+  const cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const bool fp8 = kv_dtype == MSA_KV_FP8_E4M3;
+
+  if (r.plan) {
+    PlanArgs p;
+    p.row_off = rp->input_row_offsets;
+    p.cache_len = rp->cache_lengths;
+    p.block_ids = block_ids;
+    p.num_selected = num_selected;
+    p.list = reinterpret_cast<int32_t *>(ws + r.off_list);
+    p.masks = reinterpret_cast<uint32_t *>(ws + r.off_masks);
+    p.counts = reinterpret_cast<int32_t *>(ws + r.off_counts);
+    p.dev_err = dev_err;
+    p.batch = rp->batch;
+    p.max_q_len = rp->max_q_len;
+    p.H_kv = num_kv_heads;
+    p.S = S;
+    p.max_blocks = max_blocks;
+    p.qt = r.qt;
+    p.tiles = r.tiles;
+    p.cap = r.cap;
+    if (launch_plan(p, s) != cudaSuccess) return MSA_ERR_CUDA;
+  }
+
+  CUtensorMap kmap, vmap;
+  const long long tiles = static_cast<long long>(rp->num_pages) * num_kv_heads;
+  if (!page_tensor_map(&kmap, k_cache, tiles, fp8) || !page_tensor_map(&vmap, v_cache, tiles, fp8))
+    return MSA_ERR_CUDA;
+
+  AttnArgs a;
+  a.row_off = rp->input_row_offsets;
+  a.cache_len = rp->cache_lengths;
+  a.table = rp->kv_lookup_table;
+  a.q = static_cast<const uint16_t *>(q);
+  a.block_ids = block_ids;
+  a.num_selected = num_selected;
+  a.plan_list = reinterpret_cast<const int32_t *>(ws + r.off_list);
+  a.plan_masks = reinterpret_cast<const uint32_t *>(ws + r.off_masks);
+  a.plan_counts = reinterpret_cast<const int32_t *>(ws + r.off_counts);
+  a.S = S;
+  a.cap = r.cap;
+  a.batch = rp->batch;
+  a.total_q = rp->total_q;
+  a.max_q_len = rp->max_q_len;
+  a.max_pages = rp->max_pages_per_seq;
+  a.num_pages = rp->num_pages;
+  a.H_q = num_q_heads;
+  a.H_kv = num_kv_heads;
+  a.G = G;
+  a.max_blocks = max_blocks;
+  a.qt = r.qt;
+  a.tiles = r.tiles;
+  a.splits = r.splits;
+  a.scale_log2 = scale * 1.4426950408889634f;
+  a.part_o = reinterpret_cast<float *>(ws + r.off_o);
+  a.part_lse = reinterpret_cast<float *>(ws + r.off_lse);
+  a.out = static_cast<uint16_t *>(out);
+  a.dev_err = dev_err;
+  if (launch_attention(kmap, vmap, a, fp8, r.rg, r.plan, s) != cudaSuccess) return MSA_ERR_CUDA;
+  if (r.splits > 1 &&
+      launch_combine(a.part_o, a.part_lse, r.splits, rp->total_q, num_q_heads, a.out, s) !=
+          cudaSuccess)
+    return MSA_ERR_CUDA;
+  return MSA_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,243 @@
+// indexer.cu — stage 1: block scores of the index-K cache.
+//
+// ferrox-core "Module block_sparse", "Four rules": a block's score is the MAX over its
+// positions of the raw dot product (no softmax scale), and one index head scores for one KV
+// head.  Mojo module "msa": the index-K cache is BF16 with a single head (the build also
+// accepts one index-K head per KV head).
+//
+// One CTA scores a chunk of pages of one sequence for a tile of its query tokens and all the
+// index-query heads that read one index-K head (rows = tokens x heads, at most 32).  A
+// producer warp streams the 32 KiB page tiles with TMA (128-byte swizzle) through a ring of
+// shared-memory stages; four consumer warps each take 32 of the 128 positions, compute
+// S = Q K^T with bf16 mma.sync (fp32 accumulation), mask positions after each row's query
+// position, reduce the row max with warp shuffles and then across the four warps through
+// shared memory, and write one fp32 score per (row, page).
+#include <math.h>
+
+#include "internal.h"
+#include "ptx.cuh"
+
+namespace msa {
+
+namespace {
+
+constexpr int kStages = 3;
+constexpr uint32_t kTileBytes = kBlock * kHeadDim * 2;  // one (page, head) tile, bf16
+constexpr int kConsumerWarps = 4;
+constexpr int kThreads = 32 * (kConsumerWarps + 1);
+
+constexpr size_t smem_bytes() {
+  return 1024 /*alignment slack*/ + kStages * kTileBytes + 2 * kStages * sizeof(uint64_t) +
+         kStages * sizeof(int) + 2 * kConsumerWarps * 32 * sizeof(float) + 16;
+}
+
+template <int MT>
+__global__ void __launch_bounds__(kThreads)
+    index_scores_kernel(const __grid_constant__ CUtensorMap kmap, const IndexerArgs a) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int cx = blockIdx.y, b = blockIdx.x / a.tiles, tile = blockIdx.x % a.tiles;
+  const int hk = blockIdx.z;
+  const bool reporter = threadIdx.x == 0 && cx == 0 && tile == 0 && hk == 0;
+
+  const int row0 = a.row_off[b];
+  int q_len = a.row_off[b + 1] - row0;
+  if (q_len < 0 || q_len > a.max_q_len) {
+    if (reporter) report(a.dev_err, MSA_DEVERR_LENGTHS);
+    q_len = q_len < 0 ? 0 : a.max_q_len;
+  }
+  const int tok0 = tile * a.qt;
+  if (tok0 >= q_len) return;
+  const int ntok = min(a.qt, q_len - tok0);
+  const int Hg = a.H_kv / a.H_idxk;  // index-query heads per index-K head
+  const int rows = ntok * Hg;
+  int cl = a.cache_len[b];
+  if (cl < 0) {
+    if (reporter) report(a.dev_err, MSA_DEVERR_LENGTHS);
+    cl = 0;
+  }
+  int nb_last = (cl + tok0 + ntok - 1) / kBlock + 1;  // blocks visible to the tile's last token
+  if (nb_last > a.max_blocks) {
+    if (reporter) report(a.dev_err, MSA_DEVERR_LENGTHS);
+    nb_last = a.max_blocks;
+  }
+  const int j0 = cx * a.chunk;
+  const int j_end = min(j0 + a.chunk, a.max_blocks);
+  const int j1 = min(j_end, nb_last);  // pages scored here: [j0, j1)
+
+  // Blocks of this chunk that no token of the tile can see score -inf.
+  {
+    const int f0 = max(j0, j1), nf = j_end - f0;
+    for (int idx = threadIdx.x; idx < nf * rows; idx += blockDim.x) {
+      const int r = idx / nf, j = f0 + idx % nf;
+      const int t = row0 + tok0 + r / Hg, g = hk + (r % Hg) * a.H_idxk;
+      a.scores[(static_cast<size_t>(t) * a.H_kv + g) * a.max_blocks + j] = -INFINITY;
+    }
+  }
+  const int npages = j1 - j0;
+  if (npages <= 0) return;
+
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                              ~static_cast<uintptr_t>(1023));
+  uint8_t *stages = smem;
+  uint64_t *full = reinterpret_cast<uint64_t *>(stages + kStages * kTileBytes);
+  uint64_t *empty = full + kStages;
+  int *page_ok = reinterpret_cast<int *>(empty + kStages);
+  float *red = reinterpret_cast<float *>(page_ok + kStages);  // [2][4 warps][32 rows]
+  volatile int *abort_flag = reinterpret_cast<volatile int *>(red + 2 * kConsumerWarps * 32);
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], kConsumerWarps);
+    }
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  __syncthreads();
+
+  if (warp == kConsumerWarps) {
+    // ------------------------------------------------------------ producer: TMA page ring
+    if (lane == 0) {
+      prefetch_tmap(&kmap);
+      for (int i = 0; i < npages; ++i) {
+        const int s = i % kStages;
+        if (i >= kStages && !mbar_wait(&empty[s], ((i / kStages) - 1) & 1, abort_flag)) {
+          report(a.dev_err, MSA_DEVERR_TIMEOUT);
+          *abort_flag = 1;
+          break;
+        }
+        const int page = a.table[static_cast<size_t>(b) * a.max_pages + j0 + i];
+        const bool ok = page >= 0 && page < a.num_pages;
+        page_ok[s] = ok;
+        if (ok) {
+          mbar_arrive_expect_tx(&full[s], kTileBytes);
+          const int c2 = page * a.H_idxk + hk;
+          tma_load_3d(stages + s * kTileBytes, &kmap, &full[s], 0, 0, c2);
+          tma_load_3d(stages + s * kTileBytes + kTileBytes / 2, &kmap, &full[s], 64, 0, c2);
+        } else {
+          report(a.dev_err, MSA_DEVERR_PAGE_ID);
+          mbar_arrive(&full[s]);
+        }
+      }
+    }
+    return;
+  }
+
+  // -------------------------------------------------------------- consumers
+  // A fragments of Q (rows x 128) for m16n8k16: a0a1 = (row, k), a2a3 = (row + 8, k),
+  // a4a5 = (row, k + 8), a6a7 = (row + 8, k + 8), k = 16 ks + 2 (lane % 4).
+  uint32_t qa[MT][8][4];
+  int prow[MT][2];
+#pragma unroll
+  for (int mt = 0; mt < MT; ++mt) {
+#pragma unroll
+    for (int slot = 0; slot < 2; ++slot) {
+      const int r = mt * 16 + (lane >> 2) + slot * 8;
+      prow[mt][slot] = r < rows ? cl + tok0 + r / Hg : -1;
+    }
+#pragma unroll
+    for (int ks = 0; ks < 8; ++ks) {
+#pragma unroll
+      for (int q4 = 0; q4 < 4; ++q4) {
+        const int r = mt * 16 + (lane >> 2) + (q4 & 1) * 8;
+        const int k = ks * 16 + (lane & 3) * 2 + (q4 >> 1) * 8;
+        uint32_t v = 0;
+        if (r < rows) {
+          const int t = row0 + tok0 + r / Hg, g = hk + (r % Hg) * a.H_idxk;
+          v = *reinterpret_cast<const uint32_t *>(
+              a.q_idx + (static_cast<size_t>(t) * a.H_kv + g) * kHeadDim + k);
+        }
+        qa[mt][ks][q4] = v;
+      }
+    }
+  }
+
+  const int pbase = warp * 32;  // this warp's 32 positions of every page
+  const int mi = lane >> 3, rr = lane & 7;
+  for (int i = 0; i < npages; ++i) {
+    const int s = i % kStages;
+    const int j = j0 + i;
+    bool live = mbar_wait(&full[s], (i / kStages) & 1, abort_flag);
+    if (!live) {
+      report(a.dev_err, MSA_DEVERR_TIMEOUT);
+      *abort_flag = 1;
+    }
+    const bool ok = live && page_ok[s];
+    float acc[MT][4][4];
+#pragma unroll
+    for (int mt = 0; mt < MT; ++mt)
+#pragma unroll
+      for (int nt = 0; nt < 4; ++nt)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) acc[mt][nt][e] = 0.f;
+    if (ok) {
+      const uint32_t tile_addr = smem_u32(stages + s * kTileBytes);
+#pragma unroll
+      for (int ks = 0; ks < 8; ++ks) {
+        uint32_t bf[4][2];
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          const int pos = pbase + h * 16 + (mi >> 1) * 8 + rr;
+          const int chunk = ks * 2 + (mi & 1);
+          ldsm_x4(tile_addr + sw128(pos, chunk, kTileBytes / 2), bf[2 * h][0], bf[2 * h][1],
+                  bf[2 * h + 1][0], bf[2 * h + 1][1]);
+        }
+#pragma unroll
+        for (int mt = 0; mt < MT; ++mt)
+#pragma unroll
+          for (int nt = 0; nt < 4; ++nt) mma_bf16(acc[mt][nt], qa[mt][ks], bf[nt][0], bf[nt][1]);
+      }
+    }
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&empty[s]);
+
+    // Row max over this warp's 32 positions (only positions <= the row's query position).
+    float *rbuf = red + (i & 1) * kConsumerWarps * 32;
+#pragma unroll
+    for (int mt = 0; mt < MT; ++mt) {
+#pragma unroll
+      for (int slot = 0; slot < 2; ++slot) {
+        float mx = -INFINITY;
+#pragma unroll
+        for (int nt = 0; nt < 4; ++nt)
+#pragma unroll
+          for (int e = 0; e < 2; ++e) {
+            const int pos = j * kBlock + pbase + nt * 8 + (lane & 3) * 2 + e;
+            if (ok && pos <= prow[mt][slot]) mx = fmaxf(mx, acc[mt][nt][slot * 2 + e]);
+          }
+        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
+        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
+        if ((lane & 3) == 0) rbuf[warp * 32 + mt * 16 + (lane >> 2) + slot * 8] = mx;
+      }
+    }
+    named_bar_sync(1, kConsumerWarps * 32);
+    const int r = threadIdx.x;
+    if (r < rows) {
+      float m = rbuf[r];
+#pragma unroll
+      for (int w = 1; w < kConsumerWarps; ++w) m = fmaxf(m, rbuf[w * 32 + r]);
+      const int t = row0 + tok0 + r / Hg, g = hk + (r % Hg) * a.H_idxk;
+      a.scores[(static_cast<size_t>(t) * a.H_kv + g) * a.max_blocks + j] = m;
+    }
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_index_scores(const CUtensorMap &kidx_map, const IndexerArgs &a, int mt,
+                                int chunks, cudaStream_t s) {
+  const dim3 grid(a.batch * a.tiles, chunks, a.H_idxk);
+  const size_t smem = smem_bytes();
+  const void *fn = mt == 1 ? reinterpret_cast<const void *>(&index_scores_kernel<1>)
+                           : reinterpret_cast<const void *>(&index_scores_kernel<2>);
+  cudaError_t e = ensure_smem_limit(fn, static_cast<int>(smem));
+  if (e != cudaSuccess) return e;
+  if (mt == 1)
+    index_scores_kernel<1><<<grid, kThreads, smem, s>>>(kidx_map, a);
+  else
+    index_scores_kernel<2><<<grid, kThreads, smem, s>>>(kidx_map, a);
+  return cudaGetLastError();
+}
+
+}  // namespace msa

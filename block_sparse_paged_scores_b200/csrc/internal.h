@@ -1,0 +1,78 @@
+// internal.h — argument blocks and launchers shared between the kernels and the C-ABI layer.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include "msa.h"
+
+namespace msa {
+
+constexpr int kBlock = 128;    // tokens per block == tokens per page
+constexpr int kHeadDim = 128;  // head dim of q / k / v / q_idx / k_idx
+
+// ---- stage 1: block scores (indexer.cu)
+struct IndexerArgs {
+  const int32_t *row_off, *cache_len, *table;
+  const uint16_t *q_idx;  // bf16 bits [total_q, H_kv, 128]
+  float *scores;          // [total_q, H_kv, max_blocks]
+  int32_t *dev_err;
+  int batch, max_q_len, max_pages, num_pages, H_kv, H_idxk, max_blocks;
+  int qt;     // query tokens per tile
+  int tiles;  // tiles per sequence
+  int chunk;  // pages per CTA
+};
+// mt = 16-row MMA tiles per CTA (1 or 2)
+cudaError_t launch_index_scores(const CUtensorMap &kidx_map, const IndexerArgs &a, int mt,
+                                int chunks, cudaStream_t s);
+
+// ---- stage 2: selection (select.cu)
+struct SelectArgs {
+  const int32_t *row_off, *cache_len;
+  const float *scores;
+  int32_t *block_ids, *num_selected, *dev_err;
+  int batch, total_q, H_kv, max_blocks, top_k, init_blocks, local_blocks, S;
+};
+cudaError_t launch_select(const SelectArgs &a, cudaStream_t s);
+
+// ---- per-tile union of the tokens' selections (plan.cu)
+struct PlanArgs {
+  const int32_t *row_off, *cache_len, *block_ids, *num_selected;
+  int32_t *list;     // [items, cap] ascending block ids
+  uint32_t *masks;   // [items, cap] bit i: token tok0 + i selected the block
+  int32_t *counts;   // [items]
+  int32_t *dev_err;
+  int batch, max_q_len, H_kv, S, max_blocks, qt, tiles, cap;
+};
+cudaError_t launch_plan(const PlanArgs &a, cudaStream_t s);
+
+// ---- stage 3: sparse paged attention (attention.cu)
+struct AttnArgs {
+  const int32_t *row_off, *cache_len, *table;
+  const uint16_t *q;  // bf16 bits [total_q, H_q, 128]
+  const int32_t *block_ids, *num_selected;  // decode route: the selection itself
+  const int32_t *plan_list;                 // other routes: the per-tile union
+  const uint32_t *plan_masks;
+  const int32_t *plan_counts;
+  int S, cap;
+  int batch, total_q, max_q_len, max_pages, num_pages, H_q, H_kv, G, max_blocks;
+  int qt, tiles, splits;
+  float scale_log2;  // scale * log2(e)
+  float *part_o, *part_lse;  // splits > 1
+  uint16_t *out;             // splits == 1: bf16 bits [total_q, H_q, 128]
+  int32_t *dev_err;
+};
+// rg = 16-row groups (1..4), plan = read the per-tile union instead of the selection
+cudaError_t launch_attention(const CUtensorMap &kmap, const CUtensorMap &vmap, const AttnArgs &a,
+                             bool fp8, int rg, bool plan, cudaStream_t s);
+
+// ---- split-K combine (combine.cu)
+cudaError_t launch_combine(const float *part_o, const float *part_lse, int splits, int total_q,
+                           int H_q, uint16_t *out, cudaStream_t s);
+
+// Sets the dynamic shared-memory limit of `func` once per device.
+cudaError_t ensure_smem_limit(const void *func, int bytes);
+
+}  // namespace msa

@@ -1,0 +1,201 @@
+"""ctypes binding of libmsa.so (include/msa.h), one Python function per C entry point.
+
+Argument marshalling only: every step of the path runs in the library's CUDA kernels.  Torch
+tensors supply device memory and the current CUDA stream.  The library is loaded on first use
+and a missing or unloadable library raises: there is no fallback.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libmsa.so")
+
+MSA_OK, MSA_ERR_INVALID_ARG, MSA_ERR_UNSUPPORTED, MSA_ERR_CUDA = 0, 1, 2, 3
+MSA_KV_BF16, MSA_KV_FP8_E4M3 = 0, 1
+MSA_DEVERR_PAGE_ID, MSA_DEVERR_LENGTHS, MSA_DEVERR_BLOCK_ID = 1, 2, 4
+MSA_DEVERR_NUM_SELECTED, MSA_DEVERR_TIMEOUT = 8, 16
+BLOCK = 128
+HEAD_DIM = 128
+
+
+class MSAError(RuntimeError):
+    def __init__(self, fn: str, status: int):
+        super().__init__(f"{fn} returned {msa_status_string(status)} ({status})")
+        self.status = status
+
+
+class RaggedPaged(ctypes.Structure):
+    """msa_ragged_paged_t."""
+    _fields_ = [("input_row_offsets", ctypes.c_void_p), ("cache_lengths", ctypes.c_void_p),
+                ("kv_lookup_table", ctypes.c_void_p), ("batch", ctypes.c_int32),
+                ("total_q", ctypes.c_int32), ("max_q_len", ctypes.c_int32),
+                ("max_pages_per_seq", ctypes.c_int32), ("num_pages", ctypes.c_int32)]
+
+
+_lib: Optional[ctypes.CDLL] = None
+
+
+def load(path: str = LIB_PATH) -> ctypes.CDLL:
+    """Load libmsa.so (once).  Raises if it has not been built."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(path):
+        raise RuntimeError(f"{path} is missing: build it with "
+                           "`python -m block_sparse_paged_scores_b200.build`")
+    lib = ctypes.CDLL(path)
+    P, I, F = ctypes.c_void_p, ctypes.c_int32, ctypes.c_float
+    RP = ctypes.POINTER(RaggedPaged)
+    lib.msa_index_scores.restype = I
+    lib.msa_index_scores.argtypes = [RP, P, P, I, I, I, P, P, P]
+    lib.msa_select_blocks.restype = I
+    lib.msa_select_blocks.argtypes = [RP, P, I, I, I, I, I, P, P, P, P]
+    lib.msa_sparse_attn_paged.restype = I
+    lib.msa_sparse_attn_paged.argtypes = [RP, P, P, P, I, P, P, I, I, I, I, F, I, P,
+                                          ctypes.c_size_t, P, P, P]
+    lib.msa_splitk_combine.restype = I
+    lib.msa_splitk_combine.argtypes = [P, P, I, I, I, P, P]
+    lib.msa_attn_workspace_bytes.restype = ctypes.c_size_t
+    lib.msa_attn_workspace_bytes.argtypes = [RP, I, I, I, I, I]
+    lib.msa_default_num_splits.restype = I
+    lib.msa_default_num_splits.argtypes = [I, I, I, I, I]
+    lib.msa_status_string.restype = ctypes.c_char_p
+    lib.msa_status_string.argtypes = [I]
+    _lib = lib
+    return lib
+
+
+def _ptr(t) -> Optional[int]:
+    if t is None:
+        return None
+    if isinstance(t, int):
+        return t
+    return t.data_ptr()
+
+
+def _stream(stream) -> Optional[int]:
+    if stream is None:
+        if torch.cuda.is_available():
+            return torch.cuda.current_stream().cuda_stream
+        return None
+    if isinstance(stream, int):
+        return stream
+    return stream.cuda_stream
+
+
+def _check(fn: str, status: int):
+    if status != MSA_OK:
+        raise MSAError(fn, status)
+
+
+def ragged_paged(input_row_offsets, cache_lengths, kv_lookup_table, total_q: int, max_q_len: int,
+                 num_pages: int) -> RaggedPaged:
+    """Build the msa_ragged_paged_t view of int32 device tensors (no copies)."""
+    return RaggedPaged(_ptr(input_row_offsets), _ptr(cache_lengths), _ptr(kv_lookup_table),
+                       int(input_row_offsets.numel()) - 1, int(total_q), int(max_q_len),
+                       int(kv_lookup_table.shape[-1]), int(num_pages))
+
+
+def msa_status_string(status: int) -> str:
+    return load().msa_status_string(int(status)).decode()
+
+
+def msa_default_num_splits(batch: int, max_q_len: int, num_kv_heads: int, S: int,
+                           num_sms: int) -> int:
+    return int(load().msa_default_num_splits(batch, max_q_len, num_kv_heads, S, num_sms))
+
+
+def msa_attn_workspace_bytes(rp: RaggedPaged, S: int, num_q_heads: int, num_kv_heads: int,
+                             max_blocks: int, num_splits: int) -> int:
+    return int(load().msa_attn_workspace_bytes(ctypes.byref(rp), S, num_q_heads, num_kv_heads,
+                                               max_blocks, num_splits))
+
+
+def msa_index_scores(rp: RaggedPaged, q_idx, k_idx_cache, num_kv_heads: int,
+                     num_idx_k_heads: int, max_blocks: int, scores, dev_err=None, stream=None):
+    _check("msa_index_scores", load().msa_index_scores(
+        ctypes.byref(rp), _ptr(q_idx), _ptr(k_idx_cache), num_kv_heads, num_idx_k_heads,
+        max_blocks, _ptr(scores), _ptr(dev_err), _stream(stream)))
+
+
+def msa_select_blocks(rp: RaggedPaged, scores, num_kv_heads: int, max_blocks: int, top_k: int,
+                      init_blocks: int, local_blocks: int, block_ids, num_selected, dev_err=None,
+                      stream=None):
+    _check("msa_select_blocks", load().msa_select_blocks(
+        ctypes.byref(rp), _ptr(scores), num_kv_heads, max_blocks, top_k, init_blocks,
+        local_blocks, _ptr(block_ids), _ptr(num_selected), _ptr(dev_err), _stream(stream)))
+
+
+def msa_sparse_attn_paged(rp: RaggedPaged, q, k_cache, v_cache, kv_dtype: int, block_ids,
+                          num_selected, S: int, num_q_heads: int, num_kv_heads: int,
+                          max_blocks: int, scale: float, num_splits: int, workspace, out,
+                          dev_err=None, stream=None, workspace_bytes: Optional[int] = None):
+    if workspace_bytes is None:
+        workspace_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _check("msa_sparse_attn_paged", load().msa_sparse_attn_paged(
+        ctypes.byref(rp), _ptr(q), _ptr(k_cache), _ptr(v_cache), int(kv_dtype), _ptr(block_ids),
+        _ptr(num_selected), S, num_q_heads, num_kv_heads, max_blocks, float(scale), num_splits,
+        _ptr(workspace), int(workspace_bytes), _ptr(out), _ptr(dev_err), _stream(stream)))
+
+
+def msa_splitk_combine(partial_o, partial_lse, num_splits: int, total_q: int, num_q_heads: int,
+                       out, stream=None):
+    _check("msa_splitk_combine", load().msa_splitk_combine(
+        _ptr(partial_o), _ptr(partial_lse), num_splits, total_q, num_q_heads, _ptr(out),
+        _stream(stream)))
+
+
+# ------------------------------------------------------------------ whole-path convenience
+class Path:
+    """The three stages over one problem (a dict laid out as ``workload.generate`` returns),
+    with every output and the workspace allocated once on the problem's device.  ``run()``
+    enqueues index scores -> selection -> attention on the current stream."""
+
+    def __init__(self, prob: dict, num_splits: int = 0, max_blocks: Optional[int] = None):
+        self.p = prob
+        dev = prob["q"].device
+        self.max_blocks = int(max_blocks or prob["max_blocks"])
+        self.rp = ragged_paged(prob["row_off"], prob["cache_len"], prob["table"], prob["total_q"],
+                               prob["max_q_len"], prob["num_pages"])
+        tq, hkv, S = prob["total_q"], prob["H_kv"], prob["S"]
+        self.scores = torch.empty((tq, hkv, self.max_blocks), dtype=torch.float32, device=dev)
+        self.block_ids = torch.empty((tq, hkv, S), dtype=torch.int32, device=dev)
+        self.num_selected = torch.empty((tq, hkv), dtype=torch.int32, device=dev)
+        self.out = torch.empty((tq, prob["H_q"], HEAD_DIM), dtype=torch.bfloat16, device=dev)
+        self.dev_err = torch.zeros((1,), dtype=torch.int32, device=dev)
+        self.num_splits = num_splits
+        ws = msa_attn_workspace_bytes(self.rp, S, prob["H_q"], hkv, self.max_blocks, num_splits)
+        self.workspace = torch.empty((max(ws, 1),), dtype=torch.uint8, device=dev)
+        self.workspace_bytes = ws
+        self.kv_dtype = MSA_KV_FP8_E4M3 if prob["kv_fp8"] else MSA_KV_BF16
+
+    def index_scores(self, stream=None):
+        p = self.p
+        msa_index_scores(self.rp, p["q_idx"], p["k_idx"], p["H_kv"], p["H_idxk"], self.max_blocks,
+                         self.scores, self.dev_err, stream)
+
+    def select(self, scores=None, stream=None):
+        p = self.p
+        msa_select_blocks(self.rp, self.scores if scores is None else scores, p["H_kv"],
+                          self.max_blocks, p["top_k"], p["init_blocks"], p["local_blocks"],
+                          self.block_ids, self.num_selected, self.dev_err, stream)
+
+    def attend(self, block_ids=None, num_selected=None, stream=None):
+        p = self.p
+        msa_sparse_attn_paged(self.rp, p["q"], p["k"], p["v"], self.kv_dtype,
+                              self.block_ids if block_ids is None else block_ids,
+                              self.num_selected if num_selected is None else num_selected,
+                              p["S"], p["H_q"], p["H_kv"], self.max_blocks, p["scale"],
+                              self.num_splits, self.workspace, self.out, self.dev_err, stream,
+                              workspace_bytes=self.workspace_bytes)
+
+    def run(self, stream=None):
+        self.index_scores(stream)
+        self.select(stream=stream)
+        self.attend(stream=stream)
+        return self.out

@@ -117,13 +117,13 @@ def generate(spec: WorkloadSpec, seed: int, device="cpu", poison: bool = True) -
         L = prior + q_lens
     else:
         L = _draw(spec.kv_len, spec.batch, gcpu)
-    assert bool((L >= q_lens).all()) and bool((q_lens >= 1).all())
+    assert bool((L >= q_lens).all()) and bool((q_lens >= 0).all())
     cache_len = L - q_lens
     nb = (L + BLOCK - 1) // BLOCK
     total_pages = int(nb.sum())
     pool = max(total_pages, spec.pool_pages)
     perm = torch.randperm(pool, generator=gcpu)
-    max_pages = int(nb.max())
+    max_pages = max(1, int(nb.max()))
     table = torch.full((spec.batch, max_pages), -1, dtype=torch.int32)
     cur = 0
     for b in range(spec.batch):
@@ -160,8 +160,8 @@ def generate(spec: WorkloadSpec, seed: int, device="cpu", poison: bool = True) -
         row_off=row_off.to(device), cache_len=cache_len.to(torch.int32).to(device),
         table=table.to(device), q=q, q_idx=q_idx, k_idx=k_idx, k=k, v=v,
         kv_fp8=spec.kv_dtype == "fp8",
-        batch=spec.batch, total_q=total_q, max_q_len=int(q_lens.max()),
-        max_cache_len=int(cache_len.max()), max_pages=max_pages, num_pages=pool,
+        batch=spec.batch, total_q=total_q, max_q_len=max(1, int(q_lens.max())),
+        max_cache_len=int(cache_len.max()), max_pages=max_pages, num_pages=max(pool, 1),
         max_blocks=max_pages, H_q=spec.H_q, H_kv=spec.H_kv, H_idxk=spec.H_idxk,
         top_k=spec.top_k, init_blocks=spec.init_blocks, local_blocks=spec.local_blocks,
         S=spec.S, scale=1.0 / math.sqrt(HEAD_DIM), kv_lens=L.tolist(), q_lens=q_lens.tolist(),

@@ -1,0 +1,206 @@
+/*
+ * msa.h — C ABI of libmsa.so: MiniMax-M3 block-sparse attention (MSA) over a paged KV cache,
+ * native to NVIDIA B200 (sm_100a).
+ *
+ * The path has three stages, one entry point each, plus the split-K combine:
+ *   msa_index_scores      block scores: max over a 128-token block of raw q_idx . k_idx
+ *   msa_select_blocks     forced init/local blocks + top-k of the rest, ascending
+ *   msa_sparse_attn_paged softmax attention over the selected pages (decode / speculative /
+ *                         prefill routes picked from max_q_len), split-K + combine inside
+ *   msa_splitk_combine    log-sum-exp merge of split-K partials into the ragged output
+ *
+ * Sources (page title, section):
+ *   [msa]    Mojo module "msa" (Graph-op bindings for the MiniMax-M3 block-sparse attention
+ *            kernels): module summary, the two graph ops, "Three attention routes",
+ *            MAX_SPEC_DRAFT.
+ *   [ferrox] ferrox-core "Module block_sparse": "Four rules", "The block size is an ABI",
+ *            BlockSparseConfig, block_sparse_select, positions_of_blocks.
+ *   [latent] Mojo "Struct_latent_sparse_attention_ragged_paged": the ragged / paged argument
+ *            set (input_row_offsets, cache_lengths, kv_lookup_table, scale).
+ *
+ * Conventions shared by every entry point
+ *   - Head dim and page size are both 128 and fixed ([msa] summary; [ferrox] "The block size
+ *     is an ABI").  Index-K is always BF16; main K/V is BF16 or scale-free FP8 e4m3 ([msa]).
+ *   - Every pointer argument named "device" must point to device memory owned by the caller.
+ *     The library allocates no device memory, never synchronises, and never reads device
+ *     memory from the host.  Every call only enqueues work on `stream` and returns.
+ *   - Host-side validation happens before anything is enqueued; a call that returns anything
+ *     but MSA_OK has enqueued nothing.  A failed launch returns MSA_ERR_CUDA.
+ *   - `dev_err` (device int32, nullable): kernels OR a bit mask of MSA_DEVERR_* into it when
+ *     they meet a device-side value outside the declared bounds; the offending work is skipped
+ *     (never read out of bounds, never trap).  The caller zeroes it and reads it when it likes.
+ *   - Outputs must not alias inputs.
+ *   - Query row t of sequence b is row input_row_offsets[b] + i, at position
+ *     p = cache_lengths[b] + i ([msa] "Three attention routes", speculative route).  The new
+ *     tokens' k / v / k_idx rows are already in the cache at [cache_lengths[b], L_b) with
+ *     L_b = cache_lengths[b] + q_len_b.  Block j covers positions [128 j, 128 j + 128) and is
+ *     stored in page kv_lookup_table[b * max_pages_per_seq + j].  A query at p sees the
+ *     nb(p) = p / 128 + 1 blocks whose first position is <= p.
+ */
+#ifndef MSA_H_
+#define MSA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+struct CUstream_st; /* cudaStream_t == struct CUstream_st*; NULL = the legacy default stream */
+
+#if defined(__GNUC__)
+#define MSA_API __attribute__((visibility("default")))
+#else
+#define MSA_API
+#endif
+
+#define MSA_BLOCK 128    /* tokens per block == tokens per page ([ferrox] MINIMAX_BLOCK_SIZE) */
+#define MSA_HEAD_DIM 128 /* [msa] summary: head_dim 128 */
+#define MSA_MAX_SPEC_DRAFT 8 /* [msa] MAX_SPEC_DRAFT: largest max_q_len of the speculative route */
+
+typedef enum {
+    MSA_OK = 0,
+    MSA_ERR_INVALID_ARG = 1, /* a null pointer, a size out of range, a too-small workspace */
+    MSA_ERR_UNSUPPORTED = 2, /* valid but not built: e.g. a GQA group above the kernel limit */
+    MSA_ERR_CUDA = 3         /* the CUDA runtime refused a launch or a tensor-map encode */
+} msa_status_t;
+
+typedef enum { MSA_KV_BF16 = 0, MSA_KV_FP8_E4M3 = 1 } msa_kv_dtype_t;
+
+/* Bits OR-ed into *dev_err by the kernels. */
+#define MSA_DEVERR_PAGE_ID 1u      /* a page id outside [0, num_pages): that block is skipped */
+#define MSA_DEVERR_LENGTHS 2u      /* q_len_b > max_q_len, q_len_b < 0 or nb(p) > max_blocks */
+#define MSA_DEVERR_BLOCK_ID 4u     /* a selected id outside [0, nb(p)) or not ascending */
+#define MSA_DEVERR_NUM_SELECTED 8u /* num_selected outside [0, S] */
+#define MSA_DEVERR_TIMEOUT 16u     /* a pipeline wait gave up (bounded spin); output invalid */
+
+/* The ragged batch and its page table ([latent] argument set; [msa] routes). */
+typedef struct {
+    const int32_t *input_row_offsets; /* device [batch + 1], non-decreasing, [0] == 0 */
+    const int32_t *cache_lengths;     /* device [batch], prior tokens of each sequence */
+    const int32_t *kv_lookup_table;   /* device [batch * max_pages_per_seq] physical page ids */
+    int32_t batch;                    /* host: number of sequences, >= 1 */
+    int32_t total_q;                  /* host: input_row_offsets[batch] */
+    int32_t max_q_len;                /* host: max over b of q_len_b; picks the route */
+    int32_t max_pages_per_seq;        /* host: row stride of kv_lookup_table */
+    int32_t num_pages;                /* host: pages in each paged cache pool */
+} msa_ragged_paged_t;
+
+/*
+ * msa_index_scores — stage 1 ([ferrox] "Four rules": a block's score is the MAX over its
+ * positions, no softmax scale, one index head per KV head; [msa]: the indexer op, single
+ * BF16 index-K head).
+ *
+ *   scores[t, g, j] = max over pos in [128 j, min(128 j + 127, p)] of
+ *                     sum_c q_idx[t, g, c] * k_idx[page(b, j), g % num_idx_k_heads, pos - 128 j, c]
+ *   for j < nb(p); -inf for nb(p) <= j < max_blocks.  FP32 accumulation of exact BF16
+ *   products.  Positions > p (and so every position >= L_b) never enter the max.
+ *
+ *   q_idx        device bf16 [total_q, num_kv_heads, 128]
+ *   k_idx_cache  device bf16 [num_pages, num_idx_k_heads, 128 tokens, 128], 16-byte aligned
+ *   num_idx_k_heads  1 (one index-K head shared by all index-query heads) or num_kv_heads
+ *   max_blocks   row length of `scores`; must be >= nb(p) of every query and
+ *                <= max_pages_per_seq; a larger nb(p) sets MSA_DEVERR_LENGTHS and is clipped
+ *   scores       device fp32 [total_q, num_kv_heads, max_blocks] (output)
+ */
+MSA_API msa_status_t msa_index_scores(const msa_ragged_paged_t *rp, const void *q_idx,
+                              const void *k_idx_cache, int32_t num_kv_heads,
+                              int32_t num_idx_k_heads, int32_t max_blocks, float *scores,
+                              int32_t *dev_err, struct CUstream_st *stream);
+
+/*
+ * msa_select_blocks — stage 2 ([ferrox] "Four rules": first init_blocks and newest
+ * local_blocks forced in, before any scoring; block_sparse_select returns ids ascending;
+ * BlockSparseConfig {top_k, init_blocks, local_blocks}).
+ *
+ *   F = {j < min(init_blocks, nb)} U {max(0, nb - local_blocks) <= j < nb}, nb = nb(p)
+ *   C = [0, nb) \ F;  T = the top_k blocks of C by score (equal scores: the lower id first;
+ *   -0.0 equals +0.0); all of C when |C| <= top_k.
+ *   block_ids[t, g, :] = F U T ascending, then -1 up to S = init + local + top_k;
+ *   num_selected[t, g] = |F U T| (>= 1: the selection is never empty).
+ *
+ *   scores        device fp32 [total_q, num_kv_heads, max_blocks] (as msa_index_scores)
+ *   block_ids     device int32 [total_q, num_kv_heads, S] (output)
+ *   num_selected  device int32 [total_q, num_kv_heads] (output)
+ *   init_blocks, local_blocks, top_k >= 0 with S >= 1; max_blocks <= 65536.
+ */
+MSA_API msa_status_t msa_select_blocks(const msa_ragged_paged_t *rp, const float *scores,
+                               int32_t num_kv_heads, int32_t max_blocks, int32_t top_k,
+                               int32_t init_blocks, int32_t local_blocks, int32_t *block_ids,
+                               int32_t *num_selected, int32_t *dev_err,
+                               struct CUstream_st *stream);
+
+/*
+ * msa_sparse_attn_paged — stage 3 ([ferrox] positions_of_blocks: the selected blocks'
+ * positions, ascending and causally clipped; "an ordinary masked pass over the positions
+ * those blocks cover"; [msa] "Three attention routes").
+ *
+ *   For query head h (KV head g = h / (num_q_heads / num_kv_heads)) of row t at position p:
+ *   P = positions of the blocks in block_ids[t, g, :num_selected[t, g]] that are <= p,
+ *   out[t, h] = sum_{pos in P} softmax_pos(scale * q[t, h] . k[pos]) v[pos],
+ *   FP32 accumulation, output rounded to BF16.
+ *
+ *   Route from rp->max_q_len: 1 -> decode (no causal mask needed: p = L_b - 1); 2..8 ->
+ *   speculative decode (per-token causal mask); > 8 -> prefill (per-token causal mask,
+ *   device-built plan of each tile's union of selected blocks in `workspace`).
+ *   Decode / speculative work is split over the selected blocks ("split-K") into num_splits
+ *   partitions (0 = msa_default_num_splits); with more than one partition the partials live
+ *   in `workspace` and this call also enqueues the combine that writes `out`.
+ *
+ *   q            device bf16 [total_q, num_q_heads, 128]
+ *   k_cache, v_cache  device [num_pages, num_kv_heads, 128 tokens, 128] of kv_dtype,
+ *                16-byte aligned
+ *   block_ids, num_selected  as produced by msa_select_blocks with width S
+ *   max_blocks   an upper bound on nb(p) of every query (as for msa_index_scores)
+ *   workspace    device, >= msa_attn_workspace_bytes(...) bytes, 256-byte aligned;
+ *                may be NULL when that size is 0
+ *   out          device bf16 [total_q, num_q_heads, 128] (output)
+ *   num_q_heads % num_kv_heads == 0; the group size num_q_heads / num_kv_heads <= 64.
+ */
+MSA_API msa_status_t msa_sparse_attn_paged(const msa_ragged_paged_t *rp, const void *q,
+                                   const void *k_cache, const void *v_cache,
+                                   msa_kv_dtype_t kv_dtype, const int32_t *block_ids,
+                                   const int32_t *num_selected, int32_t S, int32_t num_q_heads,
+                                   int32_t num_kv_heads, int32_t max_blocks, float scale,
+                                   int32_t num_splits, void *workspace, size_t workspace_bytes,
+                                   void *out, int32_t *dev_err, struct CUstream_st *stream);
+
+/*
+ * msa_splitk_combine — merge split-K partials ([msa] "Three attention routes": at more than
+ * one partition the partials key on the ragged global query row and a combine writes the
+ * ragged output).
+ *
+ *   out[t, h] = sum_s w_s o_s[t, h] / sum_s w_s,  w_s = exp(lse_s[t, h] - max_s lse_s[t, h]);
+ *   partitions with lse = -inf (no position) weigh nothing; a row with none at all gets 0.
+ *
+ *   partial_o    device fp32 [num_splits, total_q, num_q_heads, 128]: each partition's
+ *                softmax-normalised output over its own positions
+ *   partial_lse  device fp32 [num_splits, total_q, num_q_heads]: natural log of each
+ *                partition's sum of exp(scale * q . k)
+ *   out          device bf16 [total_q, num_q_heads, 128] (output)
+ */
+MSA_API msa_status_t msa_splitk_combine(const float *partial_o, const float *partial_lse,
+                                int32_t num_splits, int32_t total_q, int32_t num_q_heads,
+                                void *out, struct CUstream_st *stream);
+
+/* Host-only helpers (no device work, no CUDA call). */
+
+/* Bytes of `workspace` that msa_sparse_attn_paged needs for this shape (0 when none). */
+MSA_API size_t msa_attn_workspace_bytes(const msa_ragged_paged_t *rp, int32_t S, int32_t num_q_heads,
+                                int32_t num_kv_heads, int32_t max_blocks, int32_t num_splits);
+
+/* The split-K partition count the decode / speculative routes use when num_splits == 0:
+ * enough (sequence, KV head, partition) work items to fill `num_sms` SMs about twice over,
+ * never more partitions than S / 2 (at least one block pair each), and 1 for prefill. */
+MSA_API int32_t msa_default_num_splits(int32_t batch, int32_t max_q_len, int32_t num_kv_heads,
+                               int32_t S, int32_t num_sms);
+
+/* A static, human-readable name of a status code. */
+MSA_API const char *msa_status_string(msa_status_t status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MSA_H_ */

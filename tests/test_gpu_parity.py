@@ -1,0 +1,192 @@
+"""GPU parity: the CUDA path through the C ABI against the CPU oracle on the same seeded inputs.
+
+Small cases (the oracle finishes each in seconds) span several page tiles, ragged query
+lengths, partial last pages (NaN-poisoned past the sequence end), both index-K layouts,
+BF16 and FP8 KV, all three attention routes and several split-K counts.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from block_sparse_paged_scores_b200 import msa
+from block_sparse_paged_scores_b200 import workload as wl
+from parity_tools import (check_attention, check_scores, check_selection, fp32_exact,
+                          head_rows_mask, oracle_forward)
+
+pytestmark = pytest.mark.gpu
+
+W = wl.WORKLOADS
+CASES = {
+    "tiny_decode": (W["tiny_decode"], {}),
+    "bf16_decode": (W["bf16_decode"], dict(batch=4, kv_len=(2000, 9000))),
+    "bf16_decode_idxk_per_head": (W["bf16_decode"], dict(batch=3, kv_len=(1000, 5000), H_idxk=8)),
+    "short_contexts": (W["bf16_decode"], dict(batch=6, kv_len=(1, 300))),
+    "spec_decode": (W["spec_decode"], dict(batch=6, kv_len=(1500, 5000))),
+    "spec_ragged_q": (W["spec_decode"], dict(batch=6, q_len=(2, 8), kv_len=(1000, 4000))),
+    "spec_gqa4": (W["spec_decode"], dict(batch=3, G=4, H_kv=4, q_len=(2, 8), kv_len=(900, 3000))),
+    "fp8_decode": (W["fp8_long_decode"], dict(batch=4, kv_len=(3000, 12000))),
+    "fp8_spec": (W["fp8_long_decode"], dict(batch=3, q_len=(2, 6), kv_len=(2000, 6000))),
+    "prefill": (W["ragged_prefill"], dict(batch=3, q_len=(100, 600), prior_len=(0, 3000))),
+    "prefill_from_empty": (W["ragged_prefill"], dict(batch=2, q_len=(9, 300), prior_len=0)),
+    "prefill_fp8": (W["ragged_prefill"], dict(batch=2, q_len=(50, 300), prior_len=(0, 2000),
+                                              kv_dtype="fp8")),
+    "prefill_with_empty_rows": (W["ragged_prefill"], dict(batch=4, q_len=(0, 40),
+                                                          prior_len=(100, 900))),
+}
+
+
+def _problem(name):
+    spec, kw = CASES[name]
+    return wl.generate(spec.scaled(**kw), seed=1000 + sorted(CASES).index(name))
+
+
+_cache = {}
+
+
+def _oracle(name):
+    if name not in _cache:
+        p = _problem(name)
+        _cache[name] = (p, oracle_forward(p))
+    return _cache[name]
+
+
+def _gpu(prob):
+    return wl.to_device(prob, "cuda")
+
+
+@pytest.mark.parametrize("name", sorted(CASES))
+def test_index_scores_match_oracle(name):
+    p, (sc, _, _, _) = _oracle(name)
+    path = msa.Path(_gpu(p))
+    path.index_scores()
+    torch.cuda.synchronize()
+    assert int(path.dev_err.item()) == 0
+    check_scores(path.scores.cpu().numpy(), sc, p, p["max_blocks"])
+
+
+@pytest.mark.parametrize("name", sorted(CASES))
+def test_select_is_bit_exact_on_identical_scores(name):
+    p, (sc, _, _, _) = _oracle(name)
+    s32 = fp32_exact(sc)
+    ids, cnt = oracle.select_blocks(p["row_off"], p["cache_len"], s32, p["top_k"],
+                                    p["init_blocks"], p["local_blocks"])
+    path = msa.Path(_gpu(p))
+    path.select(scores=torch.from_numpy(s32.astype(np.float32)).cuda())
+    torch.cuda.synchronize()
+    assert int(path.dev_err.item()) == 0
+    assert np.array_equal(path.num_selected.cpu().numpy(), cnt)
+    assert np.array_equal(path.block_ids.cpu().numpy(), ids)
+
+
+@pytest.mark.parametrize("name", sorted(CASES))
+def test_attention_matches_oracle_on_oracle_selection(name):
+    p, (_, ids, cnt, out) = _oracle(name)
+    path = msa.Path(_gpu(p))
+    path.attend(block_ids=torch.from_numpy(ids).cuda(), num_selected=torch.from_numpy(cnt).cuda())
+    torch.cuda.synchronize()
+    assert int(path.dev_err.item()) == 0
+    check_attention(path.out.float().cpu(), out, p["kv_fp8"])
+
+
+@pytest.mark.parametrize("name", sorted(CASES))
+def test_whole_path_matches_oracle(name):
+    p, (sc, ids, cnt, out) = _oracle(name)
+    path = msa.Path(_gpu(p))
+    path.run()
+    torch.cuda.synchronize()
+    assert int(path.dev_err.item()) == 0
+    same = check_selection(path.block_ids.cpu().numpy(), path.num_selected.cpu().numpy(), ids,
+                           cnt, sc, p)
+    assert same.mean() > 0.9
+    mask = head_rows_mask(same, p["H_q"] // p["H_kv"])
+    check_attention(path.out.float().cpu(), out, p["kv_fp8"], rows_mask=mask)
+
+
+@pytest.mark.parametrize("splits", [1, 2, 3, 7, 19])
+def test_split_k_counts_agree(splits):
+    p, (_, ids, cnt, out) = _oracle("bf16_decode")
+    ref = None
+    path = msa.Path(_gpu(p), num_splits=splits)
+    path.attend(block_ids=torch.from_numpy(ids).cuda(), num_selected=torch.from_numpy(cnt).cuda())
+    torch.cuda.synchronize()
+    check_attention(path.out.float().cpu(), out, False)
+    base = msa.Path(_gpu(p), num_splits=1)
+    base.attend(block_ids=torch.from_numpy(ids).cuda(), num_selected=torch.from_numpy(cnt).cuda())
+    torch.cuda.synchronize()
+    ref = base.out.float()
+    # fp32 reassociation across partitions: at most a couple of bf16 ulps apart
+    diff = (path.out.float() - ref).abs()
+    assert float(diff.max()) <= 2 * 2 ** -7 * float(ref.abs().max())
+
+
+def test_splitk_combine_entry_point():
+    torch.manual_seed(0)
+    ns, tq, hq = 5, 7, 12
+    o = torch.randn(ns, tq, hq, 128, device="cuda")
+    lse = torch.randn(ns, tq, hq, device="cuda") * 3
+    lse[1] = -float("inf")                      # an empty partition weighs nothing
+    lse[:, 3, 4] = -float("inf")                # a row no partition saw -> 0
+    out = torch.empty(tq, hq, 128, dtype=torch.bfloat16, device="cuda")
+    msa.msa_splitk_combine(o, lse, ns, tq, hq, out)
+    torch.cuda.synchronize()
+    w = torch.softmax(lse.double(), dim=0).nan_to_num(0.0)
+    ref = (w[..., None] * o.double()).sum(0)
+    got = out.double()
+    assert torch.allclose(got, ref, atol=1e-2, rtol=1e-2)
+    assert float(got[3, 4].abs().max()) == 0.0
+
+
+def test_all_equal_scores_pick_the_lowest_ids():
+    p = wl.generate(W["bf16_decode"].scaled(batch=2, kv_len=(3000, 4000)), seed=77)
+    p["k_idx"] = torch.zeros_like(p["k_idx"])
+    sc, ids, cnt, _ = oracle_forward(p)
+    path = msa.Path(_gpu(p))
+    path.index_scores()
+    path.select()
+    torch.cuda.synchronize()
+    gpu_sc = path.scores.cpu().numpy()
+    assert np.array_equal(np.isneginf(gpu_sc), np.isneginf(sc))
+    assert np.all(gpu_sc[~np.isneginf(gpu_sc)] == 0.0)
+    assert np.array_equal(path.block_ids.cpu().numpy(), ids)
+    assert np.array_equal(path.num_selected.cpu().numpy(), cnt)
+
+
+@pytest.mark.parametrize("top_k,init,local", [(0, 1, 1), (3, 0, 0), (0, 0, 2), (500, 1, 2),
+                                              (5, 7, 0)])
+def test_selection_edge_parameters(top_k, init, local):
+    p, (sc, _, _, _) = _oracle("spec_decode")
+    p = dict(p, top_k=top_k, init_blocks=init, local_blocks=local, S=top_k + init + local)
+    s32 = fp32_exact(sc)
+    ids, cnt = oracle.select_blocks(p["row_off"], p["cache_len"], s32, top_k, init, local)
+    path = msa.Path(_gpu(p))
+    path.select(scores=torch.from_numpy(s32.astype(np.float32)).cuda())
+    torch.cuda.synchronize()
+    assert np.array_equal(path.block_ids.cpu().numpy(), ids)
+    assert np.array_equal(path.num_selected.cpu().numpy(), cnt)
+    # and attention over that selection
+    out = oracle.attention(p["row_off"], p["cache_len"], p["table"], p["q"], p["k"], p["v"],
+                           False, ids, cnt, p["scale"])
+    path.attend()
+    torch.cuda.synchronize()
+    check_attention(path.out.float().cpu(), out, False)
+
+
+def test_empty_batch_is_a_no_op():
+    p = _gpu(_oracle("tiny_decode")[0])
+    empty = dict(p, row_off=torch.zeros(2, dtype=torch.int32, device="cuda"), total_q=0)
+    empty["batch"] = 1
+    path = msa.Path(empty)
+    path.run()
+    torch.cuda.synchronize()
+    assert int(path.dev_err.item()) == 0
+
+
+def test_bad_page_id_is_reported_not_read():
+    p = _gpu(_oracle("bf16_decode")[0])
+    p["table"] = p["table"].clone()
+    p["table"][1, 3] = p["num_pages"] + 5          # outside the pool
+    path = msa.Path(p)
+    path.run()
+    torch.cuda.synchronize()
+    assert int(path.dev_err.item()) & msa.MSA_DEVERR_PAGE_ID
