@@ -276,6 +276,8 @@ def run_ours(args):
     msa.load()
 
     spec = wl.WORKLOADS[args.workload]
+    if args.batch:
+        spec = spec.scaled(batch=args.batch)
     seed = wl.SEEDS[args.workload] + 1000 * rank
     prob = wl.generate(spec, seed=seed, device=dev)
     path = msa.Path(prob, num_splits=args.splits)
@@ -329,7 +331,11 @@ def run_ours(args):
     clocks = sampler.summary(t_wall0, t_wall1) if sampler else None
 
     # ---- end to end through the public API with host buffers
-    host = {k: prob[k].cpu().pin_memory() for k in ("q", "q_idx", "row_off", "cache_len", "table")}
+    if args.no_e2e:
+        host = {}
+    else:
+        host = {k: prob[k].cpu().pin_memory()
+                for k in ("q", "q_idx", "row_off", "cache_len", "table")}
     out_host = torch.empty(path.out.shape, dtype=path.out.dtype).pin_memory()
     h2d = sum(v.numel() * v.element_size() for v in host.values())
     d2h = out_host.numel() * out_host.element_size()
@@ -384,8 +390,8 @@ def run_ours(args):
                    "top_k": prob["top_k"], "init_blocks": prob["init_blocks"],
                    "local_blocks": prob["local_blocks"], "kv_lens": f"{spec.kv_len}",
                    "num_splits": splits_used, "parallelism": f"replicas x{ws}",
-                   "l2": f"inputs larger than L2: {(idx_bytes + attn_bytes) / 1e6:.0f} MB "
-                         f"touched per step vs {L2_BYTES / 1e6:.0f} MB L2"},
+                   "l2": f"inputs larger than L2: {(idx_bytes + attn_bytes) / 2**20:.0f} MiB "
+                         f"touched per step vs {L2_BYTES / 2**20:.0f} MiB L2, no flush"},
         "roofline": {"bound": "hbm", "kernel": dom, "achieved": achieved, "peak": hbm,
                      "unit": "GB/s", "frac": achieved / hbm, "peak_source": peak_src,
                      "traffic": profiled_traffic(dom, args.workload, digest),
@@ -420,6 +426,9 @@ def main(argv=None):
     ap.add_argument("--workload", default="bf16_decode")
     ap.add_argument("--splits", type=int, default=0, help="split-K partitions (0 = heuristic)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer pass")
+    ap.add_argument("--batch", type=int, default=0, help="override the workload's batch "
+                    "(profiling runs on a smaller case; not a bench number)")
     ap.add_argument("--cpu-sample-seqs", type=int, default=4)
     ap.add_argument("--cpu-min-s", type=float, default=10.0)
     ap.add_argument("--cpu-max-s", type=float, default=30.0)
