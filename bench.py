@@ -283,12 +283,10 @@ def run_ours(args):
     path = msa.Path(prob, num_splits=args.splits)
     stream = torch.cuda.current_stream(dev)
     fp8 = prob["kv_fp8"]
-    kernels_per_step = 3 + (1 if prob["max_q_len"] > 1 else 0)
-    splits_used = 1 if prob["max_q_len"] > 8 else (args.splits or msa.msa_default_num_splits(
-        prob["batch"], prob["max_q_len"], prob["H_kv"], prob["S"],
-        torch.cuda.get_device_properties(dev).multi_processor_count))
-    if splits_used > 1:
-        kernels_per_step += 1
+    stream_route = prob["max_q_len"] <= 8  # decode / speculative: persistent kernel + combine
+    kernels_per_step = 3 + (1 if prob["max_q_len"] > 1 else 0) + (1 if stream_route else 0)
+    splits_used = msa.msa_attn_partials(path.rp, prob["S"], prob["H_q"], prob["H_kv"],
+                                        path.max_blocks, args.splits)[0] if stream_route else 1
 
     for _ in range(args.warmup):
         path.run(stream)
@@ -313,7 +311,7 @@ def run_ours(args):
     ms = max_over_ranks(ms_local, ws, dev)
 
     # ---- per-stage durations (separate K-step pass, events between the stages)
-    n_ev = 4
+    n_ev = 5
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(n_ev)] for _ in range(args.steps)]
     for k in range(args.steps):
         evs[k][0].record(stream)
@@ -321,11 +319,14 @@ def run_ours(args):
         evs[k][1].record(stream)
         path.select(stream=stream)
         evs[k][2].record(stream)
-        path.attend(stream=stream)
+        path.attend(stream=stream, combine=not stream_route)
         evs[k][3].record(stream)
+        if stream_route:
+            path.combine(stream)
+        evs[k][4].record(stream)
     torch.cuda.synchronize(dev)
     stage_ms = [sum(evs[k][i].elapsed_time(evs[k][i + 1]) for k in range(args.steps)) /
-                args.steps for i in range(3)]
+                args.steps for i in range(n_ev - 1)]
     if sampler:
         sampler.stop()
     clocks = sampler.summary(t_wall0, t_wall1) if sampler else None
@@ -389,7 +390,7 @@ def run_ours(args):
                    "H_q": prob["H_q"], "head_dim": 128, "page_size": 128,
                    "top_k": prob["top_k"], "init_blocks": prob["init_blocks"],
                    "local_blocks": prob["local_blocks"], "kv_lens": f"{spec.kv_len}",
-                   "num_splits": splits_used, "parallelism": f"replicas x{ws}",
+                   "split_k_partials": splits_used, "parallelism": f"replicas x{ws}",
                    "l2": f"inputs larger than L2: {(idx_bytes + attn_bytes) / 2**20:.0f} MiB "
                          f"touched per step vs {L2_BYTES / 2**20:.0f} MiB L2, no flush"},
         "roofline": {"bound": "hbm", "kernel": dom, "achieved": achieved, "peak": hbm,
@@ -403,7 +404,8 @@ def run_ours(args):
                      "frac_of_8TBps": (idx_bytes + attn_bytes) / (ms / args.steps * 1e-3)
                      / 8e12},
         "stages_ms": {"index_scores": stage_ms[0], "select": stage_ms[1],
-                      "attention_incl_plan_and_combine": stage_ms[2]},
+                      "attention" + ("_incl_plan" if prob["max_q_len"] > 1 else ""): stage_ms[2],
+                      "combine": stage_ms[3]},
         "gpu_launches": kernels_per_step * args.steps,
         "clocks": clocks,
         "e2e": {"value": tokens_total / (e2e_ms * 1e-3), "unit": UNIT,

@@ -9,6 +9,7 @@
 #include <math.h>
 #include <string.h>
 
+#include <algorithm>
 #include <mutex>
 
 #include "internal.h"
@@ -88,30 +89,37 @@ bool ragged_ok(const msa_ragged_paged_t *rp) {
 // ---- attention route: tiles, row groups, partitions and the workspace layout
 struct Route {
   bool plan;      // speculative / prefill: per-tile union in the workspace
+  bool stream;    // decode / speculative: the persistent split-K kernel + combine
   int qt, tiles;  // query tokens per tile, tiles per sequence
   int rg;         // 16-row groups per CTA
-  int splits;
-  int cap;        // union capacity per item
+  int cap;        // work-list slots per item
+  int items;
+  int grid;       // persistent kernel: CTAs (= split-K partitions)
+  long long R;    // slots per CTA
+  int P;          // most CTAs one item spans
+  int splits;     // partial split indices: P * position splits
   size_t off_o, off_lse, off_list, off_masks, off_counts, bytes;
 };
 
-constexpr int kMaxRows = 64;     // rows (tokens x group heads) per attention CTA
-constexpr int kMaxSplits = 256;
+constexpr int kMaxRows = 64;  // rows (tokens x group heads) per attention CTA
+constexpr int kMaxSplits = 4096;
+constexpr int kMinSlotsPerCta = 4;
 
-int default_splits(int batch, int max_q_len, int H_kv, int S, int num_sms) {
-  if (max_q_len > MSA_MAX_SPEC_DRAFT) return 1;
-  const long long units = static_cast<long long>(batch) * H_kv;
-  long long ns = (2LL * num_sms + units - 1) / (units > 0 ? units : 1);
-  const int cap = S / 2 > 1 ? S / 2 : 1;
-  if (ns > cap) ns = cap;
-  if (ns < 1) ns = 1;
-  return static_cast<int>(ns);
+int stream_grid(long long total, int num_splits, int num_sms) {
+  long long grid = num_splits > 0 ? num_splits
+                                  : std::min<long long>(num_sms,
+                                                        (total + kMinSlotsPerCta - 1) /
+                                                            kMinSlotsPerCta);
+  if (grid > total) grid = total;
+  if (grid < 1) grid = 1;
+  return static_cast<int>(grid);
 }
 
 bool make_route(const msa_ragged_paged_t *rp, int S, int H_q, int H_kv, int max_blocks,
                 int num_splits, int num_sms, Route *r) {
   const int G = H_q / H_kv;
   r->plan = rp->max_q_len > 1;
+  r->stream = rp->max_q_len <= MSA_MAX_SPEC_DRAFT;
   if (!r->plan) {
     r->qt = 1;
   } else {
@@ -123,26 +131,41 @@ bool make_route(const msa_ragged_paged_t *rp, int S, int H_q, int H_kv, int max_
   r->tiles = (rp->max_q_len + r->qt - 1) / r->qt;
   r->rg = (r->qt * G + 15) / 16;
   if (r->rg < 1 || r->rg > 4) return false;
-  if (rp->max_q_len > MSA_MAX_SPEC_DRAFT)
-    r->splits = 1;
-  else
-    r->splits = num_splits > 0 ? num_splits
-                               : default_splits(rp->batch, rp->max_q_len, H_kv, S, num_sms);
-  const long long cap = static_cast<long long>(r->qt) * S;
-  r->cap = static_cast<int>(cap < max_blocks ? cap : max_blocks);
+  const long long cap = r->plan ? std::min<long long>(static_cast<long long>(r->qt) * S, max_blocks)
+                                : S;
+  r->cap = static_cast<int>(cap);
+  const long long items = static_cast<long long>(rp->batch) * r->tiles * H_kv;
+  if (items > 0x7fffffffLL) return false;
+  r->items = static_cast<int>(items);
+  r->grid = 1;
+  r->R = 0;
+  r->P = 0;
+  r->splits = 0;
+  if (r->stream) {
+    const long long total = items * cap;
+    r->grid = stream_grid(total, num_splits, num_sms);
+    r->R = (total + r->grid - 1) / r->grid;
+    r->grid = static_cast<int>((total + r->R - 1) / r->R);
+    int P = 1;
+    for (long long it = 0; it < items; ++it) {
+      const long long first = it * cap / r->R, last = (it * cap + cap - 1) / r->R;
+      P = std::max<int>(P, static_cast<int>(last - first + 1));
+    }
+    r->P = P;
+    r->splits = P * attn_position_splits(r->rg);
+  }
   const size_t rows = static_cast<size_t>(rp->total_q) * H_q;
-  const size_t items = static_cast<size_t>(rp->batch) * r->tiles * H_kv;
   size_t off = 0;
   r->off_o = off;
-  if (r->splits > 1) off = round_up(off + rows * kHeadDim * sizeof(float) * r->splits, 256);
+  if (r->stream) off = round_up(off + rows * kHeadDim * sizeof(float) * r->splits, 256);
   r->off_lse = off;
-  if (r->splits > 1) off = round_up(off + rows * sizeof(float) * r->splits, 256);
+  if (r->stream) off = round_up(off + rows * sizeof(float) * r->splits, 256);
   r->off_list = off;
-  if (r->plan) off = round_up(off + items * r->cap * sizeof(int32_t), 256);
+  if (r->plan) off = round_up(off + static_cast<size_t>(items) * r->cap * sizeof(int32_t), 256);
   r->off_masks = off;
-  if (r->plan) off = round_up(off + items * r->cap * sizeof(uint32_t), 256);
+  if (r->plan) off = round_up(off + static_cast<size_t>(items) * r->cap * sizeof(uint32_t), 256);
   r->off_counts = off;
-  if (r->plan) off = round_up(off + items * sizeof(int32_t), 256);
+  if (r->plan) off = round_up(off + static_cast<size_t>(items) * sizeof(int32_t), 256);
   r->bytes = off;
   return true;
 }
@@ -188,8 +211,11 @@ const char *msa_status_string(msa_status_t status) {
 
 int32_t msa_default_num_splits(int32_t batch, int32_t max_q_len, int32_t num_kv_heads, int32_t S,
                                int32_t num_sms) {
-  if (batch < 1 || max_q_len < 1 || num_kv_heads < 1 || S < 1 || num_sms < 1) return 1;
-  return default_splits(batch, max_q_len, num_kv_heads, S, num_sms);
+  if (batch < 1 || max_q_len < 1 || num_kv_heads < 1 || S < 1 || num_sms < 1 ||
+      max_q_len > MSA_MAX_SPEC_DRAFT)
+    return 1;
+  const long long total = static_cast<long long>(batch) * num_kv_heads * S * max_q_len;
+  return stream_grid(total, 0, num_sms);
 }
 
 size_t msa_attn_workspace_bytes(const msa_ragged_paged_t *rp, int32_t S, int32_t num_q_heads,
@@ -202,6 +228,23 @@ size_t msa_attn_workspace_bytes(const msa_ragged_paged_t *rp, int32_t S, int32_t
   const int sms = num_splits > 0 ? 1 : num_sms_of_current_device();
   if (!make_route(rp, S, num_q_heads, num_kv_heads, max_blocks, num_splits, sms, &r)) return 0;
   return r.bytes;
+}
+
+int32_t msa_attn_partials(const msa_ragged_paged_t *rp, int32_t S, int32_t num_q_heads,
+                          int32_t num_kv_heads, int32_t max_blocks, int32_t num_splits,
+                          size_t *partial_o_offset, size_t *partial_lse_offset) {
+  if (!rp || rp->batch < 1 || rp->max_q_len < 1 || S < 1 || num_kv_heads < 1 ||
+      num_q_heads < num_kv_heads || num_q_heads % num_kv_heads || max_blocks < 1 ||
+      num_splits < 0)
+    return 0;
+  Route r;
+  const int sms = num_splits > 0 ? 1 : num_sms_of_current_device();
+  if (!make_route(rp, S, num_q_heads, num_kv_heads, max_blocks, num_splits, sms, &r) ||
+      !r.stream)
+    return 0;
+  if (partial_o_offset) *partial_o_offset = r.off_o;
+  if (partial_lse_offset) *partial_lse_offset = r.off_lse;
+  return r.splits;
 }
 
 msa_status_t msa_index_scores(const msa_ragged_paged_t *rp, const void *q_idx,
@@ -310,13 +353,14 @@ msa_status_t msa_sparse_attn_paged(const msa_ragged_paged_t *rp, const void *q,
                                    int32_t num_splits, void *workspace, size_t workspace_bytes,
                                    void *out, int32_t *dev_err, struct CUstream_st *stream) {
   if (ragged_ok(rp) && rp->total_q == 0 && S >= 1) return MSA_OK;  // nothing to attend
-  if (!ragged_ok(rp) || !q || !k_cache || !v_cache || !block_ids || !num_selected || !out ||
+  if (!ragged_ok(rp) || !q || !k_cache || !v_cache || !block_ids || !num_selected ||
       S < 1 || num_kv_heads < 1 || num_q_heads < num_kv_heads ||
       num_q_heads % num_kv_heads != 0 || max_blocks < 1 || max_blocks > rp->max_pages_per_seq ||
       !(scale > 0.f) || !isfinite(scale) || num_splits < 0 || num_splits > kMaxSplits ||
       !(kv_dtype == MSA_KV_BF16 || kv_dtype == MSA_KV_FP8_E4M3) || !aligned(q, 16) ||
       !aligned(k_cache, 16) || !aligned(v_cache, 16) || !aligned(out, 8))
     return MSA_ERR_INVALID_ARG;
+  if (!out && rp->max_q_len > MSA_MAX_SPEC_DRAFT) return MSA_ERR_INVALID_ARG;  // prefill: out
   const int G = num_q_heads / num_kv_heads;
   if (G > kMaxRows) return MSA_ERR_UNSUPPORTED;
   if (static_cast<long long>(rp->num_pages) * num_kv_heads >= (1LL << 31))
@@ -384,16 +428,22 @@ msa_status_t msa_sparse_attn_paged(const msa_ragged_paged_t *rp, const void *q,
   a.max_blocks = max_blocks;
   a.qt = r.qt;
   a.tiles = r.tiles;
-  a.splits = r.splits;
+  a.items = r.items;
+  a.R = r.R;
+  a.P = r.P;
   a.scale_log2 = scale * 1.4426950408889634f;
   a.part_o = reinterpret_cast<float *>(ws + r.off_o);
   a.part_lse = reinterpret_cast<float *>(ws + r.off_lse);
   a.out = static_cast<uint16_t *>(out);
   a.dev_err = dev_err;
-  if (launch_attention(kmap, vmap, a, fp8, r.rg, r.plan, s) != cudaSuccess) return MSA_ERR_CUDA;
-  if (r.splits > 1 &&
-      launch_combine(a.part_o, a.part_lse, r.splits, rp->total_q, num_q_heads, a.out, s) !=
-          cudaSuccess)
+  if (!r.stream)
+    return launch_attention_tiles(kmap, vmap, a, fp8, r.rg, s) == cudaSuccess ? MSA_OK
+                                                                             : MSA_ERR_CUDA;
+  if (launch_attention_stream(kmap, vmap, a, fp8, r.rg, r.plan, r.grid, s) != cudaSuccess)
+    return MSA_ERR_CUDA;
+  if (!out) return MSA_OK;  // the caller combines the partials itself
+  if (launch_combine(a.part_o, a.part_lse, r.splits, rp->total_q, num_q_heads, a.out, s) !=
+      cudaSuccess)
     return MSA_ERR_CUDA;
   return MSA_OK;
 }

@@ -1,0 +1,271 @@
+// attn_common.cuh — the per-block math of the sparse paged attention, shared by the
+// persistent decode / speculative kernel (attention_stream.cu) and the tiled kernel used for
+// prefill (attention_tile.cu).
+//
+// A consumer warp owns 16 query rows (one m16 MMA tile) and PW = 128 / PQ of the 128 positions
+// of every block, and keeps its own online-softmax state over them.  Q sits in shared memory
+// (swizzled like the TMA tiles), K and V page tiles arrive by TMA with the 128-byte swizzle.
+// QK^T and PV run on mma.sync m16n8k16 with FP32 accumulators: bf16 operands for BF16 KV;
+// for e4m3 KV the tiles are converted to f16 in registers (exact) and the MMAs take f16
+// operands (q rounded to f16, P in f16).
+#pragma once
+
+#include <math.h>
+
+#include "internal.h"
+#include "ptx.cuh"
+
+namespace msa {
+
+constexpr int kQRows = 64;                // rows of a Q buffer
+constexpr uint32_t kQSub = kQRows * 128;  // one 64-column (bf16/f16) sub-tile of Q
+constexpr uint32_t kQBuf = 2 * kQSub;     // one Q buffer
+constexpr float kLn2 = 0.69314718055994530942f;
+
+template <bool FP8>
+struct KvTile {
+  static constexpr uint32_t kBytes = FP8 ? 16384u : 32768u;  // one (page, head) tile
+  static constexpr uint32_t kSub = 16384u;                    // one swizzled [128][128 B] box
+};
+
+// Stage rows [0, kQRows) of Q for rows r = tok * G + h_local of one work item into a Q buffer
+// (zeros past `rows`).  Threads `tid` of `nthreads` share the copy.  For e4m3 KV the values
+// become f16 and, inside every 16-dim group, slot 2c+e holds dim 4c+e and slot 2c+8+e holds
+// dim 4c+2+e (c < 4, e < 2): the order in which a plain ldmatrix of an e4m3 K tile hands the
+// dims to the MMA, so that both operands agree on k.
+template <bool FP8>
+__device__ __forceinline__ void stage_q(uint8_t *qs, const uint16_t *q, int t0, int rows, int G,
+                                        int H_q, int g, int tid, int nthreads) {
+  for (int idx = tid; idx < kQRows * 8; idx += nthreads) {
+    const int r = idx >> 3, grp = idx & 7;
+    uint4 lo4 = make_uint4(0, 0, 0, 0), hi4 = make_uint4(0, 0, 0, 0);
+    if (r < rows) {
+      const int t = t0 + r / G, h = g * G + r % G;
+      const uint4 *src =
+          reinterpret_cast<const uint4 *>(q + (static_cast<size_t>(t) * H_q + h) * kHeadDim + grp * 16);
+      const uint4 x0 = src[0], x1 = src[1];
+      if (!FP8) {
+        lo4 = x0;
+        hi4 = x1;
+      } else {
+        const uint32_t wv[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
+        float f[16];
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+          f[2 * k] = __uint_as_float(wv[k] << 16);
+          f[2 * k + 1] = __uint_as_float(wv[k] & 0xffff0000u);
+        }
+        uint32_t o8[8];
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          o8[c] = pack_f16x2(f[4 * c], f[4 * c + 1]);
+          o8[4 + c] = pack_f16x2(f[4 * c + 2], f[4 * c + 3]);
+        }
+        lo4 = make_uint4(o8[0], o8[1], o8[2], o8[3]);
+        hi4 = make_uint4(o8[4], o8[5], o8[6], o8[7]);
+      }
+    }
+    *reinterpret_cast<uint4 *>(qs + sw128(r, 2 * grp, kQSub)) = lo4;
+    *reinterpret_cast<uint4 *>(qs + sw128(r, 2 * grp + 1, kQSub)) = hi4;
+  }
+}
+
+template <bool FP8, int PQ>
+struct WarpAttn {
+  static constexpr int PW = kBlock / PQ;  // positions per warp
+  static constexpr int NTW = PW / 8;      // n8 tiles of S per warp
+  static constexpr int KSW = PW / 16;     // k16 steps of PV per warp
+
+  float o[16][4];
+  float m_run[2], l_run[2];  // rows lane/4 and lane/4 + 8 (log2 domain)
+  float sc[NTW][4];
+
+  __device__ __forceinline__ void reset() {
+#pragma unroll
+    for (int n = 0; n < 16; ++n)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) o[n][e] = 0.f;
+    m_run[0] = m_run[1] = -INFINITY;
+    l_run[0] = l_run[1] = 0.f;
+  }
+
+  // sc = Q K^T for the warp's 16 rows (row base qrow0 of the Q buffer) and PW positions.
+  __device__ __forceinline__ void qk(uint32_t qs_addr, int qrow0, uint32_t kt, int pq, int lane) {
+    const int mi = lane >> 3, rr = lane & 7;
+#pragma unroll
+    for (int n = 0; n < NTW; ++n)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) sc[n][e] = 0.f;
+#pragma unroll
+    for (int ks = 0; ks < 8; ++ks) {
+      uint32_t qa[4];
+      ldsm_x4(qs_addr + sw128(qrow0 + (mi & 1) * 8 + rr, 2 * ks + (mi >> 1), kQSub), qa[0], qa[1],
+              qa[2], qa[3]);
+      if (FP8) {
+#pragma unroll
+        for (int h = 0; h < NTW / 4; ++h) {
+          uint32_t kr[4];
+          ldsm_x4(kt + sw128(pq * PW + h * 32 + mi * 8 + rr, ks, KvTile<FP8>::kSub), kr[0], kr[1],
+                  kr[2], kr[3]);
+#pragma unroll
+          for (int n = 0; n < 4; ++n)
+            mma_f16(sc[4 * h + n], qa, e4m3x2_to_f16x2(static_cast<uint16_t>(kr[n] & 0xffffu)),
+                    e4m3x2_to_f16x2(static_cast<uint16_t>(kr[n] >> 16)));
+        }
+      } else {
+        uint32_t bf[NTW][2];
+#pragma unroll
+        for (int h = 0; h < NTW / 2; ++h)
+          ldsm_x4(kt + sw128(pq * PW + h * 16 + (mi >> 1) * 8 + rr, 2 * ks + (mi & 1),
+                             KvTile<FP8>::kSub),
+                  bf[2 * h][0], bf[2 * h][1], bf[2 * h + 1][0], bf[2 * h + 1][1]);
+#pragma unroll
+        for (int n = 0; n < NTW; ++n) mma_bf16(sc[n], qa, bf[n][0], bf[n][1]);
+      }
+    }
+  }
+
+  // Mask (position <= the row's query position and the row's token selected the block),
+  // online-softmax update in the log2 domain; sc becomes P.
+  __device__ __forceinline__ void softmax(int j, int pq, int lane, const int (&prow)[2],
+                                          const uint32_t (&tbit)[2], uint32_t msk,
+                                          float scale_log2) {
+    const int c4 = lane & 3;
+    float mx[2] = {-INFINITY, -INFINITY};
+#pragma unroll
+    for (int n = 0; n < NTW; ++n)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int slot = e >> 1;
+        const int pos = j * kBlock + pq * PW + n * 8 + 2 * c4 + (e & 1);
+        const bool vis = pos <= prow[slot] && (msk & tbit[slot]);
+        const float x = vis ? sc[n][e] * scale_log2 : -INFINITY;
+        sc[n][e] = x;
+        mx[slot] = fmaxf(mx[slot], x);
+      }
+    float alpha[2], base[2];
+#pragma unroll
+    for (int slot = 0; slot < 2; ++slot) {
+      mx[slot] = fmaxf(mx[slot], __shfl_xor_sync(0xffffffffu, mx[slot], 1));
+      mx[slot] = fmaxf(mx[slot], __shfl_xor_sync(0xffffffffu, mx[slot], 2));
+      const float m_new = fmaxf(m_run[slot], mx[slot]);
+      base[slot] = m_new == -INFINITY ? 0.f : m_new;
+      alpha[slot] = fast_exp2(m_run[slot] - base[slot]);
+      m_run[slot] = m_new;
+      l_run[slot] *= alpha[slot];
+    }
+#pragma unroll
+    for (int n = 0; n < NTW; ++n)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const float pv = fast_exp2(sc[n][e] - base[e >> 1]);
+        sc[n][e] = pv;
+        l_run[e >> 1] += pv;
+      }
+#pragma unroll
+    for (int n = 0; n < 16; ++n) {
+      o[n][0] *= alpha[0];
+      o[n][1] *= alpha[0];
+      o[n][2] *= alpha[1];
+      o[n][3] *= alpha[1];
+    }
+  }
+
+  // O += P V.  Positions >= L (the sequence length) of the last page hold whatever the pool
+  // has there; their P is 0, but 0 * NaN is NaN, so those V values are zeroed first.
+  __device__ __forceinline__ void pv(uint32_t vt, int j, int pq, int lane, int L) {
+    const int mi = lane >> 3, rr = lane & 7, c4 = lane & 3;
+    uint32_t pa[KSW][4];
+#pragma unroll
+    for (int kk = 0; kk < KSW; ++kk) {
+      if (FP8) {
+        pa[kk][0] = pack_f16x2(sc[2 * kk][0], sc[2 * kk][1]);
+        pa[kk][1] = pack_f16x2(sc[2 * kk][2], sc[2 * kk][3]);
+        pa[kk][2] = pack_f16x2(sc[2 * kk + 1][0], sc[2 * kk + 1][1]);
+        pa[kk][3] = pack_f16x2(sc[2 * kk + 1][2], sc[2 * kk + 1][3]);
+      } else {
+        pa[kk][0] = pack_bf16x2(sc[2 * kk][0], sc[2 * kk][1]);
+        pa[kk][1] = pack_bf16x2(sc[2 * kk][2], sc[2 * kk][3]);
+        pa[kk][2] = pack_bf16x2(sc[2 * kk + 1][0], sc[2 * kk + 1][1]);
+        pa[kk][3] = pack_bf16x2(sc[2 * kk + 1][2], sc[2 * kk + 1][3]);
+      }
+    }
+    const bool tail = j * kBlock + kBlock > L;
+#pragma unroll
+    for (int kk = 0; kk < KSW; ++kk) {
+      const int p0 = j * kBlock + pq * PW + kk * 16 + 2 * c4;
+      const uint32_t keep0 = (p0 < L ? 0x0000ffffu : 0u) | (p0 + 1 < L ? 0xffff0000u : 0u);
+      const uint32_t keep1 = (p0 + 8 < L ? 0x0000ffffu : 0u) | (p0 + 9 < L ? 0xffff0000u : 0u);
+      const int vrow = pq * PW + kk * 16 + (mi & 1) * 8 + rr;
+      if (FP8) {
+#pragma unroll
+        for (int cp = 0; cp < 4; ++cp) {
+          uint32_t r[4];
+          ldsm_x4_t(vt + sw128(vrow, 2 * cp + (mi >> 1), KvTile<FP8>::kSub), r[0], r[1], r[2],
+                    r[3]);
+#pragma unroll
+          for (int q = 0; q < 2; ++q) {
+            const uint32_t ra = r[2 * q], rb = r[2 * q + 1];
+            uint32_t e0 = e4m3x2_to_f16x2(static_cast<uint16_t>(__byte_perm(ra, 0, 0x0020)));
+            uint32_t e1 = e4m3x2_to_f16x2(static_cast<uint16_t>(__byte_perm(rb, 0, 0x0020)));
+            uint32_t d0 = e4m3x2_to_f16x2(static_cast<uint16_t>(__byte_perm(ra, 0, 0x0031)));
+            uint32_t d1 = e4m3x2_to_f16x2(static_cast<uint16_t>(__byte_perm(rb, 0, 0x0031)));
+            if (tail) {
+              e0 &= keep0;
+              d0 &= keep0;
+              e1 &= keep1;
+              d1 &= keep1;
+            }
+            const int ch = 2 * cp + q;
+            mma_f16(o[2 * ch], pa[kk], e0, e1);
+            mma_f16(o[2 * ch + 1], pa[kk], d0, d1);
+          }
+        }
+      } else {
+#pragma unroll
+        for (int dp = 0; dp < 8; ++dp) {
+          uint32_t r[4];
+          ldsm_x4_t(vt + sw128(vrow, 2 * dp + (mi >> 1), KvTile<FP8>::kSub), r[0], r[1], r[2],
+                    r[3]);
+          if (tail) {
+            r[0] &= keep0;
+            r[1] &= keep1;
+            r[2] &= keep0;
+            r[3] &= keep1;
+          }
+          mma_bf16(o[2 * dp], pa[kk], r[0], r[1]);
+          mma_bf16(o[2 * dp + 1], pa[kk], r[2], r[3]);
+        }
+      }
+    }
+  }
+
+  // After the last block: each row's sum of P, reduced over the quad that holds the row.
+  __device__ __forceinline__ void finish_rows() {
+#pragma unroll
+    for (int slot = 0; slot < 2; ++slot) {
+      l_run[slot] += __shfl_xor_sync(0xffffffffu, l_run[slot], 1);
+      l_run[slot] += __shfl_xor_sync(0xffffffffu, l_run[slot], 2);
+    }
+  }
+
+  // This thread's part of row slot `slot` times f, as fp32, into dst (one 128-dim row); the
+  // FP8 path's dim permutation is undone here.
+  __device__ __forceinline__ void store_row(float *dst, int slot, float f, int lane) const {
+    const int c4 = lane & 3;
+    if (FP8) {
+#pragma unroll
+      for (int ch = 0; ch < 8; ++ch)
+        *reinterpret_cast<float4 *>(dst + ch * 16 + 4 * c4) =
+            make_float4(o[2 * ch][2 * slot] * f, o[2 * ch + 1][2 * slot] * f,
+                        o[2 * ch][2 * slot + 1] * f, o[2 * ch + 1][2 * slot + 1] * f);
+    } else {
+#pragma unroll
+      for (int n = 0; n < 16; ++n)
+        *reinterpret_cast<float2 *>(dst + n * 8 + 2 * c4) =
+            make_float2(o[n][2 * slot] * f, o[n][2 * slot + 1] * f);
+    }
+  }
+};
+
+}  // namespace msa

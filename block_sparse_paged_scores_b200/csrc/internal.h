@@ -48,7 +48,8 @@ struct PlanArgs {
 };
 cudaError_t launch_plan(const PlanArgs &a, cudaStream_t s);
 
-// ---- stage 3: sparse paged attention (attention.cu)
+// ---- stage 3: sparse paged attention (attention_stream.cu: decode / speculative,
+//      attention_tile.cu: prefill)
 struct AttnArgs {
   const int32_t *row_off, *cache_len, *table;
   const uint16_t *q;  // bf16 bits [total_q, H_q, 128]
@@ -56,17 +57,25 @@ struct AttnArgs {
   const int32_t *plan_list;                 // other routes: the per-tile union
   const uint32_t *plan_masks;
   const int32_t *plan_counts;
-  int S, cap;
+  int S, cap;  // cap: work-list slots per item (decode: S; others: the union capacity)
   int batch, total_q, max_q_len, max_pages, num_pages, H_q, H_kv, G, max_blocks;
-  int qt, tiles, splits;
-  float scale_log2;  // scale * log2(e)
-  float *part_o, *part_lse;  // splits > 1
-  uint16_t *out;             // splits == 1: bf16 bits [total_q, H_q, 128]
+  int qt, tiles;
+  int items;    // batch * tiles * H_kv
+  long long R;  // persistent kernel: work-list slots per CTA
+  int P;        // persistent kernel: most CTAs one item's slots can span
+  float scale_log2;          // scale * log2(e)
+  float *part_o, *part_lse;  // persistent kernel: [P * PQ][total_q][H_q][128] and [..][H_q]
+  uint16_t *out;             // tile kernel: bf16 bits [total_q, H_q, 128]
   int32_t *dev_err;
 };
-// rg = 16-row groups (1..4), plan = read the per-tile union instead of the selection
-cudaError_t launch_attention(const CUtensorMap &kmap, const CUtensorMap &vmap, const AttnArgs &a,
-                             bool fp8, int rg, bool plan, cudaStream_t s);
+// position splits (consumer warps per 16-row group) of the persistent kernel for rg groups
+int attn_position_splits(int rg);
+// rg = 16-row groups (1..4); plan = read the per-tile union instead of the selection
+cudaError_t launch_attention_stream(const CUtensorMap &kmap, const CUtensorMap &vmap,
+                                    const AttnArgs &a, bool fp8, int rg, bool plan, int grid,
+                                    cudaStream_t s);
+cudaError_t launch_attention_tiles(const CUtensorMap &kmap, const CUtensorMap &vmap,
+                                   const AttnArgs &a, bool fp8, int rg, cudaStream_t s);
 
 // ---- split-K combine (combine.cu)
 cudaError_t launch_combine(const float *part_o, const float *part_lse, int splits, int total_q,

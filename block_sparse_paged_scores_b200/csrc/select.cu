@@ -5,11 +5,12 @@
 // block_sparse_select returns the blocks each KV head may read, ascending.  The remaining
 // blocks compete on score; equal scores go to the lower block id.
 //
-// One warp per (query row, KV head).  The k-th largest candidate key is found exactly by a
-// radix select over order-preserving uint32 keys (4 passes of 8 bits, a 256-bin shared-memory
-// histogram per warp); one ascending pass over the block ids then keeps the forced blocks,
-// every candidate above the threshold key, and the lowest-id candidates equal to it until k
-// are taken.  The output comes out in ascending order with no sort.
+// One warp per (query row, KV head).  The candidates' scores become order-preserving uint32
+// keys held in registers; the exact top_k-th largest key is then built bit by bit from the top
+// (32 rounds of "how many keys are >= this prefix", one warp reduction each, no atomics).  One
+// ascending pass over the block ids keeps the forced blocks, every candidate above that
+// threshold, and the lowest-id candidates equal to it until top_k are taken, so the output
+// comes out in ascending order with no sort.
 #include <math.h>
 
 #include "internal.h"
@@ -33,13 +34,45 @@ __device__ __forceinline__ int find_sequence(const int32_t *row_off, int batch, 
   return lo;
 }
 
+// Keys of the candidate blocks (0 for blocks that are not candidates: every real key is at
+// least score_key(-inf) = 0x007fffff > 0).  KPL keys per lane stay in registers; KPL == 0
+// reads them from memory on every pass (any number of blocks).
+template <int KPL>
+struct Keys {
+  uint32_t k[KPL > 0 ? KPL : 1];
+  __device__ __forceinline__ void load(const float *srow, int nb, int lane, int init_e,
+                                       int local_lo) {
+#pragma unroll
+    for (int i = 0; i < KPL; ++i) {
+      const int j = i * 32 + lane;
+      k[i] = (j < nb && j >= init_e && j < local_lo) ? score_key(srow[j]) : 0u;
+    }
+  }
+  // number of candidate keys >= x (over the warp)
+  __device__ __forceinline__ uint32_t count_ge(uint32_t x, const float *srow, int nb, int lane,
+                                               int init_e, int local_lo) const {
+    uint32_t c = 0;
+    if (KPL > 0) {
+#pragma unroll
+      for (int i = 0; i < KPL; ++i) c += k[i] >= x;
+    } else {
+      for (int j = init_e + lane; j < local_lo; j += 32) c += score_key(srow[j]) >= x;
+    }
+    return __reduce_add_sync(0xffffffffu, c);
+  }
+  __device__ __forceinline__ uint32_t key(int i, int j, const float *srow, int init_e,
+                                          int local_lo) const {
+    if (KPL > 0) return k[i];
+    return (j >= init_e && j < local_lo) ? score_key(srow[j]) : 0u;
+  }
+};
+
+template <int KPL>
 __global__ void __launch_bounds__(32 * kWarps) select_kernel(const SelectArgs a) {
-  __shared__ uint32_t hist_all[kWarps][256];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const long long item = static_cast<long long>(blockIdx.x) * kWarps + warp;
   if (item >= static_cast<long long>(a.total_q) * a.H_kv) return;
   const int t = static_cast<int>(item / a.H_kv);
-  uint32_t *hist = hist_all[warp];
   const unsigned lt_mask = (1u << lane) - 1u;
 
   const int b = find_sequence(a.row_off, a.batch, t);
@@ -52,87 +85,54 @@ __global__ void __launch_bounds__(32 * kWarps) select_kernel(const SelectArgs a)
   const float *srow = a.scores + static_cast<size_t>(item) * a.max_blocks;
   int32_t *out = a.block_ids + static_cast<size_t>(item) * a.S;
 
+  // forced: [0, init_e) and [local_lo, nb); candidates: [init_e, local_lo)
   const int init_e = min(a.init_blocks, nb);
-  const int local_lo = max(0, nb - a.local_blocks);
-  const int n_forced = init_e + (nb - local_lo) - max(0, init_e - local_lo);
-  const int n_cand = nb - n_forced;
+  const int local_lo = max(init_e, nb - a.local_blocks);
+  const int n_cand = local_lo - init_e;
   const bool take_all = n_cand <= a.top_k;
-  auto forced = [&](int j) { return j < init_e || j >= local_lo; };
 
-  // ---- radix select of the top_k-th largest candidate key: threshold T, and how many of
-  // the candidates equal to T are still needed (need_eq).
+  Keys<KPL> keys;
   uint32_t T = 0xffffffffu;  // top_k == 0: no candidate passes
   int need_eq = 0;
   if (!take_all && a.top_k > 0) {
-    uint32_t prefix = 0, pmask = 0;
-    int kk = a.top_k;
-    for (int shift = 24; shift >= 0; shift -= 8) {
-      for (int q = lane; q < 256; q += 32) hist[q] = 0;
-      __syncwarp();
-      for (int j = lane; j < nb; j += 32) {
-        if (forced(j)) continue;
-        const uint32_t key = score_key(srow[j]);
-        if ((key & pmask) == prefix) atomicAdd(&hist[(key >> shift) & 255u], 1u);
-      }
-      __syncwarp();
-      // lane L owns digits 255-8L .. 248-8L (descending), so a lane prefix sum counts the
-      // candidates whose digit is larger.
-      uint32_t c[8], sum = 0;
-#pragma unroll
-      for (int q = 0; q < 8; ++q) {
-        c[q] = hist[255 - 8 * lane - q];
-        sum += c[q];
-      }
-      uint32_t incl = sum;
-#pragma unroll
-      for (int off = 1; off < 32; off <<= 1) {
-        const uint32_t v = __shfl_up_sync(0xffffffffu, incl, off);
-        if (lane >= off) incl += v;
-      }
-      const uint32_t excl = incl - sum;
-      const bool mine = excl < static_cast<uint32_t>(kk) && static_cast<uint32_t>(kk) <= incl;
-      const unsigned bal = __ballot_sync(0xffffffffu, mine);
-      int digit = 0, above = 0;
-      if (mine) {
-        uint32_t run = excl;
-#pragma unroll
-        for (int q = 0; q < 8; ++q) {
-          if (run + c[q] >= static_cast<uint32_t>(kk)) {
-            digit = 255 - 8 * lane - q;
-            above = static_cast<int>(run);
-            break;
-          }
-          run += c[q];
-        }
-      }
-      const int src = bal ? __ffs(bal) - 1 : 0;
-      digit = __shfl_sync(0xffffffffu, digit, src);
-      above = __shfl_sync(0xffffffffu, above, src);
-      kk -= above;
-      prefix |= static_cast<uint32_t>(digit) << shift;
-      pmask |= 255u << shift;
-      __syncwarp();
+    keys.load(srow, nb, lane, init_e, local_lo);
+    // T = the top_k-th largest candidate key: the largest x with count(key >= x) >= top_k,
+    // built one bit at a time from the top.
+    const uint32_t k = static_cast<uint32_t>(a.top_k);
+    T = 0;
+    for (int bit = 31; bit >= 0; --bit) {
+      const uint32_t x = T | (1u << bit);
+      if (keys.count_ge(x, srow, nb, lane, init_e, local_lo) >= k) T = x;
     }
-    T = prefix;
-    need_eq = kk;
+    const uint32_t above = T == 0xffffffffu
+                               ? 0u
+                               : keys.count_ge(T + 1u, srow, nb, lane, init_e, local_lo);
+    need_eq = static_cast<int>(k - above);  // how many candidates equal to T are taken
   }
 
-  // ---- one ascending pass: forced, above T, and the lowest-id ties at T.
+  // one ascending pass: forced, above T, and the lowest-id candidates equal to T
   int nsel = 0, eq_seen = 0;
-  for (int base = 0; base < nb; base += 32) {
-    const int j = base + lane;
+  const int passes = (nb + 31) / 32;
+  for (int i = 0; i < passes; ++i) {
+    const int j = i * 32 + lane;
     const bool in = j < nb;
-    const bool f = in && forced(j);
+    const bool cand = in && j >= init_e && j < local_lo;
     bool take;
     if (take_all) {
       take = in;
     } else {
-      const bool cand = in && !f;
-      const uint32_t key = cand ? score_key(srow[j]) : 0u;
+      uint32_t key = 0;
+      if (KPL > 0) {
+#pragma unroll
+        for (int q = 0; q < (KPL > 0 ? KPL : 1); ++q)
+          if (q == i) key = keys.key(q, j, srow, init_e, local_lo);
+      } else {
+        key = cand ? score_key(srow[j]) : 0u;
+      }
       const bool eq = cand && key == T;
       const unsigned eqm = __ballot_sync(0xffffffffu, eq);
       const int eq_rank = eq_seen + __popc(eqm & lt_mask);
-      take = f || (cand && key > T) || (eq && eq_rank < need_eq);
+      take = (in && !cand) || (cand && key > T) || (eq && eq_rank < need_eq);
       eq_seen += __popc(eqm);
     }
     const unsigned tm = __ballot_sync(0xffffffffu, take);
@@ -155,7 +155,14 @@ __global__ void __launch_bounds__(32 * kWarps) select_kernel(const SelectArgs a)
 cudaError_t launch_select(const SelectArgs &a, cudaStream_t s) {
   const long long items = static_cast<long long>(a.total_q) * a.H_kv;
   const unsigned blocks = static_cast<unsigned>((items + kWarps - 1) / kWarps);
-  select_kernel<<<blocks, 32 * kWarps, 0, s>>>(a);
+  if (a.max_blocks <= 4 * 32)
+    select_kernel<4><<<blocks, 32 * kWarps, 0, s>>>(a);
+  else if (a.max_blocks <= 16 * 32)
+    select_kernel<16><<<blocks, 32 * kWarps, 0, s>>>(a);
+  else if (a.max_blocks <= 32 * 32)
+    select_kernel<32><<<blocks, 32 * kWarps, 0, s>>>(a);
+  else
+    select_kernel<0><<<blocks, 32 * kWarps, 0, s>>>(a);
   return cudaGetLastError();
 }
 

@@ -64,6 +64,9 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.msa_attn_workspace_bytes.argtypes = [RP, I, I, I, I, I]
     lib.msa_default_num_splits.restype = I
     lib.msa_default_num_splits.argtypes = [I, I, I, I, I]
+    lib.msa_attn_partials.restype = I
+    lib.msa_attn_partials.argtypes = [RP, I, I, I, I, I, ctypes.POINTER(ctypes.c_size_t),
+                                      ctypes.POINTER(ctypes.c_size_t)]
     lib.msa_status_string.restype = ctypes.c_char_p
     lib.msa_status_string.argtypes = [I]
     _lib = lib
@@ -114,6 +117,15 @@ def msa_attn_workspace_bytes(rp: RaggedPaged, S: int, num_q_heads: int, num_kv_h
                              max_blocks: int, num_splits: int) -> int:
     return int(load().msa_attn_workspace_bytes(ctypes.byref(rp), S, num_q_heads, num_kv_heads,
                                                max_blocks, num_splits))
+
+
+def msa_attn_partials(rp: RaggedPaged, S: int, num_q_heads: int, num_kv_heads: int,
+                      max_blocks: int, num_splits: int):
+    """(number of partial split indices, partial_o byte offset, partial_lse byte offset)."""
+    o, l_ = ctypes.c_size_t(0), ctypes.c_size_t(0)
+    n = load().msa_attn_partials(ctypes.byref(rp), S, num_q_heads, num_kv_heads, max_blocks,
+                                 num_splits, ctypes.byref(o), ctypes.byref(l_))
+    return int(n), int(o.value), int(l_.value)
 
 
 def msa_index_scores(rp: RaggedPaged, q_idx, k_idx_cache, num_kv_heads: int,
@@ -185,14 +197,25 @@ class Path:
                           self.max_blocks, p["top_k"], p["init_blocks"], p["local_blocks"],
                           self.block_ids, self.num_selected, self.dev_err, stream)
 
-    def attend(self, block_ids=None, num_selected=None, stream=None):
+    def attend(self, block_ids=None, num_selected=None, stream=None, combine=True):
+        """Stage 3.  With combine=False on the decode / speculative routes only the split-K
+        partials are written (into the workspace); ``combine()`` then merges them."""
         p = self.p
         msa_sparse_attn_paged(self.rp, p["q"], p["k"], p["v"], self.kv_dtype,
                               self.block_ids if block_ids is None else block_ids,
                               self.num_selected if num_selected is None else num_selected,
                               p["S"], p["H_q"], p["H_kv"], self.max_blocks, p["scale"],
-                              self.num_splits, self.workspace, self.out, self.dev_err, stream,
-                              workspace_bytes=self.workspace_bytes)
+                              self.num_splits, self.workspace, self.out if combine else 0,
+                              self.dev_err, stream, workspace_bytes=self.workspace_bytes)
+
+    def partials(self):
+        n, o_off, l_off = msa_attn_partials(self.rp, self.p["S"], self.p["H_q"], self.p["H_kv"],
+                                            self.max_blocks, self.num_splits)
+        return n, self.workspace.data_ptr() + o_off, self.workspace.data_ptr() + l_off
+
+    def combine(self, stream=None):
+        n, o_ptr, l_ptr = self.partials()
+        msa_splitk_combine(o_ptr, l_ptr, n, self.p["total_q"], self.p["H_q"], self.out, stream)
 
     def run(self, stream=None):
         self.index_scores(stream)

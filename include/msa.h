@@ -142,11 +142,14 @@ MSA_API msa_status_t msa_select_blocks(const msa_ragged_paged_t *rp, const float
  *   FP32 accumulation, output rounded to BF16.
  *
  *   Route from rp->max_q_len: 1 -> decode (no causal mask needed: p = L_b - 1); 2..8 ->
- *   speculative decode (per-token causal mask); > 8 -> prefill (per-token causal mask,
- *   device-built plan of each tile's union of selected blocks in `workspace`).
- *   Decode / speculative work is split over the selected blocks ("split-K") into num_splits
- *   partitions (0 = msa_default_num_splits); with more than one partition the partials live
- *   in `workspace` and this call also enqueues the combine that writes `out`.
+ *   speculative decode (per-token causal mask); > 8 -> prefill (per-token causal mask).
+ *   Speculative and prefill steps first build, in `workspace`, each query tile's union of its
+ *   tokens' selected blocks with a per-token mask, so that a page is read once per tile.
+ *   Decode / speculative work is a list of (sequence, query tile, KV head, selected block)
+ *   entries cut into `num_splits` equal contiguous split-K partitions (0 = one per SM, a
+ *   persistent launch); their partials live in `workspace` and this call also enqueues the
+ *   combine that writes `out`.  Prefill runs one CTA per (sequence, query tile, KV head) and
+ *   ignores num_splits.
  *
  *   q            device bf16 [total_q, num_q_heads, 128]
  *   k_cache, v_cache  device [num_pages, num_kv_heads, 128 tokens, 128] of kv_dtype,
@@ -155,7 +158,9 @@ MSA_API msa_status_t msa_select_blocks(const msa_ragged_paged_t *rp, const float
  *   max_blocks   an upper bound on nb(p) of every query (as for msa_index_scores)
  *   workspace    device, >= msa_attn_workspace_bytes(...) bytes, 256-byte aligned;
  *                may be NULL when that size is 0
- *   out          device bf16 [total_q, num_q_heads, 128] (output)
+ *   out          device bf16 [total_q, num_q_heads, 128] (output).  On the decode and
+ *                speculative routes `out` may be NULL: the call then leaves the split-K
+ *                partials in `workspace` (see msa_attn_partials) and enqueues no combine.
  *   num_q_heads % num_kv_heads == 0; the group size num_q_heads / num_kv_heads <= 64.
  */
 MSA_API msa_status_t msa_sparse_attn_paged(const msa_ragged_paged_t *rp, const void *q,
@@ -190,11 +195,20 @@ MSA_API msa_status_t msa_splitk_combine(const float *partial_o, const float *par
 MSA_API size_t msa_attn_workspace_bytes(const msa_ragged_paged_t *rp, int32_t S, int32_t num_q_heads,
                                 int32_t num_kv_heads, int32_t max_blocks, int32_t num_splits);
 
-/* The split-K partition count the decode / speculative routes use when num_splits == 0:
- * enough (sequence, KV head, partition) work items to fill `num_sms` SMs about twice over,
- * never more partitions than S / 2 (at least one block pair each), and 1 for prefill. */
+/* The split-K partition count the decode / speculative routes use when num_splits == 0 for
+ * `batch` sequences of `max_q_len` new tokens: one partition per SM, fewer when the work list
+ * (batch x num_kv_heads x S x max_q_len entries) has under 4 entries per SM; 1 for prefill. */
 MSA_API int32_t msa_default_num_splits(int32_t batch, int32_t max_q_len, int32_t num_kv_heads,
                                int32_t S, int32_t num_sms);
+
+/* Where msa_sparse_attn_paged keeps its split-K partials in `workspace` for this shape:
+ * returns the number of split indices (the num_splits argument msa_splitk_combine takes) and
+ * stores the byte offsets of partial_o [n, total_q, H_q, 128] and partial_lse [n, total_q,
+ * H_q] (both fp32); returns 0 when the route writes `out` directly (prefill) or on invalid
+ * arguments.  The offsets may be NULL. */
+MSA_API int32_t msa_attn_partials(const msa_ragged_paged_t *rp, int32_t S, int32_t num_q_heads,
+                                  int32_t num_kv_heads, int32_t max_blocks, int32_t num_splits,
+                                  size_t *partial_o_offset, size_t *partial_lse_offset);
 
 /* A static, human-readable name of a status code. */
 MSA_API const char *msa_status_string(msa_status_t status);

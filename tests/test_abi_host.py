@@ -61,12 +61,12 @@ def test_status_strings(lib):
 
 
 def test_default_splits_fill_the_sms(lib):
-    # decode: (sequence, KV head) items x splits ~ 2 x SMs, capped at S/2 and >= 1
-    assert msa.msa_default_num_splits(32, 1, 8, 19, 148) == 2
-    assert msa.msa_default_num_splits(1, 1, 1, 6, 148) == 3
-    assert msa.msa_default_num_splits(128, 1, 8, 69, 148) == 1
-    assert msa.msa_default_num_splits(64, 4, 8, 35, 148) == 1
-    assert msa.msa_default_num_splits(8, 4096, 8, 67, 148) == 1  # prefill: one partition
+    # decode / speculative: one persistent partition per SM, fewer for tiny work lists
+    assert msa.msa_default_num_splits(32, 1, 8, 19, 148) == 148
+    assert msa.msa_default_num_splits(1, 1, 1, 6, 148) == 2       # 6 entries, >= 4 per CTA
+    assert msa.msa_default_num_splits(128, 1, 8, 69, 148) == 148
+    assert msa.msa_default_num_splits(64, 4, 8, 35, 148) == 148
+    assert msa.msa_default_num_splits(8, 4096, 8, 67, 148) == 1   # prefill: one partition
     assert msa.msa_default_num_splits(0, 1, 8, 19, 148) == 1
 
 
@@ -76,14 +76,20 @@ def _rp(batch=2, total_q=2, max_q_len=1, max_pages=16, num_pages=64):
 
 
 def test_workspace_bytes(lib):
-    rp = _rp(batch=4, total_q=4, max_q_len=1)
-    assert msa.msa_attn_workspace_bytes(rp, 19, 64, 8, 16, 1) == 0       # decode, one split
-    ws = msa.msa_attn_workspace_bytes(rp, 19, 64, 8, 16, 3)
     rows = 4 * 64
-    assert ws >= 3 * rows * 128 * 4 + 3 * rows * 4                       # partial o + lse
+    rp = _rp(batch=4, total_q=4, max_q_len=1)
+    # one partition covering all 4 x 8 items of 19 slots: one piece each, 4 position splits
+    ws1 = msa.msa_attn_workspace_bytes(rp, 19, 64, 8, 16, 1)
+    assert ws1 >= 4 * rows * 128 * 4 + 4 * rows * 4
+    # three partitions: some item straddles two of them -> two pieces
+    ws3 = msa.msa_attn_workspace_bytes(rp, 19, 64, 8, 16, 3)
+    assert ws3 >= 8 * rows * 128 * 4 + 8 * rows * 4
     rp = _rp(batch=2, total_q=8, max_q_len=4)
-    ws = msa.msa_attn_workspace_bytes(rp, 35, 64, 8, 16, 1)              # speculative: plan
-    assert ws >= 2 * 8 * 16 * 8
+    ws = msa.msa_attn_workspace_bytes(rp, 35, 64, 8, 16, 1)              # speculative: + plan
+    assert ws >= 4 * 8 * 64 * 128 * 4 + 2 * 8 * 16 * 8
+    rp = _rp(batch=2, total_q=600, max_q_len=300)
+    ws = msa.msa_attn_workspace_bytes(rp, 35, 64, 8, 16, 0)              # prefill: plan only
+    assert 0 < ws < 600 * 64 * 128 * 4
     assert msa.msa_attn_workspace_bytes(rp, 0, 64, 8, 16, 1) == 0        # invalid -> 0
     assert msa.msa_attn_workspace_bytes(rp, 35, 63, 8, 16, 1) == 0
 
@@ -128,6 +134,7 @@ def test_invalid_arguments_are_rejected_before_any_launch(lib):
     assert attn(k=P + 8) == msa.MSA_ERR_INVALID_ARG        # cache not 16-byte aligned
     assert attn(hq=8 * 128) == msa.MSA_ERR_UNSUPPORTED     # GQA group 128 > 64
     assert attn(ns=4) == msa.MSA_ERR_INVALID_ARG           # partials need a workspace
+    assert attn(ns=5000) == msa.MSA_ERR_INVALID_ARG        # more partitions than allowed
     stat = lib.msa_splitk_combine(None, P, 2, 4, 8, P, None)
     assert stat == msa.MSA_ERR_INVALID_ARG
     stat = lib.msa_splitk_combine(P, P, 0, 4, 8, P, None)

@@ -103,21 +103,42 @@ def test_whole_path_matches_oracle(name):
     check_attention(path.out.float().cpu(), out, p["kv_fp8"], rows_mask=mask)
 
 
-@pytest.mark.parametrize("splits", [1, 2, 3, 7, 19])
-def test_split_k_counts_agree(splits):
-    p, (_, ids, cnt, out) = _oracle("bf16_decode")
-    ref = None
+@pytest.mark.parametrize("name,splits", [("bf16_decode", n) for n in (1, 2, 3, 7, 19, 148, 700)]
+                         + [("spec_ragged_q", n) for n in (1, 5, 148)]
+                         + [("fp8_decode", n) for n in (1, 13, 148)])
+def test_split_k_partitions_agree(name, splits):
+    """Any number of split-K partitions gives the oracle's answer, and the partitions agree with
+    one another to fp32 reassociation (a couple of bf16 ulps after rounding)."""
+    p, (_, ids, cnt, out) = _oracle(name)
+    gids, gcnt = torch.from_numpy(ids).cuda(), torch.from_numpy(cnt).cuda()
     path = msa.Path(_gpu(p), num_splits=splits)
-    path.attend(block_ids=torch.from_numpy(ids).cuda(), num_selected=torch.from_numpy(cnt).cuda())
-    torch.cuda.synchronize()
-    check_attention(path.out.float().cpu(), out, False)
+    path.attend(block_ids=gids, num_selected=gcnt)
     base = msa.Path(_gpu(p), num_splits=1)
-    base.attend(block_ids=torch.from_numpy(ids).cuda(), num_selected=torch.from_numpy(cnt).cuda())
+    base.attend(block_ids=gids, num_selected=gcnt)
     torch.cuda.synchronize()
+    assert int(path.dev_err.item()) == 0
+    check_attention(path.out.float().cpu(), out, p["kv_fp8"])
     ref = base.out.float()
-    # fp32 reassociation across partitions: at most a couple of bf16 ulps apart
     diff = (path.out.float() - ref).abs()
     assert float(diff.max()) <= 2 * 2 ** -7 * float(ref.abs().max())
+
+
+@pytest.mark.parametrize("name", ["bf16_decode", "spec_decode", "fp8_spec"])
+def test_partials_then_public_combine_equal_the_fused_call(name):
+    p, (_, ids, cnt, out) = _oracle(name)
+    gids, gcnt = torch.from_numpy(ids).cuda(), torch.from_numpy(cnt).cuda()
+    fused = msa.Path(_gpu(p))
+    fused.attend(block_ids=gids, num_selected=gcnt)
+    split = msa.Path(_gpu(p))
+    split.out.fill_(float("nan"))
+    split.attend(block_ids=gids, num_selected=gcnt, combine=False)
+    torch.cuda.synchronize()
+    assert torch.isnan(split.out.float()).all()          # no combine ran
+    n, _, _ = split.partials()
+    assert n >= 2
+    split.combine()
+    torch.cuda.synchronize()
+    assert torch.equal(split.out, fused.out)
 
 
 def test_splitk_combine_entry_point():
