@@ -375,7 +375,8 @@ def run_ours(args):
         return 0
     hbm, bf16, bf16_sus, peak_src = measured_peaks()
     kinds = {"index_scores": (stage_ms[0], idx_bytes, "indexer.cu"),
-             "attention": (stage_ms[2], attn_bytes, "attention.cu")}
+             "attention": (stage_ms[2], attn_bytes,
+                           "attention_stream.cu" if stream_route else "attention_tile.cu")}
     dom = max(kinds, key=lambda k: kinds[k][0])
     d_ms, d_bytes, d_src = kinds[dom]
     achieved = d_bytes / (d_ms * 1e-3) / 1e9

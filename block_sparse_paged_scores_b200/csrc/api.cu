@@ -97,7 +97,7 @@ struct Route {
   int grid;       // persistent kernel: CTAs (= split-K partitions)
   long long R;    // slots per CTA
   int P;          // most CTAs one item spans
-  int splits;     // partial split indices: P * position splits
+  int splits;     // partial split indices (= P)
   size_t off_o, off_lse, off_list, off_masks, off_counts, bytes;
 };
 
@@ -152,7 +152,7 @@ bool make_route(const msa_ragged_paged_t *rp, int S, int H_q, int H_kv, int max_
       P = std::max<int>(P, static_cast<int>(last - first + 1));
     }
     r->P = P;
-    r->splits = P * attn_position_splits(r->rg);
+    r->splits = P;
   }
   const size_t rows = static_cast<size_t>(rp->total_q) * H_q;
   size_t off = 0;

@@ -15,14 +15,17 @@
 // plan.cu, cap = tile tokens x S), of which the first U are real.  The items' slots laid end
 // to end are cut into equal contiguous ranges of R slots, one per CTA (a split-K partition):
 // every SM streams the same number of slots.  A CTA's range meets a few items; each meeting is
-// a "segment" and each (segment, consumer warp) leaves one partial (normalised output and
-// log-sum-exp) at split index piece * PQ + position-quarter, piece = the CTA's rank among the
-// CTAs that share the item.  msa_splitk_combine's kernel merges them.
+// a "segment", merged inside the CTA into one partial (normalised output and log-sum-exp) at
+// split index `piece` = the CTA's rank among the CTAs that share the item.
+// msa_splitk_combine's kernel merges the pieces.
 //
 // Roles: one producer warp loads each segment's Q rows into a double-buffered Q slot and
 // issues the TMA loads of the K and V page tiles (128-byte swizzle) into a ring of tile slots,
-// running ahead across segment boundaries; 4 x RG consumer warps run the per-block math of
-// attn_common.cuh, releasing the K slot after QK^T and the V slot after PV.
+// running ahead across segment boundaries.  Consumer warps run the per-block math of
+// attn_common.cuh (each owns 16 rows and a share of every block's positions; with one row
+// group, two teams take alternate blocks), release the K slot after QK^T and the V slot after
+// PV, and at the end of a segment fold their online-softmax states into one per row through
+// shared memory.
 #include <math.h>
 
 #include "attn_common.cuh"
@@ -37,11 +40,30 @@ struct StreamCfg {
   static constexpr int kSlots = FP8 ? 10 : 5;  // 160 KiB of tiles in flight per SM
 };
 
-template <bool FP8>
+// Consumer layout for RG 16-row groups: PQ warps split every block's positions and NT teams
+// of RG * PQ warps take alternate blocks, so that every SM sub-partition runs two
+// independent block chains when the rows fit one group.
+template <int RG>
+constexpr int stream_pq() {
+  return RG <= 2 ? 4 : 2;
+}
+template <int RG>
+constexpr int stream_teams() {
+  return RG == 1 ? 2 : 1;
+}
+template <int RG>
+constexpr int stream_consumer_warps() {
+  return RG * stream_pq<RG>() * stream_teams<RG>();
+}
+
+template <bool FP8, int RG>
 constexpr size_t stream_smem_bytes() {
   return 1024 + StreamCfg<FP8>::kSlots * StreamCfg<FP8>::kTile + 2 * kQBuf +
+         RG * 16 * kHeadDim * sizeof(float) +                        // merge accumulator
          (2 * StreamCfg<FP8>::kSlots + 4) * sizeof(uint64_t) +
-         StreamCfg<FP8>::kSlots * 3 * sizeof(int) + 16;
+         StreamCfg<FP8>::kSlots * 3 * sizeof(int) +
+         2 * stream_consumer_warps<RG>() * 16 * sizeof(float) +       // per-warp m, l
+         2 * RG * 16 * sizeof(float) + 16;                           // per-row M, L
 }
 
 struct Item {
@@ -108,11 +130,13 @@ __device__ __forceinline__ void segment(const AttnArgs &a, int it, long long r0,
 }
 
 template <bool FP8, int RG, bool PLAN>
-__global__ void __launch_bounds__(32 * (RG * (RG <= 2 ? 4 : 2) + 1))
+__global__ void __launch_bounds__(32 * (stream_consumer_warps<RG>() + 1))
     attn_stream_kernel(const __grid_constant__ CUtensorMap kmap,
                        const __grid_constant__ CUtensorMap vmap, const AttnArgs a) {
-  constexpr int PQ = RG <= 2 ? 4 : 2;
-  constexpr int NCW = RG * PQ;
+  constexpr int PQ = stream_pq<RG>();
+  constexpr int NT = stream_teams<RG>();
+  constexpr int TEAM = RG * PQ;                    // warps of one team
+  constexpr int NCW = stream_consumer_warps<RG>();  // all consumer warps
   constexpr int NSLOT = StreamCfg<FP8>::kSlots;
   constexpr uint32_t TILE = StreamCfg<FP8>::kTile;
   using WA = WarpAttn<FP8, PQ>;
@@ -130,19 +154,24 @@ __global__ void __launch_bounds__(32 * (RG * (RG <= 2 ? 4 : 2) + 1))
                                               ~static_cast<uintptr_t>(1023));
   uint8_t *slots = smem;
   uint8_t *qbufs = slots + NSLOT * TILE;
-  uint64_t *sfull = reinterpret_cast<uint64_t *>(qbufs + 2 * kQBuf);
+  float *acc = reinterpret_cast<float *>(qbufs + 2 * kQBuf);  // [RG*16][128] merge buffer
+  uint64_t *sfull = reinterpret_cast<uint64_t *>(acc + RG * 16 * kHeadDim);
   uint64_t *sempty = sfull + NSLOT;
   uint64_t *qfull = sempty + NSLOT;
   uint64_t *qempty = qfull + 2;
   int *slot_j = reinterpret_cast<int *>(qempty + 2);
   uint32_t *slot_mask = reinterpret_cast<uint32_t *>(slot_j + NSLOT);
   int *slot_ok = reinterpret_cast<int *>(slot_mask + NSLOT);
-  volatile int *abort_flag = reinterpret_cast<volatile int *>(slot_ok + NSLOT);
+  float *mrg_m = reinterpret_cast<float *>(slot_ok + NSLOT);  // [NCW][16]
+  float *mrg_l = mrg_m + NCW * 16;                              // [NCW][16]
+  float *row_m = mrg_l + NCW * 16;                              // [RG*16]
+  float *row_l = row_m + RG * 16;                               // [RG*16]
+  volatile int *abort_flag = reinterpret_cast<volatile int *>(row_l + RG * 16);
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < NSLOT; ++s) {
       mbar_init(&sfull[s], 1);
-      mbar_init(&sempty[s], NCW);
+      mbar_init(&sempty[s], TEAM);  // each tile is read by one team
     }
     for (int q = 0; q < 2; ++q) {
       mbar_init(&qfull[q], 1);
@@ -151,7 +180,10 @@ __global__ void __launch_bounds__(32 * (RG * (RG <= 2 ? 4 : 2) + 1))
     *abort_flag = 0;
     fence_mbar_init();
   }
+  for (int i = threadIdx.x; i < RG * 16 * kHeadDim; i += blockDim.x) acc[i] = 0.f;
   __syncthreads();
+  pdl_wait();  // block ids, selection counts and the plan come from earlier kernels
+  pdl_launch_dependents();
 
   if (warp == NCW) {
     // ============================================================== producer warp
@@ -176,40 +208,55 @@ __global__ void __launch_bounds__(32 * (RG * (RG <= 2 ? 4 : 2) + 1))
       if (lane == 0) mbar_arrive(&qfull[0]);
     }
     while (it <= it_last && !dead) {
-      // ---- K and V tiles of segment n
-      if (lane == 0) {
-        for (int e = v0; e < v1 && !dead; ++e) {
-          const int j = cur.list[e];
-          const uint32_t msk = PLAN ? cur.masks[e] : 0xffffffffu;
-          const bool jok = j >= 0 && j < a.max_blocks;
-          const int page = jok ? a.table[static_cast<size_t>(cur.b) * a.max_pages + j] : -1;
-          const bool ok = jok && page >= 0 && page < a.num_pages;
-          if (!ok) report(a.dev_err, jok ? MSA_DEVERR_PAGE_ID : MSA_DEVERR_BLOCK_ID);
-          const int c2 = page * a.H_kv + cur.g;
+      // ---- K and V tiles of segment n.  The warp resolves 32 blocks' page ids at a time
+      // (one lane each) so that lane 0 never waits on a dependent lookup between two TMAs.
+      for (int base = v0; base < v1 && !dead; base += 32) {
+        const int e = base + lane;
+        int j = -1, page = -1;
+        uint32_t msk = 0u;
+        if (e < v1) {
+          j = cur.list[e];
+          msk = PLAN ? cur.masks[e] : 0xffffffffu;
+          if (j >= 0 && j < a.max_blocks)
+            page = a.table[static_cast<size_t>(cur.b) * a.max_pages + j];
+        }
+        const int cnt = min(32, v1 - base);
+        for (int i = 0; i < cnt; ++i) {
+          const int jj = __shfl_sync(0xffffffffu, j, i);
+          const int pg = __shfl_sync(0xffffffffu, page, i);
+          const uint32_t mm = __shfl_sync(0xffffffffu, msk, i);
+          if (lane == 0) {
+            const bool jok = jj >= 0 && jj < a.max_blocks;
+            const bool ok = jok && pg >= 0 && pg < a.num_pages;
+            if (!ok) report(a.dev_err, jok ? MSA_DEVERR_PAGE_ID : MSA_DEVERR_BLOCK_ID);
+            const int c2 = pg * a.H_kv + cur.g;
 #pragma unroll
-          for (int kv = 0; kv < 2; ++kv) {
-            const int s = static_cast<int>(nload % NSLOT);
-            if (nload >= static_cast<uint32_t>(NSLOT) &&
-                !mbar_wait(&sempty[s], ((nload / NSLOT) - 1) & 1, abort_flag)) {
-              report(a.dev_err, MSA_DEVERR_TIMEOUT);
-              *abort_flag = 1;
-              dead = true;
-              break;
+            for (int kv = 0; kv < 2; ++kv) {
+              const int s = static_cast<int>(nload % NSLOT);
+              if (nload >= static_cast<uint32_t>(NSLOT) &&
+                  !mbar_wait(&sempty[s], ((nload / NSLOT) - 1) & 1, abort_flag)) {
+                report(a.dev_err, MSA_DEVERR_TIMEOUT);
+                *abort_flag = 1;
+                dead = true;
+                break;
+              }
+              slot_j[s] = jj;
+              slot_mask[s] = mm;
+              slot_ok[s] = ok;
+              if (ok) {
+                const CUtensorMap *mp = kv ? &vmap : &kmap;
+                uint8_t *dst = slots + s * TILE;
+                mbar_arrive_expect_tx(&sfull[s], TILE);
+                tma_load_3d(dst, mp, &sfull[s], 0, 0, c2);
+                if (!FP8) tma_load_3d(dst + TILE / 2, mp, &sfull[s], 64, 0, c2);
+              } else {
+                mbar_arrive(&sfull[s]);
+              }
+              ++nload;
             }
-            slot_j[s] = j;
-            slot_mask[s] = msk;
-            slot_ok[s] = ok;
-            if (ok) {
-              const CUtensorMap *mp = kv ? &vmap : &kmap;
-              uint8_t *dst = slots + s * TILE;
-              mbar_arrive_expect_tx(&sfull[s], TILE);
-              tma_load_3d(dst, mp, &sfull[s], 0, 0, c2);
-              if (!FP8) tma_load_3d(dst + TILE / 2, mp, &sfull[s], 64, 0, c2);
-            } else {
-              mbar_arrive(&sfull[s]);
-            }
-            ++nload;
           }
+          dead = __shfl_sync(0xffffffffu, dead, 0);
+          if (dead) break;
         }
       }
       dead = __shfl_sync(0xffffffffu, dead, 0);
@@ -249,7 +296,9 @@ __global__ void __launch_bounds__(32 * (RG * (RG <= 2 ? 4 : 2) + 1))
   }
 
   // ================================================================ consumer warps
-  const int rg = warp / PQ, pq = warp % PQ;
+  const int team = warp / TEAM, rg = (warp % TEAM) / PQ, pq = warp % PQ;
+  const bool row_owner = team == 0 && pq == 0 && (lane & 3) == 0;  // one writer per row
+  const int nct = 32 * NCW;
   WA wa;
   uint32_t nload = 0;
   int n = 0;
@@ -261,6 +310,7 @@ __global__ void __launch_bounds__(32 * (RG * (RG <= 2 ? 4 : 2) + 1))
     const long long base = static_cast<long long>(it) * a.cap;
     const int piece = static_cast<int>(blockIdx.x - base / a.R);
     const bool last_cta = (base + a.cap - 1) / a.R == blockIdx.x;
+    const size_t split_stride = static_cast<size_t>(a.total_q) * a.H_q;
     // this thread's two rows
     int prow[2];
     uint32_t tbit[2];
@@ -275,7 +325,6 @@ __global__ void __launch_bounds__(32 * (RG * (RG <= 2 ? 4 : 2) + 1))
       tbit[slot] = rvalid[slot] ? (1u << tl) : 0u;
       orow[slot] = rvalid[slot] ? static_cast<size_t>(m.t0 + tl) * a.H_q + m.g * a.G + r % a.G : 0;
     }
-    const size_t split_stride = static_cast<size_t>(a.total_q) * a.H_q;
 
     if (v1 > v0) {
       const int buf = n & 1;
@@ -286,64 +335,119 @@ __global__ void __launch_bounds__(32 * (RG * (RG <= 2 ? 4 : 2) + 1))
       }
       const uint32_t qs_addr = smem_u32(qbufs + buf * kQBuf);
       wa.reset();
-      for (int e = v0; e < v1; ++e) {
-        // K tile
-        int s = static_cast<int>(nload % NSLOT);
-        bool live = mbar_wait(&sfull[s], (nload / NSLOT) & 1, abort_flag);
+      for (int e = v0 + team; e < v1; e += NT) {
+        const uint32_t nk = nload + 2u * static_cast<uint32_t>(e - v0);  // K tile; V is nk + 1
+        int s = static_cast<int>(nk % NSLOT);
+        bool live = mbar_wait(&sfull[s], (nk / NSLOT) & 1, abort_flag);
         const bool ok = live && qlive && slot_ok[s];
         const int j = slot_j[s];
         const uint32_t msk = slot_mask[s];
         if (ok) wa.qk(qs_addr, rg * 16, smem_u32(slots + s * TILE), pq, lane);
         __syncwarp();
         if (lane == 0) mbar_arrive(&sempty[s]);
-        ++nload;
         if (ok) wa.softmax(j, pq, lane, prow, tbit, msk, a.scale_log2);
-        // V tile
-        s = static_cast<int>(nload % NSLOT);
-        live = mbar_wait(&sfull[s], (nload / NSLOT) & 1, abort_flag) && live;
+        s = static_cast<int>((nk + 1) % NSLOT);
+        live = mbar_wait(&sfull[s], ((nk + 1) / NSLOT) & 1, abort_flag) && live;
         if (ok && live) wa.pv(smem_u32(slots + s * TILE), j, pq, lane, m.L);
         __syncwarp();
         if (lane == 0) mbar_arrive(&sempty[s]);
-        ++nload;
         if (!live) {
           report(a.dev_err, MSA_DEVERR_TIMEOUT);
           *abort_flag = 1;
         }
       }
+      nload += 2u * static_cast<uint32_t>(v1 - v0);
       __syncwarp();
       if (lane == 0) mbar_arrive(&qempty[buf]);
       ++n;
+
+      // ---- fold the NT * PQ warp states of every row into one, through shared memory
       wa.finish_rows();
-      // partial of this (segment, warp): normalised output and natural log-sum-exp
-      const size_t split = static_cast<size_t>(piece) * PQ + pq;
+      if ((lane & 3) == 0) {
 #pragma unroll
-      for (int slot = 0; slot < 2; ++slot) {
-        if (!rvalid[slot]) continue;
-        const float l = wa.l_run[slot];
-        const size_t prow_i = split * split_stride + orow[slot];
-        if (l > 0.f) {
-          wa.store_row(a.part_o + prow_i * kHeadDim, slot, 1.f / l, lane);
-          if ((lane & 3) == 0) a.part_lse[prow_i] = (wa.m_run[slot] + __log2f(l)) * kLn2;
-        } else if ((lane & 3) == 0) {
-          a.part_lse[prow_i] = -INFINITY;
+        for (int slot = 0; slot < 2; ++slot) {
+          mrg_m[warp * 16 + (lane >> 2) + slot * 8] = wa.m_run[slot];
+          mrg_l[warp * 16 + (lane >> 2) + slot * 8] = wa.l_run[slot];
         }
       }
-    } else {
+      named_bar_sync(1, nct);
+#pragma unroll
+      for (int slot = 0; slot < 2; ++slot) {
+        const int r16 = (lane >> 2) + slot * 8;
+        float M = -INFINITY;
+#pragma unroll
+        for (int t2 = 0; t2 < NT; ++t2)
+#pragma unroll
+          for (int p2 = 0; p2 < PQ; ++p2)
+            M = fmaxf(M, mrg_m[(t2 * TEAM + rg * PQ + p2) * 16 + r16]);
+        float Ls = 0.f;
+        if (M != -INFINITY) {
+#pragma unroll
+          for (int t2 = 0; t2 < NT; ++t2)
+#pragma unroll
+            for (int p2 = 0; p2 < PQ; ++p2) {
+              const int w2 = t2 * TEAM + rg * PQ + p2;
+              const float mw = mrg_m[w2 * 16 + r16];
+              if (mw != -INFINITY) Ls += mrg_l[w2 * 16 + r16] * fast_exp2(mw - M);
+            }
+        }
+        if (wa.m_run[slot] != -INFINITY) {
+          const float f = fast_exp2(wa.m_run[slot] - M);
+          float *dst = acc + (rg * 16 + r16) * kHeadDim;
+          const int c4 = lane & 3;
+          if (FP8) {
+#pragma unroll
+            for (int ch = 0; ch < 8; ++ch) {
+              red_add_shared(dst + ch * 16 + 4 * c4 + 0, wa.o[2 * ch][2 * slot] * f);
+              red_add_shared(dst + ch * 16 + 4 * c4 + 1, wa.o[2 * ch + 1][2 * slot] * f);
+              red_add_shared(dst + ch * 16 + 4 * c4 + 2, wa.o[2 * ch][2 * slot + 1] * f);
+              red_add_shared(dst + ch * 16 + 4 * c4 + 3, wa.o[2 * ch + 1][2 * slot + 1] * f);
+            }
+          } else {
+#pragma unroll
+            for (int nn = 0; nn < 16; ++nn) {
+              red_add_shared(dst + nn * 8 + 2 * c4, wa.o[nn][2 * slot] * f);
+              red_add_shared(dst + nn * 8 + 2 * c4 + 1, wa.o[nn][2 * slot + 1] * f);
+            }
+          }
+        }
+        if (row_owner) {
+          row_m[rg * 16 + r16] = M;
+          row_l[rg * 16 + r16] = Ls;
+        }
+      }
+      named_bar_sync(1, nct);
+      // ---- write this segment's partial (all consumer threads), clear the accumulator
+      const int ctid = threadIdx.x;  // consumers are threads [0, nct)
+      for (int idx = ctid; idx < RG * 16 * (kHeadDim / 4); idx += nct) {
+        const int r = idx / (kHeadDim / 4), d4 = idx % (kHeadDim / 4);
+        float4 *src = reinterpret_cast<float4 *>(acc + r * kHeadDim) + d4;
+        if (r < m.rows) {
+          const int tl = r / a.G;
+          const size_t orr = static_cast<size_t>(m.t0 + tl) * a.H_q + m.g * a.G + r % a.G;
+          const size_t pr = static_cast<size_t>(piece) * split_stride + orr;
+          const float L = row_l[r];
+          const float inv = L > 0.f ? 1.f / L : 0.f;
+          const float4 v = *src;
+          reinterpret_cast<float4 *>(a.part_o + pr * kHeadDim)[d4] =
+              make_float4(v.x * inv, v.y * inv, v.z * inv, v.w * inv);
+          if (d4 == 0) a.part_lse[pr] = L > 0.f ? (row_m[r] + __log2f(L)) * kLn2 : -INFINITY;
+        }
+        *src = make_float4(0.f, 0.f, 0.f, 0.f);
+      }
+    } else if (row_owner) {
       // a range that meets this item only in slots past its count: an empty partial
 #pragma unroll
       for (int slot = 0; slot < 2; ++slot)
-        if (rvalid[slot] && (lane & 3) == 0)
-          a.part_lse[(static_cast<size_t>(piece) * PQ + pq) * split_stride + orow[slot]] =
-              -INFINITY;
+        if (rvalid[slot]) a.part_lse[static_cast<size_t>(piece) * split_stride + orow[slot]] = -INFINITY;
     }
     // the item's last CTA marks the split indices no CTA of this item owns
-    if (last_cta) {
+    if (last_cta && row_owner) {
       for (int p2 = piece + 1; p2 < a.P; ++p2)
 #pragma unroll
         for (int slot = 0; slot < 2; ++slot)
-          if (rvalid[slot] && (lane & 3) == 0)
-            a.part_lse[(static_cast<size_t>(p2) * PQ + pq) * split_stride + orow[slot]] =
-                -INFINITY;
+          if (rvalid[slot])
+            a.part_lse[static_cast<size_t>(p2) * split_stride + orow[slot]] = -INFINITY;
     }
   }
 }
@@ -351,12 +455,12 @@ __global__ void __launch_bounds__(32 * (RG * (RG <= 2 ? 4 : 2) + 1))
 template <bool FP8, int RG, bool PLAN>
 cudaError_t launch_stream_one(const CUtensorMap &kmap, const CUtensorMap &vmap,
                               const AttnArgs &a, int grid, cudaStream_t s) {
-  const size_t smem = stream_smem_bytes<FP8>();
+  const size_t smem = stream_smem_bytes<FP8, RG>();
   auto fn = &attn_stream_kernel<FP8, RG, PLAN>;
   cudaError_t e = ensure_smem_limit(reinterpret_cast<const void *>(fn), static_cast<int>(smem));
   if (e != cudaSuccess) return e;
-  fn<<<grid, 32 * (RG * (RG <= 2 ? 4 : 2) + 1), smem, s>>>(kmap, vmap, a);
-  return cudaGetLastError();
+  return launch_pdl(fn, dim3(grid), dim3(32 * (stream_consumer_warps<RG>() + 1)), smem, s,
+                    kmap, vmap, a);
 }
 
 template <bool FP8, bool PLAN>
@@ -371,8 +475,6 @@ cudaError_t launch_stream_rg(const CUtensorMap &kmap, const CUtensorMap &vmap, c
 }
 
 }  // namespace
-
-int attn_position_splits(int rg) { return rg <= 2 ? 4 : 2; }
 
 cudaError_t launch_attention_stream(const CUtensorMap &kmap, const CUtensorMap &vmap,
                                     const AttnArgs &a, bool fp8, int rg, bool plan, int grid,

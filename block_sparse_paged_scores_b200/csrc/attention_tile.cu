@@ -43,6 +43,8 @@ template <bool FP8, int RG>
 __global__ void __launch_bounds__(32 * (RG * tile_pq<RG>() + 1))
     attn_tile_kernel(const __grid_constant__ CUtensorMap kmap,
                      const __grid_constant__ CUtensorMap vmap, const AttnArgs a) {
+  pdl_wait();
+  pdl_launch_dependents();
   using C = TileCfg<FP8>;
   constexpr int PQ = tile_pq<RG>();
   constexpr int NCW = RG * PQ, NCT = 32 * NCW, NS = C::kStages;
@@ -116,37 +118,56 @@ __global__ void __launch_bounds__(32 * (RG * tile_pq<RG>() + 1))
     if (lane == 0) {
       prefetch_tmap(&kmap);
       prefetch_tmap(&vmap);
-      for (int i = 0; i < nblk; ++i) {
-        const int s = i % NS;
-        if (i >= NS && !mbar_wait(&empty[s], ((i / NS) - 1) & 1, abort_flag)) {
-          report(a.dev_err, MSA_DEVERR_TIMEOUT);
-          *abort_flag = 1;
-          break;
-        }
-        const int j = list[i];
-        const bool jok = j >= 0 && j < a.max_blocks;
-        const int page = jok ? a.table[static_cast<size_t>(b) * a.max_pages + j] : -1;
-        const bool ok = jok && page >= 0 && page < a.num_pages;
-        st_j[s] = j;
-        st_mask[s] = masks[i];
-        st_ok[s] = ok;
-        if (ok) {
-          mbar_arrive_expect_tx(&full[s], 2 * TILE);
-          const int c2 = page * a.H_kv + g;
-          uint8_t *kd = stages + s * STAGE, *vd = kd + TILE;
-          if (FP8) {
-            tma_load_3d(kd, &kmap, &full[s], 0, 0, c2);
-            tma_load_3d(vd, &vmap, &full[s], 0, 0, c2);
+    }
+    bool dead = false;
+    // 32 blocks' page ids resolved at a time, one lane each, then issued by lane 0
+    for (int base = 0; base < nblk && !dead; base += 32) {
+      int j = -1, page = -1;
+      uint32_t msk = 0u;
+      if (base + lane < nblk) {
+        j = list[base + lane];
+        msk = masks[base + lane];
+        if (j >= 0 && j < a.max_blocks) page = a.table[static_cast<size_t>(b) * a.max_pages + j];
+      }
+      const int cnt = min(32, nblk - base);
+      for (int k = 0; k < cnt; ++k) {
+        const int jj = __shfl_sync(0xffffffffu, j, k);
+        const int pg = __shfl_sync(0xffffffffu, page, k);
+        const uint32_t mm = __shfl_sync(0xffffffffu, msk, k);
+        if (lane == 0) {
+          const int i = base + k;
+          const int s = i % NS;
+          if (i >= NS && !mbar_wait(&empty[s], ((i / NS) - 1) & 1, abort_flag)) {
+            report(a.dev_err, MSA_DEVERR_TIMEOUT);
+            *abort_flag = 1;
+            dead = true;
           } else {
-            tma_load_3d(kd, &kmap, &full[s], 0, 0, c2);
-            tma_load_3d(kd + TILE / 2, &kmap, &full[s], 64, 0, c2);
-            tma_load_3d(vd, &vmap, &full[s], 0, 0, c2);
-            tma_load_3d(vd + TILE / 2, &vmap, &full[s], 64, 0, c2);
+            const bool jok = jj >= 0 && jj < a.max_blocks;
+            const bool ok = jok && pg >= 0 && pg < a.num_pages;
+            st_j[s] = jj;
+            st_mask[s] = mm;
+            st_ok[s] = ok;
+            if (ok) {
+              mbar_arrive_expect_tx(&full[s], 2 * TILE);
+              const int c2 = pg * a.H_kv + g;
+              uint8_t *kd = stages + s * STAGE, *vd = kd + TILE;
+              if (FP8) {
+                tma_load_3d(kd, &kmap, &full[s], 0, 0, c2);
+                tma_load_3d(vd, &vmap, &full[s], 0, 0, c2);
+              } else {
+                tma_load_3d(kd, &kmap, &full[s], 0, 0, c2);
+                tma_load_3d(kd + TILE / 2, &kmap, &full[s], 64, 0, c2);
+                tma_load_3d(vd, &vmap, &full[s], 0, 0, c2);
+                tma_load_3d(vd + TILE / 2, &vmap, &full[s], 64, 0, c2);
+              }
+            } else {
+              report(a.dev_err, jok ? MSA_DEVERR_PAGE_ID : MSA_DEVERR_BLOCK_ID);
+              mbar_arrive(&full[s]);
+            }
           }
-        } else {
-          report(a.dev_err, jok ? MSA_DEVERR_PAGE_ID : MSA_DEVERR_BLOCK_ID);
-          mbar_arrive(&full[s]);
         }
+        dead = __shfl_sync(0xffffffffu, dead, 0);
+        if (dead) break;
       }
     }
     return;
@@ -247,8 +268,7 @@ cudaError_t launch_tile_one(const CUtensorMap &kmap, const CUtensorMap &vmap, co
   cudaError_t e = ensure_smem_limit(reinterpret_cast<const void *>(fn), static_cast<int>(smem));
   if (e != cudaSuccess) return e;
   const dim3 grid(a.batch * a.tiles, a.H_kv);
-  fn<<<grid, 32 * (RG * tile_pq<RG>() + 1), smem, s>>>(kmap, vmap, a);
-  return cudaGetLastError();
+  return launch_pdl(fn, grid, dim3(32 * (RG * tile_pq<RG>() + 1)), smem, s, kmap, vmap, a);
 }
 
 template <bool FP8>

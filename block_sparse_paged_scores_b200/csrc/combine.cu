@@ -17,24 +17,41 @@ namespace {
 
 constexpr int kWarps = 8;
 
+// One warp per (row, head).  All partitions' log-sum-exps are fetched at once (one lane
+// each), then every partition's output float4 is issued before any is used, so the warp
+// waits for about two memory latencies whatever the number of partitions.
 __global__ void __launch_bounds__(32 * kWarps)
     combine_kernel(const float *__restrict__ part_o, const float *__restrict__ part_lse,
                    int splits, long long rows, uint16_t *__restrict__ out) {
+  pdl_wait();
+  pdl_launch_dependents();
   const int lane = threadIdx.x & 31;
   const long long row = static_cast<long long>(blockIdx.x) * kWarps + (threadIdx.x >> 5);
   if (row >= rows) return;
-  float m = -INFINITY;
-  for (int s = lane; s < splits; s += 32) m = fmaxf(m, part_lse[s * rows + row]);
-#pragma unroll
-  for (int off = 16; off; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
   float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-  float wsum = 0.f;
-  if (m != -INFINITY) {
-    for (int s = 0; s < splits; ++s) {
-      const float lse = part_lse[s * rows + row];
-      if (lse == -INFINITY) continue;
-      const float w = expf(lse - m);
-      const float4 o = reinterpret_cast<const float4 *>(part_o + (s * rows + row) * kHeadDim)[lane];
+  float wsum = 0.f, M = -INFINITY;  // running max of the log-sum-exps seen so far
+  for (int s0 = 0; s0 < splits; s0 += 32) {
+    const int n = min(32, splits - s0);
+    const float my_lse = lane < n ? part_lse[(s0 + lane) * rows + row] : -INFINITY;
+    float m = my_lse;
+#pragma unroll
+    for (int off = 16; off; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
+    if (m == -INFINITY) continue;
+    const float m_new = fmaxf(M, m);
+    const float keep = M == -INFINITY ? 0.f : expf(M - m_new);  // rescale earlier chunks
+    acc.x *= keep;
+    acc.y *= keep;
+    acc.z *= keep;
+    acc.w *= keep;
+    wsum *= keep;
+    M = m_new;
+    const float w_lane = my_lse == -INFINITY ? 0.f : expf(my_lse - m_new);
+#pragma unroll 8
+    for (int s = 0; s < n; ++s) {
+      const float w = __shfl_sync(0xffffffffu, w_lane, s);
+      if (w == 0.f) continue;
+      const float4 o =
+          reinterpret_cast<const float4 *>(part_o + ((s0 + s) * rows + row) * kHeadDim)[lane];
       acc.x += w * o.x;
       acc.y += w * o.y;
       acc.z += w * o.z;
@@ -56,8 +73,8 @@ cudaError_t launch_combine(const float *part_o, const float *part_lse, int split
   const long long rows = static_cast<long long>(total_q) * H_q;
   if (rows == 0) return cudaSuccess;
   const unsigned blocks = static_cast<unsigned>((rows + kWarps - 1) / kWarps);
-  combine_kernel<<<blocks, 32 * kWarps, 0, s>>>(part_o, part_lse, splits, rows, out);
-  return cudaGetLastError();
+  return launch_pdl(combine_kernel, dim3(blocks), dim3(32 * kWarps), 0, s, part_o, part_lse,
+                    splits, rows, out);
 }
 
 }  // namespace msa

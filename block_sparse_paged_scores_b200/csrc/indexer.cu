@@ -34,6 +34,8 @@ constexpr size_t smem_bytes() {
 template <int MT>
 __global__ void __launch_bounds__(kThreads)
     index_scores_kernel(const __grid_constant__ CUtensorMap kmap, const IndexerArgs a) {
+  pdl_wait();
+  pdl_launch_dependents();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int cx = blockIdx.y, b = blockIdx.x / a.tiles, tile = blockIdx.x % a.tiles;
   const int hk = blockIdx.z;
@@ -98,27 +100,39 @@ __global__ void __launch_bounds__(kThreads)
 
   if (warp == kConsumerWarps) {
     // ------------------------------------------------------------ producer: TMA page ring
-    if (lane == 0) {
-      prefetch_tmap(&kmap);
-      for (int i = 0; i < npages; ++i) {
-        const int s = i % kStages;
-        if (i >= kStages && !mbar_wait(&empty[s], ((i / kStages) - 1) & 1, abort_flag)) {
-          report(a.dev_err, MSA_DEVERR_TIMEOUT);
-          *abort_flag = 1;
-          break;
+    if (lane == 0) prefetch_tmap(&kmap);
+    bool dead = false;
+    // 32 page ids fetched at a time, one lane each, then issued by lane 0
+    for (int base = 0; base < npages && !dead; base += 32) {
+      const int pg_l = base + lane < npages
+                           ? a.table[static_cast<size_t>(b) * a.max_pages + j0 + base + lane]
+                           : -1;
+      const int cnt = min(32, npages - base);
+      for (int k = 0; k < cnt; ++k) {
+        const int page = __shfl_sync(0xffffffffu, pg_l, k);
+        if (lane == 0) {
+          const int i = base + k;
+          const int s = i % kStages;
+          if (i >= kStages && !mbar_wait(&empty[s], ((i / kStages) - 1) & 1, abort_flag)) {
+            report(a.dev_err, MSA_DEVERR_TIMEOUT);
+            *abort_flag = 1;
+            dead = true;
+          } else {
+            const bool ok = page >= 0 && page < a.num_pages;
+            page_ok[s] = ok;
+            if (ok) {
+              mbar_arrive_expect_tx(&full[s], kTileBytes);
+              const int c2 = page * a.H_idxk + hk;
+              tma_load_3d(stages + s * kTileBytes, &kmap, &full[s], 0, 0, c2);
+              tma_load_3d(stages + s * kTileBytes + kTileBytes / 2, &kmap, &full[s], 64, 0, c2);
+            } else {
+              report(a.dev_err, MSA_DEVERR_PAGE_ID);
+              mbar_arrive(&full[s]);
+            }
+          }
         }
-        const int page = a.table[static_cast<size_t>(b) * a.max_pages + j0 + i];
-        const bool ok = page >= 0 && page < a.num_pages;
-        page_ok[s] = ok;
-        if (ok) {
-          mbar_arrive_expect_tx(&full[s], kTileBytes);
-          const int c2 = page * a.H_idxk + hk;
-          tma_load_3d(stages + s * kTileBytes, &kmap, &full[s], 0, 0, c2);
-          tma_load_3d(stages + s * kTileBytes + kTileBytes / 2, &kmap, &full[s], 64, 0, c2);
-        } else {
-          report(a.dev_err, MSA_DEVERR_PAGE_ID);
-          mbar_arrive(&full[s]);
-        }
+        dead = __shfl_sync(0xffffffffu, dead, 0);
+        if (dead) break;
       }
     }
     return;
@@ -233,11 +247,8 @@ cudaError_t launch_index_scores(const CUtensorMap &kidx_map, const IndexerArgs &
                            : reinterpret_cast<const void *>(&index_scores_kernel<2>);
   cudaError_t e = ensure_smem_limit(fn, static_cast<int>(smem));
   if (e != cudaSuccess) return e;
-  if (mt == 1)
-    index_scores_kernel<1><<<grid, kThreads, smem, s>>>(kidx_map, a);
-  else
-    index_scores_kernel<2><<<grid, kThreads, smem, s>>>(kidx_map, a);
-  return cudaGetLastError();
+  if (mt == 1) return launch_pdl(index_scores_kernel<1>, grid, dim3(kThreads), smem, s, kidx_map, a);
+  return launch_pdl(index_scores_kernel<2>, grid, dim3(kThreads), smem, s, kidx_map, a);
 }
 
 }  // namespace msa

@@ -6,6 +6,8 @@
 #include <stddef.h>
 #include <stdint.h>
 
+#include <utility>
+
 #include "msa.h"
 
 namespace msa {
@@ -64,12 +66,10 @@ struct AttnArgs {
   long long R;  // persistent kernel: work-list slots per CTA
   int P;        // persistent kernel: most CTAs one item's slots can span
   float scale_log2;          // scale * log2(e)
-  float *part_o, *part_lse;  // persistent kernel: [P * PQ][total_q][H_q][128] and [..][H_q]
+  float *part_o, *part_lse;  // persistent kernel: [P][total_q][H_q][128] and [P][total_q][H_q]
   uint16_t *out;             // tile kernel: bf16 bits [total_q, H_q, 128]
   int32_t *dev_err;
 };
-// position splits (consumer warps per 16-row group) of the persistent kernel for rg groups
-int attn_position_splits(int rg);
 // rg = 16-row groups (1..4); plan = read the per-tile union instead of the selection
 cudaError_t launch_attention_stream(const CUtensorMap &kmap, const CUtensorMap &vmap,
                                     const AttnArgs &a, bool fp8, int rg, bool plan, int grid,
@@ -83,5 +83,24 @@ cudaError_t launch_combine(const float *part_o, const float *part_lse, int split
 
 // Sets the dynamic shared-memory limit of `func` once per device.
 cudaError_t ensure_smem_limit(const void *func, int bytes);
+
+// Launch with programmatic stream serialization: the kernel may start while its predecessor
+// in the stream finishes; every kernel of this library calls pdl_wait() before it touches
+// global memory that an earlier kernel may write or read.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                       cudaStream_t stream, Args &&...args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
 
 }  // namespace msa

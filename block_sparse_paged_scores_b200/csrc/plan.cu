@@ -19,6 +19,8 @@ namespace {
 
 __global__ void __launch_bounds__(32) plan_kernel(const PlanArgs a) {
   extern __shared__ uint32_t psm[];
+  pdl_wait();
+  pdl_launch_dependents();
   const int lane = threadIdx.x;
   const int g = blockIdx.y, y = blockIdx.x;
   const int b = y / a.tiles, tile = y % a.tiles;
@@ -124,8 +126,7 @@ cudaError_t launch_plan(const PlanArgs &a, cudaStream_t s) {
                                     static_cast<int>(smem));
   if (e != cudaSuccess) return e;
   const dim3 grid(a.batch * a.tiles, a.H_kv);
-  plan_kernel<<<grid, 32, smem, s>>>(a);
-  return cudaGetLastError();
+  return launch_pdl(plan_kernel, grid, dim3(32), smem, s, a);
 }
 
 }  // namespace msa

@@ -69,6 +69,8 @@ struct Keys {
 
 template <int KPL>
 __global__ void __launch_bounds__(32 * kWarps) select_kernel(const SelectArgs a) {
+  pdl_wait();
+  pdl_launch_dependents();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const long long item = static_cast<long long>(blockIdx.x) * kWarps + warp;
   if (item >= static_cast<long long>(a.total_q) * a.H_kv) return;
@@ -155,15 +157,11 @@ __global__ void __launch_bounds__(32 * kWarps) select_kernel(const SelectArgs a)
 cudaError_t launch_select(const SelectArgs &a, cudaStream_t s) {
   const long long items = static_cast<long long>(a.total_q) * a.H_kv;
   const unsigned blocks = static_cast<unsigned>((items + kWarps - 1) / kWarps);
-  if (a.max_blocks <= 4 * 32)
-    select_kernel<4><<<blocks, 32 * kWarps, 0, s>>>(a);
-  else if (a.max_blocks <= 16 * 32)
-    select_kernel<16><<<blocks, 32 * kWarps, 0, s>>>(a);
-  else if (a.max_blocks <= 32 * 32)
-    select_kernel<32><<<blocks, 32 * kWarps, 0, s>>>(a);
-  else
-    select_kernel<0><<<blocks, 32 * kWarps, 0, s>>>(a);
-  return cudaGetLastError();
+  const dim3 grid(blocks), block(32 * kWarps);
+  if (a.max_blocks <= 4 * 32) return launch_pdl(select_kernel<4>, grid, block, 0, s, a);
+  if (a.max_blocks <= 16 * 32) return launch_pdl(select_kernel<16>, grid, block, 0, s, a);
+  if (a.max_blocks <= 32 * 32) return launch_pdl(select_kernel<32>, grid, block, 0, s, a);
+  return launch_pdl(select_kernel<0>, grid, block, 0, s, a);
 }
 
 }  // namespace msa

@@ -78,18 +78,22 @@ def _rp(batch=2, total_q=2, max_q_len=1, max_pages=16, num_pages=64):
 def test_workspace_bytes(lib):
     rows = 4 * 64
     rp = _rp(batch=4, total_q=4, max_q_len=1)
-    # one partition covering all 4 x 8 items of 19 slots: one piece each, 4 position splits
+    # one partition covering all 4 x 8 items of 19 slots: one piece per row
     ws1 = msa.msa_attn_workspace_bytes(rp, 19, 64, 8, 16, 1)
-    assert ws1 >= 4 * rows * 128 * 4 + 4 * rows * 4
+    assert ws1 >= rows * 128 * 4 + rows * 4
+    assert msa.msa_attn_partials(rp, 19, 64, 8, 16, 1)[0] == 1
     # three partitions: some item straddles two of them -> two pieces
     ws3 = msa.msa_attn_workspace_bytes(rp, 19, 64, 8, 16, 3)
-    assert ws3 >= 8 * rows * 128 * 4 + 8 * rows * 4
+    assert ws3 >= 2 * rows * 128 * 4 + 2 * rows * 4
+    n, o_off, l_off = msa.msa_attn_partials(rp, 19, 64, 8, 16, 3)
+    assert n == 2 and o_off == 0 and l_off >= 2 * rows * 128 * 4
     rp = _rp(batch=2, total_q=8, max_q_len=4)
     ws = msa.msa_attn_workspace_bytes(rp, 35, 64, 8, 16, 1)              # speculative: + plan
-    assert ws >= 4 * 8 * 64 * 128 * 4 + 2 * 8 * 16 * 8
+    assert ws >= 8 * 64 * 128 * 4 + 2 * 8 * 16 * 8
     rp = _rp(batch=2, total_q=600, max_q_len=300)
     ws = msa.msa_attn_workspace_bytes(rp, 35, 64, 8, 16, 0)              # prefill: plan only
     assert 0 < ws < 600 * 64 * 128 * 4
+    assert msa.msa_attn_partials(rp, 35, 64, 8, 16, 0)[0] == 0           # writes out directly
     assert msa.msa_attn_workspace_bytes(rp, 0, 64, 8, 16, 1) == 0        # invalid -> 0
     assert msa.msa_attn_workspace_bytes(rp, 35, 63, 8, 16, 1) == 0
 

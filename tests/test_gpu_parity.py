@@ -141,12 +141,15 @@ def test_partials_then_public_combine_equal_the_fused_call(name):
     assert torch.equal(split.out, fused.out)
 
 
-def test_splitk_combine_entry_point():
+@pytest.mark.parametrize("ns", [1, 5, 40, 77])
+def test_splitk_combine_entry_point(ns):
     torch.manual_seed(0)
-    ns, tq, hq = 5, 7, 12
+    tq, hq = 7, 12
     o = torch.randn(ns, tq, hq, 128, device="cuda")
     lse = torch.randn(ns, tq, hq, device="cuda") * 3
-    lse[1] = -float("inf")                      # an empty partition weighs nothing
+    lse[ns // 2] = -float("inf")                # an empty partition weighs nothing
+    if ns > 33:
+        lse[33, 2, 5] = 60.0                    # a later chunk holds the largest weight
     lse[:, 3, 4] = -float("inf")                # a row no partition saw -> 0
     out = torch.empty(tq, hq, 128, dtype=torch.bfloat16, device="cuda")
     msa.msa_splitk_combine(o, lse, ns, tq, hq, out)
@@ -156,6 +159,8 @@ def test_splitk_combine_entry_point():
     got = out.double()
     assert torch.allclose(got, ref, atol=1e-2, rtol=1e-2)
     assert float(got[3, 4].abs().max()) == 0.0
+    if ns == 1:
+        assert float((got[:3] - o[0, :3].double()).abs().max()) < 1e-2
 
 
 def test_all_equal_scores_pick_the_lowest_ids():
