@@ -180,7 +180,6 @@ __global__ void __launch_bounds__(32 * (stream_consumer_warps<RG>() + 1))
     *abort_flag = 0;
     fence_mbar_init();
   }
-  for (int i = threadIdx.x; i < RG * 16 * kHeadDim; i += blockDim.x) acc[i] = 0.f;
   __syncthreads();
   pdl_wait();  // block ids, selection counts and the plan come from earlier kernels
   pdl_launch_dependents();
@@ -371,6 +370,7 @@ __global__ void __launch_bounds__(32 * (stream_consumer_warps<RG>() + 1))
         }
       }
       named_bar_sync(1, nct);
+      float fac[2];
 #pragma unroll
       for (int slot = 0; slot < 2; ++slot) {
         const int r16 = (lane >> 2) + slot * 8;
@@ -391,49 +391,67 @@ __global__ void __launch_bounds__(32 * (stream_consumer_warps<RG>() + 1))
               if (mw != -INFINITY) Ls += mrg_l[w2 * 16 + r16] * fast_exp2(mw - M);
             }
         }
-        if (wa.m_run[slot] != -INFINITY) {
-          const float f = fast_exp2(wa.m_run[slot] - M);
-          float *dst = acc + (rg * 16 + r16) * kHeadDim;
-          const int c4 = lane & 3;
-          if (FP8) {
-#pragma unroll
-            for (int ch = 0; ch < 8; ++ch) {
-              red_add_shared(dst + ch * 16 + 4 * c4 + 0, wa.o[2 * ch][2 * slot] * f);
-              red_add_shared(dst + ch * 16 + 4 * c4 + 1, wa.o[2 * ch + 1][2 * slot] * f);
-              red_add_shared(dst + ch * 16 + 4 * c4 + 2, wa.o[2 * ch][2 * slot + 1] * f);
-              red_add_shared(dst + ch * 16 + 4 * c4 + 3, wa.o[2 * ch + 1][2 * slot + 1] * f);
-            }
-          } else {
-#pragma unroll
-            for (int nn = 0; nn < 16; ++nn) {
-              red_add_shared(dst + nn * 8 + 2 * c4, wa.o[nn][2 * slot] * f);
-              red_add_shared(dst + nn * 8 + 2 * c4 + 1, wa.o[nn][2 * slot + 1] * f);
-            }
-          }
-        }
+        fac[slot] = wa.m_run[slot] == -INFINITY ? 0.f : fast_exp2(wa.m_run[slot] - M);
         if (row_owner) {
           row_m[rg * 16 + r16] = M;
           row_l[rg * 16 + r16] = Ls;
         }
       }
-      named_bar_sync(1, nct);
-      // ---- write this segment's partial (all consumer threads), clear the accumulator
+      // fixed-order accumulation (reproducible sums): in round k the warp of each row group
+      // whose rank in the group is k adds its rescaled output; round 0 stores.
+      const int rank = team * PQ + pq;
+      for (int k = 0; k < NT * PQ; ++k) {
+        if (rank == k) {
+#pragma unroll
+          for (int slot = 0; slot < 2; ++slot) {
+            float *dst = acc + (rg * 16 + (lane >> 2) + slot * 8) * kHeadDim;
+            const int c4 = lane & 3;
+            const float f = fac[slot];
+            if (FP8) {
+#pragma unroll
+              for (int ch = 0; ch < 8; ++ch) {
+                float4 *d = reinterpret_cast<float4 *>(dst + ch * 16 + 4 * c4);
+                const float4 v = make_float4(wa.o[2 * ch][2 * slot] * f, wa.o[2 * ch + 1][2 * slot] * f,
+                                             wa.o[2 * ch][2 * slot + 1] * f,
+                                             wa.o[2 * ch + 1][2 * slot + 1] * f);
+                if (k == 0) {
+                  *d = v;
+                } else {
+                  const float4 u = *d;
+                  *d = make_float4(u.x + v.x, u.y + v.y, u.z + v.z, u.w + v.w);
+                }
+              }
+            } else {
+#pragma unroll
+              for (int nn = 0; nn < 16; ++nn) {
+                float2 *d = reinterpret_cast<float2 *>(dst + nn * 8 + 2 * c4);
+                const float2 v = make_float2(wa.o[nn][2 * slot] * f, wa.o[nn][2 * slot + 1] * f);
+                if (k == 0) {
+                  *d = v;
+                } else {
+                  const float2 u = *d;
+                  *d = make_float2(u.x + v.x, u.y + v.y);
+                }
+              }
+            }
+          }
+        }
+        named_bar_sync(1, nct);
+      }
+      // ---- write this segment's partial (all consumer threads)
       const int ctid = threadIdx.x;  // consumers are threads [0, nct)
       for (int idx = ctid; idx < RG * 16 * (kHeadDim / 4); idx += nct) {
         const int r = idx / (kHeadDim / 4), d4 = idx % (kHeadDim / 4);
-        float4 *src = reinterpret_cast<float4 *>(acc + r * kHeadDim) + d4;
-        if (r < m.rows) {
-          const int tl = r / a.G;
-          const size_t orr = static_cast<size_t>(m.t0 + tl) * a.H_q + m.g * a.G + r % a.G;
-          const size_t pr = static_cast<size_t>(piece) * split_stride + orr;
-          const float L = row_l[r];
-          const float inv = L > 0.f ? 1.f / L : 0.f;
-          const float4 v = *src;
-          reinterpret_cast<float4 *>(a.part_o + pr * kHeadDim)[d4] =
-              make_float4(v.x * inv, v.y * inv, v.z * inv, v.w * inv);
-          if (d4 == 0) a.part_lse[pr] = L > 0.f ? (row_m[r] + __log2f(L)) * kLn2 : -INFINITY;
-        }
-        *src = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (r >= m.rows) continue;
+        const int tl = r / a.G;
+        const size_t orr = static_cast<size_t>(m.t0 + tl) * a.H_q + m.g * a.G + r % a.G;
+        const size_t pr = static_cast<size_t>(piece) * split_stride + orr;
+        const float L = row_l[r];
+        const float inv = L > 0.f ? 1.f / L : 0.f;
+        const float4 v = reinterpret_cast<const float4 *>(acc + r * kHeadDim)[d4];
+        reinterpret_cast<float4 *>(a.part_o + pr * kHeadDim)[d4] =
+            make_float4(v.x * inv, v.y * inv, v.z * inv, v.w * inv);
+        if (d4 == 0) a.part_lse[pr] = L > 0.f ? (row_m[r] + __log2f(L)) * kLn2 : -INFINITY;
       }
     } else if (row_owner) {
       // a range that meets this item only in slots past its count: an empty partial
