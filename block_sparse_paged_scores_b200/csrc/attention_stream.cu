@@ -34,12 +34,6 @@ namespace msa {
 
 namespace {
 
-template <bool FP8>
-struct StreamCfg {
-  static constexpr uint32_t kTile = KvTile<FP8>::kBytes;
-  static constexpr int kSlots = FP8 ? 10 : 5;  // 160 KiB of tiles in flight per SM
-};
-
 // Consumer layout for RG 16-row groups: PQ warps split every block's positions and NT teams
 // of RG * PQ warps take alternate blocks, so that every SM sub-partition runs two
 // independent block chains when the rows fit one group.
@@ -56,12 +50,23 @@ constexpr int stream_consumer_warps() {
   return RG * stream_pq<RG>() * stream_teams<RG>();
 }
 
+// Every team has a ring of its own (a team consumes its ring strictly in order, which is what
+// makes the phase-parity waits exact): 160 KiB of tiles per SM with one team, 128 KiB (BF16)
+// or 160 KiB (FP8) with two.
+template <bool FP8, int RG>
+struct StreamCfg {
+  static constexpr uint32_t kTile = KvTile<FP8>::kBytes;
+  static constexpr int kTeams = stream_teams<RG>();
+  static constexpr int kRing = kTeams == 2 ? (FP8 ? 5 : 2) : (FP8 ? 10 : 5);  // slots per team
+  static constexpr int kSlots = kTeams * kRing;
+};
+
 template <bool FP8, int RG>
 constexpr size_t stream_smem_bytes() {
-  return 1024 + StreamCfg<FP8>::kSlots * StreamCfg<FP8>::kTile + 2 * kQBuf +
+  using C = StreamCfg<FP8, RG>;
+  return 1024 + C::kSlots * C::kTile + 2 * kQBuf +
          RG * 16 * kHeadDim * sizeof(float) +                        // merge accumulator
-         (2 * StreamCfg<FP8>::kSlots + 4) * sizeof(uint64_t) +
-         StreamCfg<FP8>::kSlots * 3 * sizeof(int) +
+         (2 * C::kSlots + 4) * sizeof(uint64_t) + C::kSlots * 3 * sizeof(int) +
          2 * stream_consumer_warps<RG>() * 16 * sizeof(float) +       // per-warp m, l
          2 * RG * 16 * sizeof(float) + 16;                           // per-row M, L
 }
@@ -137,8 +142,9 @@ __global__ void __launch_bounds__(32 * (stream_consumer_warps<RG>() + 1))
   constexpr int NT = stream_teams<RG>();
   constexpr int TEAM = RG * PQ;                    // warps of one team
   constexpr int NCW = stream_consumer_warps<RG>();  // all consumer warps
-  constexpr int NSLOT = StreamCfg<FP8>::kSlots;
-  constexpr uint32_t TILE = StreamCfg<FP8>::kTile;
+  constexpr int NSLOT = StreamCfg<FP8, RG>::kSlots;  // all rings
+  constexpr int NR = StreamCfg<FP8, RG>::kRing;      // slots of one team's ring
+  constexpr uint32_t TILE = StreamCfg<FP8, RG>::kTile;
   using WA = WarpAttn<FP8, PQ>;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -191,7 +197,8 @@ __global__ void __launch_bounds__(32 * (stream_consumer_warps<RG>() + 1))
       prefetch_tmap(&vmap);
     }
     bool dead = false;
-    uint32_t nload = 0;  // tile loads issued (two per block: K then V)
+    // tile loads issued into each team's ring (two per block: K then V)
+    uint32_t nload0 = 0, nload1 = 0;
     int n = 0;           // index of the current non-empty segment
     // first non-empty segment
     int it = it_first, v0 = 0, v1 = 0;
@@ -229,11 +236,13 @@ __global__ void __launch_bounds__(32 * (stream_consumer_warps<RG>() + 1))
             const bool ok = jok && pg >= 0 && pg < a.num_pages;
             if (!ok) report(a.dev_err, jok ? MSA_DEVERR_PAGE_ID : MSA_DEVERR_BLOCK_ID);
             const int c2 = pg * a.H_kv + cur.g;
+            const int tm = (base + i - v0) % NT;  // the team that reads this block
 #pragma unroll
             for (int kv = 0; kv < 2; ++kv) {
-              const int s = static_cast<int>(nload % NSLOT);
-              if (nload >= static_cast<uint32_t>(NSLOT) &&
-                  !mbar_wait(&sempty[s], ((nload / NSLOT) - 1) & 1, abort_flag)) {
+              const uint32_t nl = tm ? nload1 : nload0;
+              const int s = tm * NR + static_cast<int>(nl % NR);
+              if (nl >= static_cast<uint32_t>(NR) &&
+                  !mbar_wait(&sempty[s], ((nl / NR) - 1) & 1, abort_flag)) {
                 report(a.dev_err, MSA_DEVERR_TIMEOUT);
                 *abort_flag = 1;
                 dead = true;
@@ -251,7 +260,10 @@ __global__ void __launch_bounds__(32 * (stream_consumer_warps<RG>() + 1))
               } else {
                 mbar_arrive(&sfull[s]);
               }
-              ++nload;
+              if (tm)
+                nload1 = nl + 1;
+              else
+                nload0 = nl + 1;
             }
           }
           dead = __shfl_sync(0xffffffffu, dead, 0);
@@ -299,7 +311,7 @@ __global__ void __launch_bounds__(32 * (stream_consumer_warps<RG>() + 1))
   const bool row_owner = team == 0 && pq == 0 && (lane & 3) == 0;  // one writer per row
   const int nct = 32 * NCW;
   WA wa;
-  uint32_t nload = 0;
+  uint32_t nload = 0;  // loads this warp's team has consumed from its ring
   int n = 0;
   for (int it = it_first; it <= it_last; ++it) {
     const Item m = load_item<PLAN>(a, it, false);
@@ -335,9 +347,9 @@ __global__ void __launch_bounds__(32 * (stream_consumer_warps<RG>() + 1))
       const uint32_t qs_addr = smem_u32(qbufs + buf * kQBuf);
       wa.reset();
       for (int e = v0 + team; e < v1; e += NT) {
-        const uint32_t nk = nload + 2u * static_cast<uint32_t>(e - v0);  // K tile; V is nk + 1
-        int s = static_cast<int>(nk % NSLOT);
-        bool live = mbar_wait(&sfull[s], (nk / NSLOT) & 1, abort_flag);
+        const uint32_t nk = nload;  // this team's K tile; V is nk + 1
+        int s = team * NR + static_cast<int>(nk % NR);
+        bool live = mbar_wait(&sfull[s], (nk / NR) & 1, abort_flag);
         const bool ok = live && qlive && slot_ok[s];
         const int j = slot_j[s];
         const uint32_t msk = slot_mask[s];
@@ -345,17 +357,17 @@ __global__ void __launch_bounds__(32 * (stream_consumer_warps<RG>() + 1))
         __syncwarp();
         if (lane == 0) mbar_arrive(&sempty[s]);
         if (ok) wa.softmax(j, pq, lane, prow, tbit, msk, a.scale_log2);
-        s = static_cast<int>((nk + 1) % NSLOT);
-        live = mbar_wait(&sfull[s], ((nk + 1) / NSLOT) & 1, abort_flag) && live;
+        s = team * NR + static_cast<int>((nk + 1) % NR);
+        live = mbar_wait(&sfull[s], ((nk + 1) / NR) & 1, abort_flag) && live;
         if (ok && live) wa.pv(smem_u32(slots + s * TILE), j, pq, lane, m.L);
         __syncwarp();
         if (lane == 0) mbar_arrive(&sempty[s]);
+        nload = nk + 2;
         if (!live) {
           report(a.dev_err, MSA_DEVERR_TIMEOUT);
           *abort_flag = 1;
         }
       }
-      nload += 2u * static_cast<uint32_t>(v1 - v0);
       __syncwarp();
       if (lane == 0) mbar_arrive(&qempty[buf]);
       ++n;
