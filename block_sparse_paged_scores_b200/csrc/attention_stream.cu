@@ -35,29 +35,29 @@ namespace msa {
 namespace {
 
 // Consumer layout for RG 16-row groups: PQ warps split every block's positions and NT teams
-// of RG * PQ warps take alternate blocks, so that every SM sub-partition runs two
-// independent block chains when the rows fit one group.
-template <int RG>
+// of RG * PQ warps take alternate blocks.  With a single row group every SM sub-partition
+// gets two warps: BF16 splits each block eight ways; FP8 (whose K fragments come four n-tiles
+// at a time) runs two teams of four.
+template <bool FP8, int RG>
 constexpr int stream_pq() {
-  return RG <= 2 ? 4 : 2;
+  return RG == 1 ? (FP8 ? 4 : 8) : (RG == 2 ? 4 : 2);
 }
-template <int RG>
+template <bool FP8, int RG>
 constexpr int stream_teams() {
-  return RG == 1 ? 2 : 1;
+  return RG == 1 && FP8 ? 2 : 1;
 }
-template <int RG>
+template <bool FP8, int RG>
 constexpr int stream_consumer_warps() {
-  return RG * stream_pq<RG>() * stream_teams<RG>();
+  return RG * stream_pq<FP8, RG>() * stream_teams<FP8, RG>();
 }
 
 // Every team has a ring of its own (a team consumes its ring strictly in order, which is what
-// makes the phase-parity waits exact): 160 KiB of tiles per SM with one team, 128 KiB (BF16)
-// or 160 KiB (FP8) with two.
+// makes the phase-parity waits exact): 160 KiB of tiles per SM.
 template <bool FP8, int RG>
 struct StreamCfg {
   static constexpr uint32_t kTile = KvTile<FP8>::kBytes;
-  static constexpr int kTeams = stream_teams<RG>();
-  static constexpr int kRing = kTeams == 2 ? (FP8 ? 5 : 2) : (FP8 ? 10 : 5);  // slots per team
+  static constexpr int kTeams = stream_teams<FP8, RG>();
+  static constexpr int kRing = (FP8 ? 10 : 5) / kTeams;  // slots per team
   static constexpr int kSlots = kTeams * kRing;
 };
 
@@ -67,7 +67,7 @@ constexpr size_t stream_smem_bytes() {
   return 1024 + C::kSlots * C::kTile + 2 * kQBuf +
          RG * 16 * kHeadDim * sizeof(float) +                        // merge accumulator
          (2 * C::kSlots + 4) * sizeof(uint64_t) + C::kSlots * 3 * sizeof(int) +
-         2 * stream_consumer_warps<RG>() * 16 * sizeof(float) +       // per-warp m, l
+         2 * stream_consumer_warps<FP8, RG>() * 16 * sizeof(float) +       // per-warp m, l
          2 * RG * 16 * sizeof(float) + 16;                           // per-row M, L
 }
 
@@ -135,13 +135,13 @@ __device__ __forceinline__ void segment(const AttnArgs &a, int it, long long r0,
 }
 
 template <bool FP8, int RG, bool PLAN>
-__global__ void __launch_bounds__(32 * (stream_consumer_warps<RG>() + 1))
+__global__ void __launch_bounds__(32 * (stream_consumer_warps<FP8, RG>() + 1))
     attn_stream_kernel(const __grid_constant__ CUtensorMap kmap,
                        const __grid_constant__ CUtensorMap vmap, const AttnArgs a) {
-  constexpr int PQ = stream_pq<RG>();
-  constexpr int NT = stream_teams<RG>();
+  constexpr int PQ = stream_pq<FP8, RG>();
+  constexpr int NT = stream_teams<FP8, RG>();
   constexpr int TEAM = RG * PQ;                    // warps of one team
-  constexpr int NCW = stream_consumer_warps<RG>();  // all consumer warps
+  constexpr int NCW = stream_consumer_warps<FP8, RG>();  // all consumer warps
   constexpr int NSLOT = StreamCfg<FP8, RG>::kSlots;  // all rings
   constexpr int NR = StreamCfg<FP8, RG>::kRing;      // slots of one team's ring
   constexpr uint32_t TILE = StreamCfg<FP8, RG>::kTile;
@@ -489,7 +489,7 @@ cudaError_t launch_stream_one(const CUtensorMap &kmap, const CUtensorMap &vmap,
   auto fn = &attn_stream_kernel<FP8, RG, PLAN>;
   cudaError_t e = ensure_smem_limit(reinterpret_cast<const void *>(fn), static_cast<int>(smem));
   if (e != cudaSuccess) return e;
-  return launch_pdl(fn, dim3(grid), dim3(32 * (stream_consumer_warps<RG>() + 1)), smem, s,
+  return launch_pdl(fn, dim3(grid), dim3(32 * (stream_consumer_warps<FP8, RG>() + 1)), smem, s,
                     kmap, vmap, a);
 }
 
