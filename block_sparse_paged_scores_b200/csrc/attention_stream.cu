@@ -415,38 +415,8 @@ __global__ void __launch_bounds__(32 * (stream_consumer_warps<FP8, RG>() + 1))
       for (int k = 0; k < NT * PQ; ++k) {
         if (rank == k) {
 #pragma unroll
-          for (int slot = 0; slot < 2; ++slot) {
-            float *dst = acc + (rg * 16 + (lane >> 2) + slot * 8) * kHeadDim;
-            const int c4 = lane & 3;
-            const float f = fac[slot];
-            if (FP8) {
-#pragma unroll
-              for (int ch = 0; ch < 8; ++ch) {
-                float4 *d = reinterpret_cast<float4 *>(dst + ch * 16 + 4 * c4);
-                const float4 v = make_float4(wa.o[2 * ch][2 * slot] * f, wa.o[2 * ch + 1][2 * slot] * f,
-                                             wa.o[2 * ch][2 * slot + 1] * f,
-                                             wa.o[2 * ch + 1][2 * slot + 1] * f);
-                if (k == 0) {
-                  *d = v;
-                } else {
-                  const float4 u = *d;
-                  *d = make_float4(u.x + v.x, u.y + v.y, u.z + v.z, u.w + v.w);
-                }
-              }
-            } else {
-#pragma unroll
-              for (int nn = 0; nn < 16; ++nn) {
-                float2 *d = reinterpret_cast<float2 *>(dst + nn * 8 + 2 * c4);
-                const float2 v = make_float2(wa.o[nn][2 * slot] * f, wa.o[nn][2 * slot + 1] * f);
-                if (k == 0) {
-                  *d = v;
-                } else {
-                  const float2 u = *d;
-                  *d = make_float2(u.x + v.x, u.y + v.y);
-                }
-              }
-            }
-          }
+          for (int slot = 0; slot < 2; ++slot)
+            wa.store_row(acc, rg * 16 + (lane >> 2) + slot * 8, slot, fac[slot], lane, k > 0);
         }
         named_bar_sync(1, nct);
       }
@@ -460,7 +430,8 @@ __global__ void __launch_bounds__(32 * (stream_consumer_warps<FP8, RG>() + 1))
         const size_t pr = static_cast<size_t>(piece) * split_stride + orr;
         const float L = row_l[r];
         const float inv = L > 0.f ? 1.f / L : 0.f;
-        const float4 v = reinterpret_cast<const float4 *>(acc + r * kHeadDim)[d4];
+        const float4 v =
+            *reinterpret_cast<const float4 *>(acc + r * kHeadDim + acc_col(r, 4 * d4));
         reinterpret_cast<float4 *>(a.part_o + pr * kHeadDim)[d4] =
             make_float4(v.x * inv, v.y * inv, v.z * inv, v.w * inv);
         if (d4 == 0) a.part_lse[pr] = L > 0.f ? (row_m[r] + __log2f(L)) * kLn2 : -INFINITY;

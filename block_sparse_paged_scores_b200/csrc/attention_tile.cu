@@ -235,7 +235,7 @@ __global__ void __launch_bounds__(32 * (RG * tile_pq<RG>() + 1))
     }
     const float f =
         (Ls > 0.f && wa.m_run[slot] != -INFINITY) ? fast_exp2(wa.m_run[slot] - M) / Ls : 0.f;
-    wa.store_row(mo + (static_cast<size_t>(warp) * 16 + r16) * kHeadDim, slot, f, lane);
+    wa.store_row(mo + static_cast<size_t>(warp) * 16 * kHeadDim, r16, slot, f, lane, false);
   }
   named_bar_sync(1, NCT);
   for (int idx = threadIdx.x; idx < RG * 16 * (kHeadDim / 4); idx += NCT) {
@@ -245,8 +245,8 @@ __global__ void __launch_bounds__(32 * (RG * tile_pq<RG>() + 1))
     float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
     for (int w = 0; w < PQ; ++w) {
-      const float4 v = reinterpret_cast<const float4 *>(
-          mo + (static_cast<size_t>(rgr * PQ + w) * 16 + r16) * kHeadDim)[d4];
+      const float4 v = *reinterpret_cast<const float4 *>(
+          mo + (static_cast<size_t>(rgr * PQ + w) * 16 + r16) * kHeadDim + acc_col(r16, 4 * d4));
       acc.x += v.x;
       acc.y += v.y;
       acc.z += v.z;

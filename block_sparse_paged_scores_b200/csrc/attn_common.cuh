@@ -70,6 +70,10 @@ __device__ __forceinline__ void stage_q(uint8_t *qs, const uint16_t *q, int t0, 
   }
 }
 
+// Column of dim `col` in row `row` of a [rows][128] fp32 merge buffer: 32-byte chunks are
+// XOR-ed with row % 8, so that the 8 rows a warp's lanes hold fall in different banks.
+__device__ __forceinline__ int acc_col(int row, int col) { return col ^ ((row & 7) << 3); }
+
 template <bool FP8, int PQ>
 struct WarpAttn {
   static constexpr int PW = kBlock / PQ;  // positions per warp
@@ -249,21 +253,36 @@ struct WarpAttn {
     }
   }
 
-  // This thread's part of row slot `slot` times f, as fp32, into dst (one 128-dim row); the
-  // FP8 path's dim permutation is undone here.
-  __device__ __forceinline__ void store_row(float *dst, int slot, float f, int lane) const {
+  // This thread's part of row slot `slot` times f, as fp32, into row `row` of a [rows][128]
+  // fp32 buffer laid out by acc_col (the FP8 path's dim permutation is undone here).  With
+  // `add` the values are added to what the buffer holds.
+  __device__ __forceinline__ void store_row(float *buf, int row, int slot, float f, int lane,
+                                            bool add) const {
     const int c4 = lane & 3;
+    float *dst = buf + row * kHeadDim;
     if (FP8) {
 #pragma unroll
-      for (int ch = 0; ch < 8; ++ch)
-        *reinterpret_cast<float4 *>(dst + ch * 16 + 4 * c4) =
-            make_float4(o[2 * ch][2 * slot] * f, o[2 * ch + 1][2 * slot] * f,
-                        o[2 * ch][2 * slot + 1] * f, o[2 * ch + 1][2 * slot + 1] * f);
+      for (int ch = 0; ch < 8; ++ch) {
+        float4 *d = reinterpret_cast<float4 *>(dst + acc_col(row, ch * 16 + 4 * c4));
+        float4 v = make_float4(o[2 * ch][2 * slot] * f, o[2 * ch + 1][2 * slot] * f,
+                               o[2 * ch][2 * slot + 1] * f, o[2 * ch + 1][2 * slot + 1] * f);
+        if (add) {
+          const float4 u = *d;
+          v = make_float4(u.x + v.x, u.y + v.y, u.z + v.z, u.w + v.w);
+        }
+        *d = v;
+      }
     } else {
 #pragma unroll
-      for (int n = 0; n < 16; ++n)
-        *reinterpret_cast<float2 *>(dst + n * 8 + 2 * c4) =
-            make_float2(o[n][2 * slot] * f, o[n][2 * slot + 1] * f);
+      for (int n = 0; n < 16; ++n) {
+        float2 *d = reinterpret_cast<float2 *>(dst + acc_col(row, n * 8 + 2 * c4));
+        float2 v = make_float2(o[n][2 * slot] * f, o[n][2 * slot + 1] * f);
+        if (add) {
+          const float2 u = *d;
+          v = make_float2(u.x + v.x, u.y + v.y);
+        }
+        *d = v;
+      }
     }
   }
 };
