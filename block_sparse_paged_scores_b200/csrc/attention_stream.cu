@@ -16,16 +16,17 @@
 // to end are cut into equal contiguous ranges of R slots, one per CTA (a split-K partition):
 // every SM streams the same number of slots.  A CTA's range meets a few items; each meeting is
 // a "segment", merged inside the CTA into one partial (normalised output and log-sum-exp) at
-// split index `piece` = the CTA's rank among the CTAs that share the item.
-// msa_splitk_combine's kernel merges the pieces.
+// split index `piece` = the CTA's rank among the CTAs that share the item; split indices no
+// CTA fills are marked empty.  msa_splitk_combine's kernel merges the pieces.
 //
-// Roles: one producer warp loads each segment's Q rows into a double-buffered Q slot and
-// issues the TMA loads of the K and V page tiles (128-byte swizzle) into a ring of tile slots,
-// running ahead across segment boundaries.  Consumer warps run the per-block math of
-// attn_common.cuh (each owns 16 rows and a share of every block's positions; with one row
-// group, two teams take alternate blocks), release the K slot after QK^T and the V slot after
-// PV, and at the end of a segment fold their online-softmax states into one per row through
-// shared memory.
+// Roles: one producer warp walks the items, marks empty partials, loads each non-empty
+// segment's Q rows and metadata into a double-buffered Q slot and issues the TMA loads of the
+// K and V page tiles (128-byte swizzle) into the consumers' rings, running ahead across
+// segment boundaries.  Consumer warps touch no global memory but their partials: they run the
+// per-block math of attn_common.cuh (each owns 16 rows and a share of every block's positions;
+// FP8 with one row group splits into two teams taking alternate blocks), release the K slot
+// after QK^T and the V slot after PV, and at the end of a segment fold their online-softmax
+// states pairwise into one per row through shared memory.
 #include <math.h>
 
 #include "attn_common.cuh"
@@ -52,23 +53,36 @@ constexpr int stream_consumer_warps() {
 }
 
 // Every team has a ring of its own (a team consumes its ring strictly in order, which is what
-// makes the phase-parity waits exact): 160 KiB of tiles per SM.
+// makes the phase-parity waits exact): 160 KiB of tiles per SM (128 KiB with four row groups,
+// whose Q buffers and merge slices take the rest of the shared memory).
 template <bool FP8, int RG>
 struct StreamCfg {
   static constexpr uint32_t kTile = KvTile<FP8>::kBytes;
   static constexpr int kTeams = stream_teams<FP8, RG>();
-  static constexpr int kRing = (FP8 ? 10 : 5) / kTeams;  // slots per team
+  static constexpr int kRing = (RG == 4 ? (FP8 ? 8 : 4) : (FP8 ? 10 : 5)) / kTeams;
   static constexpr int kSlots = kTeams * kRing;
 };
+
+// What the producer hands the consumers with each non-empty segment's Q rows.
+struct SegMeta {
+  int valid;  // 0: no segment left
+  int t0, rows, cl, tok0, g, L, v0, v1, piece;
+};
+
+// one warp's 16 rows (padded stride), then their m and l
+template <bool FP8>
+constexpr int slice_floats() {
+  return 16 * MergeRow<FP8>::kStride + 32;
+}
 
 template <bool FP8, int RG>
 constexpr size_t stream_smem_bytes() {
   using C = StreamCfg<FP8, RG>;
-  return 1024 + C::kSlots * C::kTile + 2 * kQBuf +
-         RG * 16 * kHeadDim * sizeof(float) +                        // merge accumulator
+  constexpr int W = stream_pq<FP8, RG>() * stream_teams<FP8, RG>();  // warps per row group
+  return 1024 + C::kSlots * C::kTile + 2 * (RG * 16 * 256) +            // tiles, 2 Q buffers
+         RG * (W / 2) * slice_floats<FP8>() * sizeof(float) +           // merge slices
          (2 * C::kSlots + 4) * sizeof(uint64_t) + C::kSlots * 3 * sizeof(int) +
-         2 * stream_consumer_warps<FP8, RG>() * 16 * sizeof(float) +       // per-warp m, l
-         2 * RG * 16 * sizeof(float) + 16;                           // per-row M, L
+         2 * sizeof(SegMeta) + 16;
 }
 
 struct Item {
@@ -140,12 +154,17 @@ __global__ void __launch_bounds__(32 * (stream_consumer_warps<FP8, RG>() + 1))
                        const __grid_constant__ CUtensorMap vmap, const AttnArgs a) {
   constexpr int PQ = stream_pq<FP8, RG>();
   constexpr int NT = stream_teams<FP8, RG>();
-  constexpr int TEAM = RG * PQ;                    // warps of one team
-  constexpr int NCW = stream_consumer_warps<FP8, RG>();  // all consumer warps
-  constexpr int NSLOT = StreamCfg<FP8, RG>::kSlots;  // all rings
-  constexpr int NR = StreamCfg<FP8, RG>::kRing;      // slots of one team's ring
+  constexpr int TEAM = RG * PQ;                           // warps of one team
+  constexpr int W = NT * PQ;                              // warps sharing a row group
+  constexpr int NCW = stream_consumer_warps<FP8, RG>();   // all consumer warps
+  constexpr int NSLOT = StreamCfg<FP8, RG>::kSlots;       // all rings
+  constexpr int NR = StreamCfg<FP8, RG>::kRing;           // slots of one team's ring
   constexpr uint32_t TILE = StreamCfg<FP8, RG>::kTile;
+  constexpr int QR = RG * 16;                             // rows of a Q buffer
+  constexpr uint32_t QSUB = QR * 128, QBUF = 2 * QSUB;
   using WA = WarpAttn<FP8, PQ>;
+  constexpr int SLICE = slice_floats<FP8>();
+  constexpr int MS = MergeRow<FP8>::kStride;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const long long total = static_cast<long long>(a.items) * a.cap;
@@ -154,25 +173,23 @@ __global__ void __launch_bounds__(32 * (stream_consumer_warps<FP8, RG>() + 1))
   if (r0 >= r1) return;
   const int it_first = static_cast<int>(r0 / a.cap);
   const int it_last = static_cast<int>((r1 - 1) / a.cap);
+  const size_t split_stride = static_cast<size_t>(a.total_q) * a.H_q;
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                               ~static_cast<uintptr_t>(1023));
   uint8_t *slots = smem;
   uint8_t *qbufs = slots + NSLOT * TILE;
-  float *acc = reinterpret_cast<float *>(qbufs + 2 * kQBuf);  // [RG*16][128] merge buffer
-  uint64_t *sfull = reinterpret_cast<uint64_t *>(acc + RG * 16 * kHeadDim);
+  float *slices = reinterpret_cast<float *>(qbufs + 2 * QBUF);  // [RG][W/2][SLICE]
+  uint64_t *sfull = reinterpret_cast<uint64_t *>(slices + RG * (W / 2) * SLICE);
   uint64_t *sempty = sfull + NSLOT;
   uint64_t *qfull = sempty + NSLOT;
   uint64_t *qempty = qfull + 2;
   int *slot_j = reinterpret_cast<int *>(qempty + 2);
   uint32_t *slot_mask = reinterpret_cast<uint32_t *>(slot_j + NSLOT);
   int *slot_ok = reinterpret_cast<int *>(slot_mask + NSLOT);
-  float *mrg_m = reinterpret_cast<float *>(slot_ok + NSLOT);  // [NCW][16]
-  float *mrg_l = mrg_m + NCW * 16;                              // [NCW][16]
-  float *row_m = mrg_l + NCW * 16;                              // [RG*16]
-  float *row_l = row_m + RG * 16;                               // [RG*16]
-  volatile int *abort_flag = reinterpret_cast<volatile int *>(row_l + RG * 16);
+  SegMeta *meta = reinterpret_cast<SegMeta *>(slot_ok + NSLOT);  // [2], one per Q buffer
+  volatile int *abort_flag = reinterpret_cast<volatile int *>(meta + 2);
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < NSLOT; ++s) {
@@ -197,36 +214,76 @@ __global__ void __launch_bounds__(32 * (stream_consumer_warps<FP8, RG>() + 1))
       prefetch_tmap(&vmap);
     }
     bool dead = false;
-    // tile loads issued into each team's ring (two per block: K then V)
-    uint32_t nload0 = 0, nload1 = 0;
-    int n = 0;           // index of the current non-empty segment
-    // first non-empty segment
-    int it = it_first, v0 = 0, v1 = 0;
-    Item cur;
-    for (; it <= it_last; ++it) {
-      cur = load_item<PLAN>(a, it, lane == 0);
-      segment(a, it, r0, r1, cur.U, v0, v1);
-      if (v1 > v0) break;
-    }
-    if (it <= it_last) {
-      stage_q<FP8>(qbufs, a.q, cur.t0, cur.rows, a.G, a.H_q, cur.g, lane, 32);
+    uint32_t nload0 = 0, nload1 = 0;  // tile loads issued into each team's ring
+    int n = 0;                        // non-empty segments handed over
+    // waits (lane 0) until the consumers are done with Q buffer n & 1; false on timeout
+    auto claim_qbuf = [&](int n_) -> bool {
+      bool ok = true;
+      if (lane == 0 && n_ >= 2) ok = mbar_wait(&qempty[n_ & 1], ((n_ >> 1) - 1) & 1, abort_flag);
+      ok = __shfl_sync(0xffffffffu, ok, 0);
+      if (!ok && lane == 0) {
+        report(a.dev_err, MSA_DEVERR_TIMEOUT);
+        *abort_flag = 1;
+      }
+      return ok;
+    };
+    for (int it = it_first; it <= it_last && !dead; ++it) {
+      const Item m = load_item<PLAN>(a, it, lane == 0);
+      if (m.ntok == 0) continue;  // a tile past its sequence's end: no rows
+      int v0, v1;
+      segment(a, it, r0, r1, m.U, v0, v1);
+      const long long base = static_cast<long long>(it) * a.cap;
+      const int piece = static_cast<int>(blockIdx.x - base / a.R);
+      const bool last_cta = (base + a.cap - 1) / a.R == blockIdx.x;
+      // split indices of this item's rows that stay empty: this CTA's own when it has no real
+      // block of the item, and, from the item's last CTA, those past it
+      const int p_lo = v1 > v0 ? piece + 1 : piece;
+      const int p_hi = last_cta ? a.P : piece + 1;
+      for (int idx = lane; idx < m.rows * max(p_hi - p_lo, 0); idx += 32) {
+        const int r = idx % m.rows, p2 = p_lo + idx / m.rows;
+        const size_t orr = static_cast<size_t>(m.t0 + r / a.G) * a.H_q + m.g * a.G + r % a.G;
+        a.part_lse[static_cast<size_t>(p2) * split_stride + orr] = -INFINITY;
+      }
+      if (v1 <= v0) continue;
+
+      // ---- Q rows and metadata of this segment
+      if (!claim_qbuf(n)) {
+        dead = true;
+        break;
+      }
+      const int buf = n & 1;
+      stage_q<FP8, QR>(qbufs + buf * QBUF, a.q, m.t0, m.rows, a.G, a.H_q, m.g, lane, 32);
+      if (lane == 0) {
+        SegMeta md;
+        md.valid = 1;
+        md.t0 = m.t0;
+        md.rows = m.rows;
+        md.cl = m.cl;
+        md.tok0 = m.tok0;
+        md.g = m.g;
+        md.L = m.L;
+        md.v0 = v0;
+        md.v1 = v1;
+        md.piece = piece;
+        meta[buf] = md;
+      }
       __syncwarp();
-      if (lane == 0) mbar_arrive(&qfull[0]);
-    }
-    while (it <= it_last && !dead) {
-      // ---- K and V tiles of segment n.  The warp resolves 32 blocks' page ids at a time
-      // (one lane each) so that lane 0 never waits on a dependent lookup between two TMAs.
-      for (int base = v0; base < v1 && !dead; base += 32) {
-        const int e = base + lane;
+      if (lane == 0) mbar_arrive(&qfull[buf]);
+      ++n;
+
+      // ---- K and V tiles.  The warp resolves 32 blocks' page ids at a time (one lane
+      // each) so that lane 0 never waits on a dependent lookup between two TMAs.
+      for (int bbase = v0; bbase < v1 && !dead; bbase += 32) {
+        const int e = bbase + lane;
         int j = -1, page = -1;
         uint32_t msk = 0u;
         if (e < v1) {
-          j = cur.list[e];
-          msk = PLAN ? cur.masks[e] : 0xffffffffu;
+          j = m.list[e];
+          msk = PLAN ? m.masks[e] : 0xffffffffu;
           if (j >= 0 && j < a.max_blocks)
-            page = a.table[static_cast<size_t>(cur.b) * a.max_pages + j];
+            page = a.table[static_cast<size_t>(m.b) * a.max_pages + j];
         }
-        const int cnt = min(32, v1 - base);
+        const int cnt = min(32, v1 - bbase);
         for (int i = 0; i < cnt; ++i) {
           const int jj = __shfl_sync(0xffffffffu, j, i);
           const int pg = __shfl_sync(0xffffffffu, page, i);
@@ -235,8 +292,8 @@ __global__ void __launch_bounds__(32 * (stream_consumer_warps<FP8, RG>() + 1))
             const bool jok = jj >= 0 && jj < a.max_blocks;
             const bool ok = jok && pg >= 0 && pg < a.num_pages;
             if (!ok) report(a.dev_err, jok ? MSA_DEVERR_PAGE_ID : MSA_DEVERR_BLOCK_ID);
-            const int c2 = pg * a.H_kv + cur.g;
-            const int tm = (base + i - v0) % NT;  // the team that reads this block
+            const int c2 = pg * a.H_kv + m.g;
+            const int tm = (bbase + i - v0) % NT;  // the team that reads this block
 #pragma unroll
             for (int kv = 0; kv < 2; ++kv) {
               const uint32_t nl = tm ? nload1 : nload0;
@@ -270,185 +327,109 @@ __global__ void __launch_bounds__(32 * (stream_consumer_warps<FP8, RG>() + 1))
           if (dead) break;
         }
       }
-      dead = __shfl_sync(0xffffffffu, dead, 0);
-      if (dead) break;
-      // ---- Q rows of the next non-empty segment into the other Q buffer
-      int nit = it + 1, w0 = 0, w1 = 0;
-      Item nxt;
-      for (; nit <= it_last; ++nit) {
-        nxt = load_item<PLAN>(a, nit, lane == 0);
-        segment(a, nit, r0, r1, nxt.U, w0, w1);
-        if (w1 > w0) break;
-      }
-      if (nit <= it_last) {
-        const int buf = (n + 1) & 1;
-        bool qok = true;  // lane 0 waits for the buffer, the warp follows it
-        if (lane == 0 && n + 1 >= 2)
-          qok = mbar_wait(&qempty[buf], (((n + 1) >> 1) - 1) & 1, abort_flag);
-        qok = __shfl_sync(0xffffffffu, qok, 0);
-        if (!qok) {
-          if (lane == 0) {
-            report(a.dev_err, MSA_DEVERR_TIMEOUT);
-            *abort_flag = 1;
-          }
-          break;
-        }
-        stage_q<FP8>(qbufs + buf * kQBuf, a.q, nxt.t0, nxt.rows, a.G, a.H_q, nxt.g, lane, 32);
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&qfull[buf]);
-      }
-      cur = nxt;
-      it = nit;
-      v0 = w0;
-      v1 = w1;
-      ++n;
+    }
+    // ---- no segment left
+    if (!dead && claim_qbuf(n) && lane == 0) {
+      meta[n & 1].valid = 0;
+      mbar_arrive(&qfull[n & 1]);
     }
     return;
   }
 
   // ================================================================ consumer warps
   const int team = warp / TEAM, rg = (warp % TEAM) / PQ, pq = warp % PQ;
-  const bool row_owner = team == 0 && pq == 0 && (lane & 3) == 0;  // one writer per row
+  const int rank = team * PQ + pq;  // rank among the W warps of this row group
   const int nct = 32 * NCW;
+  float *my_slices = slices + rg * (W / 2) * SLICE;
   WA wa;
   uint32_t nload = 0;  // loads this warp's team has consumed from its ring
-  int n = 0;
-  for (int it = it_first; it <= it_last; ++it) {
-    const Item m = load_item<PLAN>(a, it, false);
-    if (m.ntok == 0) continue;  // a tile past its sequence's end: no rows
-    int v0, v1;
-    segment(a, it, r0, r1, m.U, v0, v1);
-    const long long base = static_cast<long long>(it) * a.cap;
-    const int piece = static_cast<int>(blockIdx.x - base / a.R);
-    const bool last_cta = (base + a.cap - 1) / a.R == blockIdx.x;
-    const size_t split_stride = static_cast<size_t>(a.total_q) * a.H_q;
-    // this thread's two rows
+  for (int n = 0;; ++n) {
+    const int buf = n & 1;
+    if (!mbar_wait(&qfull[buf], (n >> 1) & 1, abort_flag)) {
+      report(a.dev_err, MSA_DEVERR_TIMEOUT);
+      *abort_flag = 1;
+    }
+    named_bar_sync(1, nct);  // every consumer takes the same decision below
+    if (*abort_flag) break;
+    const SegMeta md = meta[buf];
+    if (!md.valid) break;
     int prow[2];
     uint32_t tbit[2];
-    size_t orow[2];
-    bool rvalid[2];
 #pragma unroll
     for (int slot = 0; slot < 2; ++slot) {
       const int r = rg * 16 + (lane >> 2) + slot * 8;
       const int tl = r / a.G;
-      rvalid[slot] = r < m.rows;
-      prow[slot] = rvalid[slot] ? m.cl + m.tok0 + tl : -1;
-      tbit[slot] = rvalid[slot] ? (1u << tl) : 0u;
-      orow[slot] = rvalid[slot] ? static_cast<size_t>(m.t0 + tl) * a.H_q + m.g * a.G + r % a.G : 0;
+      prow[slot] = r < md.rows ? md.cl + md.tok0 + tl : -1;
+      tbit[slot] = r < md.rows ? (1u << tl) : 0u;
     }
-
-    if (v1 > v0) {
-      const int buf = n & 1;
-      const bool qlive = mbar_wait(&qfull[buf], (n >> 1) & 1, abort_flag);
-      if (!qlive) {
+    const uint32_t qs_addr = smem_u32(qbufs + buf * QBUF);
+    wa.reset();
+    for (int e = md.v0 + team; e < md.v1; e += NT) {
+      const uint32_t nk = nload;  // this team's K tile; V is nk + 1
+      int s = team * NR + static_cast<int>(nk % NR);
+      bool live = mbar_wait(&sfull[s], (nk / NR) & 1, abort_flag);
+      const bool ok = live && slot_ok[s];
+      const int j = slot_j[s];
+      const uint32_t msk = slot_mask[s];
+      if (ok) wa.qk(qs_addr, QSUB, rg * 16, smem_u32(slots + s * TILE), pq, lane);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&sempty[s]);
+      if (ok) wa.softmax(j, pq, lane, prow, tbit, msk, a.scale_log2);
+      s = team * NR + static_cast<int>((nk + 1) % NR);
+      live = mbar_wait(&sfull[s], ((nk + 1) / NR) & 1, abort_flag) && live;
+      if (ok && live) wa.pv(smem_u32(slots + s * TILE), j, pq, lane, md.L);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&sempty[s]);
+      nload = nk + 2;
+      if (!live) {
         report(a.dev_err, MSA_DEVERR_TIMEOUT);
         *abort_flag = 1;
       }
-      const uint32_t qs_addr = smem_u32(qbufs + buf * kQBuf);
-      wa.reset();
-      for (int e = v0 + team; e < v1; e += NT) {
-        const uint32_t nk = nload;  // this team's K tile; V is nk + 1
-        int s = team * NR + static_cast<int>(nk % NR);
-        bool live = mbar_wait(&sfull[s], (nk / NR) & 1, abort_flag);
-        const bool ok = live && qlive && slot_ok[s];
-        const int j = slot_j[s];
-        const uint32_t msk = slot_mask[s];
-        if (ok) wa.qk(qs_addr, rg * 16, smem_u32(slots + s * TILE), pq, lane);
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&sempty[s]);
-        if (ok) wa.softmax(j, pq, lane, prow, tbit, msk, a.scale_log2);
-        s = team * NR + static_cast<int>((nk + 1) % NR);
-        live = mbar_wait(&sfull[s], ((nk + 1) / NR) & 1, abort_flag) && live;
-        if (ok && live) wa.pv(smem_u32(slots + s * TILE), j, pq, lane, m.L);
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&sempty[s]);
-        nload = nk + 2;
-        if (!live) {
-          report(a.dev_err, MSA_DEVERR_TIMEOUT);
-          *abort_flag = 1;
-        }
-      }
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&qempty[buf]);
-      ++n;
+    }
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&qempty[buf]);
 
-      // ---- fold the NT * PQ warp states of every row into one, through shared memory
-      wa.finish_rows();
-      if ((lane & 3) == 0) {
+    // ---- fold the W warp states of every row into rank 0: a pairwise log-sum-exp tree
+    // through shared-memory slices, in a fixed order (reproducible sums)
+    wa.finish_rows();
+#pragma unroll
+    for (int step = W / 2; step >= 1; step >>= 1) {
+      if (rank >= step && rank < 2 * step) {
+        float *sl = my_slices + (rank - step) * SLICE;
 #pragma unroll
         for (int slot = 0; slot < 2; ++slot) {
-          mrg_m[warp * 16 + (lane >> 2) + slot * 8] = wa.m_run[slot];
-          mrg_l[warp * 16 + (lane >> 2) + slot * 8] = wa.l_run[slot];
+          const int r16 = (lane >> 2) + slot * 8;
+          wa.store_row(sl, r16, slot, 1.f, lane, false);
+          if ((lane & 3) == 0) {
+            sl[16 * MS + r16] = wa.m_run[slot];
+            sl[16 * MS + 16 + r16] = wa.l_run[slot];
+          }
         }
       }
       named_bar_sync(1, nct);
-      float fac[2];
+      if (rank < step) {
+        const float *sl = my_slices + rank * SLICE;
+#pragma unroll
+        for (int slot = 0; slot < 2; ++slot) {
+          const int r16 = (lane >> 2) + slot * 8;
+          wa.merge_row(sl, r16, slot, sl[16 * MS + r16], sl[16 * MS + 16 + r16], lane);
+        }
+      }
+      named_bar_sync(1, nct);
+    }
+    // ---- rank 0 writes this segment's partial: normalised output and log-sum-exp
+    if (rank == 0) {
 #pragma unroll
       for (int slot = 0; slot < 2; ++slot) {
-        const int r16 = (lane >> 2) + slot * 8;
-        float M = -INFINITY;
-#pragma unroll
-        for (int t2 = 0; t2 < NT; ++t2)
-#pragma unroll
-          for (int p2 = 0; p2 < PQ; ++p2)
-            M = fmaxf(M, mrg_m[(t2 * TEAM + rg * PQ + p2) * 16 + r16]);
-        float Ls = 0.f;
-        if (M != -INFINITY) {
-#pragma unroll
-          for (int t2 = 0; t2 < NT; ++t2)
-#pragma unroll
-            for (int p2 = 0; p2 < PQ; ++p2) {
-              const int w2 = t2 * TEAM + rg * PQ + p2;
-              const float mw = mrg_m[w2 * 16 + r16];
-              if (mw != -INFINITY) Ls += mrg_l[w2 * 16 + r16] * fast_exp2(mw - M);
-            }
-        }
-        fac[slot] = wa.m_run[slot] == -INFINITY ? 0.f : fast_exp2(wa.m_run[slot] - M);
-        if (row_owner) {
-          row_m[rg * 16 + r16] = M;
-          row_l[rg * 16 + r16] = Ls;
-        }
+        const int r = rg * 16 + (lane >> 2) + slot * 8;
+        if (r >= md.rows) continue;
+        const size_t orr = static_cast<size_t>(md.t0 + r / a.G) * a.H_q + md.g * a.G + r % a.G;
+        const size_t pr = static_cast<size_t>(md.piece) * split_stride + orr;
+        const float l = wa.l_run[slot];
+        wa.store_global(a.part_o + pr * kHeadDim, slot, l > 0.f ? 1.f / l : 0.f, lane);
+        if ((lane & 3) == 0)
+          a.part_lse[pr] = l > 0.f ? (wa.m_run[slot] + __log2f(l)) * kLn2 : -INFINITY;
       }
-      // fixed-order accumulation (reproducible sums): in round k the warp of each row group
-      // whose rank in the group is k adds its rescaled output; round 0 stores.
-      const int rank = team * PQ + pq;
-      for (int k = 0; k < NT * PQ; ++k) {
-        if (rank == k) {
-#pragma unroll
-          for (int slot = 0; slot < 2; ++slot)
-            wa.store_row(acc, rg * 16 + (lane >> 2) + slot * 8, slot, fac[slot], lane, k > 0);
-        }
-        named_bar_sync(1, nct);
-      }
-      // ---- write this segment's partial (all consumer threads)
-      const int ctid = threadIdx.x;  // consumers are threads [0, nct)
-      for (int idx = ctid; idx < RG * 16 * (kHeadDim / 4); idx += nct) {
-        const int r = idx / (kHeadDim / 4), d4 = idx % (kHeadDim / 4);
-        if (r >= m.rows) continue;
-        const int tl = r / a.G;
-        const size_t orr = static_cast<size_t>(m.t0 + tl) * a.H_q + m.g * a.G + r % a.G;
-        const size_t pr = static_cast<size_t>(piece) * split_stride + orr;
-        const float L = row_l[r];
-        const float inv = L > 0.f ? 1.f / L : 0.f;
-        const float4 v =
-            *reinterpret_cast<const float4 *>(acc + r * kHeadDim + acc_col(r, 4 * d4));
-        reinterpret_cast<float4 *>(a.part_o + pr * kHeadDim)[d4] =
-            make_float4(v.x * inv, v.y * inv, v.z * inv, v.w * inv);
-        if (d4 == 0) a.part_lse[pr] = L > 0.f ? (row_m[r] + __log2f(L)) * kLn2 : -INFINITY;
-      }
-    } else if (row_owner) {
-      // a range that meets this item only in slots past its count: an empty partial
-#pragma unroll
-      for (int slot = 0; slot < 2; ++slot)
-        if (rvalid[slot]) a.part_lse[static_cast<size_t>(piece) * split_stride + orow[slot]] = -INFINITY;
-    }
-    // the item's last CTA marks the split indices no CTA of this item owns
-    if (last_cta && row_owner) {
-      for (int p2 = piece + 1; p2 < a.P; ++p2)
-#pragma unroll
-        for (int slot = 0; slot < 2; ++slot)
-          if (rvalid[slot])
-            a.part_lse[static_cast<size_t>(p2) * split_stride + orow[slot]] = -INFINITY;
     }
   }
 }

@@ -110,7 +110,7 @@ __global__ void __launch_bounds__(32 * (RG * tile_pq<RG>() + 1))
     *abort_flag = 0;
     fence_mbar_init();
   }
-  stage_q<FP8>(qs, a.q, t0, rows, a.G, a.H_q, g, threadIdx.x, blockDim.x);
+  stage_q<FP8, kQRows>(qs, a.q, t0, rows, a.G, a.H_q, g, threadIdx.x, blockDim.x);
   __syncthreads();
 
   if (warp == NCW) {
@@ -197,7 +197,7 @@ __global__ void __launch_bounds__(32 * (RG * tile_pq<RG>() + 1))
     if (live && st_ok[s]) {
       const int j = st_j[s];
       const uint32_t kt = smem_u32(stages + s * STAGE);
-      wa.qk(qs_addr, rg * 16, kt, pq, lane);
+      wa.qk(qs_addr, kQSub, rg * 16, kt, pq, lane);
       wa.softmax(j, pq, lane, prow, tbit, st_mask[s], a.scale_log2);
       wa.pv(kt + TILE, j, pq, lane, L);
     }
@@ -210,7 +210,8 @@ __global__ void __launch_bounds__(32 * (RG * tile_pq<RG>() + 1))
   wa.finish_rows();
   named_bar_sync(1, NCT);  // every consumer is done with the stages
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-  float *mo = reinterpret_cast<float *>(stages);  // [NCW][16][128]
+  float *mo = reinterpret_cast<float *>(stages);  // [NCW][16][padded 128]
+  constexpr int MS = MergeRow<FP8>::kStride;
   if ((lane & 3) == 0) {
 #pragma unroll
     for (int slot = 0; slot < 2; ++slot) {
@@ -235,7 +236,7 @@ __global__ void __launch_bounds__(32 * (RG * tile_pq<RG>() + 1))
     }
     const float f =
         (Ls > 0.f && wa.m_run[slot] != -INFINITY) ? fast_exp2(wa.m_run[slot] - M) / Ls : 0.f;
-    wa.store_row(mo + static_cast<size_t>(warp) * 16 * kHeadDim, r16, slot, f, lane, false);
+    wa.store_row(mo + static_cast<size_t>(warp) * 16 * MS, r16, slot, f, lane, false);
   }
   named_bar_sync(1, NCT);
   for (int idx = threadIdx.x; idx < RG * 16 * (kHeadDim / 4); idx += NCT) {
@@ -246,7 +247,7 @@ __global__ void __launch_bounds__(32 * (RG * tile_pq<RG>() + 1))
 #pragma unroll
     for (int w = 0; w < PQ; ++w) {
       const float4 v = *reinterpret_cast<const float4 *>(
-          mo + (static_cast<size_t>(rgr * PQ + w) * 16 + r16) * kHeadDim + acc_col(r16, 4 * d4));
+          mo + (static_cast<size_t>(rgr * PQ + w) * 16 + r16) * MS + 4 * d4);
       acc.x += v.x;
       acc.y += v.y;
       acc.z += v.z;

@@ -28,15 +28,16 @@ struct KvTile {
   static constexpr uint32_t kSub = 16384u;                    // one swizzled [128][128 B] box
 };
 
-// Stage rows [0, kQRows) of Q for rows r = tok * G + h_local of one work item into a Q buffer
-// (zeros past `rows`).  Threads `tid` of `nthreads` share the copy.  For e4m3 KV the values
-// become f16 and, inside every 16-dim group, slot 2c+e holds dim 4c+e and slot 2c+8+e holds
-// dim 4c+2+e (c < 4, e < 2): the order in which a plain ldmatrix of an e4m3 K tile hands the
-// dims to the MMA, so that both operands agree on k.
-template <bool FP8>
+// Stage rows [0, QR) of Q (rows r = tok * G + h_local of one work item) into a Q buffer of
+// two swizzled [QR][128 B] sub-tiles (zeros past `rows`).  Threads `tid` of `nthreads` share
+// the copy.  For e4m3 KV the values become f16 and, inside every 16-dim group, slot 2c+e holds
+// dim 4c+e and slot 2c+8+e holds dim 4c+2+e (c < 4, e < 2): the order in which a plain
+// ldmatrix of an e4m3 K tile hands the dims to the MMA, so that both operands agree on k.
+template <bool FP8, int QR>
 __device__ __forceinline__ void stage_q(uint8_t *qs, const uint16_t *q, int t0, int rows, int G,
                                         int H_q, int g, int tid, int nthreads) {
-  for (int idx = tid; idx < kQRows * 8; idx += nthreads) {
+  constexpr uint32_t sub = QR * 128;
+  for (int idx = tid; idx < QR * 8; idx += nthreads) {
     const int r = idx >> 3, grp = idx & 7;
     uint4 lo4 = make_uint4(0, 0, 0, 0), hi4 = make_uint4(0, 0, 0, 0);
     if (r < rows) {
@@ -65,14 +66,17 @@ __device__ __forceinline__ void stage_q(uint8_t *qs, const uint16_t *q, int t0, 
         hi4 = make_uint4(o8[4], o8[5], o8[6], o8[7]);
       }
     }
-    *reinterpret_cast<uint4 *>(qs + sw128(r, 2 * grp, kQSub)) = lo4;
-    *reinterpret_cast<uint4 *>(qs + sw128(r, 2 * grp + 1, kQSub)) = hi4;
+    *reinterpret_cast<uint4 *>(qs + sw128(r, 2 * grp, sub)) = lo4;
+    *reinterpret_cast<uint4 *>(qs + sw128(r, 2 * grp + 1, sub)) = hi4;
   }
 }
 
-// Column of dim `col` in row `row` of a [rows][128] fp32 merge buffer: 32-byte chunks are
-// XOR-ed with row % 8, so that the 8 rows a warp's lanes hold fall in different banks.
-__device__ __forceinline__ int acc_col(int row, int col) { return col ^ ((row & 7) << 3); }
+// Row stride (floats) of the fp32 merge buffers: padded so that the 8 rows a warp's lanes hold
+// fall in different banks for the float2 (BF16 layout) and float4 (FP8 layout) accesses.
+template <bool FP8>
+struct MergeRow {
+  static constexpr int kStride = kHeadDim + (FP8 ? 16 : 8);
+};
 
 template <bool FP8, int PQ>
 struct WarpAttn {
@@ -93,8 +97,10 @@ struct WarpAttn {
     l_run[0] = l_run[1] = 0.f;
   }
 
-  // sc = Q K^T for the warp's 16 rows (row base qrow0 of the Q buffer) and PW positions.
-  __device__ __forceinline__ void qk(uint32_t qs_addr, int qrow0, uint32_t kt, int pq, int lane) {
+  // sc = Q K^T for the warp's 16 rows (row base qrow0 of a Q buffer whose sub-tiles are
+  // qsub bytes) and PW positions.
+  __device__ __forceinline__ void qk(uint32_t qs_addr, uint32_t qsub, int qrow0, uint32_t kt,
+                                     int pq, int lane) {
     const int mi = lane >> 3, rr = lane & 7;
 #pragma unroll
     for (int n = 0; n < NTW; ++n)
@@ -103,7 +109,7 @@ struct WarpAttn {
 #pragma unroll
     for (int ks = 0; ks < 8; ++ks) {
       uint32_t qa[4];
-      ldsm_x4(qs_addr + sw128(qrow0 + (mi & 1) * 8 + rr, 2 * ks + (mi >> 1), kQSub), qa[0], qa[1],
+      ldsm_x4(qs_addr + sw128(qrow0 + (mi & 1) * 8 + rr, 2 * ks + (mi >> 1), qsub), qa[0], qa[1],
               qa[2], qa[3]);
       if (FP8) {
 #pragma unroll
@@ -253,17 +259,17 @@ struct WarpAttn {
     }
   }
 
-  // This thread's part of row slot `slot` times f, as fp32, into row `row` of a [rows][128]
-  // fp32 buffer laid out by acc_col (the FP8 path's dim permutation is undone here).  With
-  // `add` the values are added to what the buffer holds.
+  // This thread's part of row slot `slot` times f, as fp32, into row `row` of a merge buffer
+  // (rows MergeRow<FP8>::kStride floats apart; the FP8 path's dim permutation is undone
+  // here).  With `add` the values are added to what the buffer holds.
   __device__ __forceinline__ void store_row(float *buf, int row, int slot, float f, int lane,
                                             bool add) const {
     const int c4 = lane & 3;
-    float *dst = buf + row * kHeadDim;
+    float *dst = buf + row * MergeRow<FP8>::kStride;
     if (FP8) {
 #pragma unroll
       for (int ch = 0; ch < 8; ++ch) {
-        float4 *d = reinterpret_cast<float4 *>(dst + acc_col(row, ch * 16 + 4 * c4));
+        float4 *d = reinterpret_cast<float4 *>(dst + ch * 16 + 4 * c4);
         float4 v = make_float4(o[2 * ch][2 * slot] * f, o[2 * ch + 1][2 * slot] * f,
                                o[2 * ch][2 * slot + 1] * f, o[2 * ch + 1][2 * slot + 1] * f);
         if (add) {
@@ -275,7 +281,7 @@ struct WarpAttn {
     } else {
 #pragma unroll
       for (int n = 0; n < 16; ++n) {
-        float2 *d = reinterpret_cast<float2 *>(dst + acc_col(row, n * 8 + 2 * c4));
+        float2 *d = reinterpret_cast<float2 *>(dst + n * 8 + 2 * c4);
         float2 v = make_float2(o[n][2 * slot] * f, o[n][2 * slot + 1] * f);
         if (add) {
           const float2 u = *d;
@@ -283,6 +289,55 @@ struct WarpAttn {
         }
         *d = v;
       }
+    }
+  }
+
+  // Fold the state another warp left in shared memory (its output row `row` of `buf`, laid
+  // out by store_row, with max m2 and sum l2) into this thread's row slot `slot`.
+  __device__ __forceinline__ void merge_row(const float *buf, int row, int slot, float m2,
+                                            float l2, int lane) {
+    const float m1 = m_run[slot];
+    const float m = fmaxf(m1, m2);
+    const float a1 = m1 == -INFINITY ? 0.f : fast_exp2(m1 - m);
+    const float a2 = m2 == -INFINITY ? 0.f : fast_exp2(m2 - m);
+    const int c4 = lane & 3;
+    const float *src = buf + row * MergeRow<FP8>::kStride;
+    if (FP8) {
+#pragma unroll
+      for (int ch = 0; ch < 8; ++ch) {
+        const float4 u = *reinterpret_cast<const float4 *>(src + ch * 16 + 4 * c4);
+        o[2 * ch][2 * slot] = o[2 * ch][2 * slot] * a1 + u.x * a2;
+        o[2 * ch + 1][2 * slot] = o[2 * ch + 1][2 * slot] * a1 + u.y * a2;
+        o[2 * ch][2 * slot + 1] = o[2 * ch][2 * slot + 1] * a1 + u.z * a2;
+        o[2 * ch + 1][2 * slot + 1] = o[2 * ch + 1][2 * slot + 1] * a1 + u.w * a2;
+      }
+    } else {
+#pragma unroll
+      for (int n = 0; n < 16; ++n) {
+        const float2 u = *reinterpret_cast<const float2 *>(src + n * 8 + 2 * c4);
+        o[n][2 * slot] = o[n][2 * slot] * a1 + u.x * a2;
+        o[n][2 * slot + 1] = o[n][2 * slot + 1] * a1 + u.y * a2;
+      }
+    }
+    l_run[slot] = l_run[slot] * a1 + l2 * a2;
+    m_run[slot] = m;
+  }
+
+  // This thread's part of row slot `slot` times f, as fp32 in natural dim order, into a
+  // 128-dim row of global memory.
+  __device__ __forceinline__ void store_global(float *dst, int slot, float f, int lane) const {
+    const int c4 = lane & 3;
+    if (FP8) {
+#pragma unroll
+      for (int ch = 0; ch < 8; ++ch)
+        *reinterpret_cast<float4 *>(dst + ch * 16 + 4 * c4) =
+            make_float4(o[2 * ch][2 * slot] * f, o[2 * ch + 1][2 * slot] * f,
+                        o[2 * ch][2 * slot + 1] * f, o[2 * ch + 1][2 * slot + 1] * f);
+    } else {
+#pragma unroll
+      for (int n = 0; n < 16; ++n)
+        *reinterpret_cast<float2 *>(dst + n * 8 + 2 * c4) =
+            make_float2(o[n][2 * slot] * f, o[n][2 * slot + 1] * f);
     }
   }
 };
