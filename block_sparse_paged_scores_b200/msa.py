@@ -64,6 +64,9 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.msa_attn_workspace_bytes.argtypes = [RP, I, I, I, I, I]
     lib.msa_default_num_splits.restype = I
     lib.msa_default_num_splits.argtypes = [I, I, I, I, I]
+    lib.msa_sparse_attn_paged_noalloc.restype = I
+    lib.msa_sparse_attn_paged_noalloc.argtypes = [RP, P, P, P, I, P, P, I, I, I, I, F, I, P, P,
+                                                  P]
     lib.msa_attn_partials.restype = I
     lib.msa_attn_partials.argtypes = [RP, I, I, I, I, I, ctypes.POINTER(ctypes.c_size_t),
                                       ctypes.POINTER(ctypes.c_size_t)]
@@ -153,6 +156,18 @@ def msa_sparse_attn_paged(rp: RaggedPaged, q, k_cache, v_cache, kv_dtype: int, b
         ctypes.byref(rp), _ptr(q), _ptr(k_cache), _ptr(v_cache), int(kv_dtype), _ptr(block_ids),
         _ptr(num_selected), S, num_q_heads, num_kv_heads, max_blocks, float(scale), num_splits,
         _ptr(workspace), int(workspace_bytes), _ptr(out), _ptr(dev_err), _stream(stream)))
+
+
+def msa_sparse_attn_paged_noalloc(rp: RaggedPaged, q, k_cache, v_cache, kv_dtype: int,
+                                  block_ids, num_selected, S: int, num_q_heads: int,
+                                  num_kv_heads: int, max_blocks: int, scale: float,
+                                  num_splits: int, out, dev_err=None, stream=None):
+    """msa_sparse_attn_paged with its scratch in the library's own device array (for callers
+    that cannot allocate a workspace); see include/msa.h for the size limit."""
+    _check("msa_sparse_attn_paged_noalloc", load().msa_sparse_attn_paged_noalloc(
+        ctypes.byref(rp), _ptr(q), _ptr(k_cache), _ptr(v_cache), int(kv_dtype), _ptr(block_ids),
+        _ptr(num_selected), S, num_q_heads, num_kv_heads, max_blocks, float(scale), num_splits,
+        _ptr(out), _ptr(dev_err), _stream(stream)))
 
 
 def msa_splitk_combine(partial_o, partial_lse, num_splits: int, total_q: int, num_q_heads: int,

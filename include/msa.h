@@ -172,6 +172,34 @@ MSA_API msa_status_t msa_sparse_attn_paged(const msa_ragged_paged_t *rp, const v
                                    void *out, int32_t *dev_err, struct CUstream_st *stream);
 
 /*
+ * msa_sparse_attn_paged_noalloc — msa_sparse_attn_paged for callers that cannot provide a
+ * workspace.  (This entry point has no counterpart on the pages: it is a deployment aid.)
+ *
+ * Some callers cannot allocate device memory when they call in: a host runtime whose device
+ * memory plan is fixed before it starts serving and has no allocator to call afterwards, or a
+ * plugin interface that passes only an operation's inputs and outputs.  This entry point takes
+ * the same arguments as msa_sparse_attn_paged minus `workspace` / `workspace_bytes`, and keeps
+ * that scratch in a device array that is part of the library itself: MSA_NOALLOC_SCRATCH_BYTES
+ * on every GPU the library is loaded on, held until the process exits.  It allocates nothing.
+ *
+ *   - A shape whose msa_attn_workspace_bytes exceeds MSA_NOALLOC_SCRATCH_BYTES is rejected
+ *     with MSA_ERR_UNSUPPORTED before anything is enqueued (use msa_sparse_attn_paged with a
+ *     workspace of your own for it).
+ *   - The first call on a device looks the array's device address up (once per device, with
+ *     that device current); make that first call before any stream capture.
+ *   - Every call on a device shares the one array and it keeps the last call's contents
+ *     (nothing in it needs to start at zero).  Calls whose work overlaps on the GPU race on
+ *     it: run them on one stream, or order them.
+ */
+#define MSA_NOALLOC_SCRATCH_BYTES (32u << 20) /* 32 MiB */
+
+MSA_API msa_status_t msa_sparse_attn_paged_noalloc(
+    const msa_ragged_paged_t *rp, const void *q, const void *k_cache, const void *v_cache,
+    msa_kv_dtype_t kv_dtype, const int32_t *block_ids, const int32_t *num_selected, int32_t S,
+    int32_t num_q_heads, int32_t num_kv_heads, int32_t max_blocks, float scale,
+    int32_t num_splits, void *out, int32_t *dev_err, struct CUstream_st *stream);
+
+/*
  * msa_splitk_combine — merge split-K partials ([msa] "Three attention routes": at more than
  * one partition the partials key on the ragged global query row and a combine writes the
  * ragged output).
