@@ -90,6 +90,7 @@ bool ragged_ok(const msa_ragged_paged_t *rp) {
 struct Route {
   bool plan;      // speculative / prefill: per-tile union in the workspace
   bool stream;    // decode / speculative: the persistent split-K kernel + combine
+  bool tc;        // prefill on tcgen05 (BF16 KV): 128-row tiles
   int qt, tiles;  // query tokens per tile, tiles per sequence
   int rg;         // 16-row groups per CTA
   int cap;        // work-list slots per item
@@ -116,21 +117,22 @@ int stream_grid(long long total, int num_splits, int num_sms) {
 }
 
 bool make_route(const msa_ragged_paged_t *rp, int S, int H_q, int H_kv, int max_blocks,
-                int num_splits, int num_sms, Route *r) {
+                int num_splits, int num_sms, bool fp8, Route *r) {
   const int G = H_q / H_kv;
   r->plan = rp->max_q_len > 1;
   r->stream = rp->max_q_len <= MSA_MAX_SPEC_DRAFT;
+  r->tc = !r->stream && !fp8 && G <= 128 && attention_tc_supported(G, std::max(1, 128 / G));
   if (!r->plan) {
     r->qt = 1;
   } else {
-    int qt = kMaxRows / G;
+    int qt = (r->tc ? 128 : kMaxRows) / G;
     if (qt > 32) qt = 32;  // token masks are 32-bit
     if (qt > rp->max_q_len) qt = rp->max_q_len;
     r->qt = qt < 1 ? 1 : qt;
   }
   r->tiles = (rp->max_q_len + r->qt - 1) / r->qt;
   r->rg = (r->qt * G + 15) / 16;
-  if (r->rg < 1 || r->rg > 4) return false;
+  if (r->rg < 1 || (r->rg > 4 && !r->tc)) return false;
   const long long cap = r->plan ? std::min<long long>(static_cast<long long>(r->qt) * S, max_blocks)
                                 : S;
   r->cap = static_cast<int>(cap);
@@ -224,10 +226,13 @@ size_t msa_attn_workspace_bytes(const msa_ragged_paged_t *rp, int32_t S, int32_t
       num_q_heads < num_kv_heads || num_q_heads % num_kv_heads || max_blocks < 1 ||
       num_splits < 0)
     return 0;
-  Route r;
+  // the size covers either KV dtype (the prefill routes tile differently)
+  Route r, r8;
   const int sms = num_splits > 0 ? 1 : num_sms_of_current_device();
-  if (!make_route(rp, S, num_q_heads, num_kv_heads, max_blocks, num_splits, sms, &r)) return 0;
-  return r.bytes;
+  if (!make_route(rp, S, num_q_heads, num_kv_heads, max_blocks, num_splits, sms, false, &r) ||
+      !make_route(rp, S, num_q_heads, num_kv_heads, max_blocks, num_splits, sms, true, &r8))
+    return 0;
+  return std::max(r.bytes, r8.bytes);
 }
 
 int32_t msa_attn_partials(const msa_ragged_paged_t *rp, int32_t S, int32_t num_q_heads,
@@ -239,7 +244,7 @@ int32_t msa_attn_partials(const msa_ragged_paged_t *rp, int32_t S, int32_t num_q
     return 0;
   Route r;
   const int sms = num_splits > 0 ? 1 : num_sms_of_current_device();
-  if (!make_route(rp, S, num_q_heads, num_kv_heads, max_blocks, num_splits, sms, &r) ||
+  if (!make_route(rp, S, num_q_heads, num_kv_heads, max_blocks, num_splits, sms, false, &r) ||
       !r.stream)
     return 0;
   if (partial_o_offset) *partial_o_offset = r.off_o;
@@ -367,7 +372,7 @@ msa_status_t msa_sparse_attn_paged(const msa_ragged_paged_t *rp, const void *q,
     return MSA_ERR_UNSUPPORTED;
   Route r;
   if (!make_route(rp, S, num_q_heads, num_kv_heads, max_blocks, num_splits,
-                  num_sms_of_current_device(), &r))
+                  num_sms_of_current_device(), kv_dtype == MSA_KV_FP8_E4M3, &r))
     return MSA_ERR_UNSUPPORTED;
   if (r.plan && (2 * ((max_blocks + 31) / 32) + r.cap) * 4 > 200 * 1024)
     return MSA_ERR_UNSUPPORTED;
@@ -436,6 +441,8 @@ msa_status_t msa_sparse_attn_paged(const msa_ragged_paged_t *rp, const void *q,
   a.part_lse = reinterpret_cast<float *>(ws + r.off_lse);
   a.out = static_cast<uint16_t *>(out);
   a.dev_err = dev_err;
+  if (r.tc)
+    return launch_attention_tc(kmap, vmap, a, s) == cudaSuccess ? MSA_OK : MSA_ERR_CUDA;
   if (!r.stream)
     return launch_attention_tiles(kmap, vmap, a, fp8, r.rg, s) == cudaSuccess ? MSA_OK
                                                                              : MSA_ERR_CUDA;

@@ -76,6 +76,10 @@ cudaError_t launch_attention_stream(const CUtensorMap &kmap, const CUtensorMap &
                                     cudaStream_t s);
 cudaError_t launch_attention_tiles(const CUtensorMap &kmap, const CUtensorMap &vmap,
                                    const AttnArgs &a, bool fp8, int rg, cudaStream_t s);
+// prefill on tcgen05 (attention_tc.cu): BF16 KV, tiles of qt tokens x G heads <= 128 rows
+bool attention_tc_supported(int G, int qt);
+cudaError_t launch_attention_tc(const CUtensorMap &kmap, const CUtensorMap &vmap,
+                                const AttnArgs &a, cudaStream_t s);
 
 // ---- split-K combine (combine.cu)
 cudaError_t launch_combine(const float *part_o, const float *part_lse, int splits, int total_q,

@@ -33,6 +33,10 @@ CASES = {
                                               kv_dtype="fp8")),
     "prefill_with_empty_rows": (W["ragged_prefill"], dict(batch=4, q_len=(0, 40),
                                                           prior_len=(100, 900))),
+    "prefill_gqa4": (W["ragged_prefill"], dict(batch=2, q_len=(40, 200), prior_len=(0, 1500),
+                                               H_kv=2, G=4)),
+    "prefill_gqa16": (W["ragged_prefill"], dict(batch=2, q_len=(30, 150), prior_len=(100, 1200),
+                                                H_kv=1, G=16)),
 }
 
 
