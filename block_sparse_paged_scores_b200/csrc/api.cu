@@ -280,6 +280,22 @@ msa_status_t msa_index_scores(const msa_ragged_paged_t *rp, const void *q_idx,
   a.H_kv = num_kv_heads;
   a.H_idxk = num_idx_k_heads;
   a.max_blocks = max_blocks;
+  // prefill: the dense tile x page contraction runs on tcgen05 (128-row tiles)
+  const bool tc = rp->max_q_len > MSA_MAX_SPEC_DRAFT && Hg <= 128;
+  if (tc) {
+    a.qt = std::min(rp->max_q_len, std::max(1, 128 / Hg));
+    a.tiles = (rp->max_q_len + a.qt - 1) / a.qt;
+    a.chunk = max_blocks;
+    if (static_cast<long long>(rp->batch) * a.tiles > 0x7fffffffLL) return MSA_ERR_UNSUPPORTED;
+    CUtensorMap kmap;
+    if (!page_tensor_map(&kmap, k_idx_cache,
+                         static_cast<long long>(rp->num_pages) * num_idx_k_heads, false))
+      return MSA_ERR_CUDA;
+    return launch_index_scores_tc(kmap, a, reinterpret_cast<cudaStream_t>(stream)) ==
+                   cudaSuccess
+               ? MSA_OK
+               : MSA_ERR_CUDA;
+  }
   a.qt = rp->max_q_len * Hg <= 32 ? rp->max_q_len : (32 / Hg > 0 ? 32 / Hg : 1);
   a.tiles = (rp->max_q_len + a.qt - 1) / a.qt;
   const int mt = a.qt * Hg <= 16 ? 1 : 2;

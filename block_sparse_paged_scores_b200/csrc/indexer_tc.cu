@@ -1,0 +1,249 @@
+// indexer_tc.cu — stage 1 for prefill on the 5th-generation tensor cores (tcgen05 + TMEM).
+//
+// ferrox-core "Module block_sparse", "Four rules": a block's score is the MAX over its
+// positions of the raw dot product q_idx . k_idx (no softmax scale), one index head per KV
+// head.  With many new tokens per sequence the scores of a query tile against every visible
+// page are a dense contraction, so they run on tcgen05: M = 128 rows (tile tokens x the
+// index-query heads that read one index-K head), N = 128 positions of a page, K = 128 dims.
+//
+//   warp 0    producer: TMA loads of the tile's visible index-K pages (128-byte swizzle)
+//             into a 4-stage ring
+//   warp 1    TMEM owner and MMA issuer (one thread): S = Q_idx K_page^T into one of two TMEM
+//             buffers; tcgen05.commit signals the scores
+//   warps 2-5 one row per thread (its TMEM lane): the max of the row over the page's
+//             positions up to the row's query position, written as the block's score; they
+//             release the page's stage and S buffer once read.
+#include <math.h>
+
+#include "attn_common.cuh"
+
+namespace msa {
+
+namespace {
+
+constexpr int kIxRows = 128;
+constexpr uint32_t kIxTile = 32768;  // one (page, head) bf16 tile
+constexpr uint32_t kIxHalf = 16384;  // one swizzled [128][128 B] box
+constexpr int kIxStages = 4;
+constexpr uint32_t kIxQBytes = 2 * kIxHalf;
+constexpr uint32_t kIxCols = 256;  // two 128-column S buffers
+constexpr int kIxThreads = 6 * 32;
+constexpr uint32_t kIdescS = umma_idesc_bf16(128, 128, false);
+
+constexpr size_t ix_smem_bytes() {
+  return 1024 + kIxStages * kIxTile + kIxQBytes +
+         (2 * kIxStages + 2 + 2 + 1) * sizeof(uint64_t) + kIxStages * sizeof(int) + 64;
+}
+
+__device__ __forceinline__ uint64_t ix_kdesc(uint32_t base, int kstep) {
+  return umma_desc_sw128(base + (kstep >> 2) * kIxHalf + (kstep & 3) * 32, 16, 1024);
+}
+
+__global__ void __launch_bounds__(kIxThreads, 1)
+    index_scores_tc_kernel(const __grid_constant__ CUtensorMap kmap, const IndexerArgs a) {
+  pdl_wait();
+  pdl_launch_dependents();
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int b = blockIdx.x / a.tiles, tile = blockIdx.x % a.tiles;
+  const int hk = blockIdx.y;
+  const bool reporter = threadIdx.x == 0 && tile == 0 && hk == 0;
+
+  const int row0 = a.row_off[b];
+  int q_len = a.row_off[b + 1] - row0;
+  if (q_len < 0 || q_len > a.max_q_len) {
+    if (reporter) report(a.dev_err, MSA_DEVERR_LENGTHS);
+    q_len = q_len < 0 ? 0 : a.max_q_len;
+  }
+  const int tok0 = tile * a.qt;
+  if (tok0 >= q_len) return;
+  const int ntok = min(a.qt, q_len - tok0);
+  const int Hg = a.H_kv / a.H_idxk;
+  const int rows = ntok * Hg;
+  int cl = a.cache_len[b];
+  if (cl < 0) {
+    if (reporter) report(a.dev_err, MSA_DEVERR_LENGTHS);
+    cl = 0;
+  }
+  int nb_last = (cl + tok0 + ntok - 1) / kBlock + 1;
+  if (nb_last > a.max_blocks) {
+    if (reporter) report(a.dev_err, MSA_DEVERR_LENGTHS);
+    nb_last = a.max_blocks;
+  }
+  // blocks no token of the tile can see score -inf
+  for (int idx = threadIdx.x; idx < rows * (a.max_blocks - nb_last); idx += blockDim.x) {
+    const int nf = a.max_blocks - nb_last;
+    const int r = idx / nf, j = nb_last + idx % nf;
+    const int t = row0 + tok0 + r / Hg, g = hk + (r % Hg) * a.H_idxk;
+    a.scores[(static_cast<size_t>(t) * a.H_kv + g) * a.max_blocks + j] = -INFINITY;
+  }
+  const int npages = nb_last;
+
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                              ~static_cast<uintptr_t>(1023));
+  uint8_t *stages = smem;
+  uint8_t *qs = stages + kIxStages * kIxTile;
+  uint64_t *st_full = reinterpret_cast<uint64_t *>(qs + kIxQBytes);
+  uint64_t *st_empty = st_full + kIxStages;
+  uint64_t *s_full = st_empty + kIxStages;  // [2]
+  uint64_t *s_free = s_full + 2;            // [2]
+  uint64_t *mma_done = s_free + 2;
+  int *st_ok = reinterpret_cast<int *>(mma_done + 1);
+  uint32_t *tmem_base_s = reinterpret_cast<uint32_t *>(st_ok + kIxStages);
+  volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_base_s + 1);
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kIxStages; ++s) {
+      mbar_init(&st_full[s], 1);
+      mbar_init(&st_empty[s], 4);  // released by the row-max warps, after the MMA read it
+    }
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(&s_full[s], 1);
+      mbar_init(&s_free[s], 4);
+    }
+    mbar_init(mma_done, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_base_s, kIxCols);
+    tmem_relinquish();
+  }
+  // Q_idx rows r = tok * Hg + gi (index-query head hk + gi * H_idxk), K-major 128-byte swizzle
+  for (int idx = threadIdx.x; idx < kIxRows * 16; idx += blockDim.x) {
+    const int r = idx >> 4, chunk = idx & 15;
+    uint4 v = make_uint4(0, 0, 0, 0);
+    if (r < rows) {
+      const int t = row0 + tok0 + r / Hg, g = hk + (r % Hg) * a.H_idxk;
+      v = reinterpret_cast<const uint4 *>(a.q_idx + (static_cast<size_t>(t) * a.H_kv + g) *
+                                                        kHeadDim)[chunk];
+    }
+    *reinterpret_cast<uint4 *>(qs + sw128(r, chunk, kIxHalf)) = v;
+  }
+  fence_async_shared();
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tbase = *tmem_base_s;
+
+  if (warp == 0) {
+    // ============================================================== producer
+    if (lane == 0) prefetch_tmap(&kmap);
+    bool dead = false;
+    for (int base = 0; base < npages && !dead; base += 32) {
+      const int pg_l = base + lane < npages
+                           ? a.table[static_cast<size_t>(b) * a.max_pages + base + lane]
+                           : -1;
+      const int cnt = min(32, npages - base);
+      for (int k = 0; k < cnt; ++k) {
+        const int page = __shfl_sync(0xffffffffu, pg_l, k);
+        if (lane == 0) {
+          const int i = base + k;
+          const int s = i % kIxStages;
+          if (i >= kIxStages &&
+              !mbar_wait(&st_empty[s], ((i / kIxStages) - 1) & 1, abort_flag)) {
+            report(a.dev_err, MSA_DEVERR_TIMEOUT);
+            *abort_flag = 1;
+            dead = true;
+          } else {
+            const bool ok = page >= 0 && page < a.num_pages;
+            st_ok[s] = ok;
+            if (ok) {
+              mbar_arrive_expect_tx(&st_full[s], kIxTile);
+              const int c2 = page * a.H_idxk + hk;
+              tma_load_3d(stages + s * kIxTile, &kmap, &st_full[s], 0, 0, c2);
+              tma_load_3d(stages + s * kIxTile + kIxHalf, &kmap, &st_full[s], 64, 0, c2);
+            } else {
+              report(a.dev_err, MSA_DEVERR_PAGE_ID);
+              mbar_arrive(&st_full[s]);
+            }
+          }
+        }
+        dead = __shfl_sync(0xffffffffu, dead, 0);
+        if (dead) break;
+      }
+    }
+  } else if (warp == 1) {
+    // ============================================================== MMA issuer
+    if (lane == 0) {
+      const uint32_t q_addr = smem_u32(qs);
+      for (int i = 0; i < npages && !*abort_flag; ++i) {
+        const int s = i % kIxStages, sb = i & 1;
+        if (!mbar_wait(&st_full[s], (i / kIxStages) & 1, abort_flag) ||
+            (i >= 2 && !mbar_wait(&s_free[sb], ((i >> 1) - 1) & 1, abort_flag))) {
+          report(a.dev_err, MSA_DEVERR_TIMEOUT);
+          *abort_flag = 1;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t k_addr = smem_u32(stages + s * kIxTile);
+#pragma unroll
+        for (int ks = 0; ks < 8; ++ks)
+          umma_bf16_ss(tbase + sb * 128, ix_kdesc(q_addr, ks), ix_kdesc(k_addr, ks), kIdescS,
+                       ks > 0 ? 1u : 0u);
+        umma_commit(&s_full[sb]);
+      }
+      umma_commit(mma_done);
+      if (!mbar_wait(mma_done, 0, abort_flag)) report(a.dev_err, MSA_DEVERR_TIMEOUT);
+    }
+    __syncwarp();
+  } else {
+    // ============================================================== row-max warps
+    const int quarter = warp & 3;
+    const int r = quarter * 32 + lane;
+    const uint32_t lane_addr = tbase + (static_cast<uint32_t>(quarter * 32) << 16);
+    const bool valid = r < rows;
+    const int tl = r / Hg;
+    const int prow = valid ? cl + tok0 + tl : -1;
+    float *srow = valid ? a.scores + (static_cast<size_t>(row0 + tok0 + tl) * a.H_kv + hk +
+                                      (r % Hg) * a.H_idxk) * a.max_blocks
+                        : nullptr;
+    for (int i = 0; i < npages; ++i) {
+      const int s = i % kIxStages, sb = i & 1;
+      const bool live = mbar_wait(&st_full[s], (i / kIxStages) & 1, abort_flag) &&
+                        mbar_wait(&s_full[sb], (i >> 1) & 1, abort_flag);
+      if (!live) {
+        report(a.dev_err, MSA_DEVERR_TIMEOUT);
+        *abort_flag = 1;
+      }
+      tc_fence_after();
+      const bool use = live && st_ok[s];
+      const int pos0 = i * kBlock;
+      float mx = -INFINITY;
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        uint32_t v[32];
+        tmem_ld32(lane_addr + sb * 128 + c * 32, v);
+        tmem_wait_ld();
+#pragma unroll
+        for (int e = 0; e < 32; ++e)
+          if (use && pos0 + c * 32 + e <= prow) mx = fmaxf(mx, __uint_as_float(v[e]));
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) {
+        mbar_arrive(&s_free[sb]);
+        mbar_arrive(&st_empty[s]);  // the MMA finished with the page before S was signalled
+      }
+      if (valid) srow[i] = mx;
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 1) tmem_dealloc(tbase, kIxCols);
+}
+
+}  // namespace
+
+cudaError_t launch_index_scores_tc(const CUtensorMap &kidx_map, const IndexerArgs &a,
+                                   cudaStream_t s) {
+  const size_t smem = ix_smem_bytes();
+  cudaError_t e = ensure_smem_limit(reinterpret_cast<const void *>(&index_scores_tc_kernel),
+                                    static_cast<int>(smem));
+  if (e != cudaSuccess) return e;
+  const dim3 grid(a.batch * a.tiles, a.H_idxk);
+  return launch_pdl(index_scores_tc_kernel, grid, dim3(kIxThreads), smem, s, kidx_map, a);
+}
+
+}  // namespace msa

@@ -29,6 +29,10 @@ struct IndexerArgs {
 // mt = 16-row MMA tiles per CTA (1 or 2)
 cudaError_t launch_index_scores(const CUtensorMap &kidx_map, const IndexerArgs &a, int mt,
                                 int chunks, cudaStream_t s);
+// prefill on tcgen05 (indexer_tc.cu): tiles of qt tokens x (H_kv / H_idxk) heads <= 128 rows,
+// every visible page of the tile in one CTA
+cudaError_t launch_index_scores_tc(const CUtensorMap &kidx_map, const IndexerArgs &a,
+                                   cudaStream_t s);
 
 // ---- stage 2: selection (select.cu)
 struct SelectArgs {
