@@ -198,6 +198,24 @@ def algorithmic_flops(prob, block_ids, num_selected):
     return idx_flops, attn_flops
 
 
+def executed_flops_tiles(prob, block_ids, num_selected, tile_tokens):
+    """FLOPs a tile-union kernel executes: per (query tile, KV head) every block of the
+    union of its tokens' selections, on full 128-row x 128-position x 128-dim tiles
+    (QK^T and PV)."""
+    import numpy as np
+    ro = prob["row_off"].cpu().numpy()
+    ids = block_ids.cpu().numpy()
+    cnt = num_selected.cpu().numpy()
+    blocks = 0
+    for b in range(prob["batch"]):
+        for t0 in range(ro[b], ro[b + 1], tile_tokens):
+            t1 = min(t0 + tile_tokens, ro[b + 1])
+            for g in range(prob["H_kv"]):
+                sel = [ids[t, g, :cnt[t, g]] for t in range(t0, t1)]
+                blocks += len(np.unique(np.concatenate(sel))) if sel else 0
+    return float(blocks) * 4 * 128 * 128 * 128
+
+
 def source_digest(*names):
     h = hashlib.sha256()
     for n in names:
@@ -415,6 +433,12 @@ def run_ours(args):
                     "algorithmic_flops_per_launch": d_flops,
                     "note": "algorithmic FLOPs (selected, causally clipped positions only) over "
                             "the kernel's time, against the bf16 burst peak"}
+        if dom == "attention" and not fp8:
+            ex = executed_flops_tiles(prob, path.block_ids, path.num_selected,
+                                      128 // (prob["H_q"] // prob["H_kv"]))
+            roofline["executed_flops_per_launch"] = ex
+            roofline["executed_tflops"] = ex / (d_ms * 1e-3) / 1e12
+            roofline["executed_frac"] = ex / (d_ms * 1e-3) / 1e12 / bf16
     else:
         achieved = d_bytes / (d_ms * 1e-3) / 1e9
         roofline = {"bound": "hbm", "kernel": dom, "achieved": achieved, "peak": hbm,
