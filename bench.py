@@ -325,7 +325,9 @@ def run_ours(args):
     stream = torch.cuda.current_stream(dev)
     fp8 = prob["kv_fp8"]
     stream_route = prob["max_q_len"] <= 8  # decode / speculative: persistent kernel + combine
-    kernels_per_step = 3 + (1 if prob["max_q_len"] > 1 else 0) + (1 if stream_route else 0)
+    # decode / speculative: index, select, [plan], attention, combine;
+    # prefill: index, select, plan, attention
+    kernels_per_step = (4 + (1 if prob["max_q_len"] > 1 else 0)) if stream_route else 4
     splits_used = msa.msa_attn_partials(path.rp, prob["S"], prob["H_q"], prob["H_kv"],
                                         path.max_blocks, args.splits)[0] if stream_route else 1
 
@@ -351,23 +353,34 @@ def run_ours(args):
     ms_local = e0.elapsed_time(e1)
     ms = max_over_ranks(ms_local, ws, dev)
 
-    # ---- per-stage durations (separate K-step pass, events between the stages)
-    n_ev = 5
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(n_ev)] for _ in range(args.steps)]
-    for k in range(args.steps):
-        evs[k][0].record(stream)
-        path.index_scores(stream)
-        evs[k][1].record(stream)
-        path.select(stream=stream)
-        evs[k][2].record(stream)
-        path.attend(stream=stream, combine=not stream_route)
-        evs[k][3].record(stream)
-        if stream_route:
-            path.combine(stream)
-        evs[k][4].record(stream)
-    torch.cuda.synchronize(dev)
-    stage_ms = [sum(evs[k][i].elapsed_time(evs[k][i + 1]) for k in range(args.steps)) /
-                args.steps for i in range(n_ev - 1)]
+    # ---- per-stage durations (separate K-step passes, events between the launches)
+    def stage_pass(fns):
+        evs = [[torch.cuda.Event(enable_timing=True) for _ in range(len(fns) + 1)]
+               for _ in range(args.steps)]
+        for k in range(args.steps):
+            evs[k][0].record(stream)
+            for i, fn in enumerate(fns):
+                fn()
+                evs[k][i + 1].record(stream)
+        torch.cuda.synchronize(dev)
+        return [sum(evs[k][i].elapsed_time(evs[k][i + 1]) for k in range(args.steps)) /
+                args.steps for i in range(len(fns))]
+
+    attn_key = "attention" + ("_incl_plan" if prob["max_q_len"] > 1 else "")
+    if stream_route:
+        st = stage_pass([lambda: path.index_scores(stream), lambda: path.select(stream=stream),
+                         lambda: path.attend(stream=stream, combine=False),
+                         lambda: path.combine(stream)])
+        stages = {"index_scores": st[0], "select": st[1], attn_key: st[2], "combine": st[3]}
+        # the first two stages as one msa_index_select launch, for comparison
+        stages["fused_index_select"] = stage_pass([lambda: path.index_select(stream)])[0]
+        idx_kind, idx_src = "index_scores", "indexer.cu"
+    else:
+        st = stage_pass([lambda: path.index_scores(stream), lambda: path.select(stream=stream),
+                         lambda: path.attend(stream=stream)])
+        stages = {"index_scores": st[0], "select": st[1], attn_key: st[2]}
+        idx_kind, idx_src = "index_scores", "indexer_tc.cu"
+    idx_ms, attn_ms = st[0], stages[attn_key]
     if sampler:
         sampler.stop()
     clocks = sampler.summary(t_wall0, t_wall1) if sampler else None
@@ -416,8 +429,8 @@ def run_ours(args):
         return 0
     hbm, bf16, bf16_sus, peak_src = measured_peaks()
     tensor_route = prob["max_q_len"] > 8  # prefill: dense contractions on the tensor cores
-    kinds = {"index_scores": (stage_ms[0], idx_bytes, "indexer.cu"),
-             "attention": (stage_ms[2], attn_bytes,
+    kinds = {idx_kind: (idx_ms, idx_bytes, idx_src),
+             "attention": (attn_ms, attn_bytes,
                            "attention_stream.cu" if stream_route else
                            ("attention_tile.cu" if fp8 else "attention_tc.cu"))}
     dom = max(kinds, key=lambda k: kinds[k][0])
@@ -465,9 +478,7 @@ def run_ours(args):
                      / 1e9 / hbm,
                      "frac_of_8TBps": (idx_bytes + attn_bytes) / (ms / args.steps * 1e-3)
                      / 8e12},
-        "stages_ms": {"index_scores": stage_ms[0], "select": stage_ms[1],
-                      "attention" + ("_incl_plan" if prob["max_q_len"] > 1 else ""): stage_ms[2],
-                      "combine": stage_ms[3]},
+        "stages_ms": stages,
         "gpu_launches": kernels_per_step * args.steps,
         "clocks": clocks,
         "e2e": {"value": tokens_total / (e2e_ms * 1e-3), "unit": UNIT,

@@ -252,11 +252,22 @@ int32_t msa_attn_partials(const msa_ragged_paged_t *rp, int32_t S, int32_t num_q
   return r.splits;
 }
 
-msa_status_t msa_index_scores(const msa_ragged_paged_t *rp, const void *q_idx,
-                              const void *k_idx_cache, int32_t num_kv_heads,
-                              int32_t num_idx_k_heads, int32_t max_blocks, float *scores,
-                              int32_t *dev_err, struct CUstream_st *stream) {
-  if (ragged_ok(rp) && rp->total_q == 0) return MSA_OK;  // nothing to score
+namespace {
+
+// The selection to fuse into the decode indexer (nullptr: scores only).
+struct FusedSelect {
+  int32_t *counters, *block_ids, *num_selected;
+  int top_k, init_blocks, local_blocks, S;
+};
+
+bool index_uses_tc(const msa_ragged_paged_t *rp, int Hg) {
+  return rp->max_q_len > MSA_MAX_SPEC_DRAFT && Hg <= 128;
+}
+
+msa_status_t index_scores_impl(const msa_ragged_paged_t *rp, const void *q_idx,
+                               const void *k_idx_cache, int32_t num_kv_heads,
+                               int32_t num_idx_k_heads, int32_t max_blocks, float *scores,
+                               int32_t *dev_err, cudaStream_t stream, const FusedSelect *fs) {
   if (!ragged_ok(rp) || !q_idx || !k_idx_cache || !scores || num_kv_heads < 1 ||
       !(num_idx_k_heads == 1 || num_idx_k_heads == num_kv_heads) || max_blocks < 1 ||
       max_blocks > rp->max_pages_per_seq || !aligned(k_idx_cache, 16) || !aligned(q_idx, 4))
@@ -266,7 +277,7 @@ msa_status_t msa_index_scores(const msa_ragged_paged_t *rp, const void *q_idx,
   if (static_cast<long long>(rp->num_pages) * num_idx_k_heads >= (1LL << 31))
     return MSA_ERR_UNSUPPORTED;
 
-  IndexerArgs a;
+  IndexerArgs a{};
   a.row_off = rp->input_row_offsets;
   a.cache_len = rp->cache_lengths;
   a.table = rp->kv_lookup_table;
@@ -280,9 +291,10 @@ msa_status_t msa_index_scores(const msa_ragged_paged_t *rp, const void *q_idx,
   a.H_kv = num_kv_heads;
   a.H_idxk = num_idx_k_heads;
   a.max_blocks = max_blocks;
+  a.counters = nullptr;
   // prefill: the dense tile x page contraction runs on tcgen05 (128-row tiles)
-  const bool tc = rp->max_q_len > MSA_MAX_SPEC_DRAFT && Hg <= 128;
-  if (tc) {
+  if (index_uses_tc(rp, Hg)) {
+    if (fs) return MSA_ERR_UNSUPPORTED;  // the caller selects with a separate launch
     a.qt = std::min(rp->max_q_len, std::max(1, 128 / Hg));
     a.tiles = (rp->max_q_len + a.qt - 1) / a.qt;
     a.chunk = max_blocks;
@@ -291,10 +303,7 @@ msa_status_t msa_index_scores(const msa_ragged_paged_t *rp, const void *q_idx,
     if (!page_tensor_map(&kmap, k_idx_cache,
                          static_cast<long long>(rp->num_pages) * num_idx_k_heads, false))
       return MSA_ERR_CUDA;
-    return launch_index_scores_tc(kmap, a, reinterpret_cast<cudaStream_t>(stream)) ==
-                   cudaSuccess
-               ? MSA_OK
-               : MSA_ERR_CUDA;
+    return launch_index_scores_tc(kmap, a, stream) == cudaSuccess ? MSA_OK : MSA_ERR_CUDA;
   }
   a.qt = rp->max_q_len * Hg <= 32 ? rp->max_q_len : (32 / Hg > 0 ? 32 / Hg : 1);
   a.tiles = (rp->max_q_len + a.qt - 1) / a.qt;
@@ -306,20 +315,72 @@ msa_status_t msa_index_scores(const msa_ragged_paged_t *rp, const void *q_idx,
   long long chunk = (max_blocks + want - 1) / want;
   if (chunk < 4) chunk = 4;
   long long chunks = (max_blocks + chunk - 1) / chunk;
-  if (chunks > 65535) {
-    chunks = 65535;
-    chunk = (max_blocks + chunks - 1) / chunks;
-  }
   a.chunk = static_cast<int>(chunk);
+  a.chunks = static_cast<int>(chunks);
+  if (units * chunks > 0x7fffffffLL) return MSA_ERR_UNSUPPORTED;
+  if (fs) {
+    a.counters = fs->counters;
+    a.block_ids = fs->block_ids;
+    a.num_selected = fs->num_selected;
+    a.top_k = fs->top_k;
+    a.init_blocks = fs->init_blocks;
+    a.local_blocks = fs->local_blocks;
+    a.S = fs->S;
+  }
 
   CUtensorMap kmap;
   if (!page_tensor_map(&kmap, k_idx_cache, static_cast<long long>(rp->num_pages) * num_idx_k_heads,
                        false))
     return MSA_ERR_CUDA;
-  return launch_index_scores(kmap, a, mt, static_cast<int>(chunks),
-                             reinterpret_cast<cudaStream_t>(stream)) == cudaSuccess
+  return launch_index_scores(kmap, a, mt, static_cast<int>(chunks), stream) == cudaSuccess
              ? MSA_OK
              : MSA_ERR_CUDA;
+}
+
+}  // namespace
+
+msa_status_t msa_index_scores(const msa_ragged_paged_t *rp, const void *q_idx,
+                              const void *k_idx_cache, int32_t num_kv_heads,
+                              int32_t num_idx_k_heads, int32_t max_blocks, float *scores,
+                              int32_t *dev_err, struct CUstream_st *stream) {
+  if (ragged_ok(rp) && rp->total_q == 0) return MSA_OK;  // nothing to score
+  return index_scores_impl(rp, q_idx, k_idx_cache, num_kv_heads, num_idx_k_heads, max_blocks,
+                           scores, dev_err, reinterpret_cast<cudaStream_t>(stream), nullptr);
+}
+
+size_t msa_index_select_counters(const msa_ragged_paged_t *rp, int32_t num_idx_k_heads) {
+  if (!ragged_ok(rp) || num_idx_k_heads < 1) return 0;
+  return static_cast<size_t>(rp->batch) * rp->max_q_len * num_idx_k_heads;
+}
+
+msa_status_t msa_index_select(const msa_ragged_paged_t *rp, const void *q_idx,
+                              const void *k_idx_cache, int32_t num_kv_heads,
+                              int32_t num_idx_k_heads, int32_t max_blocks, int32_t top_k,
+                              int32_t init_blocks, int32_t local_blocks, float *scores,
+                              int32_t *block_ids, int32_t *num_selected, int32_t *counters,
+                              int32_t *dev_err, struct CUstream_st *stream) {
+  const long long S = static_cast<long long>(top_k) + init_blocks + local_blocks;
+  if (!ragged_ok(rp) || num_kv_heads < 1 || num_idx_k_heads < 1 || max_blocks < 1 ||
+      top_k < 0 || init_blocks < 0 || local_blocks < 0 || S < 1 || S > (1 << 20))
+    return MSA_ERR_INVALID_ARG;
+  if (rp->total_q == 0) return MSA_OK;
+  if (!block_ids || !num_selected) return MSA_ERR_INVALID_ARG;
+  const cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const bool fused = num_kv_heads % num_idx_k_heads == 0 &&
+                     !index_uses_tc(rp, num_kv_heads / num_idx_k_heads);
+  if (fused) {
+    if (!counters || !aligned(counters, 4)) return MSA_ERR_INVALID_ARG;
+    const FusedSelect fs{counters, block_ids, num_selected, top_k, init_blocks, local_blocks,
+                         static_cast<int>(S)};
+    return index_scores_impl(rp, q_idx, k_idx_cache, num_kv_heads, num_idx_k_heads, max_blocks,
+                             scores, dev_err, st, &fs);
+  }
+  const msa_status_t e = index_scores_impl(rp, q_idx, k_idx_cache, num_kv_heads,
+                                           num_idx_k_heads, max_blocks, scores, dev_err, st,
+                                           nullptr);
+  if (e != MSA_OK) return e;
+  return msa_select_blocks(rp, scores, num_kv_heads, max_blocks, top_k, init_blocks,
+                           local_blocks, block_ids, num_selected, dev_err, stream);
 }
 
 msa_status_t msa_select_blocks(const msa_ragged_paged_t *rp, const float *scores,

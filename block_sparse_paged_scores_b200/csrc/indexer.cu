@@ -12,10 +12,14 @@
 // S = Q K^T with bf16 mma.sync (fp32 accumulation), mask positions after each row's query
 // position, reduce the row max with warp shuffles and then across the four warps through
 // shared memory, and write one fp32 score per (row, page).
+//
+// With the selection fused in (decode and speculative routes), the CTAs of one (sequence,
+// tile, index-K head) count themselves out on a device counter once their scores are written;
+// the last one runs stage 2 for the unit's rows (select_row.cuh, reading the scores from L2) and
+// puts the counter back to zero, so no separate selection launch is needed.
 #include <math.h>
 
-#include "internal.h"
-#include "ptx.cuh"
+#include "select_row.cuh"
 
 namespace msa {
 
@@ -31,14 +35,53 @@ constexpr size_t smem_bytes() {
          kStages * sizeof(int) + 2 * kConsumerWarps * 32 * sizeof(float) + 16;
 }
 
-template <int MT>
+// The consumer warps (threads 0..127) of every CTA of a unit call this once the CTA's scores
+// are written; the last CTA to arrive selects for the unit's rows.
+template <int KPL>
+__device__ __forceinline__ void count_out_and_select(const IndexerArgs &a, int b, int tile,
+                                                     int hk, int row0, int tok0, int ntok,
+                                                     int cl, volatile int *is_last) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  named_bar_sync(2, kConsumerWarps * 32);  // every thread's scores written
+  if (threadIdx.x == 0) {
+    int32_t *c = a.counters + (static_cast<size_t>(b) * a.tiles + tile) * a.H_idxk + hk;
+    __threadfence();  // the CTA's scores (ordered before by the barrier), before the count
+    const bool last = atomicAdd(c, 1) == a.chunks - 1;
+    if (last) {
+      __threadfence();  // every other CTA's scores, before this CTA reads them
+      atomicExch(c, 0);
+    }
+    *is_last = last;
+  }
+  named_bar_sync(2, kConsumerWarps * 32);
+  if (!*is_last) return;
+  const int Hg = a.H_kv / a.H_idxk;
+  for (int r = warp; r < ntok * Hg; r += kConsumerWarps) {
+    const int tl = r / Hg, g = hk + (r % Hg) * a.H_idxk;
+    const size_t item = static_cast<size_t>(row0 + tok0 + tl) * a.H_kv + g;
+    const int nb = min((cl + tok0 + tl) / kBlock + 1, a.max_blocks);
+    const int nsel =
+        select_row<(KPL > 0 ? KPL : 0), true>(a.scores + item * a.max_blocks, nb, a.top_k,
+                                              a.init_blocks, a.local_blocks, a.S,
+                                              a.block_ids + item * a.S, a.dev_err, lane);
+    if (lane == 0) a.num_selected[item] = nsel;
+  }
+}
+
+// KPL < 0: scores only; KPL >= 0: selection fused, KPL keys per lane in registers (0: any
+// number of blocks, read from L2 on every pass).
+template <int MT, int KPL>
 __global__ void __launch_bounds__(kThreads)
     index_scores_kernel(const __grid_constant__ CUtensorMap kmap, const IndexerArgs a) {
   pdl_wait();
   pdl_launch_dependents();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int cx = blockIdx.y, b = blockIdx.x / a.tiles, tile = blockIdx.x % a.tiles;
-  const int hk = blockIdx.z;
+  // one CTA per (chunk, unit); a unit's chunks are launched together so that units finish one
+  // after another (and, fused, select while later units are still scoring)
+  const int cx = blockIdx.x % a.chunks;
+  const int unit = blockIdx.x / a.chunks;  // (b * tiles + tile) * H_idxk + hk
+  const int hk = unit % a.H_idxk, bt = unit / a.H_idxk;
+  const int b = bt / a.tiles, tile = bt % a.tiles;
   const bool reporter = threadIdx.x == 0 && cx == 0 && tile == 0 && hk == 0;
 
   const int row0 = a.row_off[b];
@@ -76,7 +119,6 @@ __global__ void __launch_bounds__(kThreads)
     }
   }
   const int npages = j1 - j0;
-  if (npages <= 0) return;
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -87,6 +129,16 @@ __global__ void __launch_bounds__(kThreads)
   int *page_ok = reinterpret_cast<int *>(empty + kStages);
   float *red = reinterpret_cast<float *>(page_ok + kStages);  // [2][4 warps][32 rows]
   volatile int *abort_flag = reinterpret_cast<volatile int *>(red + 2 * kConsumerWarps * 32);
+  volatile int *is_last = abort_flag + 1;
+
+  if (npages <= 0) {
+    if (KPL >= 0) {
+      __syncthreads();  // every thread's -inf fills, before the count
+      if (warp < kConsumerWarps)
+        count_out_and_select<KPL>(a, b, tile, hk, row0, tok0, ntok, cl, is_last);
+    }
+    return;
+  }
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) {
@@ -235,20 +287,35 @@ __global__ void __launch_bounds__(kThreads)
       a.scores[(static_cast<size_t>(t) * a.H_kv + g) * a.max_blocks + j] = m;
     }
   }
+  if (KPL >= 0) count_out_and_select<KPL>(a, b, tile, hk, row0, tok0, ntok, cl, is_last);
+}
+
+template <int MT, int KPL>
+cudaError_t launch_one(const CUtensorMap &kidx_map, const IndexerArgs &a, int chunks,
+                       cudaStream_t s) {
+  const dim3 grid(a.batch * a.tiles * a.H_idxk * chunks);
+  const size_t smem = smem_bytes();
+  cudaError_t e = ensure_smem_limit(reinterpret_cast<const void *>(&index_scores_kernel<MT, KPL>),
+                                    static_cast<int>(smem));
+  if (e != cudaSuccess) return e;
+  return launch_pdl(index_scores_kernel<MT, KPL>, grid, dim3(kThreads), smem, s, kidx_map, a);
+}
+
+template <int MT>
+cudaError_t launch_mt(const CUtensorMap &kidx_map, const IndexerArgs &a, int chunks,
+                      cudaStream_t s) {
+  if (!a.counters) return launch_one<MT, -1>(kidx_map, a, chunks, s);
+  if (a.max_blocks <= 4 * 32) return launch_one<MT, 4>(kidx_map, a, chunks, s);
+  if (a.max_blocks <= 16 * 32) return launch_one<MT, 16>(kidx_map, a, chunks, s);
+  if (a.max_blocks <= 32 * 32) return launch_one<MT, 32>(kidx_map, a, chunks, s);
+  return launch_one<MT, 0>(kidx_map, a, chunks, s);
 }
 
 }  // namespace
 
 cudaError_t launch_index_scores(const CUtensorMap &kidx_map, const IndexerArgs &a, int mt,
                                 int chunks, cudaStream_t s) {
-  const dim3 grid(a.batch * a.tiles, chunks, a.H_idxk);
-  const size_t smem = smem_bytes();
-  const void *fn = mt == 1 ? reinterpret_cast<const void *>(&index_scores_kernel<1>)
-                           : reinterpret_cast<const void *>(&index_scores_kernel<2>);
-  cudaError_t e = ensure_smem_limit(fn, static_cast<int>(smem));
-  if (e != cudaSuccess) return e;
-  if (mt == 1) return launch_pdl(index_scores_kernel<1>, grid, dim3(kThreads), smem, s, kidx_map, a);
-  return launch_pdl(index_scores_kernel<2>, grid, dim3(kThreads), smem, s, kidx_map, a);
+  return mt == 1 ? launch_mt<1>(kidx_map, a, chunks, s) : launch_mt<2>(kidx_map, a, chunks, s);
 }
 
 }  // namespace msa

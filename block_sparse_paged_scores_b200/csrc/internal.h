@@ -24,7 +24,14 @@ struct IndexerArgs {
   int batch, max_q_len, max_pages, num_pages, H_kv, H_idxk, max_blocks;
   int qt;     // query tokens per tile
   int tiles;  // tiles per sequence
-  int chunk;  // pages per CTA
+  int chunk;   // pages per CTA
+  int chunks;  // CTAs per (sequence, tile, index-K head)
+  // Selection fused into the decode indexer (counters == nullptr: scores only).  The CTAs of one
+  // (sequence, tile, index-K head) count themselves out on counters[(b * tiles + tile) * H_idxk
+  // + hk]; the last one selects for the unit's rows and puts the counter back to zero.
+  int32_t *counters;
+  int32_t *block_ids, *num_selected;  // [total_q, H_kv, S], [total_q, H_kv]
+  int top_k, init_blocks, local_blocks, S;
 };
 // mt = 16-row MMA tiles per CTA (1 or 2)
 cudaError_t launch_index_scores(const CUtensorMap &kidx_map, const IndexerArgs &a, int mt,

@@ -55,6 +55,10 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.msa_index_scores.argtypes = [RP, P, P, I, I, I, P, P, P]
     lib.msa_select_blocks.restype = I
     lib.msa_select_blocks.argtypes = [RP, P, I, I, I, I, I, P, P, P, P]
+    lib.msa_index_select.restype = I
+    lib.msa_index_select.argtypes = [RP, P, P, I, I, I, I, I, I, P, P, P, P, P, P]
+    lib.msa_index_select_counters.restype = ctypes.c_size_t
+    lib.msa_index_select_counters.argtypes = [RP, I]
     lib.msa_sparse_attn_paged.restype = I
     lib.msa_sparse_attn_paged.argtypes = [RP, P, P, P, I, P, P, I, I, I, I, F, I, P,
                                           ctypes.c_size_t, P, P, P]
@@ -146,6 +150,20 @@ def msa_select_blocks(rp: RaggedPaged, scores, num_kv_heads: int, max_blocks: in
         local_blocks, _ptr(block_ids), _ptr(num_selected), _ptr(dev_err), _stream(stream)))
 
 
+def msa_index_select_counters(rp: RaggedPaged, num_idx_k_heads: int) -> int:
+    return int(load().msa_index_select_counters(ctypes.byref(rp), num_idx_k_heads))
+
+
+def msa_index_select(rp: RaggedPaged, q_idx, k_idx_cache, num_kv_heads: int,
+                     num_idx_k_heads: int, max_blocks: int, top_k: int, init_blocks: int,
+                     local_blocks: int, scores, block_ids, num_selected, counters, dev_err=None,
+                     stream=None):
+    _check("msa_index_select", load().msa_index_select(
+        ctypes.byref(rp), _ptr(q_idx), _ptr(k_idx_cache), num_kv_heads, num_idx_k_heads,
+        max_blocks, top_k, init_blocks, local_blocks, _ptr(scores), _ptr(block_ids),
+        _ptr(num_selected), _ptr(counters), _ptr(dev_err), _stream(stream)))
+
+
 def msa_sparse_attn_paged(rp: RaggedPaged, q, k_cache, v_cache, kv_dtype: int, block_ids,
                           num_selected, S: int, num_q_heads: int, num_kv_heads: int,
                           max_blocks: int, scale: float, num_splits: int, workspace, out,
@@ -181,10 +199,13 @@ def msa_splitk_combine(partial_o, partial_lse, num_splits: int, total_q: int, nu
 class Path:
     """The three stages over one problem (a dict laid out as ``workload.generate`` returns),
     with every output and the workspace allocated once on the problem's device.  ``run()``
-    enqueues index scores -> selection -> attention on the current stream."""
+    enqueues index scores -> selection -> attention on the current stream (with
+    ``fused_select`` the first two as one msa_index_select call)."""
 
-    def __init__(self, prob: dict, num_splits: int = 0, max_blocks: Optional[int] = None):
+    def __init__(self, prob: dict, num_splits: int = 0, max_blocks: Optional[int] = None,
+                 fused_select: bool = False):
         self.p = prob
+        self.fused_select = fused_select
         dev = prob["q"].device
         self.max_blocks = int(max_blocks or prob["max_blocks"])
         self.rp = ragged_paged(prob["row_off"], prob["cache_len"], prob["table"], prob["total_q"],
@@ -200,11 +221,21 @@ class Path:
         self.workspace = torch.empty((max(ws, 1),), dtype=torch.uint8, device=dev)
         self.workspace_bytes = ws
         self.kv_dtype = MSA_KV_FP8_E4M3 if prob["kv_fp8"] else MSA_KV_BF16
+        nc = msa_index_select_counters(self.rp, prob["H_idxk"])
+        self.counters = torch.zeros((max(nc, 1),), dtype=torch.int32, device=dev)
 
     def index_scores(self, stream=None):
         p = self.p
         msa_index_scores(self.rp, p["q_idx"], p["k_idx"], p["H_kv"], p["H_idxk"], self.max_blocks,
                          self.scores, self.dev_err, stream)
+
+    def index_select(self, stream=None):
+        """Stages 1 and 2 in one call (one launch on the decode / speculative routes)."""
+        p = self.p
+        msa_index_select(self.rp, p["q_idx"], p["k_idx"], p["H_kv"], p["H_idxk"],
+                         self.max_blocks, p["top_k"], p["init_blocks"], p["local_blocks"],
+                         self.scores, self.block_ids, self.num_selected, self.counters,
+                         self.dev_err, stream)
 
     def select(self, scores=None, stream=None):
         p = self.p
@@ -233,7 +264,10 @@ class Path:
         msa_splitk_combine(o_ptr, l_ptr, n, self.p["total_q"], self.p["H_q"], self.out, stream)
 
     def run(self, stream=None):
-        self.index_scores(stream)
-        self.select(stream=stream)
+        if self.fused_select:
+            self.index_select(stream)
+        else:
+            self.index_scores(stream)
+            self.select(stream=stream)
         self.attend(stream=stream)
         return self.out

@@ -5,6 +5,7 @@
  * The path has three stages, one entry point each, plus the split-K combine:
  *   msa_index_scores      block scores: max over a 128-token block of raw q_idx . k_idx
  *   msa_select_blocks     forced init/local blocks + top-k of the rest, ascending
+ *   msa_index_select      the first two in one call (one launch on the decode routes)
  *   msa_sparse_attn_paged softmax attention over the selected pages (decode / speculative /
  *                         prefill routes picked from max_q_len), split-K + combine inside
  *   msa_splitk_combine    log-sum-exp merge of split-K partials into the ragged output
@@ -130,6 +131,35 @@ MSA_API msa_status_t msa_select_blocks(const msa_ragged_paged_t *rp, const float
                                int32_t init_blocks, int32_t local_blocks, int32_t *block_ids,
                                int32_t *num_selected, int32_t *dev_err,
                                struct CUstream_st *stream);
+
+/*
+ * msa_index_select — stages 1 and 2 in one call: exactly msa_index_scores followed by
+ * msa_select_blocks with the same arguments ([ferrox] "Four rules"; block_sparse_select), with
+ * bit-identical scores, block_ids and num_selected.
+ *
+ * On the decode and speculative routes (max_q_len <= MSA_MAX_SPEC_DRAFT) it is one launch: the
+ * CTAs that score one (sequence, tile of query tokens, index-K head) count themselves out on
+ * `counters`, and the last one selects for that unit's rows, so the selection needs no launch
+ * of its own.  On the prefill route it enqueues the two stages one after the other and does not
+ * touch `counters`.
+ *
+ *   scores, block_ids, num_selected  as msa_index_scores / msa_select_blocks (all outputs;
+ *                  `scores` stays valid after the call, as the selection's input)
+ *   counters      device int32 [msa_index_select_counters(rp, num_idx_k_heads)], 4-byte
+ *                 aligned, owned by the caller.  It must be all zero when the call's kernel
+ *                 starts; the kernel leaves it all zero when it ends, so the caller zeroes it
+ *                 once and reuses it.  Two calls in flight at once (on different streams) must
+ *                 not share one counters array: their counts would mix.  Required on the decode
+ *                 and speculative routes (MSA_ERR_INVALID_ARG when NULL there).
+ *   Validation is that of both stages; max_blocks <= max_pages_per_seq.
+ */
+MSA_API size_t msa_index_select_counters(const msa_ragged_paged_t *rp, int32_t num_idx_k_heads);
+MSA_API msa_status_t msa_index_select(const msa_ragged_paged_t *rp, const void *q_idx,
+                              const void *k_idx_cache, int32_t num_kv_heads,
+                              int32_t num_idx_k_heads, int32_t max_blocks, int32_t top_k,
+                              int32_t init_blocks, int32_t local_blocks, float *scores,
+                              int32_t *block_ids, int32_t *num_selected, int32_t *counters,
+                              int32_t *dev_err, struct CUstream_st *stream);
 
 /*
  * msa_sparse_attn_paged — stage 3 ([ferrox] positions_of_blocks: the selected blocks'

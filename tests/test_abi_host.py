@@ -113,6 +113,18 @@ def test_invalid_arguments_are_rejected_before_any_launch(lib):
     assert stat == msa.MSA_ERR_UNSUPPORTED
     stat = lib.msa_select_blocks(ctypes.byref(rp), P, 8, 16, 0, 0, 0, P, P, None, None)  # S = 0
     assert stat == msa.MSA_ERR_INVALID_ARG
+    # fused index + select: the decode route needs counters; S = 0 and null outputs rejected
+    fused = lambda **kw: lib.msa_index_select(
+        ctypes.byref(kw.get("rp", rp)), P, P, 8, 1, 16, kw.get("top_k", 4), 1, 1,
+        kw.get("scores", P), kw.get("ids", P), P, kw.get("counters", P), None, None)
+    assert fused(counters=None) == msa.MSA_ERR_INVALID_ARG
+    assert fused(top_k=-1) == msa.MSA_ERR_INVALID_ARG
+    assert fused(scores=None) == msa.MSA_ERR_INVALID_ARG
+    assert fused(ids=None) == msa.MSA_ERR_INVALID_ARG
+    assert fused(counters=P + 2) == msa.MSA_ERR_INVALID_ARG
+    assert lib.msa_index_select(ctypes.byref(rp), P, P, 8, 1, 16, 0, 0, 0, P, P, P, P, None,
+                                None) == msa.MSA_ERR_INVALID_ARG                   # S = 0
+    assert msa.msa_index_select_counters(_rp(batch=5, max_q_len=3, total_q=9), 8) == 5 * 3 * 8
     stat = lib.msa_select_blocks(ctypes.byref(rp), P, 8, 16, -1, 1, 1, P, P, None, None)
     assert stat == msa.MSA_ERR_INVALID_ARG
     bad = msa.RaggedPaged(P, P, P, 0, 2, 1, 16, 64)                                 # batch 0

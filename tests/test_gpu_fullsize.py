@@ -75,6 +75,17 @@ def test_full_size_workload(name):
     assert not torch.isnan(out.float()).any()
     _check_rules_on_gpu_scores(prob, scores, ids, cnt)
 
+    # the first two stages as one msa_index_select call: the same scores and selection
+    fused = msa.Path(prob, fused_select=True)
+    fused.index_select()
+    torch.cuda.synchronize()
+    assert int(fused.dev_err.item()) == 0
+    assert np.array_equal(fused.scores.cpu().numpy(), scores)
+    assert np.array_equal(fused.block_ids.cpu().numpy(), ids)
+    assert np.array_equal(fused.num_selected.cpu().numpy(), cnt)
+    assert int(fused.counters.abs().sum().item()) == 0
+    del fused
+
     # the same step again: every output bit-identical
     for _ in range(3):
         path.run()

@@ -203,6 +203,52 @@ def test_selection_edge_parameters(top_k, init, local):
     check_attention(path.out.float().cpu(), out, False)
 
 
+@pytest.mark.parametrize("name", sorted(CASES))
+def test_fused_index_select_equals_the_two_stages(name):
+    p = _gpu(_problem(name))
+    two, one = msa.Path(p), msa.Path(p)
+    two.index_scores()
+    two.select()
+    for _ in range(2):  # the counters must come back to zero for the second call
+        one.index_select()
+    torch.cuda.synchronize()
+    assert int(two.dev_err.item()) == 0 and int(one.dev_err.item()) == 0
+    assert torch.equal(one.scores, two.scores)
+    assert torch.equal(one.num_selected, two.num_selected)
+    assert torch.equal(one.block_ids, two.block_ids)
+    assert int(one.counters.abs().sum().item()) == 0
+
+
+def _pad_table(p, max_pages):
+    t = p["table"]
+    pad = torch.full((t.shape[0], max_pages - t.shape[1]), -1, dtype=t.dtype, device=t.device)
+    return dict(p, table=torch.cat([t, pad], 1))
+
+
+@pytest.mark.parametrize("top_k,init,local", [(0, 1, 1), (3, 0, 0), (0, 0, 2), (500, 1, 2),
+                                              (5, 7, 0), (16, 1, 2)])
+@pytest.mark.parametrize("name,max_blocks", [("spec_ragged_q", 0), ("bf16_decode", 0),
+                                             ("spec_decode", 300), ("bf16_decode", 700),
+                                             ("short_contexts", 1100)])
+def test_fused_selection_is_bit_exact(name, max_blocks, top_k, init, local):
+    """The fused selection against the oracle's, on the GPU's own scores; a wide score row
+    (max_blocks 700 / 1100) takes the 32-key and the from-memory key variants."""
+    p = _gpu(_problem(name))
+    p = dict(p, top_k=top_k, init_blocks=init, local_blocks=local, S=top_k + init + local)
+    if max_blocks:
+        p = _pad_table(p, max_blocks)
+    path = msa.Path(p, max_blocks=max_blocks or None)
+    path.index_select()
+    torch.cuda.synchronize()
+    assert int(path.dev_err.item()) == 0
+    sc = path.scores.cpu().numpy().astype(np.float64)
+    ids, cnt = oracle.select_blocks(p["row_off"].cpu().numpy(), p["cache_len"].cpu().numpy(), sc,
+                                    top_k, init, local)
+    assert np.array_equal(path.num_selected.cpu().numpy(), cnt)
+    assert np.array_equal(path.block_ids.cpu().numpy(), ids)
+    assert int(path.counters.abs().sum().item()) == 0
+
+
 def test_empty_batch_is_a_no_op():
     p = _gpu(_oracle("tiny_decode")[0])
     empty = dict(p, row_off=torch.zeros(2, dtype=torch.int32, device="cuda"), total_q=0)
