@@ -214,6 +214,17 @@ __device__ __forceinline__ void umma_bf16_ss(uint32_t tmem_d, uint64_t adesc, ui
       "r"(z), "r"(z)
       : "memory");
 }
+// D[tmem] (+)= A[tmem] * B[smem], issued by one thread.  A (M = 128 rows, K-major) sits in
+// TMEM: row m in lane m, two bf16 of K per 32-bit column; tmem_a points at the K-slice's first
+// column.
+__device__ __forceinline__ void umma_bf16_ts(uint32_t tmem_d, uint32_t tmem_a, uint64_t bdesc,
+                                             uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}"
+      ::"r"(tmem_d), "r"(tmem_a), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
 // Arrive on `bar` once every tcgen05 operation this thread issued before has completed.
 __device__ __forceinline__ void umma_commit(uint64_t *bar) {
   asm volatile(
