@@ -13,21 +13,22 @@
 //   warp 0     K producer: TMA loads of each block's K page tile (128-byte swizzle) into a
 //              3-stage ring, freed as soon as the block's S is computed
 //   warp 10    V producer: the V page tiles into a 2-stage ring, freed by the block's P V
-//   warp 1     TMEM owner and MMA issuer (one thread): S = Q K^T into one of three TMEM S
-//              buffers (M = N = 128, K = 16 x 8); O += P V with P read from TMEM where the
-//              softmax left it (over its S) and V as an N-major shared-memory operand;
-//              tcgen05.commit signals each
-//   warps 2-9  softmax, two warpgroups: thread (row r, half h) owns positions 64 h .. 64 h + 63
-//              of row r (its TMEM lane); one pass over S: masked partial max, the row max
-//              through shared memory, exp2 in place, P as bf16 back into TMEM over the S it
-//              came from.  The running max m only moves when a block's max exceeds it by more
-//              than 2^8 (then O is rescaled in TMEM once the previous P V is done); in between
-//              P = 2^(s - m) stays <= 2^8, well inside bf16 and fp32 range.  Zeroes
-//              the rows of a last page past the sequence end in V (0 * NaN is NaN); epilogue
-//              O / l -> bf16, each half writing its 64 dims.
+//   warp 1     TMEM owner and MMA issuer (one thread): S = Q K^T (M = N = 128, K = 16 x 8) and
+//              O += P V with P read from TMEM where the softmax left it (over its S) and V as
+//              an N-major shared-memory operand; tcgen05.commit signals each
+//   warps 2-9  softmax, two warpgroups taking alternate blocks (even / odd), each with its own
+//              S buffer, O accumulator and running max and sum: one query row per thread (its
+//              TMEM lane), one pass over the row's 128 scores (masked max, exp2, P as bf16 back
+//              into TMEM over its S).  The groups never wait for each other inside the loop, so
+//              one group's exponentials overlap the other's loads and maxima.  A group's
+//              running max only moves when a block's max exceeds it by more than 2^8 (then its
+//              O is rescaled in TMEM); in between P = 2^(s - m) stays <= 2^8, well inside bf16
+//              and fp32 range.  Zeroes the rows of a last page past the sequence end in V
+//              (0 * NaN is NaN).  Epilogue: the two groups' (m, l, O) merged by log-sum-exp,
+//              O / l -> bf16, each group writing 64 of the 128 dims.
 //
-// TMEM columns: S/P buffers [0, 128), [128, 256), [256, 384); O [384, 512).  P of buffer b
-// holds positions 0-63 in columns 128 b + [0, 32) and 64-127 in 128 b + [64, 96).
+// TMEM columns: S/P of group 0 [0, 128) and group 1 [128, 256) (P of a block in the first 64
+// columns of its S), O of group 0 [256, 384) and group 1 [384, 512).
 #include <math.h>
 
 #include "attn_common.cuh"
@@ -43,8 +44,7 @@ constexpr int kKStages = 3;
 constexpr int kVStages = 2;
 constexpr uint32_t kTcQBytes = 2 * kTcHalf;      // Q: 128 rows x 128 dims bf16
 constexpr uint32_t kTcCols = 512;                // TMEM columns allocated
-constexpr int kSBufs = 3;
-constexpr uint32_t kColO = 384;
+constexpr uint32_t kColO = 256;                  // + 128 per group
 constexpr int kSoftWarps = 8;
 constexpr int kSoftThreads = 32 * kSoftWarps;
 constexpr int kVWarp = 2 + kSoftWarps;
@@ -53,8 +53,8 @@ constexpr float kLazyLog2 = 8.f;                 // rescale only when the max gr
 
 constexpr size_t tc_smem_bytes() {
   return 1024 + (kKStages + kVStages) * kTcTile + kTcQBytes +
-         (2 * kKStages + 2 * kVStages + 2 * kSBufs + 3) * sizeof(uint64_t) +
-         (2 * 2 * kTcRows + 2 * kTcRows) * sizeof(float) + 64;
+         (2 * kKStages + 2 * kVStages + 2 * 3 + 1) * sizeof(uint64_t) +
+         2 * 2 * kTcRows * sizeof(float) + 64;
 }
 
 // S = Q K^T: A = Q (K-major, 128 rows), B = K tile (K-major, 128 positions), K = 128 dims.
@@ -71,10 +71,8 @@ __device__ __forceinline__ uint64_t nmajor_desc(uint32_t base, int kstep) {
   // 16 positions (rows) per step
   return umma_desc_sw128(base + kstep * 16 * 128, kTcHalf, 1024);
 }
-// TMEM column of P's 16-position K-slice `kstep` in S/P buffer `buf`
-__device__ __forceinline__ uint32_t p_col(int buf, int kstep) {
-  return buf * 128 + (kstep >> 2) * 64 + (kstep & 3) * 8;
-}
+// TMEM column of P's 16-position K-slice `kstep` in group `w`'s S/P buffer
+__device__ __forceinline__ uint32_t p_col(int w, int kstep) { return w * 128 + kstep * 8; }
 
 __global__ void __launch_bounds__(kTcThreads, 1)
     attn_tc_kernel(const __grid_constant__ CUtensorMap kmap,
@@ -128,13 +126,12 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   uint64_t *k_empty = k_full + kKStages;
   uint64_t *v_full = k_empty + kKStages;
   uint64_t *v_empty = v_full + kVStages;
-  uint64_t *s_full = v_empty + kVStages;  // [3] S of the buffer written
-  uint64_t *s_free = s_full + kSBufs;     // [3] the P V that read the buffer's P is done
-  uint64_t *p_full = s_free + kSBufs;
-  uint64_t *o_done = p_full + 1;
-  uint64_t *mma_done = o_done + 1;
-  float *red_m = reinterpret_cast<float *>(mma_done + 1);  // [2 parity][2 halves][128]
-  float *red_l = red_m + 2 * 2 * kTcRows;                  // [2 halves][128]
+  uint64_t *s_full = v_empty + kVStages;  // [2 groups] S of the group's block written
+  uint64_t *p_full = s_full + 2;          // [2 groups] P of the group's block written
+  uint64_t *o_done = p_full + 2;          // [2 groups] the group's P V done
+  uint64_t *mma_done = o_done + 2;
+  float *red_m = reinterpret_cast<float *>(mma_done + 1);  // [2 groups][128]
+  float *red_l = red_m + 2 * kTcRows;                      // [2 groups][128]
   uint32_t *tmem_base_s = reinterpret_cast<uint32_t *>(red_l + 2 * kTcRows);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_base_s + 1);
 
@@ -147,12 +144,11 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       mbar_init(&v_full[s], 1);
       mbar_init(&v_empty[s], 1);
     }
-    for (int s = 0; s < kSBufs; ++s) {
-      mbar_init(&s_full[s], 1);
-      mbar_init(&s_free[s], 1);
+    for (int w = 0; w < 2; ++w) {
+      mbar_init(&s_full[w], 1);
+      mbar_init(&p_full[w], kSoftWarps / 2);
+      mbar_init(&o_done[w], 1);
     }
-    mbar_init(p_full, kSoftWarps);
-    mbar_init(o_done, 1);
     mbar_init(mma_done, 1);
     *abort_flag = 0;
     fence_mbar_init();
@@ -223,43 +219,49 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     // ============================================================== MMA issuer
     if (lane == 0) {
       const uint32_t q_addr = smem_u32(qs);
-      auto pv = [&](int jb) {
-        if (!mbar_wait(p_full, jb & 1, abort_flag) ||
-            !mbar_wait(&v_full[jb % kVStages], (jb / kVStages) & 1, abort_flag)) {
-          report(a.dev_err, MSA_DEVERR_TIMEOUT);
-          *abort_flag = 1;
-          return;
-        }
-        tc_fence_after();
-        const int pb = jb % kSBufs;
-        const uint32_t v_addr = smem_u32(vst + (jb % kVStages) * kTcTile);
-#pragma unroll
-        for (int ks = 0; ks < 8; ++ks)
-          umma_bf16_ts(tbase + kColO, tbase + p_col(pb, ks), nmajor_desc(v_addr, ks), kIdescPV,
-                       (jb > 0 || ks > 0) ? 1u : 0u);
-        umma_commit(&s_free[pb]);
-        umma_commit(&v_empty[jb % kVStages]);
-        umma_commit(o_done);
+      auto fail = [&]() {
+        report(a.dev_err, MSA_DEVERR_TIMEOUT);
+        *abort_flag = 1;
       };
-      for (int i = 0; i < nblk && !*abort_flag; ++i) {
-        const int s = i % kKStages, sb = i % kSBufs;
-        if (!mbar_wait(&k_full[s], (i / kKStages) & 1, abort_flag) ||
-            (i >= kSBufs && !mbar_wait(&s_free[sb], ((i / kSBufs) - 1) & 1, abort_flag))) {
-          report(a.dev_err, MSA_DEVERR_TIMEOUT);
-          *abort_flag = 1;
-          break;
-        }
+      // S of block i into group (i & 1)'s buffer
+      auto qk = [&](int i) -> bool {
+        const int s = i % kKStages;
+        if (!mbar_wait(&k_full[s], (i / kKStages) & 1, abort_flag)) return false;
         tc_fence_after();
         const uint32_t k_addr = smem_u32(kst + s * kTcTile);
 #pragma unroll
         for (int ks = 0; ks < 8; ++ks)
-          umma_bf16_ss(tbase + sb * 128, kmajor_desc(q_addr, ks), kmajor_desc(k_addr, ks),
+          umma_bf16_ss(tbase + (i & 1) * 128, kmajor_desc(q_addr, ks), kmajor_desc(k_addr, ks),
                        kIdescQK, ks > 0 ? 1u : 0u);
-        umma_commit(&s_full[sb]);
+        umma_commit(&s_full[i & 1]);
         umma_commit(&k_empty[s]);
-        if (i >= 1) pv(i - 1);
+        return true;
+      };
+      bool alive = qk(0) && (nblk < 2 || qk(1));
+      for (int i = 0; i < nblk && alive; ++i) {
+        const int w = i & 1;
+        if (!mbar_wait(&p_full[w], (i >> 1) & 1, abort_flag) ||
+            !mbar_wait(&v_full[i % kVStages], (i / kVStages) & 1, abort_flag)) {
+          alive = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t v_addr = smem_u32(vst + (i % kVStages) * kTcTile);
+#pragma unroll
+        for (int ks = 0; ks < 8; ++ks)
+          umma_bf16_ts(tbase + kColO + w * 128, tbase + p_col(w, ks), nmajor_desc(v_addr, ks),
+                       kIdescPV, (i >= 2 || ks > 0) ? 1u : 0u);
+        umma_commit(&o_done[w]);
+        umma_commit(&v_empty[i % kVStages]);
+        // the next block of this group overwrites S (and so P) once this P V is done
+        if (i + 2 < nblk) {
+          if (!mbar_wait(&o_done[w], (i >> 1) & 1, abort_flag) || !qk(i + 2)) {
+            alive = false;
+            break;
+          }
+        }
       }
-      if (!*abort_flag) pv(nblk - 1);
+      if (!alive) fail();
       // every tcgen05 operation of this thread done before the TMEM is released
       umma_commit(mma_done);
       if (!mbar_wait(mma_done, 0, abort_flag)) report(a.dev_err, MSA_DEVERR_TIMEOUT);
@@ -267,11 +269,13 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     __syncwarp();
   } else {
     // ============================================================== softmax warpgroups
-    const int half = (warp - 2) >> 2;    // positions / dims 64 half .. 64 half + 63
+    const int w = (warp - 2) >> 2;       // this group takes blocks w, w + 2, w + 4, ...
     const int quarter = warp & 3;        // TMEM lanes 32 * quarter .. + 31
     const int r = quarter * 32 + lane;   // this thread's query row
-    const int st = (warp - 2) * 32 + lane;  // 0 .. 255
+    const int gt = (warp - 2 - 4 * w) * 32 + lane;  // 0 .. 127 within the group
     const uint32_t lane_addr = tbase + (static_cast<uint32_t>(quarter * 32) << 16);
+    const uint32_t s_addr = lane_addr + w * 128;
+    const uint32_t o_addr = lane_addr + kColO + w * 128;
     const int tl = r / a.G;
     const bool valid = r < rows;
     const int prow = valid ? cl + tok0 + tl : -1;
@@ -292,96 +296,118 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     int nj;
     uint32_t nmsk;
     bool nok;
-    block_meta(0, nj, nmsk, nok);
-    for (int i = 0; i < nblk; ++i) {
-      const int sb = i % kSBufs;
+    block_meta(w, nj, nmsk, nok);
+    for (int i = w; i < nblk; i += 2) {
       const int j = nj;
       const uint32_t msk = nmsk;
       const bool ok = nok;
-      block_meta(i + 1, nj, nmsk, nok);
-      const bool live = mbar_wait(&s_full[sb], (i / kSBufs) & 1, abort_flag);
+      block_meta(i + 2, nj, nmsk, nok);
+      const bool live = mbar_wait(&s_full[w], (i >> 1) & 1, abort_flag);
       if (!live) {
         report(a.dev_err, MSA_DEVERR_TIMEOUT);
         *abort_flag = 1;
       }
       tc_fence_after();
       const bool use = live && ok && (msk & tbit);
-      const int pos0 = j * kBlock + 64 * half;   // this thread's first position
-      const int lim = prow - pos0;               // element e is visible iff e <= lim
-      const bool full = use && lim >= 63;
-      const uint32_t s_addr = lane_addr + sb * 128 + 64 * half;
-      uint32_t v[64];
-      tmem_ld32(s_addr, *reinterpret_cast<uint32_t(*)[32]>(v));
-      tmem_ld32(s_addr + 32, *reinterpret_cast<uint32_t(*)[32]>(v + 32));
-      tmem_wait_ld();
-      // masked max over this half (eight independent chains), then the row's max through
-      // shared memory
-      float mx = -INFINITY;
-      {
-        float m8[8];
+      const int pos0 = j * kBlock;
+      const int lim = prow - pos0;               // position e is visible iff e <= lim
+      // Per warp, one of three paths (lanes of a warp are 32 / G tokens that selected
+      // different blocks, so a per-lane choice would run both code paths):
+      //   none   no row of the warp uses the block: P = 0, nothing else;
+      //   plain  every row either does not use it or sees all 128 positions: no per-position
+      //          mask (a row that does not use the block gets scale 0 and offset -inf, and its
+      //          scores are finite: some row of the warp sees the whole block, so it lies below
+      //          the sequence end);
+      //   masked the diagonal blocks.
+      const bool any_use = __any_sync(0xffffffffu, use);
+      const bool plain = __all_sync(0xffffffffu, !use || lim >= kBlock - 1);
+      float m8[8];
 #pragma unroll
-        for (int k = 0; k < 8; ++k) m8[k] = -INFINITY;
-        if (full) {
+      for (int k = 0; k < 8; ++k) m8[k] = -INFINITY;
+      if (any_use) {
+        // row max, 64 scores at a time (eight independent chains)
 #pragma unroll
-          for (int e = 0; e < 64; ++e) m8[e & 7] = fmaxf(m8[e & 7], __uint_as_float(v[e]));
-        } else if (use) {
+        for (int h = 0; h < 2; ++h) {
+          uint32_t v[64];
+          tmem_ld32(s_addr + 64 * h, *reinterpret_cast<uint32_t(*)[32]>(v));
+          tmem_ld32(s_addr + 64 * h + 32, *reinterpret_cast<uint32_t(*)[32]>(v + 32));
+          tmem_wait_ld();
+          if (plain) {
 #pragma unroll
-          for (int e = 0; e < 64; ++e)
-            if (e <= lim) m8[e & 7] = fmaxf(m8[e & 7], __uint_as_float(v[e]));
+            for (int e = 0; e < 64; ++e) m8[e & 7] = fmaxf(m8[e & 7], __uint_as_float(v[e]));
+          } else {
+#pragma unroll
+            for (int e = 0; e < 64; ++e)
+              if (use && 64 * h + e <= lim) m8[e & 7] = fmaxf(m8[e & 7], __uint_as_float(v[e]));
+          }
         }
 #pragma unroll
         for (int k = 0; k < 4; ++k) m8[k] = fmaxf(m8[k], m8[k + 4]);
-        mx = fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3]));
       }
-      float *rm = red_m + (i & 1) * 2 * kTcRows;
-      rm[half * kTcRows + r] = mx;
-      named_bar_sync(1, kSoftThreads);
-      const float mb = fmaxf(mx, rm[(half ^ 1) * kTcRows + r]) * a.scale_log2;
+      const float mrow = fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3]));
+      const float mb = use ? mrow * a.scale_log2 : -INFINITY;
       const float m_cand = fmaxf(m_run, mb);
       float alpha = 1.f;
       if (m_cand > m_run + kLazyLog2) {  // also the first visible block (m_run = -inf)
         alpha = fast_exp2(m_run - m_cand);
         m_run = m_cand;
       }
-      const float nbase = m_run == -INFINITY ? 0.f : -m_run;
-      // P = 2^(scale log2e S - m) as bf16 into TMEM over this half's S (four sum chains)
+      // x = s * sc + nb: P = 2^(scale log2e S - m) where the row uses the block, else 0
+      const float sc = use ? a.scale_log2 : 0.f;
+      const float nb = use ? -m_run : -INFINITY;
       float ps4[4] = {0.f, 0.f, 0.f, 0.f};
-      uint32_t pk[32];
-      if (full) {
+      if (!any_use) {
+        uint32_t z[32];
 #pragma unroll
-        for (int e = 0; e < 64; e += 2) {
-          const float e0 = fast_exp2(fmaf(__uint_as_float(v[e]), a.scale_log2, nbase));
-          const float e1 = fast_exp2(fmaf(__uint_as_float(v[e + 1]), a.scale_log2, nbase));
-          ps4[(e >> 1) & 3] += e0 + e1;
-          pk[e >> 1] = pack_bf16x2(e0, e1);
-        }
+        for (int e = 0; e < 32; ++e) z[e] = 0u;
+        tmem_st32(s_addr, z);
+        tmem_st32(s_addr + 32, z);
       } else {
+        // P as bf16 into TMEM over the first 64 columns of S; the scores are read again, 64
+        // at a time (P of positions 0-63 overwrites their columns after they were read back)
 #pragma unroll
-        for (int e = 0; e < 64; e += 2) {
-          const float x0 = (use && e <= lim) ? fmaf(__uint_as_float(v[e]), a.scale_log2, nbase)
-                                             : -INFINITY;
-          const float x1 = (use && e + 1 <= lim)
-                               ? fmaf(__uint_as_float(v[e + 1]), a.scale_log2, nbase)
-                               : -INFINITY;
-          const float e0 = fast_exp2(x0), e1 = fast_exp2(x1);
-          ps4[(e >> 1) & 3] += e0 + e1;
-          pk[e >> 1] = pack_bf16x2(e0, e1);
+        for (int h = 0; h < 2; ++h) {
+          uint32_t v[64];
+          tmem_ld32(s_addr + 64 * h, *reinterpret_cast<uint32_t(*)[32]>(v));
+          tmem_ld32(s_addr + 64 * h + 32, *reinterpret_cast<uint32_t(*)[32]>(v + 32));
+          tmem_wait_ld();
+          uint32_t pk[32];
+          if (plain) {
+#pragma unroll
+            for (int e = 0; e < 64; e += 2) {
+              const float e0 = fast_exp2(fmaf(__uint_as_float(v[e]), sc, nb));
+              const float e1 = fast_exp2(fmaf(__uint_as_float(v[e + 1]), sc, nb));
+              ps4[(e >> 1) & 3] += e0 + e1;
+              pk[e >> 1] = pack_bf16x2(e0, e1);
+            }
+          } else {
+#pragma unroll
+            for (int e = 0; e < 64; e += 2) {
+              const int pe = 64 * h + e;
+              const float x0 = (use && pe <= lim) ? fmaf(__uint_as_float(v[e]), sc, nb)
+                                                  : -INFINITY;
+              const float x1 = (use && pe + 1 <= lim)
+                                   ? fmaf(__uint_as_float(v[e + 1]), sc, nb)
+                                   : -INFINITY;
+              const float e0 = fast_exp2(x0), e1 = fast_exp2(x1);
+              ps4[(e >> 1) & 3] += e0 + e1;
+              pk[e >> 1] = pack_bf16x2(e0, e1);
+            }
+          }
+          tmem_st32(s_addr + 32 * h, pk);
         }
       }
-      const float psum = (ps4[0] + ps4[1]) + (ps4[2] + ps4[3]);
-      tmem_st32(s_addr, pk);
-      l_run = l_run * alpha + psum;
-      // the previous P V must be done before O is rescaled (and, every block, so that the
-      // o_done phases are waited in order)
-      if (i >= 1 && !mbar_wait(o_done, (i - 1) & 1, abort_flag)) {
+      l_run = l_run * alpha + ((ps4[0] + ps4[1]) + (ps4[2] + ps4[3]));
+      // this group's previous P V (done before this block's S was written; waited here so
+      // that every phase is observed in order) before its O is rescaled
+      if (i >= 2 && !mbar_wait(&o_done[w], ((i >> 1) - 1) & 1, abort_flag)) {
         report(a.dev_err, MSA_DEVERR_TIMEOUT);
         *abort_flag = 1;
       }
       tc_fence_after();
-      if (i >= 1 && __any_sync(0xffffffffu, alpha < 1.f)) {
-        const uint32_t o_addr = lane_addr + kColO + 64 * half;
+      if (i >= 2 && __any_sync(0xffffffffu, alpha < 1.f)) {
 #pragma unroll
-        for (int c = 0; c < 2; ++c) {
+        for (int c = 0; c < 4; ++c) {
           uint32_t o[32];
           tmem_ld32(o_addr + c * 32, o);
           tmem_wait_ld();
@@ -394,15 +420,14 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       // positions past the sequence end in a last page: V rows there become zeros.  The V
       // tile of block i has landed, or is the next phase of its barrier to complete: V(i + 2)
       // waits for this block's P V, and V(i - 2) was read by a P V already waited for.
-      const int bpos = j * kBlock;
-      if (bpos + kBlock > L && live && ok) {
-        const int first = max(L - bpos, 0);
+      if (pos0 + kBlock > L && live && ok) {
+        const int first = max(L - pos0, 0);
         if (!mbar_wait(&v_full[i % kVStages], (i / kVStages) & 1, abort_flag)) {
           report(a.dev_err, MSA_DEVERR_TIMEOUT);
           *abort_flag = 1;
         }
         uint8_t *vt = vst + (i % kVStages) * kTcTile;
-        for (int idx = st; idx < (kBlock - first) * 16; idx += kSoftThreads) {
+        for (int idx = gt; idx < (kBlock - first) * 16; idx += 128) {
           const int rr = first + idx / 16, ch = idx % 16;
           *reinterpret_cast<uint4 *>(vt + sw128(rr, ch, kTcHalf)) = make_uint4(0, 0, 0, 0);
         }
@@ -410,33 +435,50 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       }
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(p_full);
+      if (lane == 0) mbar_arrive(&p_full[w]);
     }
-    // ---- epilogue: O / l, bf16, into the ragged output (each half: its 64 dims)
-    if (!mbar_wait(o_done, (nblk - 1) & 1, abort_flag)) {
+    // ---- epilogue: the two groups merged by log-sum-exp, O / l, bf16 (group w: dims 64 w ..)
+    const int nw = (nblk - w + 1) / 2;  // blocks this group took
+    if (nw > 0 && !mbar_wait(&o_done[w], (nw - 1) & 1, abort_flag)) {
       report(a.dev_err, MSA_DEVERR_TIMEOUT);
       *abort_flag = 1;
     }
     tc_fence_after();
-    red_l[half * kTcRows + r] = l_run;
+    red_m[w * kTcRows + r] = m_run;
+    red_l[w * kTcRows + r] = l_run;
     named_bar_sync(1, kSoftThreads);
-    const float l_tot = red_l[r] + red_l[kTcRows + r];
+    const float m0 = red_m[r], m1 = red_m[kTcRows + r];
+    const float m = fmaxf(m0, m1);
+    // a group with no block (nblk == 1) never wrote its O: its weight must be exactly 0
+    const float f0 = m0 == -INFINITY ? 0.f : fast_exp2(m0 - m);
+    const float f1 = (nblk < 2 || m1 == -INFINITY) ? 0.f : fast_exp2(m1 - m);
+    const float l_tot = red_l[r] * f0 + red_l[kTcRows + r] * f1;
     const float inv = l_tot > 0.f ? 1.f / l_tot : 0.f;
+    const float g0 = f0 * inv, g1 = f1 * inv;
     const size_t orow = static_cast<size_t>(t0 + tl) * a.H_q + g * a.G + r % a.G;
+    const uint32_t o0 = lane_addr + kColO + 64 * w, o1 = o0 + 128;
 #pragma unroll
     for (int c = 0; c < 2; ++c) {
-      uint32_t v[32];
-      tmem_ld32(lane_addr + kColO + 64 * half + c * 32, v);
+      uint32_t x0[32], x1[32];
+      tmem_ld32(o0 + c * 32, x0);
+      tmem_ld32(o1 + c * 32, x1);
       tmem_wait_ld();
+      float y[32];
+#pragma unroll
+      for (int e = 0; e < 32; ++e) {
+        // a zero weight contributes nothing, whatever the (possibly unwritten) O holds
+        const float a0 = g0 != 0.f ? __uint_as_float(x0[e]) * g0 : 0.f;
+        const float a1 = g1 != 0.f ? __uint_as_float(x1[e]) * g1 : 0.f;
+        y[e] = a0 + a1;
+      }
       if (valid) {
-        uint4 *dst = reinterpret_cast<uint4 *>(a.out + orow * kHeadDim + 64 * half + c * 32);
+        uint4 *dst = reinterpret_cast<uint4 *>(a.out + orow * kHeadDim + 64 * w + c * 32);
 #pragma unroll
         for (int q4 = 0; q4 < 4; ++q4)
-          dst[q4] = make_uint4(
-              pack_bf16x2(__uint_as_float(v[8 * q4 + 0]) * inv, __uint_as_float(v[8 * q4 + 1]) * inv),
-              pack_bf16x2(__uint_as_float(v[8 * q4 + 2]) * inv, __uint_as_float(v[8 * q4 + 3]) * inv),
-              pack_bf16x2(__uint_as_float(v[8 * q4 + 4]) * inv, __uint_as_float(v[8 * q4 + 5]) * inv),
-              pack_bf16x2(__uint_as_float(v[8 * q4 + 6]) * inv, __uint_as_float(v[8 * q4 + 7]) * inv));
+          dst[q4] = make_uint4(pack_bf16x2(y[8 * q4 + 0], y[8 * q4 + 1]),
+                               pack_bf16x2(y[8 * q4 + 2], y[8 * q4 + 3]),
+                               pack_bf16x2(y[8 * q4 + 4], y[8 * q4 + 5]),
+                               pack_bf16x2(y[8 * q4 + 6], y[8 * q4 + 7]));
       }
     }
   }

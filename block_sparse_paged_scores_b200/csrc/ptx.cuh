@@ -45,23 +45,37 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
       : "memory");
   return ok != 0;
 }
+// The same test, but a thread whose phase is not complete yet is suspended until it
+// completes or about `hint_ns` have passed (it then issues nothing while it waits).
+__device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t *bar, uint32_t parity,
+                                                    uint32_t hint_ns) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity), "r"(hint_ns)
+      : "memory");
+  return ok != 0;
+}
 __device__ __forceinline__ uint64_t global_timer_ns() {
   uint64_t t;
   asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
   return t;
 }
 // Waits for the phase with the given parity to complete.  Gives up after kWaitTimeoutNs or
-// as soon as *abort is set, and then returns false (the caller reports and unwinds).
+// as soon as *abort is set, and then returns false (the caller reports and unwinds).  After
+// the first test the thread sleeps in the barrier between tests (at most 0.5 ms each), so
+// waiting warps take no issue slots from the working ones.
 __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity,
                                           volatile int *abort) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = global_timer_ns();
-  for (uint32_t it = 1;; ++it) {
-    if (mbar_try_wait(bar, parity)) return true;
-    if ((it & 63) == 0) {
-      if (*abort) return false;
-      if (global_timer_ns() - t0 > kWaitTimeoutNs) return false;
-    }
+  for (;;) {
+    if (mbar_try_wait_sleep(bar, parity, 500000u)) return true;
+    if (*abort) return false;
+    if (global_timer_ns() - t0 > kWaitTimeoutNs) return false;
   }
 }
 
