@@ -325,11 +325,12 @@ def run_ours(args):
     stream = torch.cuda.current_stream(dev)
     fp8 = prob["kv_fp8"]
     stream_route = prob["max_q_len"] <= 8  # decode / speculative: persistent kernel + combine
-    # decode / speculative: index, select, [plan], attention, combine;
-    # prefill: index, select, plan, attention
-    kernels_per_step = (4 + (1 if prob["max_q_len"] > 1 else 0)) if stream_route else 4
     splits_used = msa.msa_attn_partials(path.rp, prob["S"], prob["H_q"], prob["H_kv"],
                                         path.max_blocks, args.splits)[0] if stream_route else 1
+    # decode / speculative: index, select, [plan], attention, [combine: only with more than one
+    # split-K partition]; prefill: index, select, plan, attention
+    kernels_per_step = (3 + (1 if prob["max_q_len"] > 1 else 0) + (1 if splits_used > 1 else 0)
+                        if stream_route else 4)
 
     for _ in range(args.warmup):
         path.run(stream)
@@ -367,11 +368,16 @@ def run_ours(args):
                 args.steps for i in range(len(fns))]
 
     attn_key = "attention" + ("_incl_plan" if prob["max_q_len"] > 1 else "")
-    if stream_route:
+    if stream_route and splits_used > 1:
         st = stage_pass([lambda: path.index_scores(stream), lambda: path.select(stream=stream),
                          lambda: path.attend(stream=stream, combine=False),
                          lambda: path.combine(stream)])
         stages = {"index_scores": st[0], "select": st[1], attn_key: st[2], "combine": st[3]}
+    elif stream_route:  # one partition: the attention kernel writes the output, no combine
+        st = stage_pass([lambda: path.index_scores(stream), lambda: path.select(stream=stream),
+                         lambda: path.attend(stream=stream)])
+        stages = {"index_scores": st[0], "select": st[1], attn_key: st[2]}
+    if stream_route:
         # the first two stages as one msa_index_select launch, for comparison
         stages["fused_index_select"] = stage_pass([lambda: path.index_select(stream)])[0]
         idx_kind, idx_src = "index_scores", "indexer.cu"

@@ -104,7 +104,7 @@ struct Route {
 
 constexpr int kMaxRows = 64;  // rows (tokens x group heads) per attention CTA
 constexpr int kMaxSplits = 4096;
-constexpr int kMinSlotsPerCta = 4;
+constexpr int kMinSlotsPerCta = 8;
 
 int stream_grid(long long total, int num_splits, int num_sms) {
   long long grid = num_splits > 0 ? num_splits
@@ -270,7 +270,7 @@ msa_status_t index_scores_impl(const msa_ragged_paged_t *rp, const void *q_idx,
                                int32_t *dev_err, cudaStream_t stream, const FusedSelect *fs) {
   if (!ragged_ok(rp) || !q_idx || !k_idx_cache || !scores || num_kv_heads < 1 ||
       !(num_idx_k_heads == 1 || num_idx_k_heads == num_kv_heads) || max_blocks < 1 ||
-      max_blocks > rp->max_pages_per_seq || !aligned(k_idx_cache, 16) || !aligned(q_idx, 4))
+      max_blocks > rp->max_pages_per_seq || !aligned(k_idx_cache, 16) || !aligned(q_idx, 16))
     return MSA_ERR_INVALID_ARG;
   const int Hg = num_kv_heads / num_idx_k_heads;
   if (Hg > 32) return MSA_ERR_UNSUPPORTED;
@@ -440,7 +440,7 @@ msa_status_t msa_sparse_attn_paged(const msa_ragged_paged_t *rp, const void *q,
       num_q_heads % num_kv_heads != 0 || max_blocks < 1 || max_blocks > rp->max_pages_per_seq ||
       !(scale > 0.f) || !isfinite(scale) || num_splits < 0 || num_splits > kMaxSplits ||
       !(kv_dtype == MSA_KV_BF16 || kv_dtype == MSA_KV_FP8_E4M3) || !aligned(q, 16) ||
-      !aligned(k_cache, 16) || !aligned(v_cache, 16) || !aligned(out, 8))
+      !aligned(k_cache, 16) || !aligned(v_cache, 16) || !aligned(out, 16))
     return MSA_ERR_INVALID_ARG;
   if (!out && rp->max_q_len > MSA_MAX_SPEC_DRAFT) return MSA_ERR_INVALID_ARG;  // prefill: out
   const int G = num_q_heads / num_kv_heads;
@@ -517,6 +517,8 @@ msa_status_t msa_sparse_attn_paged(const msa_ragged_paged_t *rp, const void *q,
   a.part_o = reinterpret_cast<float *>(ws + r.off_o);
   a.part_lse = reinterpret_cast<float *>(ws + r.off_lse);
   a.out = static_cast<uint16_t *>(out);
+  // one partition: every item lies inside one CTA, which then writes the output itself
+  a.direct = r.stream && r.splits == 1 && out != nullptr;
   a.dev_err = dev_err;
   if (r.tc)
     return launch_attention_tc(kmap, vmap, a, s) == cudaSuccess ? MSA_OK : MSA_ERR_CUDA;
@@ -525,7 +527,7 @@ msa_status_t msa_sparse_attn_paged(const msa_ragged_paged_t *rp, const void *q,
                                                                              : MSA_ERR_CUDA;
   if (launch_attention_stream(kmap, vmap, a, fp8, r.rg, r.plan, r.grid, s) != cudaSuccess)
     return MSA_ERR_CUDA;
-  if (!out) return MSA_OK;  // the caller combines the partials itself
+  if (!out || a.direct) return MSA_OK;  // no partials, or the caller combines them itself
   if (launch_combine(a.part_o, a.part_lse, r.splits, rp->total_q, num_q_heads, a.out, s) !=
       cudaSuccess)
     return MSA_ERR_CUDA;

@@ -242,7 +242,12 @@ __global__ void __launch_bounds__(32 * (stream_consumer_warps<FP8, RG>() + 1))
       for (int idx = lane; idx < m.rows * max(p_hi - p_lo, 0); idx += 32) {
         const int r = idx % m.rows, p2 = p_lo + idx / m.rows;
         const size_t orr = static_cast<size_t>(m.t0 + r / a.G) * a.H_q + m.g * a.G + r % a.G;
-        a.part_lse[static_cast<size_t>(p2) * split_stride + orr] = -INFINITY;
+        if (a.direct) {  // a row that saw nothing: zeros, as the combine would give
+          uint4 *dst = reinterpret_cast<uint4 *>(a.out + orr * kHeadDim);
+          for (int c = 0; c < kHeadDim / 8; ++c) dst[c] = make_uint4(0, 0, 0, 0);
+        } else {
+          a.part_lse[static_cast<size_t>(p2) * split_stride + orr] = -INFINITY;
+        }
       }
       if (v1 <= v0) continue;
 
@@ -424,8 +429,12 @@ __global__ void __launch_bounds__(32 * (stream_consumer_warps<FP8, RG>() + 1))
         const int r = rg * 16 + (lane >> 2) + slot * 8;
         if (r >= md.rows) continue;
         const size_t orr = static_cast<size_t>(md.t0 + r / a.G) * a.H_q + md.g * a.G + r % a.G;
-        const size_t pr = static_cast<size_t>(md.piece) * split_stride + orr;
         const float l = wa.l_run[slot];
+        if (a.direct) {
+          wa.store_bf16(a.out + orr * kHeadDim, slot, l > 0.f ? 1.f / l : 0.f, lane);
+          continue;
+        }
+        const size_t pr = static_cast<size_t>(md.piece) * split_stride + orr;
         wa.store_global(a.part_o + pr * kHeadDim, slot, l > 0.f ? 1.f / l : 0.f, lane);
         if ((lane & 3) == 0)
           a.part_lse[pr] = l > 0.f ? (wa.m_run[slot] + __log2f(l)) * kLn2 : -INFINITY;

@@ -323,6 +323,23 @@ struct WarpAttn {
     m_run[slot] = m;
   }
 
+  // This thread's part of row slot `slot` times f, as bf16 in natural dim order, into a
+  // 128-dim row of global memory.
+  __device__ __forceinline__ void store_bf16(uint16_t *dst, int slot, float f, int lane) const {
+    const int c4 = lane & 3;
+    if (FP8) {
+#pragma unroll
+      for (int ch = 0; ch < 8; ++ch)
+        *reinterpret_cast<uint2 *>(dst + ch * 16 + 4 * c4) =
+            make_uint2(pack_bf16x2(o[2 * ch][2 * slot] * f, o[2 * ch + 1][2 * slot] * f),
+                       pack_bf16x2(o[2 * ch][2 * slot + 1] * f, o[2 * ch + 1][2 * slot + 1] * f));
+    } else {
+#pragma unroll
+      for (int n = 0; n < 16; ++n)
+        *reinterpret_cast<uint32_t *>(dst + n * 8 + 2 * c4) =
+            pack_bf16x2(o[n][2 * slot] * f, o[n][2 * slot + 1] * f);
+    }
+  }
   // This thread's part of row slot `slot` times f, as fp32 in natural dim order, into a
   // 128-dim row of global memory.
   __device__ __forceinline__ void store_global(float *dst, int slot, float f, int lane) const {

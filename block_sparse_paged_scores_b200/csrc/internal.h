@@ -78,7 +78,10 @@ struct AttnArgs {
   int P;        // persistent kernel: most CTAs one item's slots can span
   float scale_log2;          // scale * log2(e)
   float *part_o, *part_lse;  // persistent kernel: [P][total_q][H_q][128] and [P][total_q][H_q]
-  uint16_t *out;             // tile kernel: bf16 bits [total_q, H_q, 128]
+  uint16_t *out;             // bf16 bits [total_q, H_q, 128]: tile kernels, and the persistent
+                             // kernel when `direct`
+  int direct;                // persistent kernel with P == 1 (every item inside one CTA): write
+                             // O / l to `out` instead of partials (no combine follows)
   int32_t *dev_err;
 };
 // rg = 16-row groups (1..4); plan = read the per-tile union instead of the selection

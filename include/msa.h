@@ -98,7 +98,7 @@ typedef struct {
  *   for j < nb(p); -inf for nb(p) <= j < max_blocks.  FP32 accumulation of exact BF16
  *   products.  Positions > p (and so every position >= L_b) never enter the max.
  *
- *   q_idx        device bf16 [total_q, num_kv_heads, 128]
+ *   q_idx        device bf16 [total_q, num_kv_heads, 128], 16-byte aligned
  *   k_idx_cache  device bf16 [num_pages, num_idx_k_heads, 128 tokens, 128], 16-byte aligned
  *   num_idx_k_heads  1 (one index-K head shared by all index-query heads) or num_kv_heads
  *   max_blocks   row length of `scores`; must be >= nb(p) of every query and
@@ -176,10 +176,11 @@ MSA_API msa_status_t msa_index_select(const msa_ragged_paged_t *rp, const void *
  *   Speculative and prefill steps first build, in `workspace`, each query tile's union of its
  *   tokens' selected blocks with a per-token mask, so that a page is read once per tile.
  *   Decode / speculative work is a list of (sequence, query tile, KV head, selected block)
- *   entries cut into `num_splits` equal contiguous split-K partitions (0 = one per SM, a
- *   persistent launch); their partials live in `workspace` and this call also enqueues the
- *   combine that writes `out`.  Prefill runs one CTA per (sequence, query tile, KV head) and
- *   ignores num_splits.
+ *   entries cut into `num_splits` equal contiguous split-K partitions (0 = one per SM and at
+ *   least 8 blocks per partition, a persistent launch); their partials live in `workspace` and
+ *   this call also enqueues the combine that writes `out`.  With a single partition the
+ *   attention kernel writes `out` itself and no combine is enqueued.  Prefill runs one CTA per
+ *   (sequence, query tile, KV head) and ignores num_splits.
  *
  *   q            device bf16 [total_q, num_q_heads, 128]
  *   k_cache, v_cache  device [num_pages, num_kv_heads, 128 tokens, 128] of kv_dtype,
@@ -188,9 +189,10 @@ MSA_API msa_status_t msa_index_select(const msa_ragged_paged_t *rp, const void *
  *   max_blocks   an upper bound on nb(p) of every query (as for msa_index_scores)
  *   workspace    device, >= msa_attn_workspace_bytes(...) bytes, 256-byte aligned;
  *                may be NULL when that size is 0
- *   out          device bf16 [total_q, num_q_heads, 128] (output).  On the decode and
- *                speculative routes `out` may be NULL: the call then leaves the split-K
- *                partials in `workspace` (see msa_attn_partials) and enqueues no combine.
+ *   out          device bf16 [total_q, num_q_heads, 128] (output), 16-byte aligned.  On the
+ *                decode and speculative routes `out` may be NULL: the call then leaves the
+ *                split-K partials in `workspace` (see msa_attn_partials) and enqueues no
+ *                combine.
  *   num_q_heads % num_kv_heads == 0; the group size num_q_heads / num_kv_heads <= 64.
  */
 MSA_API msa_status_t msa_sparse_attn_paged(const msa_ragged_paged_t *rp, const void *q,
@@ -255,7 +257,7 @@ MSA_API size_t msa_attn_workspace_bytes(const msa_ragged_paged_t *rp, int32_t S,
 
 /* The split-K partition count the decode / speculative routes use when num_splits == 0 for
  * `batch` sequences of `max_q_len` new tokens: one partition per SM, fewer when the work list
- * (batch x num_kv_heads x S x max_q_len entries) has under 4 entries per SM; 1 for prefill. */
+ * (batch x num_kv_heads x S x max_q_len entries) has under 8 entries per SM; 1 for prefill. */
 MSA_API int32_t msa_default_num_splits(int32_t batch, int32_t max_q_len, int32_t num_kv_heads,
                                int32_t S, int32_t num_sms);
 

@@ -63,7 +63,8 @@ def test_status_strings(lib):
 def test_default_splits_fill_the_sms(lib):
     # decode / speculative: one persistent partition per SM, fewer for tiny work lists
     assert msa.msa_default_num_splits(32, 1, 8, 19, 148) == 148
-    assert msa.msa_default_num_splits(1, 1, 1, 6, 148) == 2       # 6 entries, >= 4 per CTA
+    assert msa.msa_default_num_splits(1, 1, 1, 6, 148) == 1       # 6 entries, >= 8 per CTA
+    assert msa.msa_default_num_splits(1, 1, 4, 6, 148) == 3       # 24 entries
     assert msa.msa_default_num_splits(128, 1, 8, 69, 148) == 148
     assert msa.msa_default_num_splits(64, 4, 8, 35, 148) == 148
     assert msa.msa_default_num_splits(8, 4096, 8, 67, 148) == 1   # prefill: one partition
@@ -109,6 +110,8 @@ def test_invalid_arguments_are_rejected_before_any_launch(lib):
     assert stat == msa.MSA_ERR_INVALID_ARG
     stat = lib.msa_index_scores(ctypes.byref(rp), P, P + 2, 8, 1, 16, P, None, None)  # align
     assert stat == msa.MSA_ERR_INVALID_ARG
+    stat = lib.msa_index_scores(ctypes.byref(rp), P + 8, P, 8, 1, 16, P, None, None)  # q_idx
+    assert stat == msa.MSA_ERR_INVALID_ARG
     stat = lib.msa_index_scores(ctypes.byref(rp), P, P, 64, 1, 16, P, None, None)  # group > 32
     assert stat == msa.MSA_ERR_UNSUPPORTED
     stat = lib.msa_select_blocks(ctypes.byref(rp), P, 8, 16, 0, 0, 0, P, P, None, None)  # S = 0
@@ -148,6 +151,7 @@ def test_invalid_arguments_are_rejected_before_any_launch(lib):
     assert attn(scale=float("nan")) == msa.MSA_ERR_INVALID_ARG
     assert attn(ns=-1) == msa.MSA_ERR_INVALID_ARG
     assert attn(k=P + 8) == msa.MSA_ERR_INVALID_ARG        # cache not 16-byte aligned
+    assert attn(out=P + 8) == msa.MSA_ERR_INVALID_ARG      # output not 16-byte aligned
     assert attn(hq=8 * 128) == msa.MSA_ERR_UNSUPPORTED     # GQA group 128 > 64
     assert attn(ns=4) == msa.MSA_ERR_INVALID_ARG           # partials need a workspace
     assert attn(ns=5000) == msa.MSA_ERR_INVALID_ARG        # more partitions than allowed
