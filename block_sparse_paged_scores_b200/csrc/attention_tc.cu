@@ -237,28 +237,48 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         umma_commit(&k_empty[s]);
         return true;
       };
+      // Event loop: the P V of the next block once its P (and V) is there, and the QK^T of the
+      // next block once the P V that read its group's buffer is done, both in block order, so
+      // that neither group waits behind the other's step.  Every barrier's phases are polled
+      // in order.
       bool alive = qk(0) && (nblk < 2 || qk(1));
-      for (int i = 0; i < nblk && alive; ++i) {
-        const int w = i & 1;
-        if (!mbar_wait(&p_full[w], (i >> 1) & 1, abort_flag) ||
-            !mbar_wait(&v_full[i % kVStages], (i / kVStages) & 1, abort_flag)) {
-          alive = false;
-          break;
-        }
-        tc_fence_after();
-        const uint32_t v_addr = smem_u32(vst + (i % kVStages) * kTcTile);
+      int next_pv = 0, next_qk = 2;
+      uint64_t t_idle = 0;
+      uint32_t idle = 0;
+      while (alive && next_pv < nblk) {
+        bool progress = false;
+        {
+          const int i = next_pv, w = i & 1;
+          if (mbar_try_wait(&p_full[w], (i >> 1) & 1) &&
+              mbar_try_wait(&v_full[i % kVStages], (i / kVStages) & 1)) {
+            tc_fence_after();
+            const uint32_t v_addr = smem_u32(vst + (i % kVStages) * kTcTile);
 #pragma unroll
-        for (int ks = 0; ks < 8; ++ks)
-          umma_bf16_ts(tbase + kColO + w * 128, tbase + p_col(w, ks), nmajor_desc(v_addr, ks),
-                       kIdescPV, (i >= 2 || ks > 0) ? 1u : 0u);
-        umma_commit(&o_done[w]);
-        umma_commit(&v_empty[i % kVStages]);
-        // the next block of this group overwrites S (and so P) once this P V is done
-        if (i + 2 < nblk) {
-          if (!mbar_wait(&o_done[w], (i >> 1) & 1, abort_flag) || !qk(i + 2)) {
-            alive = false;
-            break;
+            for (int ks = 0; ks < 8; ++ks)
+              umma_bf16_ts(tbase + kColO + w * 128, tbase + p_col(w, ks),
+                           nmajor_desc(v_addr, ks), kIdescPV, (i >= 2 || ks > 0) ? 1u : 0u);
+            umma_commit(&o_done[w]);
+            umma_commit(&v_empty[i % kVStages]);
+            ++next_pv;
+            progress = true;
           }
+        }
+        if (next_qk < nblk && next_qk - 2 < next_pv) {
+          const int i = next_qk, w = i & 1;
+          // the group's previous P V read P from the buffer this S overwrites
+          if (mbar_try_wait(&o_done[w], ((i >> 1) - 1) & 1) &&
+              mbar_try_wait(&k_full[i % kKStages], (i / kKStages) & 1)) {
+            alive = qk(i);
+            ++next_qk;
+            progress = true;
+          }
+        }
+        if (progress) {
+          idle = 0;
+        } else if ((++idle & 255) == 1) {
+          const uint64_t now = global_timer_ns();
+          if (idle == 1) t_idle = now;
+          if (*abort_flag || now - t_idle > kWaitTimeoutNs) alive = false;
         }
       }
       if (!alive) fail();
@@ -281,27 +301,28 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     const int prow = valid ? cl + tok0 + tl : -1;
     const uint32_t tbit = valid ? (1u << tl) : 0u;
     float m_run = -INFINITY, l_run = 0.f;
-    // the block's id, token mask and page validity, read one block ahead from the plan
-    auto block_meta = [&](int i, int &j, uint32_t &msk, bool &ok) {
-      j = -1, msk = 0u, ok = false;
-      if (i < nblk) {
-        j = list[i];
-        msk = masks[i];
-        if (j >= 0 && j < a.max_blocks) {
-          const int pg = a.table[static_cast<size_t>(b) * a.max_pages + j];
-          ok = pg >= 0 && pg < a.num_pages;
-        }
-      }
+    // The block's id, token mask and page validity come from the plan and the page table
+    // through a two-deep register pipeline, so that no load is waited for in the block that
+    // issues it: the list entries of this group's block after next, and the page of its next.
+    const int32_t *trow = a.table + static_cast<size_t>(b) * a.max_pages;
+    auto list_at = [&](int i, int &j, uint32_t &msk) {
+      j = i < nblk ? list[i] : -1;
+      msk = i < nblk ? masks[i] : 0u;
     };
-    int nj;
-    uint32_t nmsk;
-    bool nok;
-    block_meta(w, nj, nmsk, nok);
+    auto page_of = [&](int j) { return (j >= 0 && j < a.max_blocks) ? trow[j] : -1; };
+    int j_n, j_nn;
+    uint32_t msk_n, msk_nn;
+    list_at(w, j_n, msk_n);
+    list_at(w + 2, j_nn, msk_nn);
+    int pg_n = page_of(j_n);
     for (int i = w; i < nblk; i += 2) {
-      const int j = nj;
-      const uint32_t msk = nmsk;
-      const bool ok = nok;
-      block_meta(i + 2, nj, nmsk, nok);
+      const int j = j_n;
+      const uint32_t msk = msk_n;
+      const bool ok = pg_n >= 0 && pg_n < a.num_pages;
+      j_n = j_nn;
+      msk_n = msk_nn;
+      pg_n = page_of(j_n);
+      list_at(i + 4, j_nn, msk_nn);
       const bool live = mbar_wait(&s_full[w], (i >> 1) & 1, abort_flag);
       if (!live) {
         report(a.dev_err, MSA_DEVERR_TIMEOUT);

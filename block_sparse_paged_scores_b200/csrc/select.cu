@@ -13,14 +13,17 @@ namespace {
 
 constexpr int kWarps = 4;
 
-__device__ __forceinline__ int find_sequence(const int32_t *row_off, int batch, int t) {
-  int lo = 0, hi = batch;  // row_off[lo] <= t < row_off[hi]
-  while (hi - lo > 1) {
-    const int mid = (lo + hi) >> 1;
-    if (row_off[mid] <= t)
-      lo = mid;
-    else
-      hi = mid;
+// The sequence of row t: the largest b < batch with row_off[b] <= t, by a warp-wide 32-ary
+// search (one load per lane per level: one level up to 32 sequences, two up to 1024).
+__device__ __forceinline__ int find_sequence(const int32_t *row_off, int batch, int t, int lane) {
+  int lo = 0, n = batch;  // row_off[lo] <= t, and t < row_off[lo + n] unless lo + n == batch
+  while (n > 1) {
+    const int step = (n + 31) / 32;
+    const bool le = lane * step < n && row_off[lo + lane * step] <= t;
+    const unsigned m = __ballot_sync(0xffffffffu, le);  // lane 0 always set
+    const int last = 31 - __clz(m);
+    lo += last * step;
+    n = min(step, n - last * step);
   }
   return lo;
 }
@@ -34,7 +37,7 @@ __global__ void __launch_bounds__(32 * kWarps) select_kernel(const SelectArgs a)
   if (item >= static_cast<long long>(a.total_q) * a.H_kv) return;
   const int t = static_cast<int>(item / a.H_kv);
 
-  const int b = find_sequence(a.row_off, a.batch, t);
+  const int b = find_sequence(a.row_off, a.batch, t, lane);
   const int p = a.cache_len[b] + (t - a.row_off[b]);
   int nb = (p < 0 ? 0 : p) / kBlock + 1;
   if (nb > a.max_blocks) {

@@ -43,18 +43,40 @@ struct SelKeys {
       k[i] = (j < nb && j >= init_e && j < local_lo) ? score_key(load_score<CG>(srow + j)) : 0u;
     }
   }
-  // number of candidate keys >= x (over the warp)
+  // number of candidate keys >= x (over the warp); four independent partial counts
   __device__ __forceinline__ uint32_t count_ge(uint32_t x, const float *srow, int lane,
                                                int init_e, int local_lo) const {
     uint32_t c = 0;
     if (KPL > 0) {
+      uint32_t c4[4] = {0u, 0u, 0u, 0u};
 #pragma unroll
-      for (int i = 0; i < KPL; ++i) c += k[i] >= x;
+      for (int i = 0; i < KPL; ++i) c4[i & 3] += k[i] >= x;
+      c = (c4[0] + c4[1]) + (c4[2] + c4[3]);
     } else {
       for (int j = init_e + lane; j < local_lo; j += 32)
         c += score_key(load_score<CG>(srow + j)) >= x;
     }
     return __reduce_add_sync(0xffffffffu, c);
+  }
+  // largest and smallest candidate key over the warp
+  __device__ __forceinline__ void range(const float *srow, int lane, int init_e, int local_lo,
+                                        uint32_t &kmax, uint32_t &kmin) const {
+    uint32_t hi = 0u, lo = 0xffffffffu;
+    if (KPL > 0) {
+#pragma unroll
+      for (int i = 0; i < KPL; ++i) {
+        hi = max(hi, k[i]);
+        if (k[i] != 0u) lo = min(lo, k[i]);
+      }
+    } else {
+      for (int j = init_e + lane; j < local_lo; j += 32) {
+        const uint32_t key = score_key(load_score<CG>(srow + j));
+        hi = max(hi, key);
+        lo = min(lo, key);
+      }
+    }
+    kmax = __reduce_max_sync(0xffffffffu, hi);
+    kmin = __reduce_min_sync(0xffffffffu, lo);
   }
 };
 
@@ -77,10 +99,15 @@ __device__ __forceinline__ int select_row(const float *srow, int nb, int top_k, 
   if (!take_all && top_k > 0) {
     keys.load(srow, nb, lane, init_e, local_lo);
     // T = the top_k-th largest candidate key: the largest x with count(key >= x) >= top_k,
-    // built one bit at a time from the top.
+    // built one bit at a time from the top.  Every candidate key lies in [kmin, kmax], so T
+    // shares their common leading bits and only the bits below can still be open.
     const uint32_t k = static_cast<uint32_t>(top_k);
-    T = 0;
-    for (int bit = 31; bit >= 0; --bit) {
+    uint32_t kmax, kmin;
+    keys.range(srow, lane, init_e, local_lo, kmax, kmin);
+    const uint32_t diff = kmax ^ kmin;
+    const int top = diff == 0u ? -1 : 31 - __clz(diff);  // highest bit where they differ
+    T = top < 0 ? kmax : (kmax & ~((2u << top) - 1u));
+    for (int bit = top; bit >= 0; --bit) {
       const uint32_t x = T | (1u << bit);
       if (keys.count_ge(x, srow, lane, init_e, local_lo) >= k) T = x;
     }

@@ -267,3 +267,35 @@ def test_bad_page_id_is_reported_not_read():
     path.run()
     torch.cuda.synchronize()
     assert int(path.dev_err.item()) & msa.MSA_DEVERR_PAGE_ID
+
+
+@pytest.mark.parametrize("kw", [
+    # 8192 one-to-three-page units (per-head index-K): most CTAs of the indexer have no page
+    # to score, and the fused selection's last-CTA counting runs over thousands of units
+    dict(batch=2048, kv_len=(1, 260), H_kv=4, G=1, H_idxk=4, top_k=1, init_blocks=1,
+         local_blocks=0),
+    dict(batch=2100, kv_len=(1, 300), H_kv=1, G=1, top_k=1, init_blocks=1, local_blocks=0),
+])
+def test_indexer_for_many_short_sequences(kw):
+    spec = W["bf16_decode"].scaled(**kw)
+    p = wl.generate(spec, seed=4242, device="cuda")
+    path = msa.Path(p)
+    path.index_scores()
+    path.select()
+    fused = msa.Path(p)
+    fused.index_select()
+    torch.cuda.synchronize()
+    assert int(path.dev_err.item()) == 0 and int(fused.dev_err.item()) == 0
+    assert torch.equal(fused.scores, path.scores)
+    assert torch.equal(fused.block_ids, path.block_ids)
+    assert torch.equal(fused.num_selected, path.num_selected)
+    assert int(fused.counters.abs().sum().item()) == 0
+    cpu = {k: (v.cpu() if torch.is_tensor(v) else v) for k, v in p.items()}
+    sc = oracle.index_scores(cpu["row_off"], cpu["cache_len"], cpu["table"], cpu["q_idx"],
+                             cpu["k_idx"], p["max_blocks"])
+    check_scores(path.scores.cpu().numpy(), sc, cpu, p["max_blocks"])
+    gsc = path.scores.cpu().numpy().astype(np.float64)
+    ids, cnt = oracle.select_blocks(cpu["row_off"], cpu["cache_len"], gsc, p["top_k"],
+                                    p["init_blocks"], p["local_blocks"])
+    assert np.array_equal(path.num_selected.cpu().numpy(), cnt)
+    assert np.array_equal(path.block_ids.cpu().numpy(), ids)
