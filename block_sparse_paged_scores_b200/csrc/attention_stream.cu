@@ -367,15 +367,18 @@ __global__ void __launch_bounds__(32 * (stream_consumer_warps<FP8, RG>() + 1))
       prow[slot] = r < md.rows ? md.cl + md.tok0 + tl : -1;
       tbit[slot] = r < md.rows ? (1u << tl) : 0u;
     }
+    // the tokens of this warp's row group: a block none of them selected leaves its rows'
+    // state unchanged, so its math is skipped (speculative tiles walk their tokens' union)
+    const uint32_t rg_bits = __reduce_or_sync(0xffffffffu, tbit[0] | tbit[1]);
     const uint32_t qs_addr = smem_u32(qbufs + buf * QBUF);
     wa.reset();
     for (int e = md.v0 + team; e < md.v1; e += NT) {
       const uint32_t nk = nload;  // this team's K tile; V is nk + 1
       int s = team * NR + static_cast<int>(nk % NR);
       bool live = mbar_wait(&sfull[s], (nk / NR) & 1, abort_flag);
-      const bool ok = live && slot_ok[s];
       const int j = slot_j[s];
       const uint32_t msk = slot_mask[s];
+      const bool ok = live && slot_ok[s] && (msk & rg_bits) != 0;
       if (ok) wa.qk(qs_addr, QSUB, rg * 16, smem_u32(slots + s * TILE), pq, lane);
       __syncwarp();
       if (lane == 0) mbar_arrive(&sempty[s]);

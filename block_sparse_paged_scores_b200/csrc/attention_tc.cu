@@ -12,14 +12,15 @@
 //
 //   warp 0     K producer: TMA loads of each block's K page tile (128-byte swizzle) into a
 //              3-stage ring, freed as soon as the block's S is computed
-//   warp 10    V producer: the V page tiles into a 2-stage ring, freed by the block's P V
+//   warp 2     V producer: the V page tiles into a 2-stage ring, freed by the block's P V
 //   warp 1     TMEM owner and MMA issuer (one thread): S = Q K^T (M = N = 128, K = 16 x 8) and
 //              O += P V with P read from TMEM where the softmax left it (over its S) and V as
 //              an N-major shared-memory operand; tcgen05.commit signals each
-//   warps 2-9  softmax, two warpgroups taking alternate blocks (even / odd), each with its own
+//   warps 4-11 softmax, two warpgroups taking alternate blocks (even / odd), each with its own
 //              S buffer, O accumulator and running max and sum: one query row per thread (its
-//              TMEM lane), one pass over the row's 128 scores (masked max, exp2, P as bf16 back
-//              into TMEM over its S).  The groups never wait for each other inside the loop, so
+//              TMEM lane), one pass over the row's 128 scores held in registers (masked max,
+//              exp2, P as bf16 back into TMEM over its S).  The first warpgroup (producers, MMA
+//              issuer, one idle warp) hands registers to the softmax warpgroups (setmaxnreg).  The groups never wait for each other inside the loop, so
 //              one group's exponentials overlap the other's loads and maxima.  A group's
 //              running max only moves when a block's max exceeds it by more than 2^8 (then its
 //              O is rescaled in TMEM); in between P = 2^(s - m) stays <= 2^8, well inside bf16
@@ -47,8 +48,15 @@ constexpr uint32_t kTcCols = 512;                // TMEM columns allocated
 constexpr uint32_t kColO = 256;                  // + 128 per group
 constexpr int kSoftWarps = 8;
 constexpr int kSoftThreads = 32 * kSoftWarps;
-constexpr int kVWarp = 2 + kSoftWarps;
-constexpr int kTcThreads = 32 * (3 + kSoftWarps);
+constexpr int kVWarp = 2;
+constexpr int kTcThreads = 32 * (4 + kSoftWarps);  // warpgroup 0: roles; 1 and 2: softmax
+// Registers per thread after the split: the kernel is launched with kRegsLaunch per thread
+// (384 threads, 65536 registers), warpgroup 0 gives up to kRegsRoles and the two softmax
+// warpgroups take kRegsSoftmax; the split never asks for more than the launch holds (an
+// increase waits until the registers are free, so a larger one would wait forever).
+constexpr int kRegsLaunch = 168, kRegsRoles = 56, kRegsSoftmax = 224;
+static_assert(128 * kRegsRoles + 256 * kRegsSoftmax <= kTcThreads * kRegsLaunch,
+              "register split must fit in the launch's registers");
 constexpr float kLazyLog2 = 8.f;                 // rescale only when the max grows by > 2^8
 
 constexpr size_t tc_smem_bytes() {
@@ -165,6 +173,9 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   tc_fence_after();
   const uint32_t tbase = *tmem_base_s;
 
+  if (warp < 4) {
+  // warpgroup 0: the roles, on few registers (each branch keeps its own budget to the end)
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegsRoles));
   if (warp == 0 || warp == kVWarp) {
     // ============================================================== K or V producer
     const bool is_k = warp == 0;
@@ -287,12 +298,15 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       if (!mbar_wait(mma_done, 0, abort_flag)) report(a.dev_err, MSA_DEVERR_TIMEOUT);
     }
     __syncwarp();
+  }
+  // warp 3: no role of its own (its registers went to the softmax warpgroups)
   } else {
     // ============================================================== softmax warpgroups
-    const int w = (warp - 2) >> 2;       // this group takes blocks w, w + 2, w + 4, ...
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kRegsSoftmax));
+    const int w = (warp - 4) >> 2;       // this group takes blocks w, w + 2, w + 4, ...
     const int quarter = warp & 3;        // TMEM lanes 32 * quarter .. + 31
     const int r = quarter * 32 + lane;   // this thread's query row
-    const int gt = (warp - 2 - 4 * w) * 32 + lane;  // 0 .. 127 within the group
+    const int gt = (warp - 4 - 4 * w) * 32 + lane;  // 0 .. 127 within the group
     const uint32_t lane_addr = tbase + (static_cast<uint32_t>(quarter * 32) << 16);
     const uint32_t s_addr = lane_addr + w * 128;
     const uint32_t o_addr = lane_addr + kColO + w * 128;
@@ -345,22 +359,20 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       float m8[8];
 #pragma unroll
       for (int k = 0; k < 8; ++k) m8[k] = -INFINITY;
+      uint32_t v[128];  // the row's 128 scores
       if (any_use) {
-        // row max, 64 scores at a time (eight independent chains)
 #pragma unroll
-        for (int h = 0; h < 2; ++h) {
-          uint32_t v[64];
-          tmem_ld32(s_addr + 64 * h, *reinterpret_cast<uint32_t(*)[32]>(v));
-          tmem_ld32(s_addr + 64 * h + 32, *reinterpret_cast<uint32_t(*)[32]>(v + 32));
-          tmem_wait_ld();
-          if (plain) {
+        for (int c = 0; c < 4; ++c)
+          tmem_ld32(s_addr + 32 * c, *reinterpret_cast<uint32_t(*)[32]>(v + 32 * c));
+        tmem_wait_ld();
+        // row max (eight independent chains)
+        if (plain) {
 #pragma unroll
-            for (int e = 0; e < 64; ++e) m8[e & 7] = fmaxf(m8[e & 7], __uint_as_float(v[e]));
-          } else {
+          for (int e = 0; e < 128; ++e) m8[e & 7] = fmaxf(m8[e & 7], __uint_as_float(v[e]));
+        } else {
 #pragma unroll
-            for (int e = 0; e < 64; ++e)
-              if (use && 64 * h + e <= lim) m8[e & 7] = fmaxf(m8[e & 7], __uint_as_float(v[e]));
-          }
+          for (int e = 0; e < 128; ++e)
+            if (use && e <= lim) m8[e & 7] = fmaxf(m8[e & 7], __uint_as_float(v[e]));
         }
 #pragma unroll
         for (int k = 0; k < 4; ++k) m8[k] = fmaxf(m8[k], m8[k + 4]);
@@ -384,20 +396,15 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         tmem_st32(s_addr, z);
         tmem_st32(s_addr + 32, z);
       } else {
-        // P as bf16 into TMEM over the first 64 columns of S; the scores are read again, 64
-        // at a time (P of positions 0-63 overwrites their columns after they were read back)
+        // P as bf16 into TMEM over the first 64 columns of S (the scores were read already)
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
-          uint32_t v[64];
-          tmem_ld32(s_addr + 64 * h, *reinterpret_cast<uint32_t(*)[32]>(v));
-          tmem_ld32(s_addr + 64 * h + 32, *reinterpret_cast<uint32_t(*)[32]>(v + 32));
-          tmem_wait_ld();
           uint32_t pk[32];
           if (plain) {
 #pragma unroll
             for (int e = 0; e < 64; e += 2) {
-              const float e0 = fast_exp2(fmaf(__uint_as_float(v[e]), sc, nb));
-              const float e1 = fast_exp2(fmaf(__uint_as_float(v[e + 1]), sc, nb));
+              const float e0 = fast_exp2(fmaf(__uint_as_float(v[64 * h + e]), sc, nb));
+              const float e1 = fast_exp2(fmaf(__uint_as_float(v[64 * h + e + 1]), sc, nb));
               ps4[(e >> 1) & 3] += e0 + e1;
               pk[e >> 1] = pack_bf16x2(e0, e1);
             }
@@ -405,10 +412,10 @@ __global__ void __launch_bounds__(kTcThreads, 1)
 #pragma unroll
             for (int e = 0; e < 64; e += 2) {
               const int pe = 64 * h + e;
-              const float x0 = (use && pe <= lim) ? fmaf(__uint_as_float(v[e]), sc, nb)
+              const float x0 = (use && pe <= lim) ? fmaf(__uint_as_float(v[pe]), sc, nb)
                                                   : -INFINITY;
               const float x1 = (use && pe + 1 <= lim)
-                                   ? fmaf(__uint_as_float(v[e + 1]), sc, nb)
+                                   ? fmaf(__uint_as_float(v[pe + 1]), sc, nb)
                                    : -INFINITY;
               const float e0 = fast_exp2(x0), e1 = fast_exp2(x1);
               ps4[(e >> 1) & 3] += e0 + e1;
@@ -515,6 +522,19 @@ bool attention_tc_supported(int G, int qt) { return qt * G <= kTcRows && qt <= 3
 
 cudaError_t launch_attention_tc(const CUtensorMap &kmap, const CUtensorMap &vmap,
                                 const AttnArgs &a, cudaStream_t s) {
+  // The register split is only valid for a launch with exactly kRegsLaunch registers per
+  // thread (a larger split than the launch holds would wait forever): checked once per device.
+  static int checked[64] = {0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+  if (!checked[dev]) {
+    cudaFuncAttributes fa;
+    cudaError_t e = cudaFuncGetAttributes(&fa, reinterpret_cast<const void *>(&attn_tc_kernel));
+    if (e != cudaSuccess) return e;
+    if (fa.numRegs != kRegsLaunch || fa.maxThreadsPerBlock < kTcThreads)
+      return cudaErrorInvalidConfiguration;
+    checked[dev] = 1;
+  }
   const size_t smem = tc_smem_bytes();
   cudaError_t e = ensure_smem_limit(reinterpret_cast<const void *>(&attn_tc_kernel),
                                     static_cast<int>(smem));
