@@ -10,6 +10,8 @@
 // One warp per item: a shared-memory bitmap of the blocks marks the union, a warp prefix sum
 // of the word popcounts gives each block its union index, and each token ORs its bit into
 // the mask of every block it selected.
+#include <climits>
+
 #include "internal.h"
 #include "ptx.cuh"
 
@@ -43,28 +45,51 @@ __global__ void __launch_bounds__(32) plan_kernel(const PlanArgs a) {
   }
   const int ntok = min(a.qt, q_len - tok0);
   const int cl = a.cache_len[b];
+  // the tokens' selection counts, one lane each (ntok <= 32), read all at once
+  int n_l = 0;
+  if (lane < ntok) {
+    n_l = a.num_selected[static_cast<size_t>(row0 + tok0 + lane) * a.H_kv + g];
+    if (n_l < 0 || n_l > a.S) {
+      report(a.dev_err, MSA_DEVERR_NUM_SELECTED);
+      n_l = n_l < 0 ? 0 : a.S;
+    }
+  }
+  // Every (token, slot) pair of the tile, kR per lane at a time, so that the loads of all the
+  // tokens' ids are in flight together; `fn(i, j)` is called for each valid id j of token i.
+  constexpr int kR = 8;
+  const int total = ntok * a.S;
+  auto for_each_id = [&](auto fn) {
+    for (int k0 = 0; k0 < total; k0 += 32 * kR) {
+      int jr[kR], ir[kR];
+#pragma unroll
+      for (int r = 0; r < kR; ++r) {
+        const int k = k0 + r * 32 + lane;
+        const int i = k < total ? k / a.S : 0, sl = k - i * a.S;
+        const int n = __shfl_sync(0xffffffffu, n_l, i);
+        ir[r] = i;
+        jr[r] = (k < total && sl < n)
+                    ? a.block_ids[(static_cast<size_t>(row0 + tok0 + i) * a.H_kv + g) * a.S + sl]
+                    : INT_MIN;
+      }
+#pragma unroll
+      for (int r = 0; r < kR; ++r) {
+        if (jr[r] == INT_MIN) continue;
+        const int nb = (cl + tok0 + ir[r]) / kBlock + 1;
+        fn(ir[r], jr[r], jr[r] >= 0 && jr[r] < nb && jr[r] < a.max_blocks);
+      }
+    }
+  };
 
   for (int w = lane; w < words; w += 32) bitmap[w] = 0;
   __syncwarp();
   // mark the union
-  for (int i = 0; i < ntok; ++i) {
-    const size_t sel = static_cast<size_t>(row0 + tok0 + i) * a.H_kv + g;
-    int n = a.num_selected[sel];
-    if (n < 0 || n > a.S) {
-      if (lane == 0) report(a.dev_err, MSA_DEVERR_NUM_SELECTED);
-      n = n < 0 ? 0 : a.S;
+  for_each_id([&](int, int j, bool valid) {
+    if (!valid) {
+      report(a.dev_err, MSA_DEVERR_BLOCK_ID);
+      return;
     }
-    const int nb = (cl + tok0 + i) / kBlock + 1;
-    const int32_t *ids = a.block_ids + sel * a.S;
-    for (int s = lane; s < n; s += 32) {
-      const int j = ids[s];
-      if (j < 0 || j >= nb || j >= a.max_blocks) {
-        report(a.dev_err, MSA_DEVERR_BLOCK_ID);
-        continue;
-      }
-      atomicOr(&bitmap[j >> 5], 1u << (j & 31));
-    }
-  }
+    atomicOr(&bitmap[j >> 5], 1u << (j & 31));
+  });
   __syncwarp();
   // exclusive prefix of the word popcounts
   uint32_t carry = 0;
@@ -84,19 +109,12 @@ __global__ void __launch_bounds__(32) plan_kernel(const PlanArgs a) {
   for (int e = lane; e < U; e += 32) mask_s[e] = 0;
   __syncwarp();
   // token masks
-  for (int i = 0; i < ntok; ++i) {
-    const size_t sel = static_cast<size_t>(row0 + tok0 + i) * a.H_kv + g;
-    const int n = min(max(a.num_selected[sel], 0), a.S);
-    const int nb = (cl + tok0 + i) / kBlock + 1;
-    const int32_t *ids = a.block_ids + sel * a.S;
-    for (int s = lane; s < n; s += 32) {
-      const int j = ids[s];
-      if (j < 0 || j >= nb || j >= a.max_blocks) continue;
-      const uint32_t w = bitmap[j >> 5];
-      const int e = static_cast<int>(wprefix[j >> 5]) + __popc(w & ((1u << (j & 31)) - 1u));
-      if (e < U) atomicOr(&mask_s[e], 1u << i);
-    }
-  }
+  for_each_id([&](int i, int j, bool valid) {
+    if (!valid) return;
+    const uint32_t w = bitmap[j >> 5];
+    const int e = static_cast<int>(wprefix[j >> 5]) + __popc(w & ((1u << (j & 31)) - 1u));
+    if (e < U) atomicOr(&mask_s[e], 1u << i);
+  });
   __syncwarp();
   // write the CSR row
   int32_t *list = a.list + item * a.cap;
