@@ -25,7 +25,7 @@ namespace msa {
 
 namespace {
 
-constexpr int kStages = 3;
+constexpr int kStages = 2;  // two 32 KiB stages: three CTAs per SM hide latency better than deeper rings
 constexpr uint32_t kTileBytes = kBlock * kHeadDim * 2;  // one (page, head) tile, bf16
 constexpr int kConsumerWarps = 4;
 constexpr int kThreads = 32 * (kConsumerWarps + 1);
