@@ -17,7 +17,10 @@
 // every SM streams the same number of slots.  A CTA's range meets a few items; each meeting is
 // a "segment", merged inside the CTA into one partial (normalised output and log-sum-exp) at
 // split index `piece` = the CTA's rank among the CTAs that share the item; split indices no
-// CTA fills are marked empty.  msa_splitk_combine's kernel merges the pieces.
+// CTA fills are marked empty.  msa_splitk_combine's kernel merges the pieces.  With a single
+// partition (every item inside one CTA) the kernel writes the bf16 output itself instead.
+// On speculative tiles a row group (16 rows: two draft tokens) skips the math of a union block
+// that neither of its tokens selected: their state would not change.
 //
 // Roles: one producer warp walks the items, marks empty partials, loads each non-empty
 // segment's Q rows and metadata into a double-buffered Q slot and issues the TMA loads of the

@@ -249,9 +249,10 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         return true;
       };
       // Event loop: the P V of the next block once its P (and V) is there, and the QK^T of the
-      // next block once the P V that read its group's buffer is done, both in block order, so
-      // that neither group waits behind the other's step.  Every barrier's phases are polled
-      // in order.
+      // next block once the P V that read its group's buffer is done, each in block order, so
+      // that a QK^T never waits behind a P V that is not ready.  Every barrier's phases are
+      // polled in order.  (Issuing per group out of block order measured slower: the groups
+      // drift apart and the shared K ring serialises them anyway.)
       bool alive = qk(0) && (nblk < 2 || qk(1));
       int next_pv = 0, next_qk = 2;
       uint64_t t_idle = 0;
