@@ -327,10 +327,15 @@ def run_ours(args):
     stream_route = prob["max_q_len"] <= 8  # decode / speculative: persistent kernel + combine
     splits_used = msa.msa_attn_partials(path.rp, prob["S"], prob["H_q"], prob["H_kv"],
                                         path.max_blocks, args.splits)[0] if stream_route else 1
-    # decode / speculative: index, select, [plan], attention, [combine: only with more than one
-    # split-K partition]; prefill: index, select, plan, attention
-    kernels_per_step = (3 + (1 if prob["max_q_len"] > 1 else 0) + (1 if splits_used > 1 else 0)
-                        if stream_route else 4)
+    # decode: index, attention with the selection inside, [combine: only with more than one
+    # split-K partition]; speculative: index, select, plan, attention, [combine];
+    # prefill: index, select, plan, attention
+    if prob["max_q_len"] == 1 and prob["H_q"] // prob["H_kv"] <= 16:
+        kernels_per_step = 2 + (1 if splits_used > 1 else 0)
+    elif stream_route:
+        kernels_per_step = 4 + (1 if splits_used > 1 else 0)
+    else:
+        kernels_per_step = 4
 
     for _ in range(args.warmup):
         path.run(stream)
@@ -395,8 +400,13 @@ def run_ours(args):
                          lambda: path.attend(stream=stream)])
         stages = {"index_scores": st[0], "select": st[1], attn_key: st[2]}
     if stream_route:
-        # the first two stages as one msa_index_select launch, for comparison
+        # the first two stages as one msa_index_select launch, and the last two (with the
+        # combine) as one msa_select_sparse_attn_paged call, for comparison
         stages["fused_index_select"] = stage_pass([lambda: path.index_select(stream)])[0]
+        stages["select_in_attention"] = stage_pass([lambda: path.select_attend(stream)])[0]
+        stages["step_with_separate_select"] = stage_pass(
+            [lambda: (path.index_scores(stream), path.select(stream=stream),
+                      path.attend(stream=stream))])[0]
         idx_kind, idx_src = "index_scores", "indexer.cu"
     else:
         st = stage_pass([lambda: path.index_scores(stream), lambda: path.select(stream=stream),

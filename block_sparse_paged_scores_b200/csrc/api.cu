@@ -427,13 +427,31 @@ msa_status_t msa_splitk_combine(const float *partial_o, const float *partial_lse
              : MSA_ERR_CUDA;
 }
 
-msa_status_t msa_sparse_attn_paged(const msa_ragged_paged_t *rp, const void *q,
-                                   const void *k_cache, const void *v_cache,
-                                   msa_kv_dtype_t kv_dtype, const int32_t *block_ids,
-                                   const int32_t *num_selected, int32_t S, int32_t num_q_heads,
-                                   int32_t num_kv_heads, int32_t max_blocks, float scale,
-                                   int32_t num_splits, void *workspace, size_t workspace_bytes,
-                                   void *out, int32_t *dev_err, struct CUstream_st *stream) {
+}  // extern "C"
+
+namespace {
+
+// The selection to run inside the decode attention kernel (msa_select_sparse_attn_paged).
+struct AttnSelect {
+  const float *scores;
+  int32_t *block_ids, *num_selected;
+  int top_k, init_blocks, local_blocks;
+};
+
+// Whether msa_select_sparse_attn_paged selects inside the attention kernel for this shape: the
+// decode route with one 16-row group per item.
+bool select_in_attention(const msa_ragged_paged_t *rp, int num_q_heads, int num_kv_heads) {
+  return rp->max_q_len == 1 && num_q_heads / num_kv_heads <= 16;
+}
+
+// msa_sparse_attn_paged's body.  dry_run: validate only (nothing enqueued); sel: select inside
+// the decode attention kernel (block_ids / num_selected are then its outputs).
+msa_status_t attn_impl(const msa_ragged_paged_t *rp, const void *q, const void *k_cache,
+                       const void *v_cache, msa_kv_dtype_t kv_dtype, const int32_t *block_ids,
+                       const int32_t *num_selected, int32_t S, int32_t num_q_heads,
+                       int32_t num_kv_heads, int32_t max_blocks, float scale, int32_t num_splits,
+                       void *workspace, size_t workspace_bytes, void *out, int32_t *dev_err,
+                       struct CUstream_st *stream, bool dry_run, const AttnSelect *sel) {
   if (ragged_ok(rp) && rp->total_q == 0 && S >= 1) return MSA_OK;  // nothing to attend
   if (!ragged_ok(rp) || !q || !k_cache || !v_cache || !block_ids || !num_selected ||
       S < 1 || num_kv_heads < 1 || num_q_heads < num_kv_heads ||
@@ -456,6 +474,8 @@ msa_status_t msa_sparse_attn_paged(const msa_ragged_paged_t *rp, const void *q,
   if (static_cast<long long>(rp->batch) * r.tiles > 0x7fffffffLL) return MSA_ERR_UNSUPPORTED;
   if (r.bytes > 0 && (!workspace || workspace_bytes < r.bytes || !aligned(workspace, 256)))
     return MSA_ERR_INVALID_ARG;
+  if (sel && (!r.stream || r.plan || r.rg != 1)) return MSA_ERR_UNSUPPORTED;
+  if (dry_run) return MSA_OK;
 
   uint8_t *ws = static_cast<uint8_t *>(workspace);
   const cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
@@ -520,6 +540,12 @@ msa_status_t msa_sparse_attn_paged(const msa_ragged_paged_t *rp, const void *q,
   // one partition: every item lies inside one CTA, which then writes the output itself
   a.direct = r.stream && r.splits == 1 && out != nullptr;
   a.dev_err = dev_err;
+  a.scores = sel ? sel->scores : nullptr;
+  a.sel_ids = sel ? sel->block_ids : nullptr;
+  a.sel_counts = sel ? sel->num_selected : nullptr;
+  a.top_k = sel ? sel->top_k : 0;
+  a.init_blocks = sel ? sel->init_blocks : 0;
+  a.local_blocks = sel ? sel->local_blocks : 0;
   if (r.tc)
     return launch_attention_tc(kmap, vmap, a, s) == cudaSuccess ? MSA_OK : MSA_ERR_CUDA;
   if (!r.stream)
@@ -532,6 +558,57 @@ msa_status_t msa_sparse_attn_paged(const msa_ragged_paged_t *rp, const void *q,
       cudaSuccess)
     return MSA_ERR_CUDA;
   return MSA_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+msa_status_t msa_sparse_attn_paged(const msa_ragged_paged_t *rp, const void *q,
+                                   const void *k_cache, const void *v_cache,
+                                   msa_kv_dtype_t kv_dtype, const int32_t *block_ids,
+                                   const int32_t *num_selected, int32_t S, int32_t num_q_heads,
+                                   int32_t num_kv_heads, int32_t max_blocks, float scale,
+                                   int32_t num_splits, void *workspace, size_t workspace_bytes,
+                                   void *out, int32_t *dev_err, struct CUstream_st *stream) {
+  return attn_impl(rp, q, k_cache, v_cache, kv_dtype, block_ids, num_selected, S, num_q_heads,
+                   num_kv_heads, max_blocks, scale, num_splits, workspace, workspace_bytes, out,
+                   dev_err, stream, false, nullptr);
+}
+
+msa_status_t msa_select_sparse_attn_paged(
+    const msa_ragged_paged_t *rp, const float *scores, int32_t top_k, int32_t init_blocks,
+    int32_t local_blocks, const void *q, const void *k_cache, const void *v_cache,
+    msa_kv_dtype_t kv_dtype, int32_t num_q_heads, int32_t num_kv_heads, int32_t max_blocks,
+    float scale, int32_t num_splits, void *workspace, size_t workspace_bytes,
+    int32_t *block_ids, int32_t *num_selected, void *out, int32_t *dev_err,
+    struct CUstream_st *stream) {
+  const long long S = static_cast<long long>(top_k) + init_blocks + local_blocks;
+  if (!ragged_ok(rp) || top_k < 0 || init_blocks < 0 || local_blocks < 0 || S < 1 ||
+      S > (1 << 20) || num_kv_heads < 1 || num_q_heads < num_kv_heads)
+    return MSA_ERR_INVALID_ARG;
+  if (rp->total_q == 0) return MSA_OK;
+  if (!scores || !block_ids || !num_selected) return MSA_ERR_INVALID_ARG;
+  const int Si = static_cast<int>(S);
+  // everything validated before anything is enqueued
+  const msa_status_t v = attn_impl(rp, q, k_cache, v_cache, kv_dtype, block_ids, num_selected,
+                                   Si, num_q_heads, num_kv_heads, max_blocks, scale, num_splits,
+                                   workspace, workspace_bytes, out, dev_err, stream, true,
+                                   nullptr);
+  if (v != MSA_OK) return v;
+  if (select_in_attention(rp, num_q_heads, num_kv_heads)) {
+    const AttnSelect sel{scores, block_ids, num_selected, top_k, init_blocks, local_blocks};
+    return attn_impl(rp, q, k_cache, v_cache, kv_dtype, block_ids, num_selected, Si,
+                     num_q_heads, num_kv_heads, max_blocks, scale, num_splits, workspace,
+                     workspace_bytes, out, dev_err, stream, false, &sel);
+  }
+  const msa_status_t e = msa_select_blocks(rp, scores, num_kv_heads, max_blocks, top_k,
+                                           init_blocks, local_blocks, block_ids, num_selected,
+                                           dev_err, stream);
+  if (e != MSA_OK) return e;
+  return attn_impl(rp, q, k_cache, v_cache, kv_dtype, block_ids, num_selected, Si, num_q_heads,
+                   num_kv_heads, max_blocks, scale, num_splits, workspace, workspace_bytes, out,
+                   dev_err, stream, false, nullptr);
 }
 
 }  // extern "C"

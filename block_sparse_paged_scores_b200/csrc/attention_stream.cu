@@ -33,6 +33,7 @@
 #include <math.h>
 
 #include "attn_common.cuh"
+#include "select_row.cuh"
 
 namespace msa {
 
@@ -151,7 +152,9 @@ __device__ __forceinline__ void segment(const AttnArgs &a, int it, long long r0,
   v1 = min(s1, U);
 }
 
-template <bool FP8, int RG, bool PLAN>
+// SEL >= 0: decode with the selection in the kernel (select_row with SEL keys per lane in
+// registers, 0: from memory); SEL < 0: the selection comes from an earlier launch.
+template <bool FP8, int RG, bool PLAN, int SEL>
 __global__ void __launch_bounds__(32 * (stream_consumer_warps<FP8, RG>() + 1))
     attn_stream_kernel(const __grid_constant__ CUtensorMap kmap,
                        const __grid_constant__ CUtensorMap vmap, const AttnArgs a) {
@@ -207,8 +210,32 @@ __global__ void __launch_bounds__(32 * (stream_consumer_warps<FP8, RG>() + 1))
     fence_mbar_init();
   }
   __syncthreads();
-  pdl_wait();  // block ids, selection counts and the plan come from earlier kernels
+  pdl_wait();  // block ids, selection counts and the plan (or the scores) come from earlier kernels
   pdl_launch_dependents();
+
+  if constexpr (SEL >= 0) {
+    // Decode: every warp of the CTA selects rows of the CTA's items (one query row per item;
+    // block_sparse_select as in select.cu), before any of them is streamed.  Items shared
+    // with a neighbouring CTA are selected by both, with identical results.
+    const int n_items = it_last - it_first + 1;
+    for (int k = warp; k < n_items; k += NCW + 1) {
+      const int it = it_first + k;
+      const int g = it % a.H_kv, b = it / a.H_kv;  // one query tile per sequence
+      const int row0 = a.row_off[b];
+      if (a.row_off[b + 1] - row0 <= 0) continue;  // no query row
+      int nb = max(a.cache_len[b], 0) / kBlock + 1;
+      if (nb > a.max_blocks) {
+        if (lane == 0) report(a.dev_err, MSA_DEVERR_LENGTHS);
+        nb = a.max_blocks;
+      }
+      const size_t sel = static_cast<size_t>(row0) * a.H_kv + g;
+      const int nsel = select_row<(SEL > 0 ? SEL : 0), false>(
+          a.scores + sel * a.max_blocks, nb, a.top_k, a.init_blocks, a.local_blocks, a.S,
+          a.sel_ids + sel * a.S, a.dev_err, lane);
+      if (lane == 0) a.sel_counts[sel] = nsel;
+    }
+    __syncthreads();  // the producer reads the selection back
+  }
 
   if (warp == NCW) {
     // ============================================================== producer warp
@@ -449,11 +476,11 @@ __global__ void __launch_bounds__(32 * (stream_consumer_warps<FP8, RG>() + 1))
   }
 }
 
-template <bool FP8, int RG, bool PLAN>
+template <bool FP8, int RG, bool PLAN, int SEL>
 cudaError_t launch_stream_one(const CUtensorMap &kmap, const CUtensorMap &vmap,
                               const AttnArgs &a, int grid, cudaStream_t s) {
   const size_t smem = stream_smem_bytes<FP8, RG>();
-  auto fn = &attn_stream_kernel<FP8, RG, PLAN>;
+  auto fn = &attn_stream_kernel<FP8, RG, PLAN, SEL>;
   cudaError_t e = ensure_smem_limit(reinterpret_cast<const void *>(fn), static_cast<int>(smem));
   if (e != cudaSuccess) return e;
   return launch_pdl(fn, dim3(grid), dim3(32 * (stream_consumer_warps<FP8, RG>() + 1)), smem, s,
@@ -464,11 +491,21 @@ template <bool FP8, bool PLAN>
 cudaError_t launch_stream_rg(const CUtensorMap &kmap, const CUtensorMap &vmap, const AttnArgs &a,
                              int rg, int grid, cudaStream_t s) {
   switch (rg) {
-    case 1: return launch_stream_one<FP8, 1, PLAN>(kmap, vmap, a, grid, s);
-    case 2: return launch_stream_one<FP8, 2, PLAN>(kmap, vmap, a, grid, s);
-    case 3: return launch_stream_one<FP8, 3, PLAN>(kmap, vmap, a, grid, s);
-    default: return launch_stream_one<FP8, 4, PLAN>(kmap, vmap, a, grid, s);
+    case 1: return launch_stream_one<FP8, 1, PLAN, -1>(kmap, vmap, a, grid, s);
+    case 2: return launch_stream_one<FP8, 2, PLAN, -1>(kmap, vmap, a, grid, s);
+    case 3: return launch_stream_one<FP8, 3, PLAN, -1>(kmap, vmap, a, grid, s);
+    default: return launch_stream_one<FP8, 4, PLAN, -1>(kmap, vmap, a, grid, s);
   }
+}
+
+// decode with the selection inside: one row group, keys per lane chosen by the row length
+template <bool FP8>
+cudaError_t launch_stream_sel(const CUtensorMap &kmap, const CUtensorMap &vmap, const AttnArgs &a,
+                              int grid, cudaStream_t s) {
+  if (a.max_blocks <= 4 * 32) return launch_stream_one<FP8, 1, false, 4>(kmap, vmap, a, grid, s);
+  if (a.max_blocks <= 16 * 32) return launch_stream_one<FP8, 1, false, 16>(kmap, vmap, a, grid, s);
+  if (a.max_blocks <= 32 * 32) return launch_stream_one<FP8, 1, false, 32>(kmap, vmap, a, grid, s);
+  return launch_stream_one<FP8, 1, false, 0>(kmap, vmap, a, grid, s);
 }
 
 }  // namespace
@@ -476,6 +513,11 @@ cudaError_t launch_stream_rg(const CUtensorMap &kmap, const CUtensorMap &vmap, c
 cudaError_t launch_attention_stream(const CUtensorMap &kmap, const CUtensorMap &vmap,
                                     const AttnArgs &a, bool fp8, int rg, bool plan, int grid,
                                     cudaStream_t s) {
+  if (a.sel_ids) {  // decode (rg == 1, no plan) with the selection inside
+    if (plan || rg != 1) return cudaErrorInvalidValue;
+    return fp8 ? launch_stream_sel<true>(kmap, vmap, a, grid, s)
+               : launch_stream_sel<false>(kmap, vmap, a, grid, s);
+  }
   if (fp8)
     return plan ? launch_stream_rg<true, true>(kmap, vmap, a, rg, grid, s)
                 : launch_stream_rg<true, false>(kmap, vmap, a, rg, grid, s);

@@ -25,11 +25,15 @@ namespace msa {
 
 namespace {
 
-constexpr int kStages = 2;  // two 32 KiB stages: three CTAs per SM hide latency better than deeper rings
+// Ring depth: two 32 KiB stages (three CTAs per SM) for CTAs with a short chunk of pages, three
+// (two CTAs per SM) for long ones: the same bytes in flight per SM, but more pages in process at
+// once wins on short chunks, a deeper ring on long streams.
+constexpr int kLongChunk = 32;  // pages per CTA from which the deeper ring is used
 constexpr uint32_t kTileBytes = kBlock * kHeadDim * 2;  // one (page, head) tile, bf16
 constexpr int kConsumerWarps = 4;
 constexpr int kThreads = 32 * (kConsumerWarps + 1);
 
+template <int kStages>
 constexpr size_t smem_bytes() {
   return 1024 /*alignment slack*/ + kStages * kTileBytes + 2 * kStages * sizeof(uint64_t) +
          kStages * sizeof(int) + 2 * kConsumerWarps * 32 * sizeof(float) + 16;
@@ -70,7 +74,7 @@ __device__ __forceinline__ void count_out_and_select(const IndexerArgs &a, int b
 
 // KPL < 0: scores only; KPL >= 0: selection fused, KPL keys per lane in registers (0: any
 // number of blocks, read from L2 on every pass).
-template <int MT, int KPL>
+template <int MT, int KPL, int kStages>
 __global__ void __launch_bounds__(kThreads)
     index_scores_kernel(const __grid_constant__ CUtensorMap kmap, const IndexerArgs a) {
   pdl_wait();
@@ -290,25 +294,32 @@ __global__ void __launch_bounds__(kThreads)
   if (KPL >= 0) count_out_and_select<KPL>(a, b, tile, hk, row0, tok0, ntok, cl, is_last);
 }
 
-template <int MT, int KPL>
+template <int MT, int KPL, int ST>
 cudaError_t launch_one(const CUtensorMap &kidx_map, const IndexerArgs &a, int chunks,
                        cudaStream_t s) {
   const dim3 grid(a.batch * a.tiles * a.H_idxk * chunks);
-  const size_t smem = smem_bytes();
-  cudaError_t e = ensure_smem_limit(reinterpret_cast<const void *>(&index_scores_kernel<MT, KPL>),
-                                    static_cast<int>(smem));
+  const size_t smem = smem_bytes<ST>();
+  cudaError_t e = ensure_smem_limit(
+      reinterpret_cast<const void *>(&index_scores_kernel<MT, KPL, ST>), static_cast<int>(smem));
   if (e != cudaSuccess) return e;
-  return launch_pdl(index_scores_kernel<MT, KPL>, grid, dim3(kThreads), smem, s, kidx_map, a);
+  return launch_pdl(index_scores_kernel<MT, KPL, ST>, grid, dim3(kThreads), smem, s, kidx_map, a);
+}
+
+template <int MT, int KPL>
+cudaError_t launch_st(const CUtensorMap &kidx_map, const IndexerArgs &a, int chunks,
+                      cudaStream_t s) {
+  return a.chunk >= kLongChunk ? launch_one<MT, KPL, 3>(kidx_map, a, chunks, s)
+                               : launch_one<MT, KPL, 2>(kidx_map, a, chunks, s);
 }
 
 template <int MT>
 cudaError_t launch_mt(const CUtensorMap &kidx_map, const IndexerArgs &a, int chunks,
                       cudaStream_t s) {
-  if (!a.counters) return launch_one<MT, -1>(kidx_map, a, chunks, s);
-  if (a.max_blocks <= 4 * 32) return launch_one<MT, 4>(kidx_map, a, chunks, s);
-  if (a.max_blocks <= 16 * 32) return launch_one<MT, 16>(kidx_map, a, chunks, s);
-  if (a.max_blocks <= 32 * 32) return launch_one<MT, 32>(kidx_map, a, chunks, s);
-  return launch_one<MT, 0>(kidx_map, a, chunks, s);
+  if (!a.counters) return launch_st<MT, -1>(kidx_map, a, chunks, s);
+  if (a.max_blocks <= 4 * 32) return launch_st<MT, 4>(kidx_map, a, chunks, s);
+  if (a.max_blocks <= 16 * 32) return launch_st<MT, 16>(kidx_map, a, chunks, s);
+  if (a.max_blocks <= 32 * 32) return launch_st<MT, 32>(kidx_map, a, chunks, s);
+  return launch_st<MT, 0>(kidx_map, a, chunks, s);
 }
 
 }  // namespace

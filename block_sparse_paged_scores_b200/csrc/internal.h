@@ -82,6 +82,11 @@ struct AttnArgs {
                              // kernel when `direct`
   int direct;                // persistent kernel with P == 1 (every item inside one CTA): write
                              // O / l to `out` instead of partials (no combine follows)
+  // Selection inside the decode attention kernel (sel_ids != nullptr): every CTA first selects
+  // the rows of its items from `scores` into sel_ids / sel_counts (== block_ids / num_selected).
+  const float *scores;
+  int32_t *sel_ids, *sel_counts;
+  int top_k, init_blocks, local_blocks;
   int32_t *dev_err;
 };
 // rg = 16-row groups (1..4); plan = read the per-tile union instead of the selection

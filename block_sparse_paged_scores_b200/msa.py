@@ -62,6 +62,9 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.msa_sparse_attn_paged.restype = I
     lib.msa_sparse_attn_paged.argtypes = [RP, P, P, P, I, P, P, I, I, I, I, F, I, P,
                                           ctypes.c_size_t, P, P, P]
+    lib.msa_select_sparse_attn_paged.restype = I
+    lib.msa_select_sparse_attn_paged.argtypes = [RP, P, I, I, I, P, P, P, I, I, I, I, F, I, P,
+                                                 ctypes.c_size_t, P, P, P, P, P]
     lib.msa_splitk_combine.restype = I
     lib.msa_splitk_combine.argtypes = [P, P, I, I, I, P, P]
     lib.msa_attn_workspace_bytes.restype = ctypes.c_size_t
@@ -176,6 +179,21 @@ def msa_sparse_attn_paged(rp: RaggedPaged, q, k_cache, v_cache, kv_dtype: int, b
         _ptr(workspace), int(workspace_bytes), _ptr(out), _ptr(dev_err), _stream(stream)))
 
 
+def msa_select_sparse_attn_paged(rp: RaggedPaged, scores, top_k: int, init_blocks: int,
+                                 local_blocks: int, q, k_cache, v_cache, kv_dtype: int,
+                                 num_q_heads: int, num_kv_heads: int, max_blocks: int,
+                                 scale: float, num_splits: int, workspace, block_ids,
+                                 num_selected, out, dev_err=None, stream=None,
+                                 workspace_bytes: Optional[int] = None):
+    if workspace_bytes is None:
+        workspace_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _check("msa_select_sparse_attn_paged", load().msa_select_sparse_attn_paged(
+        ctypes.byref(rp), _ptr(scores), top_k, init_blocks, local_blocks, _ptr(q), _ptr(k_cache),
+        _ptr(v_cache), int(kv_dtype), num_q_heads, num_kv_heads, max_blocks, float(scale),
+        num_splits, _ptr(workspace), int(workspace_bytes), _ptr(block_ids), _ptr(num_selected),
+        _ptr(out), _ptr(dev_err), _stream(stream)))
+
+
 def msa_sparse_attn_paged_noalloc(rp: RaggedPaged, q, k_cache, v_cache, kv_dtype: int,
                                   block_ids, num_selected, S: int, num_q_heads: int,
                                   num_kv_heads: int, max_blocks: int, scale: float,
@@ -199,13 +217,16 @@ def msa_splitk_combine(partial_o, partial_lse, num_splits: int, total_q: int, nu
 class Path:
     """The three stages over one problem (a dict laid out as ``workload.generate`` returns),
     with every output and the workspace allocated once on the problem's device.  ``run()``
-    enqueues index scores -> selection -> attention on the current stream (with
-    ``fused_select`` the first two as one msa_index_select call)."""
+    enqueues index scores -> selection -> attention on the current stream: by default the
+    last two as one msa_select_sparse_attn_paged call (``select_in_attention``); with
+    ``fused_select`` the first two as one msa_index_select call; with neither, three separate
+    calls."""
 
     def __init__(self, prob: dict, num_splits: int = 0, max_blocks: Optional[int] = None,
-                 fused_select: bool = False):
+                 fused_select: bool = False, select_in_attention: bool = True):
         self.p = prob
         self.fused_select = fused_select
+        self.select_in_attention = select_in_attention
         dev = prob["q"].device
         self.max_blocks = int(max_blocks or prob["max_blocks"])
         self.rp = ragged_paged(prob["row_off"], prob["cache_len"], prob["table"], prob["total_q"],
@@ -254,6 +275,16 @@ class Path:
                               self.num_splits, self.workspace, self.out if combine else 0,
                               self.dev_err, stream, workspace_bytes=self.workspace_bytes)
 
+    def select_attend(self, stream=None):
+        """Stages 2 and 3 in one call (msa_select_sparse_attn_paged: one launch on decode)."""
+        p = self.p
+        msa_select_sparse_attn_paged(self.rp, self.scores, p["top_k"], p["init_blocks"],
+                                     p["local_blocks"], p["q"], p["k"], p["v"], self.kv_dtype,
+                                     p["H_q"], p["H_kv"], self.max_blocks, p["scale"],
+                                     self.num_splits, self.workspace, self.block_ids,
+                                     self.num_selected, self.out, self.dev_err, stream,
+                                     workspace_bytes=self.workspace_bytes)
+
     def partials(self):
         n, o_off, l_off = msa_attn_partials(self.rp, self.p["S"], self.p["H_q"], self.p["H_kv"],
                                             self.max_blocks, self.num_splits)
@@ -266,6 +297,10 @@ class Path:
     def run(self, stream=None):
         if self.fused_select:
             self.index_select(stream)
+        elif self.select_in_attention:
+            self.index_scores(stream)
+            self.select_attend(stream)
+            return self.out
         else:
             self.index_scores(stream)
             self.select(stream=stream)

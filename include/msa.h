@@ -6,6 +6,7 @@
  *   msa_index_scores      block scores: max over a 128-token block of raw q_idx . k_idx
  *   msa_select_blocks     forced init/local blocks + top-k of the rest, ascending
  *   msa_index_select      the first two in one call (one launch on the decode routes)
+ *   msa_select_sparse_attn_paged  the last two in one call (one launch on the decode route)
  *   msa_sparse_attn_paged softmax attention over the selected pages (decode / speculative /
  *                         prefill routes picked from max_q_len), split-K + combine inside
  *   msa_splitk_combine    log-sum-exp merge of split-K partials into the ragged output
@@ -202,6 +203,31 @@ MSA_API msa_status_t msa_sparse_attn_paged(const msa_ragged_paged_t *rp, const v
                                    int32_t num_kv_heads, int32_t max_blocks, float scale,
                                    int32_t num_splits, void *workspace, size_t workspace_bytes,
                                    void *out, int32_t *dev_err, struct CUstream_st *stream);
+
+/*
+ * msa_select_sparse_attn_paged — stages 2 and 3 in one call: exactly msa_select_blocks
+ * followed by msa_sparse_attn_paged with the same arguments ([ferrox] block_sparse_select,
+ * positions_of_blocks; [msa] "Three attention routes"), with bit-identical block_ids and
+ * num_selected and the same output.
+ *
+ * On the decode route (max_q_len == 1) with a GQA group of at most 16 the selection runs inside
+ * the attention launch: each CTA of the persistent kernel first selects the rows of the items in
+ * its share of the work, then streams them, so the selection needs no launch of its own.  On the
+ * other routes it enqueues the two stages one after the other.
+ *
+ *   scores, top_k, init_blocks, local_blocks  as msa_select_blocks (S = init + local + top_k)
+ *   block_ids, num_selected  device int32 [total_q, num_kv_heads, S] / [total_q, num_kv_heads]
+ *                  (outputs, as msa_select_blocks writes them)
+ *   the rest      as msa_sparse_attn_paged.
+ *   Validation is that of both stages, all of it before anything is enqueued.
+ */
+MSA_API msa_status_t msa_select_sparse_attn_paged(
+    const msa_ragged_paged_t *rp, const float *scores, int32_t top_k, int32_t init_blocks,
+    int32_t local_blocks, const void *q, const void *k_cache, const void *v_cache,
+    msa_kv_dtype_t kv_dtype, int32_t num_q_heads, int32_t num_kv_heads, int32_t max_blocks,
+    float scale, int32_t num_splits, void *workspace, size_t workspace_bytes,
+    int32_t *block_ids, int32_t *num_selected, void *out, int32_t *dev_err,
+    struct CUstream_st *stream);
 
 /*
  * msa_sparse_attn_paged_noalloc — msa_sparse_attn_paged for callers that cannot provide a

@@ -128,6 +128,17 @@ def test_invalid_arguments_are_rejected_before_any_launch(lib):
     assert lib.msa_index_select(ctypes.byref(rp), P, P, 8, 1, 16, 0, 0, 0, P, P, P, P, None,
                                 None) == msa.MSA_ERR_INVALID_ARG                   # S = 0
     assert msa.msa_index_select_counters(_rp(batch=5, max_q_len=3, total_q=9), 8) == 5 * 3 * 8
+    # select + attention in one call: the selection's and the attention's validation, up front
+    sa = lambda **kw: lib.msa_select_sparse_attn_paged(
+        ctypes.byref(rp), kw.get("scores", P), kw.get("top_k", 4), 1, 1, P, P, P, 0, 64, 8, 16,
+        ctypes.c_float(kw.get("scale", 0.088)), 0, None, 0, kw.get("ids", P), P,
+        kw.get("out", P), None, None)
+    assert sa(scores=None) == msa.MSA_ERR_INVALID_ARG
+    assert sa(top_k=-1) == msa.MSA_ERR_INVALID_ARG
+    assert sa(ids=None) == msa.MSA_ERR_INVALID_ARG
+    assert sa(scale=0.0) == msa.MSA_ERR_INVALID_ARG
+    assert sa(out=P + 8) == msa.MSA_ERR_INVALID_ARG
+    assert sa() == msa.MSA_ERR_INVALID_ARG          # the decode route needs a workspace
     stat = lib.msa_select_blocks(ctypes.byref(rp), P, 8, 16, -1, 1, 1, P, P, None, None)
     assert stat == msa.MSA_ERR_INVALID_ARG
     bad = msa.RaggedPaged(P, P, P, 0, 2, 1, 16, 64)                                 # batch 0

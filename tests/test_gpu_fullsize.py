@@ -86,6 +86,16 @@ def test_full_size_workload(name):
     assert int(fused.counters.abs().sum().item()) == 0
     del fused
 
+    # the last two stages as one msa_select_sparse_attn_paged call: the same selection and output
+    inatt = msa.Path(prob, select_in_attention=True)
+    inatt.run()
+    torch.cuda.synchronize()
+    assert int(inatt.dev_err.item()) == 0
+    assert np.array_equal(inatt.block_ids.cpu().numpy(), ids)
+    assert np.array_equal(inatt.num_selected.cpu().numpy(), cnt)
+    assert torch.equal(inatt.out, out)
+    del inatt
+
     # the same step again: every output bit-identical
     for _ in range(3):
         path.run()

@@ -219,6 +219,47 @@ def test_fused_index_select_equals_the_two_stages(name):
     assert int(one.counters.abs().sum().item()) == 0
 
 
+@pytest.mark.parametrize("name", sorted(CASES))
+def test_select_in_attention_equals_the_two_stages(name):
+    """msa_select_sparse_attn_paged (the selection inside the decode attention launch, two
+    launches elsewhere) against msa_select_blocks + msa_sparse_attn_paged."""
+    p = _gpu(_problem(name))
+    two, one = msa.Path(p, select_in_attention=False), msa.Path(p, select_in_attention=True)
+    two.run()
+    for _ in range(2):
+        one.run()
+    torch.cuda.synchronize()
+    assert int(two.dev_err.item()) == 0 and int(one.dev_err.item()) == 0
+    assert torch.equal(one.num_selected, two.num_selected)
+    assert torch.equal(one.block_ids, two.block_ids)
+    assert torch.equal(one.out, two.out)
+
+
+@pytest.mark.parametrize("top_k,init,local", [(0, 1, 1), (3, 0, 0), (0, 0, 2), (500, 1, 2),
+                                              (5, 7, 0)])
+@pytest.mark.parametrize("name,max_blocks", [("bf16_decode", 0), ("fp8_decode", 0),
+                                             ("bf16_decode", 700), ("short_contexts", 1100)])
+def test_selection_inside_attention_is_bit_exact(name, max_blocks, top_k, init, local):
+    """The in-kernel selection (every register-key variant) against the oracle's on the GPU's
+    own scores, and the output against the oracle's attention over that selection."""
+    p = _gpu(_problem(name))
+    p = dict(p, top_k=top_k, init_blocks=init, local_blocks=local, S=top_k + init + local)
+    if max_blocks:
+        p = _pad_table(p, max_blocks)
+    path = msa.Path(p, max_blocks=max_blocks or None, select_in_attention=True)
+    path.run()
+    torch.cuda.synchronize()
+    assert int(path.dev_err.item()) == 0
+    cpu = {k: (v.cpu() if torch.is_tensor(v) else v) for k, v in p.items()}
+    sc = path.scores.cpu().numpy().astype(np.float64)
+    ids, cnt = oracle.select_blocks(cpu["row_off"], cpu["cache_len"], sc, top_k, init, local)
+    assert np.array_equal(path.num_selected.cpu().numpy(), cnt)
+    assert np.array_equal(path.block_ids.cpu().numpy(), ids)
+    out = oracle.attention(cpu["row_off"], cpu["cache_len"], cpu["table"], cpu["q"], cpu["k"],
+                           cpu["v"], p["kv_fp8"], ids, cnt, p["scale"])
+    check_attention(path.out.float().cpu(), out, p["kv_fp8"])
+
+
 def _pad_table(p, max_pages):
     t = p["table"]
     pad = torch.full((t.shape[0], max_pages - t.shape[1]), -1, dtype=t.dtype, device=t.device)
