@@ -306,3 +306,74 @@ class Path:
             self.select(stream=stream)
         self.attend(stream=stream)
         return self.out
+
+
+class HostPipeline:
+    """Steps whose per-step inputs arrive in pinned host memory and whose output goes back to
+    pinned host memory, pipelined two deep: step i's host->device copy runs on one copy stream
+    while step i-1 computes, and its device->host copy on another while step i+1 computes.
+
+    The KV caches (``k``, ``v``, ``k_idx``) stay resident and are shared; the per-step inputs
+    (``PER_STEP``) and every output live twice on the device, one set per Path, and alternate
+    between steps.  Stream order keeps each buffer's writer after its last reader:
+    copy-in(i) waits for compute(i-2), compute(i) waits for copy-in(i) and for copy-out(i-2),
+    copy-out(i) waits for compute(i).
+    """
+
+    PER_STEP = ("q", "q_idx", "row_off", "cache_len", "table")
+
+    def __init__(self, prob: dict, **path_kw):
+        self.paths = []
+        for b in range(2):
+            p = dict(prob)
+            if b:
+                for k in self.PER_STEP:
+                    p[k] = prob[k].clone()
+            self.paths.append(Path(p, **path_kw))
+        dev = prob["q"].device
+        self.compute = torch.cuda.Stream(dev)
+        self.h2d = torch.cuda.Stream(dev)
+        self.d2h = torch.cuda.Stream(dev)
+        self.copied_in = [torch.cuda.Event() for _ in range(2)]
+        self.computed = [torch.cuda.Event() for _ in range(2)]
+        self.copied_out = [torch.cuda.Event() for _ in range(2)]
+        self.i = 0
+
+    def h2d_bytes(self, host_in: dict) -> int:
+        return sum(host_in[k].numel() * host_in[k].element_size() for k in self.PER_STEP)
+
+    def start(self, after: Optional[torch.cuda.Event] = None):
+        """Order the three streams after ``after`` (e.g. a timing event) and restart at step 0."""
+        for s in (self.compute, self.h2d, self.d2h):
+            if after is not None:
+                s.wait_event(after)
+        self.i = 0
+
+    def submit(self, host_in: dict, host_out: torch.Tensor) -> torch.cuda.Event:
+        """Enqueue one step: ``host_in`` holds the PER_STEP tensors in pinned host memory,
+        ``host_out`` receives the step's output.  Returns the event after which ``host_out``
+        holds it."""
+        b = self.i % 2
+        path = self.paths[b]
+        with torch.cuda.stream(self.h2d):
+            if self.i >= 2:
+                self.h2d.wait_event(self.computed[b])
+            for k in self.PER_STEP:
+                path.p[k].copy_(host_in[k], non_blocking=True)
+            self.copied_in[b].record(self.h2d)
+        self.compute.wait_event(self.copied_in[b])
+        if self.i >= 2:
+            self.compute.wait_event(self.copied_out[b])
+        path.run(self.compute)
+        self.computed[b].record(self.compute)
+        with torch.cuda.stream(self.d2h):
+            self.d2h.wait_event(self.computed[b])
+            host_out.copy_(path.out, non_blocking=True)
+            self.copied_out[b].record(self.d2h)
+        self.i += 1
+        return self.copied_out[b]
+
+    def finish(self, stream: torch.cuda.Stream):
+        """Order ``stream`` after every step submitted so far."""
+        for s in (self.compute, self.h2d, self.d2h):
+            stream.wait_stream(s)
