@@ -32,6 +32,8 @@
 // states pairwise into one per row through shared memory.
 #include <math.h>
 
+#include <type_traits>
+
 #include "attn_common.cuh"
 #include "select_row.cuh"
 
@@ -154,7 +156,8 @@ __device__ __forceinline__ void segment(const AttnArgs &a, int it, long long r0,
 
 // SEL >= 0: decode with the selection in the kernel (select_row with SEL keys per lane in
 // registers, 0: from memory); SEL < 0: the selection comes from an earlier launch.
-template <bool FP8, int RG, bool PLAN, int SEL>
+// SWAP: decode items of at most 8 rows, on the swapped-operand math (WarpAttnSwap).
+template <bool FP8, int RG, bool PLAN, int SEL, bool SWAP>
 __global__ void __launch_bounds__(32 * (stream_consumer_warps<FP8, RG>() + 1))
     attn_stream_kernel(const __grid_constant__ CUtensorMap kmap,
                        const __grid_constant__ CUtensorMap vmap, const AttnArgs a) {
@@ -168,7 +171,8 @@ __global__ void __launch_bounds__(32 * (stream_consumer_warps<FP8, RG>() + 1))
   constexpr uint32_t TILE = StreamCfg<FP8, RG>::kTile;
   constexpr int QR = RG * 16;                             // rows of a Q buffer
   constexpr uint32_t QSUB = QR * 128, QBUF = 2 * QSUB;
-  using WA = WarpAttn<FP8, PQ>;
+  static_assert(!SWAP || (RG == 1 && !PLAN), "swapped math: one decode row group");
+  using WA = std::conditional_t<SWAP, WarpAttnSwap<FP8, PQ>, WarpAttn<FP8, PQ>>;
   constexpr int SLICE = slice_floats<FP8>();
   constexpr int MS = MergeRow<FP8>::kStride;
 
@@ -392,7 +396,7 @@ __global__ void __launch_bounds__(32 * (stream_consumer_warps<FP8, RG>() + 1))
     uint32_t tbit[2];
 #pragma unroll
     for (int slot = 0; slot < 2; ++slot) {
-      const int r = rg * 16 + (lane >> 2) + slot * 8;
+      const int r = SWAP ? 2 * (lane & 3) + slot : rg * 16 + (lane >> 2) + slot * 8;
       const int tl = r / a.G;
       prow[slot] = r < md.rows ? md.cl + md.tok0 + tl : -1;
       tbit[slot] = r < md.rows ? (1u << tl) : 0u;
@@ -402,6 +406,7 @@ __global__ void __launch_bounds__(32 * (stream_consumer_warps<FP8, RG>() + 1))
     const uint32_t rg_bits = __reduce_or_sync(0xffffffffu, tbit[0] | tbit[1]);
     const uint32_t qs_addr = smem_u32(qbufs + buf * QBUF);
     wa.reset();
+    if constexpr (SWAP) wa.load_q(qs_addr, QSUB, lane);
     for (int e = md.v0 + team; e < md.v1; e += NT) {
       const uint32_t nk = nload;  // this team's K tile; V is nk + 1
       int s = team * NR + static_cast<int>(nk % NR);
@@ -432,55 +437,101 @@ __global__ void __launch_bounds__(32 * (stream_consumer_warps<FP8, RG>() + 1))
     wa.finish_rows();
 #pragma unroll
     for (int step = W / 2; step >= 1; step >>= 1) {
-      if (rank >= step && rank < 2 * step) {
-        float *sl = my_slices + (rank - step) * SLICE;
+      if constexpr (SWAP) {
+        if (rank >= step && rank < 2 * step)
+          wa.store_rows(my_slices + (rank - step) * SLICE, {1.f, 1.f}, lane);
+        named_bar_sync(1, nct);
+        if (rank < step) wa.merge_rows(my_slices + rank * SLICE, lane);
+        named_bar_sync(1, nct);
+      } else {
+        if (rank >= step && rank < 2 * step) {
+          float *sl = my_slices + (rank - step) * SLICE;
 #pragma unroll
-        for (int slot = 0; slot < 2; ++slot) {
-          const int r16 = (lane >> 2) + slot * 8;
-          wa.store_row(sl, r16, slot, 1.f, lane, false);
-          if ((lane & 3) == 0) {
-            sl[16 * MS + r16] = wa.m_run[slot];
-            sl[16 * MS + 16 + r16] = wa.l_run[slot];
+          for (int slot = 0; slot < 2; ++slot) {
+            const int r16 = (lane >> 2) + slot * 8;
+            wa.store_row(sl, r16, slot, 1.f, lane, false);
+            if ((lane & 3) == 0) {
+              sl[16 * MS + r16] = wa.m_run[slot];
+              sl[16 * MS + 16 + r16] = wa.l_run[slot];
+            }
+          }
+        }
+        named_bar_sync(1, nct);
+        if (rank < step) {
+          const float *sl = my_slices + rank * SLICE;
+#pragma unroll
+          for (int slot = 0; slot < 2; ++slot) {
+            const int r16 = (lane >> 2) + slot * 8;
+            wa.merge_row(sl, r16, slot, sl[16 * MS + r16], sl[16 * MS + 16 + r16], lane);
+          }
+        }
+        named_bar_sync(1, nct);
+      }
+    }
+    // ---- rank 0 writes this segment's partial: normalised output and log-sum-exp
+    if constexpr (SWAP) {
+      // through its own slice (rank 0 read it last), so that the rows leave in whole 16-byte
+      // pieces
+      if (rank == 0) {
+        float *sl = my_slices;
+        const float f[2] = {wa.l_run[0] > 0.f ? 1.f / wa.l_run[0] : 0.f,
+                            wa.l_run[1] > 0.f ? 1.f / wa.l_run[1] : 0.f};
+        wa.store_rows(sl, f, lane);
+        __syncwarp();
+        for (int idx = lane; idx < md.rows * 32; idx += 32) {
+          const int r = idx >> 5, c4 = idx & 31;
+          const size_t orr =
+              static_cast<size_t>(md.t0 + r / a.G) * a.H_q + md.g * a.G + r % a.G;
+          const float4 v = *reinterpret_cast<const float4 *>(sl + r * MS + 4 * c4);
+          if (a.direct) {
+            *reinterpret_cast<uint2 *>(a.out + orr * kHeadDim + 4 * c4) =
+                make_uint2(pack_bf16x2(v.x, v.y), pack_bf16x2(v.z, v.w));
+          } else {
+            const size_t pr = static_cast<size_t>(md.piece) * split_stride + orr;
+            *reinterpret_cast<float4 *>(a.part_o + pr * kHeadDim + 4 * c4) = v;
+          }
+        }
+        if (!a.direct && lane < 4) {
+#pragma unroll
+          for (int slot = 0; slot < 2; ++slot) {
+            const int r = 2 * lane + slot;
+            if (r >= md.rows) continue;
+            const size_t orr =
+                static_cast<size_t>(md.t0 + r / a.G) * a.H_q + md.g * a.G + r % a.G;
+            const float l = wa.l_run[slot];
+            a.part_lse[static_cast<size_t>(md.piece) * split_stride + orr] =
+                l > 0.f ? (wa.m_run[slot] + __log2f(l)) * kLn2 : -INFINITY;
           }
         }
       }
-      named_bar_sync(1, nct);
-      if (rank < step) {
-        const float *sl = my_slices + rank * SLICE;
+    } else {
+      if (rank == 0) {
 #pragma unroll
         for (int slot = 0; slot < 2; ++slot) {
-          const int r16 = (lane >> 2) + slot * 8;
-          wa.merge_row(sl, r16, slot, sl[16 * MS + r16], sl[16 * MS + 16 + r16], lane);
+          const int r = rg * 16 + (lane >> 2) + slot * 8;
+          if (r >= md.rows) continue;
+          const size_t orr =
+              static_cast<size_t>(md.t0 + r / a.G) * a.H_q + md.g * a.G + r % a.G;
+          const float l = wa.l_run[slot];
+          if (a.direct) {
+            wa.store_bf16(a.out + orr * kHeadDim, slot, l > 0.f ? 1.f / l : 0.f, lane);
+            continue;
+          }
+          const size_t pr = static_cast<size_t>(md.piece) * split_stride + orr;
+          wa.store_global(a.part_o + pr * kHeadDim, slot, l > 0.f ? 1.f / l : 0.f, lane);
+          if ((lane & 3) == 0)
+            a.part_lse[pr] = l > 0.f ? (wa.m_run[slot] + __log2f(l)) * kLn2 : -INFINITY;
         }
-      }
-      named_bar_sync(1, nct);
-    }
-    // ---- rank 0 writes this segment's partial: normalised output and log-sum-exp
-    if (rank == 0) {
-#pragma unroll
-      for (int slot = 0; slot < 2; ++slot) {
-        const int r = rg * 16 + (lane >> 2) + slot * 8;
-        if (r >= md.rows) continue;
-        const size_t orr = static_cast<size_t>(md.t0 + r / a.G) * a.H_q + md.g * a.G + r % a.G;
-        const float l = wa.l_run[slot];
-        if (a.direct) {
-          wa.store_bf16(a.out + orr * kHeadDim, slot, l > 0.f ? 1.f / l : 0.f, lane);
-          continue;
-        }
-        const size_t pr = static_cast<size_t>(md.piece) * split_stride + orr;
-        wa.store_global(a.part_o + pr * kHeadDim, slot, l > 0.f ? 1.f / l : 0.f, lane);
-        if ((lane & 3) == 0)
-          a.part_lse[pr] = l > 0.f ? (wa.m_run[slot] + __log2f(l)) * kLn2 : -INFINITY;
       }
     }
   }
 }
 
-template <bool FP8, int RG, bool PLAN, int SEL>
+template <bool FP8, int RG, bool PLAN, int SEL, bool SWAP = false>
 cudaError_t launch_stream_one(const CUtensorMap &kmap, const CUtensorMap &vmap,
                               const AttnArgs &a, int grid, cudaStream_t s) {
   const size_t smem = stream_smem_bytes<FP8, RG>();
-  auto fn = &attn_stream_kernel<FP8, RG, PLAN, SEL>;
+  auto fn = &attn_stream_kernel<FP8, RG, PLAN, SEL, SWAP>;
   cudaError_t e = ensure_smem_limit(reinterpret_cast<const void *>(fn), static_cast<int>(smem));
   if (e != cudaSuccess) return e;
   return launch_pdl(fn, dim3(grid), dim3(32 * (stream_consumer_warps<FP8, RG>() + 1)), smem, s,
@@ -491,7 +542,10 @@ template <bool FP8, bool PLAN>
 cudaError_t launch_stream_rg(const CUtensorMap &kmap, const CUtensorMap &vmap, const AttnArgs &a,
                              int rg, int grid, cudaStream_t s) {
   switch (rg) {
-    case 1: return launch_stream_one<FP8, 1, PLAN, -1>(kmap, vmap, a, grid, s);
+    case 1:
+      if (!PLAN && a.G <= 8)
+        return launch_stream_one<FP8, 1, false, -1, true>(kmap, vmap, a, grid, s);
+      return launch_stream_one<FP8, 1, PLAN, -1>(kmap, vmap, a, grid, s);
     case 2: return launch_stream_one<FP8, 2, PLAN, -1>(kmap, vmap, a, grid, s);
     case 3: return launch_stream_one<FP8, 3, PLAN, -1>(kmap, vmap, a, grid, s);
     default: return launch_stream_one<FP8, 4, PLAN, -1>(kmap, vmap, a, grid, s);
@@ -499,13 +553,22 @@ cudaError_t launch_stream_rg(const CUtensorMap &kmap, const CUtensorMap &vmap, c
 }
 
 // decode with the selection inside: one row group, keys per lane chosen by the row length
+template <bool FP8, bool SWAP>
+cudaError_t launch_stream_sel_math(const CUtensorMap &kmap, const CUtensorMap &vmap,
+                                   const AttnArgs &a, int grid, cudaStream_t s) {
+  if (a.max_blocks <= 4 * 32)
+    return launch_stream_one<FP8, 1, false, 4, SWAP>(kmap, vmap, a, grid, s);
+  if (a.max_blocks <= 16 * 32)
+    return launch_stream_one<FP8, 1, false, 16, SWAP>(kmap, vmap, a, grid, s);
+  if (a.max_blocks <= 32 * 32)
+    return launch_stream_one<FP8, 1, false, 32, SWAP>(kmap, vmap, a, grid, s);
+  return launch_stream_one<FP8, 1, false, 0, SWAP>(kmap, vmap, a, grid, s);
+}
 template <bool FP8>
 cudaError_t launch_stream_sel(const CUtensorMap &kmap, const CUtensorMap &vmap, const AttnArgs &a,
                               int grid, cudaStream_t s) {
-  if (a.max_blocks <= 4 * 32) return launch_stream_one<FP8, 1, false, 4>(kmap, vmap, a, grid, s);
-  if (a.max_blocks <= 16 * 32) return launch_stream_one<FP8, 1, false, 16>(kmap, vmap, a, grid, s);
-  if (a.max_blocks <= 32 * 32) return launch_stream_one<FP8, 1, false, 32>(kmap, vmap, a, grid, s);
-  return launch_stream_one<FP8, 1, false, 0>(kmap, vmap, a, grid, s);
+  return a.G <= 8 ? launch_stream_sel_math<FP8, true>(kmap, vmap, a, grid, s)
+                  : launch_stream_sel_math<FP8, false>(kmap, vmap, a, grid, s);
 }
 
 }  // namespace

@@ -359,4 +359,247 @@ struct WarpAttn {
   }
 };
 
+
+// ---- decode math with the operands swapped (at most 8 query rows)
+//
+// A decode item has one query token, so its rows are the G <= 8 heads of one KV head and an
+// m16 tile of query rows is at least half padding.  Here the MMAs run transposed: S^T = K Q^T
+// takes 16 of the block's positions as M and the query rows as N (n8), and O^T += V^T P^T takes
+// 16 head dims as M, the rows as N and the positions as K, so no MMA computes padding and the
+// softmax touches half the values.  P^T moves from the C layout of S^T to the B layout of the
+// P V MMA through movmatrix (an 8x8 transpose in registers).  Lane (g, c) = (lane / 4,
+// lane % 4) holds query rows 2c and 2c + 1; its online-softmax state covers its own positions
+// (the max is reduced over the eight lanes of the same c, the sum at finish_rows).
+// For e4m3 KV the K rows arrive in the same per-16-dim order as stage_q gives Q, and the V^T
+// tiles of 32 dims split into an even-dim and an odd-dim m16 tile (dim_lo / dim_hi say which
+// dims a lane's accumulators hold).
+template <bool FP8, int PQ>
+struct WarpAttnSwap {
+  static constexpr int PW = kBlock / PQ;  // positions per warp
+  static constexpr int MT = PW / 16;      // m16 tiles of S^T per warp
+
+  float o[8][4];  // O^T tile t: [s] = (dim_lo(t), row 2c + s), [2 + s] = (dim_hi(t), row 2c + s)
+  float m_run[2], l_run[2];  // rows 2c and 2c + 1 (log2 domain)
+  float st[MT][4];           // S^T, then P^T: [s] = (position g, row 2c + s), [2 + s] = (g + 8, .)
+  uint32_t qb[8][2];         // Q^T B fragments of the eight k16 steps
+
+  __device__ static __forceinline__ int dim_lo(int t, int g) {
+    return FP8 ? 32 * (t >> 1) + 2 * g + (t & 1) : 16 * t + g;
+  }
+  __device__ static __forceinline__ int dim_hi(int t, int g) {
+    return dim_lo(t, g) + (FP8 ? 16 : 8);
+  }
+
+  __device__ __forceinline__ void reset() {
+#pragma unroll
+    for (int t = 0; t < 8; ++t)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) o[t][e] = 0.f;
+    m_run[0] = m_run[1] = -INFINITY;
+    l_run[0] = l_run[1] = 0.f;
+  }
+
+  // Q rows 0..7 of a Q buffer (sub-tiles qsub bytes apart) as the B operand of every k step.
+  __device__ __forceinline__ void load_q(uint32_t qs_addr, uint32_t qsub, int lane) {
+    const int r = lane & 7, hi = (lane >> 3) & 1;
+#pragma unroll
+    for (int ks = 0; ks < 8; ++ks)
+      ldsm_x2(qs_addr + sw128(r, 2 * ks + hi, qsub), qb[ks][0], qb[ks][1]);
+  }
+
+  // st = K Q^T over the warp's PW positions (the Q arguments are those of WarpAttn::qk; the
+  // fragments come from load_q).
+  __device__ __forceinline__ void qk(uint32_t, uint32_t, int, uint32_t kt, int pq, int lane) {
+    const int q = lane >> 3, r = lane & 7;
+#pragma unroll
+    for (int mt = 0; mt < MT; ++mt) {
+#pragma unroll
+      for (int e = 0; e < 4; ++e) st[mt][e] = 0.f;
+      const int row = pq * PW + mt * 16 + (q & 1) * 8 + r;  // the position this lane addresses
+      if (FP8) {
+#pragma unroll
+        for (int jd = 0; jd < 4; ++jd) {  // 32 dims (two k steps) per load
+          uint32_t kr[4];
+          ldsm_x4(kt + sw128(row, 2 * jd + (q >> 1), KvTile<FP8>::kSub), kr[0], kr[1], kr[2],
+                  kr[3]);
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            const uint32_t a[4] = {
+                e4m3x2_to_f16x2(static_cast<uint16_t>(kr[2 * h] & 0xffffu)),
+                e4m3x2_to_f16x2(static_cast<uint16_t>(kr[2 * h + 1] & 0xffffu)),
+                e4m3x2_to_f16x2(static_cast<uint16_t>(kr[2 * h] >> 16)),
+                e4m3x2_to_f16x2(static_cast<uint16_t>(kr[2 * h + 1] >> 16))};
+            mma_f16(st[mt], a, qb[2 * jd + h][0], qb[2 * jd + h][1]);
+          }
+        }
+      } else {
+#pragma unroll
+        for (int ks = 0; ks < 8; ++ks) {
+          uint32_t a[4];
+          ldsm_x4(kt + sw128(row, 2 * ks + (q >> 1), KvTile<FP8>::kSub), a[0], a[1], a[2], a[3]);
+          mma_bf16(st[mt], a, qb[ks][0], qb[ks][1]);
+        }
+      }
+    }
+  }
+
+  // Mask (position <= the row's query position, the row's token selected the block) and the
+  // online-softmax update in the log2 domain; st becomes P^T.
+  __device__ __forceinline__ void softmax(int j, int pq, int lane, const int (&prow)[2],
+                                          const uint32_t (&tbit)[2], uint32_t msk,
+                                          float scale_log2) {
+    const int g = lane >> 2;
+    float mx[2] = {-INFINITY, -INFINITY};
+#pragma unroll
+    for (int mt = 0; mt < MT; ++mt)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int s = e & 1;
+        const int pos = j * kBlock + pq * PW + mt * 16 + g + (e >> 1) * 8;
+        const bool vis = pos <= prow[s] && (msk & tbit[s]);
+        const float x = vis ? st[mt][e] * scale_log2 : -INFINITY;
+        st[mt][e] = x;
+        mx[s] = fmaxf(mx[s], x);
+      }
+    float alpha[2], base[2];
+#pragma unroll
+    for (int s = 0; s < 2; ++s) {
+#pragma unroll
+      for (int off = 4; off < 32; off <<= 1)
+        mx[s] = fmaxf(mx[s], __shfl_xor_sync(0xffffffffu, mx[s], off));
+      const float m_new = fmaxf(m_run[s], mx[s]);
+      base[s] = m_new == -INFINITY ? 0.f : m_new;
+      alpha[s] = fast_exp2(m_run[s] - base[s]);
+      m_run[s] = m_new;
+      l_run[s] *= alpha[s];
+    }
+#pragma unroll
+    for (int mt = 0; mt < MT; ++mt)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const float pv = fast_exp2(st[mt][e] - base[e & 1]);
+        st[mt][e] = pv;
+        l_run[e & 1] += pv;
+      }
+#pragma unroll
+    for (int t = 0; t < 8; ++t) {
+      o[t][0] *= alpha[0];
+      o[t][1] *= alpha[1];
+      o[t][2] *= alpha[0];
+      o[t][3] *= alpha[1];
+    }
+  }
+
+  // O^T += V^T P^T.  V values at positions >= L (the sequence length) are zeroed first (P is 0
+  // there, but the pool may hold NaN).
+  __device__ __forceinline__ void pv(uint32_t vt, int j, int pq, int lane, int L) {
+    const int c = lane & 3, q = lane >> 3, r = lane & 7;
+    const bool tail = j * kBlock + kBlock > L;
+#pragma unroll
+    for (int kk = 0; kk < MT; ++kk) {
+      uint32_t x0, x1;
+      if (FP8) {
+        x0 = pack_f16x2(st[kk][0], st[kk][1]);
+        x1 = pack_f16x2(st[kk][2], st[kk][3]);
+      } else {
+        x0 = pack_bf16x2(st[kk][0], st[kk][1]);
+        x1 = pack_bf16x2(st[kk][2], st[kk][3]);
+      }
+      const uint32_t b0 = movmatrix_t(x0), b1 = movmatrix_t(x1);  // (positions 2c.., row g)
+      const int p0 = j * kBlock + pq * PW + kk * 16 + 2 * c;
+      const uint32_t keep0 = (p0 < L ? 0x0000ffffu : 0u) | (p0 + 1 < L ? 0xffff0000u : 0u);
+      const uint32_t keep1 = (p0 + 8 < L ? 0x0000ffffu : 0u) | (p0 + 9 < L ? 0xffff0000u : 0u);
+      const int vrow = pq * PW + kk * 16 + (q >> 1) * 8 + r;  // the position this lane addresses
+      if (FP8) {
+#pragma unroll
+        for (int qd = 0; qd < 4; ++qd) {  // dims 32 qd .. 32 qd + 31
+          uint32_t rr[4];
+          ldsm_x4_t(vt + sw128(vrow, 2 * qd + (q & 1), KvTile<FP8>::kSub), rr[0], rr[1], rr[2],
+                    rr[3]);
+#pragma unroll
+          for (int sd = 0; sd < 2; ++sd) {  // even, odd dims
+            const uint32_t sel = sd ? 0x0031u : 0x0020u;
+            uint32_t a[4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+              a[i] = e4m3x2_to_f16x2(static_cast<uint16_t>(__byte_perm(rr[i], 0, sel)));
+            if (tail) {
+              a[0] &= keep0;
+              a[1] &= keep0;
+              a[2] &= keep1;
+              a[3] &= keep1;
+            }
+            mma_f16(o[2 * qd + sd], a, b0, b1);
+          }
+        }
+      } else {
+#pragma unroll
+        for (int d = 0; d < 8; ++d) {  // dims 16 d .. 16 d + 15
+          uint32_t a[4];
+          ldsm_x4_t(vt + sw128(vrow, 2 * d + (q & 1), KvTile<FP8>::kSub), a[0], a[1], a[2],
+                    a[3]);
+          if (tail) {
+            a[0] &= keep0;
+            a[1] &= keep0;
+            a[2] &= keep1;
+            a[3] &= keep1;
+          }
+          mma_bf16(o[d], a, b0, b1);
+        }
+      }
+    }
+  }
+
+  // After the last block: each row's sum of P over all of the warp's positions.
+  __device__ __forceinline__ void finish_rows() {
+#pragma unroll
+    for (int s = 0; s < 2; ++s)
+#pragma unroll
+      for (int off = 4; off < 32; off <<= 1)
+        l_run[s] += __shfl_xor_sync(0xffffffffu, l_run[s], off);
+  }
+
+  // Rows 2c and 2c + 1 times f[0] / f[1], as fp32 rows of buf (kStride floats apart, natural
+  // dim order), and (from the lanes with g == 0) their m and l after the 16 rows.
+  __device__ __forceinline__ void store_rows(float *buf, const float (&f)[2], int lane) const {
+    constexpr int MS = MergeRow<FP8>::kStride;
+    const int g = lane >> 2, c = lane & 3;
+#pragma unroll
+    for (int s = 0; s < 2; ++s) {
+      float *row = buf + (2 * c + s) * MS;
+#pragma unroll
+      for (int t = 0; t < 8; ++t) {
+        row[dim_lo(t, g)] = o[t][s] * f[s];
+        row[dim_hi(t, g)] = o[t][2 + s] * f[s];
+      }
+      if (g == 0) {
+        buf[16 * MS + 2 * c + s] = m_run[s];
+        buf[16 * MS + 16 + 2 * c + s] = l_run[s];
+      }
+    }
+  }
+
+  // Fold another warp's state, left in buf by store_rows (f = 1), into this lane's rows.
+  __device__ __forceinline__ void merge_rows(const float *buf, int lane) {
+    constexpr int MS = MergeRow<FP8>::kStride;
+    const int g = lane >> 2, c = lane & 3;
+#pragma unroll
+    for (int s = 0; s < 2; ++s) {
+      const float m2 = buf[16 * MS + 2 * c + s], l2 = buf[16 * MS + 16 + 2 * c + s];
+      const float m1 = m_run[s];
+      const float m = fmaxf(m1, m2);
+      const float a1 = m1 == -INFINITY ? 0.f : fast_exp2(m1 - m);
+      const float a2 = m2 == -INFINITY ? 0.f : fast_exp2(m2 - m);
+      const float *row = buf + (2 * c + s) * MS;
+#pragma unroll
+      for (int t = 0; t < 8; ++t) {
+        o[t][s] = o[t][s] * a1 + row[dim_lo(t, g)] * a2;
+        o[t][2 + s] = o[t][2 + s] * a1 + row[dim_hi(t, g)] * a2;
+      }
+      l_run[s] = l_run[s] * a1 + l2 * a2;
+      m_run[s] = m;
+    }
+  }
+};
+
 }  // namespace msa
