@@ -313,24 +313,34 @@ class HostPipeline:
     pinned host memory, pipelined two deep: step i's host->device copy runs on one copy stream
     while step i-1 computes, and its device->host copy on another while step i+1 computes.
 
-    The KV caches (``k``, ``v``, ``k_idx``) stay resident and are shared; the per-step inputs
-    (``PER_STEP``) and every output live twice on the device, one set per Path, and alternate
-    between steps.  Stream order keeps each buffer's writer after its last reader:
-    copy-in(i) waits for compute(i-2), compute(i) waits for copy-in(i) and for copy-out(i-2),
-    copy-out(i) waits for compute(i).
+    The KV caches (``k``, ``v``, ``k_idx``) stay resident and are shared.  The per-step inputs
+    (``PER_STEP``) of one step travel as one packed buffer (``pack``: each tensor at a 256-byte
+    aligned offset), so a step costs one host->device copy; on the device they live twice, in
+    two staging buffers that the two Paths read in place, and alternate between steps with every
+    output.  Stream order keeps each buffer's writer after its last reader: copy-in(i) waits for
+    compute(i-2), compute(i) waits for copy-in(i) and for copy-out(i-2), copy-out(i) waits for
+    compute(i).
     """
 
     PER_STEP = ("q", "q_idx", "row_off", "cache_len", "table")
 
     def __init__(self, prob: dict, **path_kw):
+        self.layout, off = [], 0
+        for k in self.PER_STEP:
+            t = prob[k]
+            n = t.numel() * t.element_size()
+            self.layout.append((k, off, t.dtype, tuple(t.shape), n))
+            off = (off + n + 255) // 256 * 256
+        self.step_bytes = off
+        dev = prob["q"].device
+        self.stage = [torch.empty((off,), dtype=torch.uint8, device=dev) for _ in range(2)]
         self.paths = []
         for b in range(2):
             p = dict(prob)
-            if b:
-                for k in self.PER_STEP:
-                    p[k] = prob[k].clone()
+            for k, o, dt, shape, n in self.layout:
+                p[k] = self.stage[b][o:o + n].view(dt).view(shape)
+                p[k].copy_(prob[k])
             self.paths.append(Path(p, **path_kw))
-        dev = prob["q"].device
         self.compute = torch.cuda.Stream(dev)
         self.h2d = torch.cuda.Stream(dev)
         self.d2h = torch.cuda.Stream(dev)
@@ -339,8 +349,14 @@ class HostPipeline:
         self.copied_out = [torch.cuda.Event() for _ in range(2)]
         self.i = 0
 
-    def h2d_bytes(self, host_in: dict) -> int:
-        return sum(host_in[k].numel() * host_in[k].element_size() for k in self.PER_STEP)
+    def pack(self, host_in: dict) -> torch.Tensor:
+        """One step's PER_STEP tensors (host) packed into a new pinned buffer for submit()."""
+        buf = torch.empty((self.step_bytes,), dtype=torch.uint8).pin_memory()
+        for k, o, dt, shape, n in self.layout:
+            t = host_in[k]
+            assert t.dtype == dt and tuple(t.shape) == shape, k
+            buf[o:o + n].view(dt).view(shape).copy_(t)
+        return buf
 
     def start(self, after: Optional[torch.cuda.Event] = None):
         """Order the three streams after ``after`` (e.g. a timing event) and restart at step 0."""
@@ -349,17 +365,16 @@ class HostPipeline:
                 s.wait_event(after)
         self.i = 0
 
-    def submit(self, host_in: dict, host_out: torch.Tensor) -> torch.cuda.Event:
-        """Enqueue one step: ``host_in`` holds the PER_STEP tensors in pinned host memory,
-        ``host_out`` receives the step's output.  Returns the event after which ``host_out``
+    def submit(self, host_packed: torch.Tensor, host_out: torch.Tensor) -> torch.cuda.Event:
+        """Enqueue one step: ``host_packed`` is a pinned buffer from pack(), ``host_out``
+        (pinned) receives the step's output.  Returns the event after which ``host_out``
         holds it."""
         b = self.i % 2
         path = self.paths[b]
         with torch.cuda.stream(self.h2d):
             if self.i >= 2:
                 self.h2d.wait_event(self.computed[b])
-            for k in self.PER_STEP:
-                path.p[k].copy_(host_in[k], non_blocking=True)
+            self.stage[b].copy_(host_packed, non_blocking=True)
             self.copied_in[b].record(self.h2d)
         self.compute.wait_event(self.copied_in[b])
         if self.i >= 2:

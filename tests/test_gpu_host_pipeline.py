@@ -54,7 +54,8 @@ def test_pipelined_steps_equal_serial_steps(name):
     pipe = msa.HostPipeline(prob)
     outs = [torch.empty(ref_path.out.shape, dtype=ref_path.out.dtype).pin_memory()
             for _ in steps]
-    done = [pipe.submit(s, o) for s, o in zip(steps, outs)]
+    packed = [pipe.pack(s) for s in steps]
+    done = [pipe.submit(s, o) for s, o in zip(packed, outs)]
     pipe.finish(torch.cuda.current_stream())
     torch.cuda.synchronize()
     for p in pipe.paths:
