@@ -22,6 +22,12 @@ CASES = {
     "bf16_decode": (W["bf16_decode"], dict(batch=4, kv_len=(2000, 9000))),
     "bf16_decode_idxk_per_head": (W["bf16_decode"], dict(batch=3, kv_len=(1000, 5000), H_idxk=8)),
     "short_contexts": (W["bf16_decode"], dict(batch=6, kv_len=(1, 300))),
+    # decode groups off the swapped-operand path (G > 8) and with padding rows (G = 3)
+    "decode_gqa16": (W["bf16_decode"], dict(batch=3, kv_len=(1500, 6000), H_kv=2, G=16)),
+    "decode_gqa3": (W["bf16_decode"], dict(batch=4, kv_len=(900, 5000), H_kv=3, G=3)),
+    "fp8_decode_gqa16": (W["fp8_long_decode"], dict(batch=2, kv_len=(2000, 7000), H_kv=2,
+                                                     G=16)),
+    "fp8_decode_gqa5": (W["fp8_long_decode"], dict(batch=3, kv_len=(1000, 4000), H_kv=2, G=5)),
     "spec_decode": (W["spec_decode"], dict(batch=6, kv_len=(1500, 5000))),
     "spec_ragged_q": (W["spec_decode"], dict(batch=6, q_len=(2, 8), kv_len=(1000, 4000))),
     "spec_gqa4": (W["spec_decode"], dict(batch=3, G=4, H_kv=4, q_len=(2, 8), kv_len=(900, 3000))),
@@ -109,7 +115,9 @@ def test_whole_path_matches_oracle(name):
 
 @pytest.mark.parametrize("name,splits", [("bf16_decode", n) for n in (1, 2, 3, 7, 19, 148, 700)]
                          + [("spec_ragged_q", n) for n in (1, 5, 148)]
-                         + [("fp8_decode", n) for n in (1, 13, 148)])
+                         + [("fp8_decode", n) for n in (1, 13, 148)]
+                         + [("decode_gqa16", n) for n in (1, 5, 148)]
+                         + [("fp8_decode_gqa5", n) for n in (1, 13)])
 def test_split_k_partitions_agree(name, splits):
     """Any number of split-K partitions gives the oracle's answer, and the partitions agree with
     one another to fp32 reassociation (a couple of bf16 ulps after rounding)."""
