@@ -210,14 +210,27 @@ __global__ void __launch_bounds__(kIxThreads, 1)
       const bool use = live && st_ok[s];
       const int pos0 = i * kBlock;
       float mx = -INFINITY;
+      uint32_t v[4][32];
 #pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        uint32_t v[32];
-        tmem_ld32(lane_addr + sb * 128 + c * 32, v);
-        tmem_wait_ld();
+      for (int c = 0; c < 4; ++c) tmem_ld32(lane_addr + sb * 128 + c * 32, v[c]);
+      tmem_wait_ld();
+      if (use && pos0 + kBlock - 1 <= prow) {
+        // the whole page is visible to this row: four independent three-input max chains
+        float m4[4];
 #pragma unroll
-        for (int e = 0; e < 32; ++e)
-          if (use && pos0 + c * 32 + e <= prow) mx = fmaxf(mx, __uint_as_float(v[e]));
+        for (int c = 0; c < 4; ++c) {
+          m4[c] = fmaxf(__uint_as_float(v[c][0]), __uint_as_float(v[c][1]));
+#pragma unroll
+          for (int e = 2; e < 32; e += 2)
+            m4[c] = fmax3(m4[c], __uint_as_float(v[c][e]), __uint_as_float(v[c][e + 1]));
+        }
+        mx = fmax3(fmaxf(m4[0], m4[1]), m4[2], m4[3]);
+      } else if (use) {  // the diagonal page: positions up to the row's own
+#pragma unroll
+        for (int c = 0; c < 4; ++c)
+#pragma unroll
+          for (int e = 0; e < 32; ++e)
+            if (pos0 + c * 32 + e <= prow) mx = fmaxf(mx, __uint_as_float(v[c][e]));
       }
       tc_fence_before();
       __syncwarp();

@@ -163,6 +163,12 @@ __device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi) {
   asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
   return r;
 }
+// max(a, b, c) in one instruction (a NaN operand is ignored, as by fmaxf).
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
 // 2^x on the SFU (MUFU.EX2), flushing subnormal results to zero.
 __device__ __forceinline__ float fast_exp2(float x) {
   float y;
