@@ -20,8 +20,9 @@
 //              S buffer, O accumulator and running max and sum: one query row per thread (its
 //              TMEM lane), one pass over the row's 128 scores held in registers (masked max,
 //              exp2, P as bf16 back into TMEM over its S).  The first warpgroup (producers, MMA
-//              issuer, one idle warp) hands registers to the softmax warpgroups (setmaxnreg).  The groups never wait for each other inside the loop, so
-//              one group's exponentials overlap the other's loads and maxima.  A group's
+//              issuer, one idle warp) hands registers to the softmax warpgroups (setmaxnreg).
+//              The groups never wait for each other inside the loop, so one group's
+//              exponentials overlap the other's loads and maxima.  A group's
 //              running max only moves when a block's max exceeds it by more than 2^8 (then its
 //              O is rescaled in TMEM); in between P = 2^(s - m) stays <= 2^8, well inside bf16
 //              and fp32 range.  Zeroes the rows of a last page past the sequence end in V
@@ -366,10 +367,14 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         for (int c = 0; c < 4; ++c)
           tmem_ld32(s_addr + 32 * c, *reinterpret_cast<uint32_t(*)[32]>(v + 32 * c));
         tmem_wait_ld();
-        // row max (eight independent chains)
+        // row max (independent chains; three-input max where no position is masked)
         if (plain) {
 #pragma unroll
-          for (int e = 0; e < 128; ++e) m8[e & 7] = fmaxf(m8[e & 7], __uint_as_float(v[e]));
+          for (int e = 0; e < 128; e += 8)
+#pragma unroll
+            for (int k = 0; k < 4; ++k)
+              m8[k] = fmax3(m8[k], __uint_as_float(v[e + 2 * k]),
+                            __uint_as_float(v[e + 2 * k + 1]));
         } else {
 #pragma unroll
           for (int e = 0; e < 128; ++e)
@@ -390,6 +395,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       const float sc = use ? a.scale_log2 : 0.f;
       const float nb = use ? -m_run : -INFINITY;
       float ps4[4] = {0.f, 0.f, 0.f, 0.f};
+      float2 ps2[4] = {{0.f, 0.f}, {0.f, 0.f}, {0.f, 0.f}, {0.f, 0.f}};
       if (!any_use) {
         uint32_t z[32];
 #pragma unroll
@@ -401,12 +407,14 @@ __global__ void __launch_bounds__(kTcThreads, 1)
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
           uint32_t pk[32];
-          if (plain) {
+          if (plain) {  // pairs on the packed fp32x2 pipe: one FMA and one add per pair
 #pragma unroll
             for (int e = 0; e < 64; e += 2) {
-              const float e0 = fast_exp2(fmaf(__uint_as_float(v[64 * h + e]), sc, nb));
-              const float e1 = fast_exp2(fmaf(__uint_as_float(v[64 * h + e + 1]), sc, nb));
-              ps4[(e >> 1) & 3] += e0 + e1;
+              const float2 x = fma2(make_float2(__uint_as_float(v[64 * h + e]),
+                                                __uint_as_float(v[64 * h + e + 1])),
+                                    make_float2(sc, sc), make_float2(nb, nb));
+              const float e0 = fast_exp2(x.x), e1 = fast_exp2(x.y);
+              ps2[(e >> 1) & 3] = add2(ps2[(e >> 1) & 3], make_float2(e0, e1));
               pk[e >> 1] = pack_bf16x2(e0, e1);
             }
           } else {
@@ -426,6 +434,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           tmem_st32(s_addr + 32 * h, pk);
         }
       }
+#pragma unroll
+      for (int k = 0; k < 4; ++k) ps4[k] += ps2[k].x + ps2[k].y;
       l_run = l_run * alpha + ((ps4[0] + ps4[1]) + (ps4[2] + ps4[3]));
       // this group's previous P V (done before this block's S was written; waited here so
       // that every phase is observed in order) before its O is rescaled
@@ -441,7 +451,12 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           tmem_ld32(o_addr + c * 32, o);
           tmem_wait_ld();
 #pragma unroll
-          for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
+          for (int e = 0; e < 32; e += 2) {
+            const float2 r = mul2(make_float2(__uint_as_float(o[e]), __uint_as_float(o[e + 1])),
+                                  make_float2(alpha, alpha));
+            o[e] = __float_as_uint(r.x);
+            o[e + 1] = __float_as_uint(r.y);
+          }
           tmem_st32(o_addr + c * 32, o);
         }
       }

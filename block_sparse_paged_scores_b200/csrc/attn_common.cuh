@@ -42,8 +42,8 @@ __device__ __forceinline__ void stage_q(uint8_t *qs, const uint16_t *q, int t0, 
     uint4 lo4 = make_uint4(0, 0, 0, 0), hi4 = make_uint4(0, 0, 0, 0);
     if (r < rows) {
       const int t = t0 + r / G, h = g * G + r % G;
-      const uint4 *src =
-          reinterpret_cast<const uint4 *>(q + (static_cast<size_t>(t) * H_q + h) * kHeadDim + grp * 16);
+      const uint4 *src = reinterpret_cast<const uint4 *>(
+          q + (static_cast<size_t>(t) * H_q + h) * kHeadDim + grp * 16);
       const uint4 x0 = src[0], x1 = src[1];
       if (!FP8) {
         lo4 = x0;

@@ -278,8 +278,9 @@ MSA_API msa_status_t msa_splitk_combine(const float *partial_o, const float *par
 /* Host-only helpers (no device work, no CUDA call). */
 
 /* Bytes of `workspace` that msa_sparse_attn_paged needs for this shape (0 when none). */
-MSA_API size_t msa_attn_workspace_bytes(const msa_ragged_paged_t *rp, int32_t S, int32_t num_q_heads,
-                                int32_t num_kv_heads, int32_t max_blocks, int32_t num_splits);
+MSA_API size_t msa_attn_workspace_bytes(const msa_ragged_paged_t *rp, int32_t S,
+                                        int32_t num_q_heads, int32_t num_kv_heads,
+                                        int32_t max_blocks, int32_t num_splits);
 
 /* The split-K partition count the decode / speculative routes use when num_splits == 0 for
  * `batch` sequences of `max_q_len` new tokens: one partition per SM, fewer when the work list
