@@ -219,14 +219,15 @@ def executed_flops_tiles(prob, block_ids, num_selected, tile_tokens):
 
 def source_digest(*names):
     """Digest of a kernel's code: its source file and the headers that hold its math, with
-    comments and blank space removed (a comment edit does not make a profile stale)."""
+    comments and all white space removed (a comment or layout edit does not make a profile
+    stale)."""
     h = hashlib.sha256()
     for n in names:
         with open(os.path.join(ROOT, "block_sparse_paged_scores_b200", "csrc", n)) as f:
             src = f.read()
         src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
         src = re.sub(r"//[^\n]*", "", src)
-        h.update("\n".join(l.strip() for l in src.splitlines() if l.strip()).encode())
+        h.update(re.sub(r"\s+", "", src).encode())
     return h.hexdigest()[:16]
 
 
