@@ -11,11 +11,18 @@ Recipe (all draws from ``torch.Generator`` seeded with the workload's seed, in t
   3. q, q_idx, k_idx, K, V as standard normals on the target device, rounded to bf16 (RNE),
      or for e4m3 KV clamped to +-448 and cast with torch's float8_e4m3fn (RNE);
   4. poison: every pool page no sequence uses, and every position >= L_b of a sequence's
-     last page, is set to NaN (bf16 0x7FC0, e4m3 0x7F) so that a stray read shows up.
+     last page, is set to NaN (bf16 0x7FC0, e4m3 0x7F) so that a stray read shows up;
+  5. a scaled index-K cache ("fp8" / "fp4" index dtype) is the N(0,1) index-K of step 3,
+     quantised: fp8 with one float32 scale per token (its largest |value| / 448, then each
+     element rounded to e4m3), fp4 with one UE8M0 exponent per 32 elements (the smallest
+     2^e with largest |value| / 2^e <= 6, then each element rounded to the nearest E2M1
+     value); poisoned positions get a NaN scale (fp8) or the NaN exponent 0xFF (fp4).
 
 Layouts (the C-ABI's):
   q      bf16 [total_q, H_q, 128]         q_idx  bf16 [total_q, H_kv, 128]
-  k_idx  bf16 [num_pages, H_idxk, 128, 128]
+  k_idx  bf16 [num_pages, H_idxk, 128, 128], or for a scaled index-K cache
+         fp8: uint8 e4m3 codes [num_pages, H_idxk, 128, 128] + k_idx_scale f32 [.., 128]
+         fp4: uint8 e2m1 pairs [num_pages, H_idxk, 128, 64] + k_idx_scale u8 [.., 128, 4]
   k, v   bf16 | float8_e4m3fn [num_pages, H_kv, 128, 128]
   row_off int32 [batch+1], cache_len int32 [batch], table int32 [batch, max_pages] (-1 unused)
 """
@@ -48,6 +55,8 @@ class WorkloadSpec:
     H_idxk: int = 1            # index-K heads: 1 (shared) or H_kv
     prior_len: Optional[IntOrRange] = None   # prefill: prior cache length, L_b = prior + q_len
     pool_pages: int = 0        # minimum pool size (extra pages stay unused and poisoned)
+    idx_dtype: str = "bf16"    # index-K cache: "bf16" | "fp8" (e4m3 + f32 scale per token)
+                               # | "fp4" (e2m1 + ue8m0 exponent per 32 elements)
 
     @property
     def H_q(self) -> int:
@@ -108,6 +117,46 @@ def _fill_nan(t: torch.Tensor, index):
         t[index] = float("nan")
 
 
+# E2M1 magnitudes by code and the midpoints between neighbours (a value on a midpoint goes to
+# the lower code)
+_E2M1_MID = (0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5.0)
+
+
+def quantize_index_k(x: torch.Tensor, idx_dtype: str, chunk_pages: int = 4096):
+    """(codes, scales) of an index-K cache ``x`` (bf16 [pages, H, 128, 128]) in the scaled
+    format ``idx_dtype``, computed on x's device page-chunk by page-chunk."""
+    P, H = x.shape[0], x.shape[1]
+    dev = x.device
+    if idx_dtype == "fp8":
+        codes = torch.empty((P, H, BLOCK, HEAD_DIM), dtype=torch.uint8, device=dev)
+        scales = torch.empty((P, H, BLOCK), dtype=torch.float32, device=dev)
+    else:
+        codes = torch.empty((P, H, BLOCK, HEAD_DIM // 2), dtype=torch.uint8, device=dev)
+        scales = torch.empty((P, H, BLOCK, HEAD_DIM // 32), dtype=torch.uint8, device=dev)
+        mids = torch.tensor(_E2M1_MID, dtype=torch.float32, device=dev)
+    for s in range(0, P, chunk_pages):
+        e = min(P, s + chunk_pages)
+        v = x[s:e].float()
+        if idx_dtype == "fp8":
+            amax = v.abs().amax(-1)
+            sc = torch.where(amax > 0, amax / 448.0, torch.ones_like(amax))
+            codes[s:e] = (v / sc[..., None]).clamp(-448.0, 448.0).to(
+                torch.float8_e4m3fn).view(torch.uint8)
+            scales[s:e] = sc
+        else:
+            g = v.reshape(e - s, H, BLOCK, HEAD_DIM // 32, 32)
+            amax = g.abs().amax(-1)
+            ex = torch.ceil(torch.log2(torch.clamp(amax / 6.0, min=2.0 ** -126)))
+            ex = torch.clamp(ex, -126, 127)
+            y = g / torch.exp2(ex)[..., None]
+            mag = torch.bucketize(y.abs().clamp(max=6.0), mids).to(torch.uint8)   # 0..7
+            code = mag | ((y < 0).to(torch.uint8) << 3)
+            code = code.reshape(e - s, H, BLOCK, HEAD_DIM // 2, 2)
+            codes[s:e] = code[..., 0] | (code[..., 1] << 4)
+            scales[s:e] = (ex + 127).to(torch.uint8)
+    return codes, scales
+
+
 def generate(spec: WorkloadSpec, seed: int, device="cpu", poison: bool = True) -> dict:
     """Draw one seeded problem for ``spec``; tensors live on ``device``."""
     gcpu = torch.Generator().manual_seed(seed)
@@ -155,10 +204,25 @@ def generate(spec: WorkloadSpec, seed: int, device="cpu", poison: bool = True) -
                 for t in (k_idx, k, v):
                     _fill_nan(t, (last, slice(None), slice(tail, None)))
 
+    k_idx_scale = None
+    if spec.idx_dtype != "bf16":
+        k_idx, k_idx_scale = quantize_index_k(k_idx, spec.idx_dtype)
+        if poison:
+            # the NaN scale / exponent reaches every element of a poisoned token
+            bad = 0xFF if spec.idx_dtype == "fp4" else float("nan")
+            if unused.numel():
+                k_idx_scale[unused] = bad
+            for b in range(spec.batch):
+                tail = int(L[b]) % BLOCK
+                if tail:
+                    last = int(table[b, int(nb[b]) - 1])
+                    k_idx_scale[last, :, tail:] = bad
+
     return dict(
         name=spec.name, spec=spec, seed=seed,
         row_off=row_off.to(device), cache_len=cache_len.to(torch.int32).to(device),
-        table=table.to(device), q=q, q_idx=q_idx, k_idx=k_idx, k=k, v=v,
+        table=table.to(device), q=q, q_idx=q_idx, k_idx=k_idx, k_idx_scale=k_idx_scale,
+        idx_dtype=spec.idx_dtype, k=k, v=v,
         kv_fp8=spec.kv_dtype == "fp8",
         batch=spec.batch, total_q=total_q, max_q_len=max(1, int(q_lens.max())),
         max_cache_len=int(cache_len.max()), max_pages=max_pages, num_pages=max(pool, 1),

@@ -51,8 +51,12 @@ def _load():
         lib.orc_bf16_value.argtypes = [ctypes.c_uint16]
         lib.orc_e4m3_value.restype = ctypes.c_double
         lib.orc_e4m3_value.argtypes = [ctypes.c_uint8]
+        lib.orc_e2m1_value.restype = ctypes.c_double
+        lib.orc_e2m1_value.argtypes = [ctypes.c_uint8]
+        lib.orc_ue8m0_value.restype = ctypes.c_double
+        lib.orc_ue8m0_value.argtypes = [ctypes.c_uint8]
         lib.orc_index_scores.restype = None
-        lib.orc_index_scores.argtypes = [I, P, P, P, I, P, P, I, I, I, P]
+        lib.orc_index_scores.argtypes = [I, P, P, P, I, P, I, P, P, I, I, I, P]
         lib.orc_select_blocks.restype = None
         lib.orc_select_blocks.argtypes = [I, P, P, I, I, P, I, I, I, I, P, P]
         lib.orc_attention.restype = None
@@ -73,6 +77,17 @@ def bf16_value(bits: int) -> float:
 
 def e4m3_value(code: int) -> float:
     return _load().orc_e4m3_value(int(code))
+
+
+def e2m1_value(code: int) -> float:
+    return _load().orc_e2m1_value(int(code))
+
+
+def ue8m0_value(code: int) -> float:
+    return _load().orc_ue8m0_value(int(code))
+
+
+IDX_FORMATS = {"bf16": 0, "fp8": 1, "fp4": 2}
 
 
 def _bits16(x):
@@ -96,23 +111,41 @@ def _ints(x):
     return np.asarray(x, dtype=np.int32)
 
 
-def index_scores(row_off, cache_len, table, q_idx, k_idx, max_blocks):
+def index_scores(row_off, cache_len, table, q_idx, k_idx, max_blocks, k_idx_scale=None,
+                 idx_dtype="bf16"):
     """Block scores [total_q, H_kv, max_blocks] in fp64 (-inf where the block is not visible).
 
-    q_idx bf16 [total_q, H_kv, 128]; k_idx bf16 [num_pages, H_idxk, 128, 128].
+    q_idx bf16 [total_q, H_kv, 128]; k_idx by ``idx_dtype``: "bf16" bf16 [num_pages, H_idxk,
+    128, 128]; "fp8" e4m3 bytes [num_pages, H_idxk, 128, 128] with k_idx_scale float32
+    [num_pages, H_idxk, 128]; "fp4" e2m1 pairs uint8 [num_pages, H_idxk, 128, 64] with
+    k_idx_scale ue8m0 uint8 [num_pages, H_idxk, 128, 4].
     """
     lib = _load()
+    fmt = IDX_FORMATS[idx_dtype]
     row_off, p_off = _c(_ints(row_off), np.int32)
     cache_len, p_cl = _c(_ints(cache_len), np.int32)
     table, p_tab = _c(_ints(table), np.int32)
     qb, p_q = _c(_bits16(q_idx), np.uint16)
-    kb, p_k = _c(_bits16(k_idx), np.uint16)
+    if fmt == 0:
+        kb, p_k = _c(_bits16(k_idx), np.uint16)
+        p_s = None
+    else:
+        kb, p_k = _c(_bytes8(k_idx), np.uint8)
+        assert kb.shape[3] == (128 if fmt == 1 else 64), kb.shape
+        if fmt == 1:
+            sc = np.asarray(k_idx_scale.detach().cpu().numpy() if hasattr(k_idx_scale, "detach")
+                            else k_idx_scale, dtype=np.float32)
+            sc, p_s = _c(sc, np.float32)
+            assert sc.shape == kb.shape[:3]
+        else:
+            sc, p_s = _c(_bytes8(k_idx_scale), np.uint8)
+            assert sc.shape == kb.shape[:3] + (4,)
     total_q, H_kv, _ = qb.shape
     H_idxk = kb.shape[1]
     batch = row_off.shape[0] - 1
     out = np.empty((total_q, H_kv, max_blocks), dtype=np.float64)
-    lib.orc_index_scores(batch, p_off, p_cl, p_tab, table.shape[1], p_q, p_k, H_kv, H_idxk,
-                         max_blocks, out.ctypes.data_as(ctypes.c_void_p))
+    lib.orc_index_scores(batch, p_off, p_cl, p_tab, table.shape[1], p_q, fmt, p_k, p_s, H_kv,
+                         H_idxk, max_blocks, out.ctypes.data_as(ctypes.c_void_p))
     return out
 
 
@@ -165,7 +198,8 @@ def forward(inp, top_k, init_blocks, local_blocks, scale, max_blocks):
     """The whole path: scores -> selection -> attention.  ``inp`` is a mapping with the
     tensors named as in the C-ABI (row_off, cache_len, table, q, q_idx, k_idx, k, v, kv_fp8)."""
     sc = index_scores(inp["row_off"], inp["cache_len"], inp["table"], inp["q_idx"],
-                      inp["k_idx"], max_blocks)
+                      inp["k_idx"], max_blocks, inp.get("k_idx_scale"),
+                      inp.get("idx_dtype", "bf16"))
     ids, counts = select_blocks(inp["row_off"], inp["cache_len"], sc, top_k, init_blocks,
                                 local_blocks)
     out = attention(inp["row_off"], inp["cache_len"], inp["table"], inp["q"], inp["k"],

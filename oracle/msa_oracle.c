@@ -14,6 +14,8 @@
  *             single index-K head, scale-free FP8 e4m3 main KV, FP32 accumulation) and the
  *             "Three attention routes" list (query position = cache_lengths[batch] +
  *             tok_in_seq; logical KV start of a selected block = block id * BN).
+ *   [trtllm]  TensorRT-LLM "DeepSeekSparseAttentionConfig", field indexer_k_dtype (the
+ *             scaled FP8 / FP4 index-K formats; below, before stage 1).
  *   [ferrox]  ferrox-core "Module block_sparse": "Four rules" (max over the block, no
  *             softmax scale, per-KV-head selection, forced init/local blocks),
  *             "The block size is an ABI", and the functions block_sparse_select
@@ -33,7 +35,9 @@
  * Memory layouts (the same host bytes the GPU path consumes):
  *   q        bf16 bits  [total_q][H_q][128]
  *   q_idx    bf16 bits  [total_q][H_kv][128]
- *   k_idx    bf16 bits  [num_pages][H_idxk][128 tokens][128]
+ *   k_idx    bf16 bits  [num_pages][H_idxk][128 tokens][128], or
+ *            fp8: e4m3 bytes [num_pages][H_idxk][128 tokens][128] + f32 [..][128 tokens],
+ *            fp4: e2m1 pairs [num_pages][H_idxk][128 tokens][64] + ue8m0 [..][128 tokens][4]
  *   k, v     bf16 bits or e4m3 bytes [num_pages][H_kv][128 tokens][128]
  *   table    int32      [batch][max_pages]  (logical block j of sequence b -> page)
  *   scores   fp64       [total_q][H_kv][max_blocks]
@@ -73,6 +77,57 @@ double orc_e4m3_value(uint8_t x)
     return sign ? -v : v;
 }
 
+/* ---------------------------------------------------------------------------------------
+ * Scaled index-K formats: TensorRT-LLM "DeepSeekSparseAttentionConfig", field
+ * indexer_k_dtype.  fp8: one E4M3 byte per element and one float32 scale for the token's 128
+ * elements (132 B per token); fp4: two E2M1 codes per byte and one UE8M0 exponent per 32
+ * elements (68 B per token).  Readings where the page is silent: element c of a token's fp4
+ * codes is in byte c / 2, in the low nibble when c is even; the exponent byte x stands for
+ * 2^(x - 127); an element's value is its code's value times its scale.
+ * ------------------------------------------------------------------------------------- */
+
+/* E2M1 (1 sign bit, 2 exponent bits with bias 1, 1 mantissa bit; no inf, no NaN) -> value. */
+double orc_e2m1_value(uint8_t code)
+{
+    int sign = (code >> 3) & 1;
+    int e = (code >> 1) & 3;
+    int m = code & 1;
+    double v = (e == 0) ? 0.5 * m                          /* subnormal: 0.m * 2^(1-1) */
+                        : ldexp(1.0 + 0.5 * m, e - 1);     /* 1.m * 2^(e-1) */
+    return sign ? -v : v;
+}
+
+/* UE8M0 (8 exponent bits, bias 127, no sign, no mantissa; 0xFF is NaN) -> value. */
+double orc_ue8m0_value(uint8_t x)
+{
+    if (x == 0xFF)
+        return NAN;
+    return ldexp(1.0, (int)x - 127);
+}
+
+#define ORC_IDX_BF16 0
+#define ORC_IDX_FP8 1
+#define ORC_IDX_FP4 2
+
+/* Element c of index-K row r (r = (page * H_idxk + head) * 128 + token) in format fmt:
+ * bf16 codes [rows][128] u16; fp8 codes [rows][128] u8 with scales [rows] f32; fp4 codes
+ * [rows][64] u8 with exponents [rows][4] u8. */
+static double idx_k_value(int fmt, const void *codes, const void *scales, size_t r, int c)
+{
+    if (fmt == ORC_IDX_FP8) {
+        float s;
+        memcpy(&s, (const uint8_t *)scales + r * sizeof(float), sizeof s);
+        return orc_e4m3_value(((const uint8_t *)codes)[r * ORC_D + c]) * (double)s;
+    }
+    if (fmt == ORC_IDX_FP4) {
+        uint8_t byte = ((const uint8_t *)codes)[r * (ORC_D / 2) + c / 2];
+        uint8_t code = (c & 1) ? (uint8_t)(byte >> 4) : (uint8_t)(byte & 15);
+        uint8_t e = ((const uint8_t *)scales)[r * (ORC_D / 32) + c / 32];
+        return orc_e2m1_value(code) * orc_ue8m0_value(e);
+    }
+    return orc_bf16_value(((const uint16_t *)codes)[r * ORC_D + c]);
+}
+
 /* Query position of row i of sequence b: [msa] "Three attention routes",
  * speculative route: position = cache_lengths[batch] + tok_in_seq. */
 static int query_position(const int32_t *cache_len, int b, int i) { return cache_len[b] + i; }
@@ -87,8 +142,8 @@ static int visible_blocks(int p) { return p / ORC_BLOCK + 1; }
  * ------------------------------------------------------------------------------------- */
 void orc_index_scores(int batch, const int32_t *row_off, const int32_t *cache_len,
                       const int32_t *table, int max_pages, const uint16_t *q_idx,
-                      const uint16_t *k_idx, int H_kv, int H_idxk, int max_blocks,
-                      double *scores)
+                      int k_idx_fmt, const void *k_idx, const void *k_idx_scale, int H_kv,
+                      int H_idxk, int max_blocks, double *scores)
 {
     for (int b = 0; b < batch; ++b) {
         int q_len = row_off[b + 1] - row_off[b];
@@ -110,11 +165,11 @@ void orc_index_scores(int batch, const int32_t *row_off, const int32_t *cache_le
                             last = p;
                         for (int pos = j * ORC_BLOCK; pos <= last; ++pos) {
                             int tok = pos - j * ORC_BLOCK;
-                            const uint16_t *kv =
-                                k_idx + (((size_t)page * H_idxk + hk) * ORC_BLOCK + tok) * ORC_D;
+                            size_t r = ((size_t)page * H_idxk + hk) * ORC_BLOCK + (size_t)tok;
                             double dot = 0.0;
                             for (int c = 0; c < ORC_D; ++c)
-                                dot += orc_bf16_value(qv[c]) * orc_bf16_value(kv[c]);
+                                dot += orc_bf16_value(qv[c]) *
+                                       idx_k_value(k_idx_fmt, k_idx, k_idx_scale, r, c);
                             if (dot > best)
                                 best = dot;
                         }

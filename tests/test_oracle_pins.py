@@ -45,6 +45,28 @@ def test_e4m3_decoder_matches_torch_on_every_code():
     assert np.array_equal(got[~nan], ref[~nan])
 
 
+def test_e2m1_decoder_matches_ml_dtypes_on_every_code():
+    import ml_dtypes
+    codes = np.arange(16, dtype=np.uint8)
+    ref = codes.view(ml_dtypes.float4_e2m1fn).astype(np.float64)
+    got = np.array([oracle.e2m1_value(int(c)) for c in codes])
+    assert np.array_equal(got, ref)
+    assert np.array_equal(np.signbit(got), np.signbit(ref))   # -0.0 for code 8
+
+
+def test_ue8m0_decoder_matches_torch_and_ml_dtypes_on_every_code():
+    import ml_dtypes
+    codes = np.arange(256, dtype=np.uint8)
+    ref_t = torch.from_numpy(codes.copy()).view(torch.float8_e8m0fnu).double().numpy()
+    ref_m = codes.view(ml_dtypes.float8_e8m0fnu).astype(np.float64)
+    got = np.array([oracle.ue8m0_value(int(c)) for c in codes])
+    for ref in (ref_t, ref_m):
+        nan = np.isnan(ref)
+        assert nan.sum() == 1 and nan[255]
+        assert np.array_equal(np.isnan(got), nan)
+        assert np.array_equal(got[~nan], ref[~nan])
+
+
 # ----------------------------------------------------------------------------- helpers
 def _small(name, **kw):
     base = wl.WORKLOADS[name]
@@ -95,6 +117,65 @@ def test_scores_equal_numpy_brute_force(name, kw):
             assert np.array_equal(np.isinf(got), np.isinf(ref))
             fin = np.isfinite(ref)
             np.testing.assert_allclose(got[fin], ref[fin], rtol=1e-12, atol=1e-11)
+
+
+def _dequantized_index_k(p):
+    """The scaled index-K cache of ``p`` as fp64 values, decoded with library routines (torch
+    for e4m3 and e8m0, ml_dtypes for e2m1): [num_pages, H_idxk, 128, 128]."""
+    import ml_dtypes
+    codes = p["k_idx"].numpy()
+    if p["idx_dtype"] == "fp8":
+        v = torch.from_numpy(codes.copy()).view(torch.float8_e4m3fn).double().numpy()
+        return v * p["k_idx_scale"].double().numpy()[..., None]
+    lo = (codes & 15).view(ml_dtypes.float4_e2m1fn).astype(np.float64)
+    hi = (codes >> 4).view(ml_dtypes.float4_e2m1fn).astype(np.float64)
+    v = np.stack([lo, hi], axis=-1).reshape(codes.shape[:3] + (128,))
+    ex = torch.from_numpy(p["k_idx_scale"].numpy().copy()).view(torch.float8_e8m0fnu)
+    return v * np.repeat(ex.double().numpy(), 32, axis=-1)
+
+
+@pytest.mark.parametrize("idx_dtype", ["fp8", "fp4"])
+@pytest.mark.parametrize("name,kw", SCORE_CASES)
+def test_scaled_index_k_scores_equal_numpy_brute_force(name, kw, idx_dtype):
+    p = _small(name, idx_dtype=idx_dtype, **kw)
+    sc = oracle.index_scores(p["row_off"], p["cache_len"], p["table"], p["q_idx"], p["k_idx"],
+                             p["max_blocks"], p["k_idx_scale"], idx_dtype)
+    kv = torch.from_numpy(_dequantized_index_k(p))
+    ro, cl = p["row_off"].tolist(), p["cache_len"].tolist()
+    for b in range(p["batch"]):
+        L = p["kv_lens"][b]
+        for g in range(p["H_kv"]):
+            K = _dense_rows(kv, p["table"][b], L, g % p["H_idxk"])
+            Q = p["q_idx"][ro[b]:ro[b + 1], g].double().numpy()
+            full = np.full((Q.shape[0], p["max_blocks"] * BLOCK), -np.inf)
+            full[:, :L] = Q @ K.T
+            pos_q = cl[b] + np.arange(Q.shape[0])
+            full[np.arange(full.shape[1])[None, :] > pos_q[:, None]] = -np.inf
+            ref = full.reshape(Q.shape[0], p["max_blocks"], BLOCK).max(axis=2)
+            got = sc[ro[b]:ro[b + 1], g]
+            assert np.array_equal(np.isinf(got), np.isinf(ref))
+            assert not np.isnan(got).any()
+            fin = np.isfinite(ref)
+            np.testing.assert_allclose(got[fin], ref[fin], rtol=1e-12, atol=1e-11)
+
+
+@pytest.mark.parametrize("idx_dtype", ["fp8", "fp4"])
+def test_scaled_index_k_is_close_to_the_bf16_cache_it_quantises(idx_dtype):
+    """The quantised cache keeps the scores within the formats' rounding (fp8: 2^-4 relative
+    per element, fp4: a quarter of the group's scale), and a poisoned token reads as NaN."""
+    p16 = _small("bf16_decode", batch=2, kv_len=(300, 900))
+    pq = _small("bf16_decode", batch=2, kv_len=(300, 900), idx_dtype=idx_dtype)
+    s16 = oracle.index_scores(p16["row_off"], p16["cache_len"], p16["table"], p16["q_idx"],
+                              p16["k_idx"], p16["max_blocks"])
+    sq = oracle.index_scores(pq["row_off"], pq["cache_len"], pq["table"], pq["q_idx"],
+                             pq["k_idx"], pq["max_blocks"], pq["k_idx_scale"], idx_dtype)
+    fin = np.isfinite(s16)
+    rel = 2.0 ** -4 if idx_dtype == "fp8" else 0.5
+    qn = np.linalg.norm(p16["q_idx"].double().numpy(), axis=-1)[..., None]
+    assert np.all(np.abs(sq[fin] - s16[fin]) <= rel * np.broadcast_to(qn, s16.shape)[fin] * 12)
+    # every pool page beyond the used ones is poisoned through its scale
+    assert torch.isnan(pq["k_idx_scale"].float()).any() if idx_dtype == "fp8" else \
+        bool((pq["k_idx_scale"] == 0xFF).any())
 
 
 def test_block_score_is_max_not_mean():
