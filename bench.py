@@ -1,15 +1,21 @@
 """Benchmark of the block-sparse paged attention hot path on B200.
 
 One step = one pass of the whole path over one batch: block scores -> selection -> sparse
-paged attention (split-K + combine), through the C ABI, on the BF16-decode workload (batch 32,
-1 query token, 8 KV heads x 8 query heads, head dim 128, context U[16384, 65536], page 128,
-top_k 16, init 1, local 2) unless --workload says otherwise.
+paged attention (split-K + combine), through the C ABI.  The headline workload is the largest
+single-GPU configuration, FP8 long-context decode (batch 128, 1 query token, 8 KV heads x 8
+query heads, head dim 128, context 131072, e4m3 KV, BF16 index-K, page 128, top_k 64, init 1,
+local 4: 6.6 GB of algorithmic HBM traffic per step); the four other workloads are measured
+the same way in the same run and reported under "workloads".
 
-    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--only]
+                    [--impl ours|reference]
 
+Timing: W warm-up steps, then blocks of exactly K steps (CUDA events on the launching stream,
+synchronize and barrier on both sides) repeated for about a second; the median block gives
+the value.  Per-launch times come from separate passes with events between the launch groups.
 Under torchrun every rank runs an independent replica (the path does not shard: no
-collective), timed on the device between barriers, and rank 0 prints one JSON line whose
-value is the query tokens of all ranks divided by the slowest rank's time.
+collective), and rank 0 prints one JSON line whose value is the query tokens of all ranks
+divided by the slowest rank's time.
 """
 from __future__ import annotations
 
@@ -17,6 +23,7 @@ import argparse
 import datetime
 import hashlib
 import json
+import math
 import os
 import re
 import statistics
@@ -281,6 +288,63 @@ def cpu_threads():
     return int(n) if n else len(os.sched_getaffinity(0))
 
 
+# ------------------------------------------------------------------ timing helpers
+def _events(n):
+    return [torch.cuda.Event(enable_timing=True) for _ in range(n)]
+
+
+def blocks_for(block_ms: float, min_s: float, ws: int, dev) -> int:
+    """How many K-step blocks fill about ``min_s`` seconds (at least 3): the same count on every
+    rank (the largest over ranks), so that every rank takes the same steps."""
+    n = max(3, min(2000, math.ceil(min_s * 1e3 / max(block_ms, 1e-3))))
+    return int(max_over_ranks(n, ws, dev))
+
+
+def time_block(step, steps: int, stream, flush_buf=None) -> float:
+    """Device time (ms) of one block of ``steps`` calls of step() on ``stream``, from CUDA
+    events on that stream with a synchronize on both sides.  With ``flush_buf`` L2 is flushed
+    before every step (a write of twice its size, outside the step's own events) and the
+    steps' own intervals are summed."""
+    torch.cuda.synchronize()
+    if flush_buf is None:
+        e0, e1 = _events(2)
+        e0.record(stream)
+        for _ in range(steps):
+            step()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        return e0.elapsed_time(e1)
+    evs = [_events(2) for _ in range(steps)]
+    for a_, b_ in evs:
+        flush_buf.fill_(1)
+        a_.record(stream)
+        step()
+        b_.record(stream)
+    torch.cuda.synchronize()
+    return sum(a_.elapsed_time(b_) for a_, b_ in evs)
+
+
+def stage_times(groups, steps: int, stream, min_s: float):
+    """Each launch group's average device time per step (ms): K-step passes with an event
+    between consecutive groups, repeated until about ``min_s`` seconds have passed (at least
+    three passes); the median over the passes."""
+    per = [[] for _ in groups]
+    t0 = time.perf_counter()
+    while True:
+        evs = [_events(len(groups) + 1) for _ in range(steps)]
+        for k in range(steps):
+            evs[k][0].record(stream)
+            for i, fn in enumerate(groups):
+                fn()
+                evs[k][i + 1].record(stream)
+        torch.cuda.synchronize()
+        for i in range(len(groups)):
+            per[i].append(sum(evs[k][i].elapsed_time(evs[k][i + 1]) for k in range(steps))
+                          / steps)
+        if len(per[0]) >= 3 and time.perf_counter() - t0 >= min_s:
+            return [statistics.median(x) for x in per]
+
+
 # ------------------------------------------------------------------ arms
 def run_reference(args):
     """The CPU oracle as the reference arm: each step is the whole path on a bounded sample
@@ -315,6 +379,230 @@ def run_reference(args):
     return 0
 
 
+def bench_workload(name, args, ws, rank, dev, sampler, with_cpu):
+    """Every measurement of one workload: the timed whole-path step (median of repeated
+    K-step blocks), per-launch times of the same launches, the roofline of the dominant one,
+    the end-to-end figure with host buffers and, when asked, the CPU oracle baseline."""
+    from block_sparse_paged_scores_b200 import msa
+    from block_sparse_paged_scores_b200 import workload as wl
+
+    spec = wl.WORKLOADS[name]
+    if args.batch:
+        spec = spec.scaled(batch=args.batch)
+    prob = wl.generate(spec, seed=wl.SEEDS[name] + 1000 * rank, device=dev)
+    path = msa.Path(prob, num_splits=args.splits)
+    stream = torch.cuda.current_stream(dev)
+    fp8 = prob["kv_fp8"]
+    G = prob["H_q"] // prob["H_kv"]
+    decode = prob["max_q_len"] == 1 and G <= 16      # the selection runs inside the attention
+    stream_route = prob["max_q_len"] <= 8            # persistent split-K kernel (+ combine)
+    tensor_route = not stream_route                  # prefill: dense contractions, tcgen05
+    splits = msa.msa_attn_partials(path.rp, prob["S"], prob["H_q"], prob["H_kv"],
+                                   path.max_blocks, args.splits)[0] if stream_route else 1
+    combine = stream_route and splits > 1
+    if decode:          # index, attention with the selection inside, [combine]
+        launches = 2 + int(combine)
+    elif stream_route:  # index, select, plan, attention, [combine]
+        launches = 4 + int(combine)
+    else:               # index, select, plan, attention
+        launches = 4
+    step = lambda: path.run(stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(dev)
+    assert int(path.dev_err.item()) == 0, f"device error flag set during warm-up ({name})"
+
+    idx_bytes, attn_bytes = algorithmic_bytes(prob, path.block_ids, path.num_selected)
+    flush = idx_bytes + attn_bytes < L2_BYTES
+    flush_buf = torch.empty(2 * L2_BYTES, dtype=torch.uint8, device=dev) if flush else None
+
+    # ---- the timed region: blocks of exactly K steps between barriers, repeated for about
+    # args.min_seconds; the median block is the number
+    first = time_block(step, args.steps, stream, flush_buf)
+    n_blocks = blocks_for(first, args.min_seconds, ws, dev)
+    barrier(ws, dev)
+    torch.cuda.synchronize(dev)
+    t_wall0 = time.time()
+    blocks = [time_block(step, args.steps, stream, flush_buf) for _ in range(n_blocks)]
+    barrier(ws, dev)
+    t_wall1 = time.time()
+    ms_block = max_over_ranks(statistics.median(blocks), ws, dev)
+    tokens = sum_over_ranks(prob["total_q"], ws, dev)
+    assert int(path.dev_err.item()) == 0, f"device error flag set ({name})"
+
+    # ---- the same launches, one group at a time (events between them)
+    if decode:
+        groups = {"index_scores": lambda: path.index_scores(stream)}
+        if combine:
+            groups["attention_with_selection"] = lambda: path.select_attend(stream,
+                                                                            combine=False)
+            groups["combine"] = lambda: path.combine(stream)
+        else:
+            groups["attention_with_selection"] = lambda: path.select_attend(stream)
+        attn_key = "attention_with_selection"
+        attn_src = ("attention_stream.cu", "attn_common.cuh", "select_row.cuh")
+    else:
+        groups = {"index_scores": lambda: path.index_scores(stream),
+                  "select": lambda: path.select(stream=stream)}
+        attn_key = "attention_incl_plan"
+        if combine:
+            groups[attn_key] = lambda: path.attend(stream=stream, combine=False)
+            groups["combine"] = lambda: path.combine(stream)
+        else:
+            groups[attn_key] = lambda: path.attend(stream=stream)
+        attn_src = (("attention_stream.cu", "attn_common.cuh", "select_row.cuh")
+                    if stream_route else
+                    (("attention_tile.cu", "attn_common.cuh") if fp8 else ("attention_tc.cu",)))
+    idx_src = ("indexer.cu", "select_row.cuh") if stream_route else ("indexer_tc.cu",)
+    st = stage_times(list(groups.values()), args.steps, stream, args.stage_seconds)
+    stages = dict(zip(groups, st))
+    if stream_route:
+        # for comparison: the first two stages as one msa_index_select launch
+        stages["fused_index_select"] = stage_times([lambda: path.index_select(stream)],
+                                                   args.steps, stream,
+                                                   args.stage_seconds / 2)[0]
+
+    # ---- roofline of the dominant launch group of the step
+    hbm, bf16, bf16_sus, peak_src = measured_peaks()
+    kinds = {"index_scores": (stages["index_scores"], idx_src),
+             attn_key: (stages[attn_key], attn_src)}
+    dom = max(kinds, key=lambda k: kinds[k][0])
+    d_ms, d_src = kinds[dom]
+    traffic_kernel = "index_scores" if dom == "index_scores" else "attention"
+    traffic = profiled_traffic(traffic_kernel, name, source_digest(*d_src))
+    if tensor_route:
+        idx_flops, attn_flops = algorithmic_flops(prob, path.block_ids, path.num_selected)
+        d_flops = idx_flops if dom == "index_scores" else attn_flops
+        achieved = d_flops / (d_ms * 1e-3) / 1e12
+        roofline = {"bound": "tensor", "kernel": dom, "achieved": achieved, "peak": bf16,
+                    "unit": "TFLOP/s", "frac": achieved / bf16, "peak_source": peak_src,
+                    "frac_of_sustained_peak": achieved / bf16_sus, "traffic": traffic,
+                    "algorithmic_flops_per_launch": d_flops,
+                    "note": "algorithmic FLOPs (selected, causally clipped positions only) over "
+                            "the launch group's median time, against the measured bf16 burst "
+                            "peak"}
+        if dom != "index_scores" and not fp8:
+            ex = executed_flops_tiles(prob, path.block_ids, path.num_selected, 128 // G)
+            roofline["executed_flops_per_launch"] = ex
+            roofline["executed_tflops"] = ex / (d_ms * 1e-3) / 1e12
+            roofline["executed_frac"] = ex / (d_ms * 1e-3) / 1e12 / bf16
+        work = {"algorithmic_tflop": (idx_flops + attn_flops) / 1e12,
+                "achieved_TFLOPs": (idx_flops + attn_flops) / (ms_block / args.steps * 1e-3)
+                / 1e12}
+    else:
+        d_bytes = idx_bytes if dom == "index_scores" else attn_bytes
+        achieved = d_bytes / (d_ms * 1e-3) / 1e9
+        roofline = {"bound": "hbm", "kernel": dom, "achieved": achieved, "peak": hbm,
+                    "unit": "GB/s", "frac": achieved / hbm, "peak_source": peak_src,
+                    "frac_of_8TBps": achieved / 8000.0, "traffic": traffic,
+                    "algorithmic_bytes_per_launch": d_bytes}
+        step_s = ms_block / args.steps * 1e-3
+        work = {"algorithmic_bytes": idx_bytes + attn_bytes,
+                "achieved_GBps": (idx_bytes + attn_bytes) / step_s / 1e9,
+                "frac_of_measured": (idx_bytes + attn_bytes) / step_s / 1e9 / hbm,
+                "frac_of_8TBps": (idx_bytes + attn_bytes) / step_s / 8e12}
+
+    # ---- end to end through the public API with host buffers: every step copies its inputs
+    # from pinned host memory and its output back, both inside the timed region
+    e2e = None
+    if not args.no_e2e:
+        host = {k: prob[k].cpu().pin_memory() for k in msa.HostPipeline.PER_STEP}
+        outs = [torch.empty(path.out.shape, dtype=path.out.dtype).pin_memory()
+                for _ in range(2)]
+        d2h = outs[0].numel() * outs[0].element_size()
+
+        def serial_step():
+            for k_, v_ in host.items():
+                prob[k_].copy_(v_, non_blocking=True)
+            path.run(stream)
+            outs[0].copy_(path.out, non_blocking=True)
+
+        for _ in range(max(1, args.warmup)):
+            serial_step()
+        serial_ms = statistics.median(time_block(serial_step, args.steps, stream)
+                                      for _ in range(3))
+        pipe = msa.HostPipeline(prob, num_splits=args.splits)
+        packed = pipe.pack(host)  # the step's inputs as one pinned buffer: one copy per step
+        for i in range(max(2, args.warmup)):
+            pipe.submit(packed, outs[i % 2])
+        pipe.finish(stream)
+        torch.cuda.synchronize(dev)
+
+        def pipe_block():
+            x0, x1 = _events(2)
+            x0.record(stream)
+            pipe.start(after=x0)
+            for i in range(args.steps):
+                pipe.submit(packed, outs[i % 2])
+            pipe.finish(stream)
+            x1.record(stream)
+            torch.cuda.synchronize(dev)
+            return x0.elapsed_time(x1)
+
+        pipe_ms = statistics.median(pipe_block() for _ in range(3))
+        for p_ in pipe.paths:
+            assert int(p_.dev_err.item()) == 0, "device error flag set (host pipeline)"
+        assert torch.equal(outs[(args.steps - 1) % 2].to(dev), path.out), \
+            "host pipeline output differs from the device-resident step"
+        pipe_ms = max_over_ranks(pipe_ms, ws, dev)
+        serial_ms = max_over_ranks(serial_ms, ws, dev)
+        e2e = {"value": tokens * args.steps / (pipe_ms * 1e-3), "unit": UNIT,
+               "h2d_bytes_per_step": packed.numel(), "d2h_bytes_per_step": d2h,
+               "serial_value": tokens * args.steps / (serial_ms * 1e-3),
+               "note": "per-step inputs (q, q_idx, row offsets, cache lengths, page table) "
+                       "copied from pinned host memory and the output read back, every step "
+                       "inside the timed region (median of 3 K-step blocks); value: two-deep "
+                       "pipeline (the step's inputs packed in one pinned buffer, one copy; "
+                       "step i+1's copy in and step i-1's copy out on their own streams while "
+                       "step i computes); serial_value: one copy per input, compute, copy "
+                       "out, all on one stream; the caches stay resident"}
+        del pipe
+
+    cpu = None
+    if with_cpu:
+        sample, desc = oracle_sample(name, args.cpu_sample_seqs, seed=7)
+        v, el, reps = time_oracle(sample, args.cpu_min_s, args.cpu_max_s)
+        cpu = {"value": v, "unit": UNIT, "cores": cpu_threads(), "kind": "oracle",
+               "sample": f"{desc}, seed 7, {reps} pass(es), {el:.1f} s"}
+
+    l2 = ((f"{(idx_bytes + attn_bytes) / 2**20:.1f} MiB touched per step, under the "
+           f"{L2_BYTES / 2**20:.0f} MiB L2: L2 flushed before every step (a "
+           f"{2 * L2_BYTES / 2**20:.0f} MiB write outside the step's events), time = sum of "
+           f"the steps' own intervals") if flush else
+          (f"inputs larger than L2: {(idx_bytes + attn_bytes) / 2**20:.0f} MiB touched per "
+           f"step vs {L2_BYTES / 2**20:.0f} MiB L2, no flush"))
+    res = {
+        "value": tokens * args.steps / (ms_block * 1e-3),
+        "ms_per_step": ms_block / args.steps,
+        "dtype": "fp8-e4m3 kv / bf16" if fp8 else "bf16",
+        "config": {"workload": name, "batch": prob["batch"],
+                   "q_tokens_per_step": prob["total_q"], "H_kv": prob["H_kv"],
+                   "H_q": prob["H_q"], "head_dim": 128, "page_size": 128,
+                   "top_k": prob["top_k"], "init_blocks": prob["init_blocks"],
+                   "local_blocks": prob["local_blocks"],
+                   "kv_lens": f"{spec.kv_len}" if spec.prior_len is None else
+                   f"prior {spec.prior_len} + new {spec.q_len}",
+                   "kv_dtype": spec.kv_dtype, "index_k_dtype": "bf16",
+                   "split_k_partials": splits, "parallelism": f"replicas x{ws}", "l2": l2},
+        "timing": {"blocks": n_blocks, "steps_per_block": args.steps,
+                   "block_ms_min_median_max": [min(blocks), statistics.median(blocks),
+                                               max(blocks)],
+                   "note": "value and ms_per_step from the median block (max over ranks)"},
+        "roofline": roofline,
+        ("step_flops" if tensor_route else "step_hbm"): work,
+        "stages_ms": stages,
+        "launches_per_step": launches,
+        "gpu_launches": launches * args.steps * n_blocks,
+        "clocks": sampler.summary(t_wall0, t_wall1) if sampler else None,
+        "e2e": e2e,
+        "cpu_baseline": cpu,
+    }
+    del path, prob, flush_buf
+    torch.cuda.empty_cache()
+    return res
+
+
 def run_ours(args):
     from block_sparse_paged_scores_b200 import build as msa_build
     from block_sparse_paged_scores_b200 import msa
@@ -329,244 +617,31 @@ def run_ours(args):
     barrier(ws, dev)
     msa.load()
 
-    spec = wl.WORKLOADS[args.workload]
-    if args.batch:
-        spec = spec.scaled(batch=args.batch)
-    seed = wl.SEEDS[args.workload] + 1000 * rank
-    prob = wl.generate(spec, seed=seed, device=dev)
-    path = msa.Path(prob, num_splits=args.splits)
-    stream = torch.cuda.current_stream(dev)
-    fp8 = prob["kv_fp8"]
-    stream_route = prob["max_q_len"] <= 8  # decode / speculative: persistent kernel + combine
-    splits_used = msa.msa_attn_partials(path.rp, prob["S"], prob["H_q"], prob["H_kv"],
-                                        path.max_blocks, args.splits)[0] if stream_route else 1
-    # decode: index, attention with the selection inside, [combine: only with more than one
-    # split-K partition]; speculative: index, select, plan, attention, [combine];
-    # prefill: index, select, plan, attention
-    if prob["max_q_len"] == 1 and prob["H_q"] // prob["H_kv"] <= 16:
-        kernels_per_step = 2 + (1 if splits_used > 1 else 0)
-    elif stream_route:
-        kernels_per_step = 4 + (1 if splits_used > 1 else 0)
-    else:
-        kernels_per_step = 4
-
-    for _ in range(args.warmup):
-        path.run(stream)
-    torch.cuda.synchronize(dev)
-    assert int(path.dev_err.item()) == 0, "device error flag set during warm-up"
-
     sampler = ClockSampler(local).start() if rank == 0 else None
     time.sleep(0.3 if sampler else 0)
-    # a step that touches less than L2 is timed cold: L2 is flushed (a write of twice its size)
-    # before every step, outside the step's own events
-    idx_bytes, attn_bytes = algorithmic_bytes(prob, path.block_ids, path.num_selected)
-    flush = idx_bytes + attn_bytes < L2_BYTES
-    flush_buf = torch.empty(2 * L2_BYTES, dtype=torch.uint8, device=dev) if flush else None
-
-    # ---- device-timed region: exactly K steps between barriers
-    barrier(ws, dev)
-    torch.cuda.synchronize(dev)
-    t_wall0 = time.time()
-    if flush:
-        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-               for _ in range(args.steps)]
-        for a_, b_ in evs:
-            flush_buf.fill_(1)
-            a_.record(stream)
-            path.run(stream)
-            b_.record(stream)
-        torch.cuda.synchronize(dev)
-        ms_local = sum(a_.elapsed_time(b_) for a_, b_ in evs)
-    else:
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e0.record(stream)
-        for _ in range(args.steps):
-            path.run(stream)
-        e1.record(stream)
-        torch.cuda.synchronize(dev)
-        ms_local = e0.elapsed_time(e1)
-    barrier(ws, dev)
-    t_wall1 = time.time()
-    ms = max_over_ranks(ms_local, ws, dev)
-
-    # ---- per-stage durations (separate K-step passes, events between the launches)
-    def stage_pass(fns):
-        evs = [[torch.cuda.Event(enable_timing=True) for _ in range(len(fns) + 1)]
-               for _ in range(args.steps)]
-        for k in range(args.steps):
-            evs[k][0].record(stream)
-            for i, fn in enumerate(fns):
-                fn()
-                evs[k][i + 1].record(stream)
-        torch.cuda.synchronize(dev)
-        return [sum(evs[k][i].elapsed_time(evs[k][i + 1]) for k in range(args.steps)) /
-                args.steps for i in range(len(fns))]
-
-    attn_key = "attention" + ("_incl_plan" if prob["max_q_len"] > 1 else "")
-    if stream_route and splits_used > 1:
-        st = stage_pass([lambda: path.index_scores(stream), lambda: path.select(stream=stream),
-                         lambda: path.attend(stream=stream, combine=False),
-                         lambda: path.combine(stream)])
-        stages = {"index_scores": st[0], "select": st[1], attn_key: st[2], "combine": st[3]}
-    elif stream_route:  # one partition: the attention kernel writes the output, no combine
-        st = stage_pass([lambda: path.index_scores(stream), lambda: path.select(stream=stream),
-                         lambda: path.attend(stream=stream)])
-        stages = {"index_scores": st[0], "select": st[1], attn_key: st[2]}
-    if stream_route:
-        # the first two stages as one msa_index_select launch, and the last two (with the
-        # combine) as one msa_select_sparse_attn_paged call, for comparison
-        stages["fused_index_select"] = stage_pass([lambda: path.index_select(stream)])[0]
-        stages["select_in_attention"] = stage_pass([lambda: path.select_attend(stream)])[0]
-        stages["step_with_separate_select"] = stage_pass(
-            [lambda: (path.index_scores(stream), path.select(stream=stream),
-                      path.attend(stream=stream))])[0]
-        idx_kind, idx_src = "index_scores", ("indexer.cu", "select_row.cuh")
-    else:
-        st = stage_pass([lambda: path.index_scores(stream), lambda: path.select(stream=stream),
-                         lambda: path.attend(stream=stream)])
-        stages = {"index_scores": st[0], "select": st[1], attn_key: st[2]}
-        idx_kind, idx_src = "index_scores", ("indexer_tc.cu",)
-    idx_ms, attn_ms = st[0], stages[attn_key]
+    head = bench_workload(args.workload, args, ws, rank, dev, sampler,
+                          with_cpu=rank == 0 and ws == 1 and not args.no_cpu_baseline)
+    others = {}
+    if not args.only:
+        # the other workloads, each measured the same way (every rank takes the same steps)
+        for name in wl.WORKLOADS:
+            if name != args.workload:
+                others[name] = bench_workload(name, args, ws, rank, dev, sampler, False)
     if sampler:
         sampler.stop()
-    clocks = sampler.summary(t_wall0, t_wall1) if sampler else None
-
-    # ---- end to end through the public API with host buffers: every step copies its inputs
-    # from pinned host memory and its output back, both inside the timed region.  The pipelined
-    # figure (HostPipeline, two deep) is the headline; the serial one (copy in, compute, copy
-    # out on one stream) is reported beside it.
-    e2e_ms = e2e_serial_ms = None
-    h2d = d2h = 0
-    if not args.no_e2e:
-        host = {k: prob[k].cpu().pin_memory() for k in msa.HostPipeline.PER_STEP}
-        outs = [torch.empty(path.out.shape, dtype=path.out.dtype).pin_memory() for _ in range(2)]
-        h2d = sum(v.numel() * v.element_size() for v in host.values())
-        d2h = outs[0].numel() * outs[0].element_size()
-        for _ in range(max(1, args.warmup)):
-            for k_, v_ in host.items():
-                prob[k_].copy_(v_, non_blocking=True)
-            path.run(stream)
-            outs[0].copy_(path.out, non_blocking=True)
-        torch.cuda.synchronize(dev)
-        barrier(ws, dev)
-        x0, x1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        x0.record(stream)
-        for _ in range(args.steps):
-            for k_, v_ in host.items():
-                prob[k_].copy_(v_, non_blocking=True)
-            path.run(stream)
-            outs[0].copy_(path.out, non_blocking=True)
-        x1.record(stream)
-        torch.cuda.synchronize(dev)
-        e2e_serial_ms = max_over_ranks(x0.elapsed_time(x1), ws, dev)
-
-        pipe = msa.HostPipeline(prob, num_splits=args.splits)
-        packed = pipe.pack(host)  # the step's inputs as one pinned buffer: one copy per step
-        for i in range(max(2, args.warmup)):
-            pipe.submit(packed, outs[i % 2])
-        pipe.finish(stream)
-        torch.cuda.synchronize(dev)
-        barrier(ws, dev)
-        x0.record(stream)
-        pipe.start(after=x0)
-        for i in range(args.steps):
-            pipe.submit(packed, outs[i % 2])
-        pipe.finish(stream)
-        x1.record(stream)
-        torch.cuda.synchronize(dev)
-        e2e_ms = max_over_ranks(x0.elapsed_time(x1), ws, dev)
-        h2d = packed.numel()
-        for p_ in pipe.paths:
-            assert int(p_.dev_err.item()) == 0, "device error flag set (host pipeline)"
-        assert torch.equal(outs[(args.steps - 1) % 2].to(dev), path.out), \
-            "host pipeline output differs from the device-resident step"
-        del pipe
-
-    # ---- the realised work of this step, for the roofline (idx_bytes, attn_bytes above)
-    tokens_total = sum_over_ranks(prob["total_q"], ws, dev) * args.steps
-    assert int(path.dev_err.item()) == 0, "device error flag set"
-
-    cpu = None
-    if rank == 0 and ws == 1 and not args.no_cpu_baseline:
-        sample, desc = oracle_sample(args.workload, args.cpu_sample_seqs, seed=7)
-        v, el, reps = time_oracle(sample, args.cpu_min_s, args.cpu_max_s)
-        cpu = {"value": v, "unit": UNIT, "cores": cpu_threads(), "kind": "oracle",
-               "sample": f"{desc}, seed 7, {reps} pass(es), {el:.1f} s"}
-
     if rank != 0:
         return 0
-    hbm, bf16, bf16_sus, peak_src = measured_peaks()
-    tensor_route = prob["max_q_len"] > 8  # prefill: dense contractions on the tensor cores
-    kinds = {idx_kind: (idx_ms, idx_bytes, idx_src),
-             "attention": (attn_ms, attn_bytes,
-                           ("attention_stream.cu", "attn_common.cuh", "select_row.cuh")
-                           if stream_route else
-                           (("attention_tile.cu", "attn_common.cuh") if fp8
-                            else ("attention_tc.cu",)))}
-    dom = max(kinds, key=lambda k: kinds[k][0])
-    d_ms, d_bytes, d_src = kinds[dom]
-    digest = source_digest(*d_src)
-    if tensor_route:
-        idx_flops, attn_flops = algorithmic_flops(prob, path.block_ids, path.num_selected)
-        d_flops = attn_flops if dom == "attention" else idx_flops
-        achieved = d_flops / (d_ms * 1e-3) / 1e12
-        roofline = {"bound": "tensor", "kernel": dom, "achieved": achieved, "peak": bf16,
-                    "unit": "TFLOP/s", "frac": achieved / bf16, "peak_source": peak_src,
-                    "traffic": profiled_traffic(dom, args.workload, digest),
-                    "algorithmic_flops_per_launch": d_flops,
-                    "note": "algorithmic FLOPs (selected, causally clipped positions only) over "
-                            "the kernel's time, against the bf16 burst peak"}
-        if dom == "attention" and not fp8:
-            ex = executed_flops_tiles(prob, path.block_ids, path.num_selected,
-                                      128 // (prob["H_q"] // prob["H_kv"]))
-            roofline["executed_flops_per_launch"] = ex
-            roofline["executed_tflops"] = ex / (d_ms * 1e-3) / 1e12
-            roofline["executed_frac"] = ex / (d_ms * 1e-3) / 1e12 / bf16
-    else:
-        achieved = d_bytes / (d_ms * 1e-3) / 1e9
-        roofline = {"bound": "hbm", "kernel": dom, "achieved": achieved, "peak": hbm,
-                    "unit": "GB/s", "frac": achieved / hbm, "peak_source": peak_src,
-                    "traffic": profiled_traffic(dom, args.workload, digest),
-                    "algorithmic_bytes_per_launch": d_bytes}
-    line = {
-        "metric": METRIC, "value": tokens_total / (ms * 1e-3), "unit": UNIT, "n_gpus": ws,
-        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms / args.steps,
-        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-        "dtype": "fp8-e4m3 kv / bf16" if fp8 else "bf16", "data": "synthetic",
-        "config": {"workload": args.workload, "batch": prob["batch"],
-                   "q_tokens_per_step": prob["total_q"], "H_kv": prob["H_kv"],
-                   "H_q": prob["H_q"], "head_dim": 128, "page_size": 128,
-                   "top_k": prob["top_k"], "init_blocks": prob["init_blocks"],
-                   "local_blocks": prob["local_blocks"], "kv_lens": f"{spec.kv_len}",
-                   "split_k_partials": splits_used, "parallelism": f"replicas x{ws}",
-                   "l2": (f"{(idx_bytes + attn_bytes) / 2**20:.1f} MiB touched per step, under "
-                          f"the {L2_BYTES / 2**20:.0f} MiB L2: L2 flushed before every step (a "
-                          f"{2 * L2_BYTES / 2**20:.0f} MiB write outside the step's events), "
-                          f"time = sum of the steps' own intervals") if flush else
-                         (f"inputs larger than L2: {(idx_bytes + attn_bytes) / 2**20:.0f} MiB "
-                          f"touched per step vs {L2_BYTES / 2**20:.0f} MiB L2, no flush")},
-        "roofline": roofline,
-        "step_hbm": {"algorithmic_bytes": idx_bytes + attn_bytes,
-                     "achieved_GBps": (idx_bytes + attn_bytes) / (ms / args.steps * 1e-3) / 1e9,
-                     "frac_of_measured": (idx_bytes + attn_bytes) / (ms / args.steps * 1e-3)
-                     / 1e9 / hbm,
-                     "frac_of_8TBps": (idx_bytes + attn_bytes) / (ms / args.steps * 1e-3)
-                     / 8e12},
-        "stages_ms": stages,
-        "gpu_launches": kernels_per_step * args.steps,
-        "clocks": clocks,
-        "e2e": None if e2e_ms is None else {
-            "value": tokens_total / (e2e_ms * 1e-3), "unit": UNIT,
-            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-            "serial_value": tokens_total / (e2e_serial_ms * 1e-3),
-            "note": "per-step inputs (q, q_idx, row offsets, cache lengths, page table) copied "
-                    "from pinned host memory and the output read back, every step inside the "
-                    "timed region; value: two-deep pipeline (the step's inputs packed in one "
-                    "pinned buffer, one copy; step i+1's copy in and step i-1's copy out on "
-                    "their own streams while step i computes); serial_value: one copy per "
-                    "input, compute, copy out, all on one stream; the caches stay resident"},
-        "cpu_baseline": cpu,
-    }
+    line = {"metric": METRIC, "value": head["value"], "unit": UNIT, "n_gpus": ws,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": head["ms_per_step"],
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": head["dtype"], "data": "synthetic"}
+    line.update({k: v for k, v in head.items() if k not in ("value", "ms_per_step", "dtype")})
+    if others:
+        line["workloads"] = {
+            n: {k: r[k] for k in ("value", "ms_per_step", "dtype", "config", "timing",
+                                  "roofline", "step_hbm", "step_flops", "stages_ms",
+                                  "launches_per_step", "clocks", "e2e") if k in r}
+            for n, r in others.items()}
     print(json.dumps(line), flush=True)
     return 0
 
@@ -574,14 +649,20 @@ def run_ours(args):
 def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__)
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=200)
-    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", default="bf16_decode")
+    ap.add_argument("--workload", default="fp8_long_decode",
+                    help="the headline workload (the largest single-GPU configuration)")
+    ap.add_argument("--only", action="store_true",
+                    help="measure the headline workload only (not the other four)")
     ap.add_argument("--splits", type=int, default=0, help="split-K partitions (0 = heuristic)")
+    ap.add_argument("--min-seconds", type=float, default=1.0,
+                    help="repeat K-step blocks for about this long; the median block counts")
+    ap.add_argument("--stage-seconds", type=float, default=0.5)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer pass")
-    ap.add_argument("--batch", type=int, default=0, help="override the workload's batch "
+    ap.add_argument("--batch", type=int, default=0, help="override the workloads' batch "
                     "(profiling runs on a smaller case; not a bench number)")
     ap.add_argument("--cpu-sample-seqs", type=int, default=4)
     ap.add_argument("--cpu-min-s", type=float, default=10.0)

@@ -41,14 +41,17 @@ EncodeTiledFn encode_fn() {
 // A paged cache [tiles = num_pages * heads][128 tokens][128 dims] as a 3-D tensor map whose
 // box is one (page, head) tile: 128 tokens x 64 bf16 (two loads per tile) or 128 x 128 e4m3,
 // written to shared memory with the 128-byte swizzle.
-bool page_tensor_map(CUtensorMap *map, const void *base, long long tiles, bool fp8) {
+// `rows` < 128 views a tile of 1-byte elements as `rows` rows of 128 bytes (the fp4 index-K
+// tile: 64 rows, two tokens' code pairs each).
+bool page_tensor_map(CUtensorMap *map, const void *base, long long tiles, bool fp8,
+                     int rows = kBlock) {
   EncodeTiledFn fn = encode_fn();
   if (!fn) return false;
   const cuuint64_t esz = fp8 ? 1 : 2;
-  const cuuint64_t dims[3] = {static_cast<cuuint64_t>(kHeadDim), static_cast<cuuint64_t>(kBlock),
+  const cuuint64_t dims[3] = {static_cast<cuuint64_t>(kHeadDim), static_cast<cuuint64_t>(rows),
                               static_cast<cuuint64_t>(tiles)};
-  const cuuint64_t strides[2] = {kHeadDim * esz, kHeadDim * kBlock * esz};
-  const cuuint32_t box[3] = {fp8 ? 128u : 64u, static_cast<cuuint32_t>(kBlock), 1u};
+  const cuuint64_t strides[2] = {kHeadDim * esz, kHeadDim * rows * esz};
+  const cuuint32_t box[3] = {fp8 ? 128u : 64u, static_cast<cuuint32_t>(rows), 1u};
   const cuuint32_t estr[3] = {1, 1, 1};
   memset(map, 0, sizeof(*map));
   const CUresult r = fn(map, fp8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16,
@@ -260,18 +263,32 @@ struct FusedSelect {
   int top_k, init_blocks, local_blocks, S;
 };
 
-bool index_uses_tc(const msa_ragged_paged_t *rp, int Hg) {
-  return rp->max_q_len > MSA_MAX_SPEC_DRAFT && Hg <= 128;
+// The prefill route scores BF16 index-K on tcgen05; the scaled formats take the warp-MMA
+// kernel on every route.
+bool index_uses_tc(const msa_ragged_paged_t *rp, int Hg, int idx_fmt) {
+  return idx_fmt == kIdxBf16 && rp->max_q_len > MSA_MAX_SPEC_DRAFT && Hg <= 128;
+}
+
+bool index_k_ok(const msa_index_k_t *k, int32_t num_kv_heads) {
+  if (!k || !k->codes || !aligned(k->codes, 16) ||
+      !(k->num_heads == 1 || k->num_heads == num_kv_heads))
+    return false;
+  if (k->dtype == MSA_IDX_BF16) return true;
+  if (k->dtype == MSA_IDX_FP8_E4M3 || k->dtype == MSA_IDX_FP4_E2M1)
+    return k->scales && aligned(k->scales, 16);
+  return false;
 }
 
 msa_status_t index_scores_impl(const msa_ragged_paged_t *rp, const void *q_idx,
-                               const void *k_idx_cache, int32_t num_kv_heads,
-                               int32_t num_idx_k_heads, int32_t max_blocks, float *scores,
-                               int32_t *dev_err, cudaStream_t stream, const FusedSelect *fs) {
-  if (!ragged_ok(rp) || !q_idx || !k_idx_cache || !scores || num_kv_heads < 1 ||
-      !(num_idx_k_heads == 1 || num_idx_k_heads == num_kv_heads) || max_blocks < 1 ||
-      max_blocks > rp->max_pages_per_seq || !aligned(k_idx_cache, 16) || !aligned(q_idx, 16))
+                               const msa_index_k_t *kidx, int32_t num_kv_heads,
+                               int32_t max_blocks, float *scores, int32_t *dev_err,
+                               cudaStream_t stream, const FusedSelect *fs) {
+  if (!ragged_ok(rp) || !q_idx || !scores || num_kv_heads < 1 || !index_k_ok(kidx, num_kv_heads) ||
+      max_blocks < 1 || max_blocks > rp->max_pages_per_seq || !aligned(q_idx, 16))
     return MSA_ERR_INVALID_ARG;
+  const void *k_idx_cache = kidx->codes;
+  const int32_t num_idx_k_heads = kidx->num_heads;
+  const int idx_fmt = static_cast<int>(kidx->dtype);
   const int Hg = num_kv_heads / num_idx_k_heads;
   if (Hg > 32) return MSA_ERR_UNSUPPORTED;
   if (static_cast<long long>(rp->num_pages) * num_idx_k_heads >= (1LL << 31))
@@ -292,8 +309,10 @@ msa_status_t index_scores_impl(const msa_ragged_paged_t *rp, const void *q_idx,
   a.H_idxk = num_idx_k_heads;
   a.max_blocks = max_blocks;
   a.counters = nullptr;
+  a.idx_fmt = idx_fmt;
+  a.k_idx_scale = kidx->scales;
   // prefill: the dense tile x page contraction runs on tcgen05 (128-row tiles)
-  if (index_uses_tc(rp, Hg)) {
+  if (index_uses_tc(rp, Hg, idx_fmt)) {
     if (fs) return MSA_ERR_UNSUPPORTED;  // the caller selects with a separate launch
     a.qt = std::min(rp->max_q_len, std::max(1, 128 / Hg));
     a.tiles = (rp->max_q_len + a.qt - 1) / a.qt;
@@ -329,28 +348,81 @@ msa_status_t index_scores_impl(const msa_ragged_paged_t *rp, const void *q_idx,
   }
 
   CUtensorMap kmap;
-  if (!page_tensor_map(&kmap, k_idx_cache, static_cast<long long>(rp->num_pages) * num_idx_k_heads,
-                       false))
-    return MSA_ERR_CUDA;
+  const long long ktiles = static_cast<long long>(rp->num_pages) * num_idx_k_heads;
+  const bool ok_map = idx_fmt == kIdxBf16 ? page_tensor_map(&kmap, k_idx_cache, ktiles, false)
+                      : idx_fmt == kIdxFp8
+                          ? page_tensor_map(&kmap, k_idx_cache, ktiles, true)
+                          : page_tensor_map(&kmap, k_idx_cache, ktiles, true, kBlock / 2);
+  if (!ok_map) return MSA_ERR_CUDA;
   return launch_index_scores(kmap, a, mt, static_cast<int>(chunks), stream) == cudaSuccess
              ? MSA_OK
              : MSA_ERR_CUDA;
 }
 
+msa_index_k_t bf16_index_k(const void *k_idx_cache, int32_t num_idx_k_heads) {
+  msa_index_k_t k;
+  k.dtype = MSA_IDX_BF16;
+  k.codes = k_idx_cache;
+  k.scales = nullptr;
+  k.num_heads = num_idx_k_heads;
+  return k;
+}
+
 }  // namespace
+
+msa_status_t msa_index_scores_k(const msa_ragged_paged_t *rp, const void *q_idx,
+                                const msa_index_k_t *k_idx, int32_t num_kv_heads,
+                                int32_t max_blocks, uint32_t flags, float *scores,
+                                int32_t *dev_err, struct CUstream_st *stream) {
+  if (flags != 0) return MSA_ERR_INVALID_ARG;
+  if (ragged_ok(rp) && rp->total_q == 0) return MSA_OK;  // nothing to score
+  return index_scores_impl(rp, q_idx, k_idx, num_kv_heads, max_blocks, scores, dev_err,
+                           reinterpret_cast<cudaStream_t>(stream), nullptr);
+}
 
 msa_status_t msa_index_scores(const msa_ragged_paged_t *rp, const void *q_idx,
                               const void *k_idx_cache, int32_t num_kv_heads,
                               int32_t num_idx_k_heads, int32_t max_blocks, float *scores,
                               int32_t *dev_err, struct CUstream_st *stream) {
-  if (ragged_ok(rp) && rp->total_q == 0) return MSA_OK;  // nothing to score
-  return index_scores_impl(rp, q_idx, k_idx_cache, num_kv_heads, num_idx_k_heads, max_blocks,
-                           scores, dev_err, reinterpret_cast<cudaStream_t>(stream), nullptr);
+  const msa_index_k_t k = bf16_index_k(k_idx_cache, num_idx_k_heads);
+  return msa_index_scores_k(rp, q_idx, &k, num_kv_heads, max_blocks, 0u, scores, dev_err,
+                            stream);
 }
 
 size_t msa_index_select_counters(const msa_ragged_paged_t *rp, int32_t num_idx_k_heads) {
   if (!ragged_ok(rp) || num_idx_k_heads < 1) return 0;
   return static_cast<size_t>(rp->batch) * rp->max_q_len * num_idx_k_heads;
+}
+
+msa_status_t msa_index_select_k(const msa_ragged_paged_t *rp, const void *q_idx,
+                                const msa_index_k_t *k_idx, int32_t num_kv_heads,
+                                int32_t max_blocks, int32_t top_k, int32_t init_blocks,
+                                int32_t local_blocks, uint32_t flags, float *scores,
+                                int32_t *block_ids, int32_t *num_selected, int32_t *counters,
+                                int32_t *dev_err, struct CUstream_st *stream) {
+  const long long S = static_cast<long long>(top_k) + init_blocks + local_blocks;
+  if (!ragged_ok(rp) || num_kv_heads < 1 || !k_idx || k_idx->num_heads < 1 || max_blocks < 1 ||
+      top_k < 0 || init_blocks < 0 || local_blocks < 0 || S < 1 || S > (1 << 20) ||
+      flags != 0)
+    return MSA_ERR_INVALID_ARG;
+  if (rp->total_q == 0) return MSA_OK;
+  if (!block_ids || !num_selected) return MSA_ERR_INVALID_ARG;
+  const cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const bool fused =
+      num_kv_heads % k_idx->num_heads == 0 &&
+      !index_uses_tc(rp, num_kv_heads / k_idx->num_heads, static_cast<int>(k_idx->dtype));
+  if (fused) {
+    if (!counters || !aligned(counters, 4)) return MSA_ERR_INVALID_ARG;
+    const FusedSelect fs{counters, block_ids, num_selected, top_k, init_blocks, local_blocks,
+                         static_cast<int>(S)};
+    return index_scores_impl(rp, q_idx, k_idx, num_kv_heads, max_blocks, scores, dev_err, st,
+                             &fs);
+  }
+  const msa_status_t e =
+      index_scores_impl(rp, q_idx, k_idx, num_kv_heads, max_blocks, scores, dev_err, st, nullptr);
+  if (e != MSA_OK) return e;
+  return msa_select_blocks(rp, scores, num_kv_heads, max_blocks, top_k, init_blocks,
+                           local_blocks, block_ids, num_selected, dev_err, stream);
 }
 
 msa_status_t msa_index_select(const msa_ragged_paged_t *rp, const void *q_idx,
@@ -359,28 +431,10 @@ msa_status_t msa_index_select(const msa_ragged_paged_t *rp, const void *q_idx,
                               int32_t init_blocks, int32_t local_blocks, float *scores,
                               int32_t *block_ids, int32_t *num_selected, int32_t *counters,
                               int32_t *dev_err, struct CUstream_st *stream) {
-  const long long S = static_cast<long long>(top_k) + init_blocks + local_blocks;
-  if (!ragged_ok(rp) || num_kv_heads < 1 || num_idx_k_heads < 1 || max_blocks < 1 ||
-      top_k < 0 || init_blocks < 0 || local_blocks < 0 || S < 1 || S > (1 << 20))
-    return MSA_ERR_INVALID_ARG;
-  if (rp->total_q == 0) return MSA_OK;
-  if (!block_ids || !num_selected) return MSA_ERR_INVALID_ARG;
-  const cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  const bool fused = num_kv_heads % num_idx_k_heads == 0 &&
-                     !index_uses_tc(rp, num_kv_heads / num_idx_k_heads);
-  if (fused) {
-    if (!counters || !aligned(counters, 4)) return MSA_ERR_INVALID_ARG;
-    const FusedSelect fs{counters, block_ids, num_selected, top_k, init_blocks, local_blocks,
-                         static_cast<int>(S)};
-    return index_scores_impl(rp, q_idx, k_idx_cache, num_kv_heads, num_idx_k_heads, max_blocks,
-                             scores, dev_err, st, &fs);
-  }
-  const msa_status_t e = index_scores_impl(rp, q_idx, k_idx_cache, num_kv_heads,
-                                           num_idx_k_heads, max_blocks, scores, dev_err, st,
-                                           nullptr);
-  if (e != MSA_OK) return e;
-  return msa_select_blocks(rp, scores, num_kv_heads, max_blocks, top_k, init_blocks,
-                           local_blocks, block_ids, num_selected, dev_err, stream);
+  const msa_index_k_t k = bf16_index_k(k_idx_cache, num_idx_k_heads);
+  return msa_index_select_k(rp, q_idx, &k, num_kv_heads, max_blocks, top_k, init_blocks,
+                            local_blocks, 0u, scores, block_ids, num_selected, counters, dev_err,
+                            stream);
 }
 
 msa_status_t msa_select_blocks(const msa_ragged_paged_t *rp, const float *scores,

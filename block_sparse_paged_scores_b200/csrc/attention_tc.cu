@@ -19,7 +19,9 @@
 //   warps 4-11 softmax, two warpgroups taking alternate blocks (even / odd), each with its own
 //              S buffer, O accumulator and running max and sum: one query row per thread (its
 //              TMEM lane), one pass over the row's 128 scores held in registers (masked max,
-//              exp2, P as bf16 back into TMEM over its S).  The first warpgroup (producers, MMA
+//              exp2, P as bf16 back into TMEM over its S; the row sum adds the same rounded
+//              P that the P V MMA reads, so that numerator and denominator weigh every
+//              position alike).  The first warpgroup (producers, MMA
 //              issuer, one idle warp) hands registers to the softmax warpgroups (setmaxnreg).
 //              The groups never wait for each other inside the loop, so one group's
 //              exponentials overlap the other's loads and maxima.  A group's
@@ -413,9 +415,9 @@ __global__ void __launch_bounds__(kTcThreads, 1)
               const float2 x = fma2(make_float2(__uint_as_float(v[64 * h + e]),
                                                 __uint_as_float(v[64 * h + e + 1])),
                                     make_float2(sc, sc), make_float2(nb, nb));
-              const float e0 = fast_exp2(x.x), e1 = fast_exp2(x.y);
-              ps2[(e >> 1) & 3] = add2(ps2[(e >> 1) & 3], make_float2(e0, e1));
-              pk[e >> 1] = pack_bf16x2(e0, e1);
+              const uint32_t pb = pack_bf16x2(fast_exp2(x.x), fast_exp2(x.y));
+              pk[e >> 1] = pb;
+              ps2[(e >> 1) & 3] = add2(ps2[(e >> 1) & 3], bf16x2_to_float2(pb));
             }
           } else {
 #pragma unroll
@@ -426,9 +428,10 @@ __global__ void __launch_bounds__(kTcThreads, 1)
               const float x1 = (use && pe + 1 <= lim)
                                    ? fmaf(__uint_as_float(v[pe + 1]), sc, nb)
                                    : -INFINITY;
-              const float e0 = fast_exp2(x0), e1 = fast_exp2(x1);
-              ps4[(e >> 1) & 3] += e0 + e1;
-              pk[e >> 1] = pack_bf16x2(e0, e1);
+              const uint32_t pb = pack_bf16x2(fast_exp2(x0), fast_exp2(x1));
+              pk[e >> 1] = pb;
+              const float2 pf = bf16x2_to_float2(pb);
+              ps4[(e >> 1) & 3] += pf.x + pf.y;
             }
           }
           tmem_st32(s_addr + 32 * h, pk);

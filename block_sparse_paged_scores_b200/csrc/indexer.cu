@@ -13,6 +13,18 @@
 // position, reduce the row max with warp shuffles and then across the four warps through
 // shared memory, and write one fp32 score per (row, page).
 //
+// Scaled index-K caches (TensorRT-LLM "DeepSeekSparseAttentionConfig", indexer_k_dtype): fp8
+// (e4m3 codes, one fp32 scale per token) and fp4 (e2m1 code pairs, one UE8M0 exponent per 32
+// elements).  The codes stream by TMA like the bf16 tile and the token's 512 bytes of scales by
+// one bulk copy on the same barrier.  The consumers turn two codes into an f16 pair with one
+// cvt and run f16 mma.sync against q_idx turned into f16 once per CTA (each row prescaled by a
+// power of two that keeps it below 2^15, undone exactly on its scores).  The 128 dims are
+// visited in an order of the consumers' own (the same on both operands, so the dot product is
+// unchanged) in which a thread reads one 32-bit word of its position's codes per k-step, and
+// in which every k-step of the fp4 layout stays inside one 32-element exponent group: each
+// group's partial product is then scaled by its exponent, and an fp8 row by its token's scale,
+// before the max.
+//
 // With the selection fused in (decode and speculative routes), the CTAs of one (sequence,
 // tile, index-K head) count themselves out on a device counter once their scores are written;
 // the last one runs stage 2 for the unit's rows (select_row.cuh, reading the scores from L2) and
@@ -29,14 +41,42 @@ namespace {
 // (two CTAs per SM) for long ones: the same bytes in flight per SM, but more pages in process at
 // once wins on short chunks, a deeper ring on long streams.
 constexpr int kLongChunk = 32;  // pages per CTA from which the deeper ring is used
-constexpr uint32_t kTileBytes = kBlock * kHeadDim * 2;  // one (page, head) tile, bf16
 constexpr int kConsumerWarps = 4;
 constexpr int kThreads = 32 * (kConsumerWarps + 1);
 
-template <int kStages>
+// Index-K formats (IndexerArgs::idx_fmt), one (page, head) tile each: bf16 32 KiB; fp8 16 KiB
+// of codes + 128 fp32 scales; fp4 8 KiB of code pairs (viewed as 64 rows of 128 bytes: tokens
+// 2r and 2r + 1 in row r) + 128 x 4 exponent bytes.
+template <int IF>
+constexpr uint32_t tile_bytes() {
+  return IF == kIdxBf16 ? 32768u : (IF == kIdxFp8 ? 16384u : 8192u);
+}
+template <int IF>
+constexpr uint32_t scale_bytes() { return IF == kIdxBf16 ? 0u : 512u; }
+// The ring keeps the same bytes in flight for every format: smaller tiles, more stages.
+template <int ST, int IF>
+constexpr int ring_stages() { return ST * static_cast<int>(32768u / tile_bytes<IF>()); }
+
+template <int kStages, int IF>
 constexpr size_t smem_bytes() {
-  return 1024 /*alignment slack*/ + kStages * kTileBytes + 2 * kStages * sizeof(uint64_t) +
-         kStages * sizeof(int) + 2 * kConsumerWarps * 32 * sizeof(float) + 16;
+  return 1024 /*alignment slack*/ + kStages * (tile_bytes<IF>() + scale_bytes<IF>()) +
+         2 * kStages * sizeof(uint64_t) + kStages * sizeof(int) +
+         2 * kConsumerWarps * 32 * sizeof(float) + 16;
+}
+
+// First of the four dims of k-step ks that lane j (lane % 4) holds, in the scaled formats'
+// visiting order: fp8 dims 16 ks + 4 j .. + 3 (one word of codes); fp4 dims 32 g + 8 j + 4 h
+// .. + 3 for ks = 2 g + h (half a word of code pairs, inside exponent group g).  The first
+// two of the four are the MMA's k slots 2j, 2j + 1, the last two 2j + 8, 2j + 9.
+template <int IF>
+__device__ __forceinline__ int scaled_dim(int ks, int j) {
+  return IF == kIdxFp8 ? 16 * ks + 4 * j : 32 * (ks >> 1) + 8 * j + 4 * (ks & 1);
+}
+
+// 2^(x - 127) of a UE8M0 byte (0xFF: NaN)
+__device__ __forceinline__ float ue8m0_to_float(uint32_t x) {
+  return x == 0xFFu ? __uint_as_float(0x7fc00000u)
+                    : (x == 0u ? __uint_as_float(0x00400000u) : __uint_as_float(x << 23));
 }
 
 // The consumer warps (threads 0..127) of every CTA of a unit call this once the CTA's scores
@@ -74,9 +114,11 @@ __device__ __forceinline__ void count_out_and_select(const IndexerArgs &a, int b
 
 // KPL < 0: scores only; KPL >= 0: selection fused, KPL keys per lane in registers (0: any
 // number of blocks, read from L2 on every pass).
-template <int MT, int KPL, int kStages>
+template <int MT, int KPL, int kStages, int IF>
 __global__ void __launch_bounds__(kThreads)
     index_scores_kernel(const __grid_constant__ CUtensorMap kmap, const IndexerArgs a) {
+  constexpr uint32_t kTileBytes = tile_bytes<IF>();
+  constexpr uint32_t kScaleBytes = scale_bytes<IF>();
   pdl_wait();
   pdl_launch_dependents();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -128,7 +170,8 @@ __global__ void __launch_bounds__(kThreads)
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                               ~static_cast<uintptr_t>(1023));
   uint8_t *stages = smem;
-  uint64_t *full = reinterpret_cast<uint64_t *>(stages + kStages * kTileBytes);
+  uint8_t *scale_st = stages + kStages * kTileBytes;  // [kStages][kScaleBytes]
+  uint64_t *full = reinterpret_cast<uint64_t *>(scale_st + kStages * kScaleBytes);
   uint64_t *empty = full + kStages;
   int *page_ok = reinterpret_cast<int *>(empty + kStages);
   float *red = reinterpret_cast<float *>(page_ok + kStages);  // [2][4 warps][32 rows]
@@ -177,10 +220,19 @@ __global__ void __launch_bounds__(kThreads)
             const bool ok = page >= 0 && page < a.num_pages;
             page_ok[s] = ok;
             if (ok) {
-              mbar_arrive_expect_tx(&full[s], kTileBytes);
+              mbar_arrive_expect_tx(&full[s], kTileBytes + kScaleBytes);
               const int c2 = page * a.H_idxk + hk;
-              tma_load_3d(stages + s * kTileBytes, &kmap, &full[s], 0, 0, c2);
-              tma_load_3d(stages + s * kTileBytes + kTileBytes / 2, &kmap, &full[s], 64, 0, c2);
+              if constexpr (IF == kIdxBf16) {
+                tma_load_3d(stages + s * kTileBytes, &kmap, &full[s], 0, 0, c2);
+                tma_load_3d(stages + s * kTileBytes + kTileBytes / 2, &kmap, &full[s], 64, 0,
+                            c2);
+              } else {
+                tma_load_3d(stages + s * kTileBytes, &kmap, &full[s], 0, 0, c2);
+                bulk_load(scale_st + s * kScaleBytes,
+                          static_cast<const uint8_t *>(a.k_idx_scale) +
+                              static_cast<size_t>(c2) * kScaleBytes,
+                          kScaleBytes, &full[s]);
+              }
             } else {
               report(a.dev_err, MSA_DEVERR_PAGE_ID);
               mbar_arrive(&full[s]);
@@ -197,21 +249,27 @@ __global__ void __launch_bounds__(kThreads)
   // -------------------------------------------------------------- consumers
   // A fragments of Q (rows x 128) for m16n8k16: a0a1 = (row, k), a2a3 = (row + 8, k),
   // a4a5 = (row, k + 8), a6a7 = (row + 8, k + 8), k = 16 ks + 2 (lane % 4).
+  // Scaled formats: the fragments hold f16 pairs of the dims scaled_dim() names, each row
+  // multiplied by qscale = 2^-k (k >= 0, 1 unless the row holds |values| >= 2^15) and its
+  // scores by 1 / qscale.
   uint32_t qa[MT][8][4];
   int prow[MT][2];
+  float qinv[MT][2];
 #pragma unroll
   for (int mt = 0; mt < MT; ++mt) {
 #pragma unroll
     for (int slot = 0; slot < 2; ++slot) {
       const int r = mt * 16 + (lane >> 2) + slot * 8;
       prow[mt][slot] = r < rows ? cl + tok0 + r / Hg : -1;
+      qinv[mt][slot] = 1.f;
     }
 #pragma unroll
     for (int ks = 0; ks < 8; ++ks) {
 #pragma unroll
       for (int q4 = 0; q4 < 4; ++q4) {
         const int r = mt * 16 + (lane >> 2) + (q4 & 1) * 8;
-        const int k = ks * 16 + (lane & 3) * 2 + (q4 >> 1) * 8;
+        const int k = IF == kIdxBf16 ? ks * 16 + (lane & 3) * 2 + (q4 >> 1) * 8
+                                     : scaled_dim<IF>(ks, lane & 3) + (q4 >> 1) * 2;
         uint32_t v = 0;
         if (r < rows) {
           const int t = row0 + tok0 + r / Hg, g = hk + (r % Hg) * a.H_idxk;
@@ -219,6 +277,34 @@ __global__ void __launch_bounds__(kThreads)
               a.q_idx + (static_cast<size_t>(t) * a.H_kv + g) * kHeadDim + k);
         }
         qa[mt][ks][q4] = v;
+      }
+    }
+    if constexpr (IF != kIdxBf16) {
+#pragma unroll
+      for (int slot = 0; slot < 2; ++slot) {
+        float m = 0.f;
+#pragma unroll
+        for (int ks = 0; ks < 8; ++ks)
+#pragma unroll
+          for (int hi = 0; hi < 2; ++hi) {
+            const float2 f = bf16x2_to_float2(qa[mt][ks][slot + 2 * hi]);
+            m = fmaxf(m, fmaxf(fabsf(f.x), fabsf(f.y)));
+          }
+        m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 1));
+        m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 2));
+        float qs = 1.f;
+        if (m >= 32768.f) {  // 2^k with m * 2^-k < 2^15 (m < 2^(e + 1), e = its exponent)
+          const int k = static_cast<int>((__float_as_uint(m) >> 23) & 0xff) - 127 - 14;
+          qs = __uint_as_float(static_cast<uint32_t>(127 - k) << 23);
+          qinv[mt][slot] = __uint_as_float(static_cast<uint32_t>(127 + k) << 23);
+        }
+#pragma unroll
+        for (int ks = 0; ks < 8; ++ks)
+#pragma unroll
+          for (int hi = 0; hi < 2; ++hi) {
+            const float2 f = bf16x2_to_float2(qa[mt][ks][slot + 2 * hi]);
+            qa[mt][ks][slot + 2 * hi] = pack_f16x2(f.x * qs, f.y * qs);
+          }
       }
     }
   }
@@ -243,20 +329,80 @@ __global__ void __launch_bounds__(kThreads)
         for (int e = 0; e < 4; ++e) acc[mt][nt][e] = 0.f;
     if (ok) {
       const uint32_t tile_addr = smem_u32(stages + s * kTileBytes);
+      if constexpr (IF == kIdxBf16) {
 #pragma unroll
-      for (int ks = 0; ks < 8; ++ks) {
-        uint32_t bf[4][2];
+        for (int ks = 0; ks < 8; ++ks) {
+          uint32_t bf[4][2];
 #pragma unroll
-        for (int h = 0; h < 2; ++h) {
-          const int pos = pbase + h * 16 + (mi >> 1) * 8 + rr;
-          const int chunk = ks * 2 + (mi & 1);
-          ldsm_x4(tile_addr + sw128(pos, chunk, kTileBytes / 2), bf[2 * h][0], bf[2 * h][1],
-                  bf[2 * h + 1][0], bf[2 * h + 1][1]);
+          for (int h = 0; h < 2; ++h) {
+            const int pos = pbase + h * 16 + (mi >> 1) * 8 + rr;
+            const int chunk = ks * 2 + (mi & 1);
+            ldsm_x4(tile_addr + sw128(pos, chunk, kTileBytes / 2), bf[2 * h][0], bf[2 * h][1],
+                    bf[2 * h + 1][0], bf[2 * h + 1][1]);
+          }
+#pragma unroll
+          for (int mt = 0; mt < MT; ++mt)
+#pragma unroll
+            for (int nt = 0; nt < 4; ++nt)
+              mma_bf16(acc[mt][nt], qa[mt][ks], bf[nt][0], bf[nt][1]);
         }
+      } else {
+        const uint8_t *sc = scale_st + s * kScaleBytes;
+        const int j4 = lane & 3;
 #pragma unroll
-        for (int mt = 0; mt < MT; ++mt)
+        for (int nt = 0; nt < 4; ++nt) {
+          const int pos = pbase + nt * 8 + (lane >> 2);         // this lane's B column
+          const int c0 = pbase + nt * 8 + 2 * j4;                // its two C columns
+          if constexpr (IF == kIdxFp8) {
 #pragma unroll
-          for (int nt = 0; nt < 4; ++nt) mma_bf16(acc[mt][nt], qa[mt][ks], bf[nt][0], bf[nt][1]);
+            for (int ks = 0; ks < 8; ++ks) {
+              const uint32_t w = *reinterpret_cast<const uint32_t *>(
+                  stages + s * kTileBytes + sw128(pos, ks, kTileBytes) + 4 * j4);
+              const uint32_t b0 = e4m3x2_to_f16x2(static_cast<uint16_t>(w & 0xffffu));
+              const uint32_t b1 = e4m3x2_to_f16x2(static_cast<uint16_t>(w >> 16));
+#pragma unroll
+              for (int mt = 0; mt < MT; ++mt) mma_f16(acc[mt][nt], qa[mt][ks], b0, b1);
+            }
+            const float2 ts = *reinterpret_cast<const float2 *>(sc + 4 * c0);  // token scales
+#pragma unroll
+            for (int mt = 0; mt < MT; ++mt)
+#pragma unroll
+              for (int e = 0; e < 4; ++e)
+                acc[mt][nt][e] *= ((e & 1) ? ts.y : ts.x) * qinv[mt][e >> 1];
+          } else {
+            const uint32_t ex0 = *reinterpret_cast<const uint32_t *>(sc + 4 * c0);
+            const uint32_t ex1 = *reinterpret_cast<const uint32_t *>(sc + 4 * c0 + 4);
+#pragma unroll
+            for (int gq = 0; gq < 4; ++gq) {
+              const uint32_t w = *reinterpret_cast<const uint32_t *>(
+                  stages + s * kTileBytes + sw128(pos >> 1, 4 * (pos & 1) + gq, kTileBytes) +
+                  4 * j4);
+              float cg[MT][4];
+#pragma unroll
+              for (int mt = 0; mt < MT; ++mt)
+#pragma unroll
+                for (int e = 0; e < 4; ++e) cg[mt][e] = 0.f;
+#pragma unroll
+              for (int h = 0; h < 2; ++h) {
+                const uint32_t b0 = e2m1x2_to_f16x2((w >> (16 * h)) & 0xffu);
+                const uint32_t b1 = e2m1x2_to_f16x2((w >> (16 * h + 8)) & 0xffu);
+#pragma unroll
+                for (int mt = 0; mt < MT; ++mt) mma_f16(cg[mt], qa[mt][2 * gq + h], b0, b1);
+              }
+              const float e0 = ue8m0_to_float((ex0 >> (8 * gq)) & 0xffu);
+              const float e1 = ue8m0_to_float((ex1 >> (8 * gq)) & 0xffu);
+#pragma unroll
+              for (int mt = 0; mt < MT; ++mt)
+#pragma unroll
+                for (int e = 0; e < 4; ++e)
+                  acc[mt][nt][e] = fmaf(cg[mt][e], (e & 1) ? e1 : e0, acc[mt][nt][e]);
+            }
+#pragma unroll
+            for (int mt = 0; mt < MT; ++mt)
+#pragma unroll
+              for (int e = 0; e < 4; ++e) acc[mt][nt][e] *= qinv[mt][e >> 1];
+          }
+        }
       }
     }
     __syncwarp();
@@ -294,39 +440,52 @@ __global__ void __launch_bounds__(kThreads)
   if (KPL >= 0) count_out_and_select<KPL>(a, b, tile, hk, row0, tok0, ntok, cl, is_last);
 }
 
-template <int MT, int KPL, int ST>
+template <int MT, int KPL, int ST, int IF>
 cudaError_t launch_one(const CUtensorMap &kidx_map, const IndexerArgs &a, int chunks,
                        cudaStream_t s) {
+  constexpr int kStages = ring_stages<ST, IF>();
   const dim3 grid(a.batch * a.tiles * a.H_idxk * chunks);
-  const size_t smem = smem_bytes<ST>();
-  cudaError_t e = ensure_smem_limit(
-      reinterpret_cast<const void *>(&index_scores_kernel<MT, KPL, ST>), static_cast<int>(smem));
+  const size_t smem = smem_bytes<kStages, IF>();
+  auto *kernel = &index_scores_kernel<MT, KPL, kStages, IF>;
+  cudaError_t e = ensure_smem_limit(reinterpret_cast<const void *>(kernel),
+                                    static_cast<int>(smem));
   if (e != cudaSuccess) return e;
-  return launch_pdl(index_scores_kernel<MT, KPL, ST>, grid, dim3(kThreads), smem, s, kidx_map, a);
+  return launch_pdl(kernel, grid, dim3(kThreads), smem, s, kidx_map, a);
 }
 
-template <int MT, int KPL>
+template <int MT, int KPL, int IF>
 cudaError_t launch_st(const CUtensorMap &kidx_map, const IndexerArgs &a, int chunks,
                       cudaStream_t s) {
-  return a.chunk >= kLongChunk ? launch_one<MT, KPL, 3>(kidx_map, a, chunks, s)
-                               : launch_one<MT, KPL, 2>(kidx_map, a, chunks, s);
+  return a.chunk >= kLongChunk ? launch_one<MT, KPL, 3, IF>(kidx_map, a, chunks, s)
+                               : launch_one<MT, KPL, 2, IF>(kidx_map, a, chunks, s);
 }
 
-template <int MT>
+template <int MT, int IF>
 cudaError_t launch_mt(const CUtensorMap &kidx_map, const IndexerArgs &a, int chunks,
                       cudaStream_t s) {
-  if (!a.counters) return launch_st<MT, -1>(kidx_map, a, chunks, s);
-  if (a.max_blocks <= 4 * 32) return launch_st<MT, 4>(kidx_map, a, chunks, s);
-  if (a.max_blocks <= 16 * 32) return launch_st<MT, 16>(kidx_map, a, chunks, s);
-  if (a.max_blocks <= 32 * 32) return launch_st<MT, 32>(kidx_map, a, chunks, s);
-  return launch_st<MT, 0>(kidx_map, a, chunks, s);
+  if (!a.counters) return launch_st<MT, -1, IF>(kidx_map, a, chunks, s);
+  if (a.max_blocks <= 4 * 32) return launch_st<MT, 4, IF>(kidx_map, a, chunks, s);
+  if (a.max_blocks <= 16 * 32) return launch_st<MT, 16, IF>(kidx_map, a, chunks, s);
+  if (a.max_blocks <= 32 * 32) return launch_st<MT, 32, IF>(kidx_map, a, chunks, s);
+  return launch_st<MT, 0, IF>(kidx_map, a, chunks, s);
+}
+
+template <int IF>
+cudaError_t launch_if(const CUtensorMap &kidx_map, const IndexerArgs &a, int mt, int chunks,
+                      cudaStream_t s) {
+  return mt == 1 ? launch_mt<1, IF>(kidx_map, a, chunks, s)
+                 : launch_mt<2, IF>(kidx_map, a, chunks, s);
 }
 
 }  // namespace
 
 cudaError_t launch_index_scores(const CUtensorMap &kidx_map, const IndexerArgs &a, int mt,
                                 int chunks, cudaStream_t s) {
-  return mt == 1 ? launch_mt<1>(kidx_map, a, chunks, s) : launch_mt<2>(kidx_map, a, chunks, s);
+  switch (a.idx_fmt) {
+    case kIdxFp8: return launch_if<kIdxFp8>(kidx_map, a, mt, chunks, s);
+    case kIdxFp4: return launch_if<kIdxFp4>(kidx_map, a, mt, chunks, s);
+    default: return launch_if<kIdxBf16>(kidx_map, a, mt, chunks, s);
+  }
 }
 
 }  // namespace msa

@@ -16,9 +16,12 @@ constexpr int kBlock = 128;    // tokens per block == tokens per page
 constexpr int kHeadDim = 128;  // head dim of q / k / v / q_idx / k_idx
 
 // ---- stage 1: block scores (indexer.cu)
+constexpr int kIdxBf16 = 0, kIdxFp8 = 1, kIdxFp4 = 2;  // index-K formats (msa_idx_dtype_t)
 struct IndexerArgs {
   const int32_t *row_off, *cache_len, *table;
   const uint16_t *q_idx;  // bf16 bits [total_q, H_kv, 128]
+  int idx_fmt;               // kIdxBf16 / kIdxFp8 / kIdxFp4
+  const void *k_idx_scale;   // fp8: f32 [pages, H_idxk, 128]; fp4: u8 [pages, H_idxk, 128, 4]
   float *scores;          // [total_q, H_kv, max_blocks]
   int32_t *dev_err;
   int batch, max_q_len, max_pages, num_pages, H_kv, H_idxk, max_blocks;

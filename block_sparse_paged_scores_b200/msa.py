@@ -17,6 +17,8 @@ LIB_PATH = os.path.join(_HERE, "libmsa.so")
 
 MSA_OK, MSA_ERR_INVALID_ARG, MSA_ERR_UNSUPPORTED, MSA_ERR_CUDA = 0, 1, 2, 3
 MSA_KV_BF16, MSA_KV_FP8_E4M3 = 0, 1
+MSA_IDX_BF16, MSA_IDX_FP8_E4M3, MSA_IDX_FP4_E2M1 = 0, 1, 2
+IDX_DTYPES = {"bf16": MSA_IDX_BF16, "fp8": MSA_IDX_FP8_E4M3, "fp4": MSA_IDX_FP4_E2M1}
 MSA_DEVERR_PAGE_ID, MSA_DEVERR_LENGTHS, MSA_DEVERR_BLOCK_ID = 1, 2, 4
 MSA_DEVERR_NUM_SELECTED, MSA_DEVERR_TIMEOUT = 8, 16
 BLOCK = 128
@@ -35,6 +37,17 @@ class RaggedPaged(ctypes.Structure):
                 ("kv_lookup_table", ctypes.c_void_p), ("batch", ctypes.c_int32),
                 ("total_q", ctypes.c_int32), ("max_q_len", ctypes.c_int32),
                 ("max_pages_per_seq", ctypes.c_int32), ("num_pages", ctypes.c_int32)]
+
+
+class IndexK(ctypes.Structure):
+    """msa_index_k_t: the index-K cache in one of the msa_idx_dtype_t formats."""
+    _fields_ = [("dtype", ctypes.c_int32), ("codes", ctypes.c_void_p),
+                ("scales", ctypes.c_void_p), ("num_heads", ctypes.c_int32)]
+
+
+def index_k(codes, scales, num_heads: int, idx_dtype: str = "bf16") -> IndexK:
+    """The msa_index_k_t view of an index-K cache (no copies)."""
+    return IndexK(IDX_DTYPES[idx_dtype], _ptr(codes), _ptr(scales), int(num_heads))
 
 
 _lib: Optional[ctypes.CDLL] = None
@@ -57,6 +70,12 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.msa_select_blocks.argtypes = [RP, P, I, I, I, I, I, P, P, P, P]
     lib.msa_index_select.restype = I
     lib.msa_index_select.argtypes = [RP, P, P, I, I, I, I, I, I, P, P, P, P, P, P]
+    IK = ctypes.POINTER(IndexK)
+    U = ctypes.c_uint32
+    lib.msa_index_scores_k.restype = I
+    lib.msa_index_scores_k.argtypes = [RP, P, IK, I, I, U, P, P, P]
+    lib.msa_index_select_k.restype = I
+    lib.msa_index_select_k.argtypes = [RP, P, IK, I, I, I, I, I, U, P, P, P, P, P, P]
     lib.msa_index_select_counters.restype = ctypes.c_size_t
     lib.msa_index_select_counters.argtypes = [RP, I]
     lib.msa_sparse_attn_paged.restype = I
@@ -77,6 +96,8 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.msa_attn_partials.restype = I
     lib.msa_attn_partials.argtypes = [RP, I, I, I, I, I, ctypes.POINTER(ctypes.c_size_t),
                                       ctypes.POINTER(ctypes.c_size_t)]
+    lib.msa_selftest_bounded_wait.restype = I
+    lib.msa_selftest_bounded_wait.argtypes = [ctypes.c_uint32, P, P, P]
     lib.msa_status_string.restype = ctypes.c_char_p
     lib.msa_status_string.argtypes = [I]
     _lib = lib
@@ -153,6 +174,23 @@ def msa_select_blocks(rp: RaggedPaged, scores, num_kv_heads: int, max_blocks: in
         local_blocks, _ptr(block_ids), _ptr(num_selected), _ptr(dev_err), _stream(stream)))
 
 
+def msa_index_scores_k(rp: RaggedPaged, q_idx, k_idx: IndexK, num_kv_heads: int,
+                       max_blocks: int, flags: int, scores, dev_err=None, stream=None):
+    _check("msa_index_scores_k", load().msa_index_scores_k(
+        ctypes.byref(rp), _ptr(q_idx), ctypes.byref(k_idx), num_kv_heads, max_blocks,
+        int(flags), _ptr(scores), _ptr(dev_err), _stream(stream)))
+
+
+def msa_index_select_k(rp: RaggedPaged, q_idx, k_idx: IndexK, num_kv_heads: int,
+                       max_blocks: int, top_k: int, init_blocks: int, local_blocks: int,
+                       flags: int, scores, block_ids, num_selected, counters, dev_err=None,
+                       stream=None):
+    _check("msa_index_select_k", load().msa_index_select_k(
+        ctypes.byref(rp), _ptr(q_idx), ctypes.byref(k_idx), num_kv_heads, max_blocks, top_k,
+        init_blocks, local_blocks, int(flags), _ptr(scores), _ptr(block_ids),
+        _ptr(num_selected), _ptr(counters), _ptr(dev_err), _stream(stream)))
+
+
 def msa_index_select_counters(rp: RaggedPaged, num_idx_k_heads: int) -> int:
     return int(load().msa_index_select_counters(ctypes.byref(rp), num_idx_k_heads))
 
@@ -206,6 +244,12 @@ def msa_sparse_attn_paged_noalloc(rp: RaggedPaged, q, k_cache, v_cache, kv_dtype
         _ptr(out), _ptr(dev_err), _stream(stream)))
 
 
+def msa_selftest_bounded_wait(limit_us: int, dev_err, result, stream=None):
+    """Diagnostic: the library's bounded pipeline wait made to run out (see include/msa.h)."""
+    _check("msa_selftest_bounded_wait", load().msa_selftest_bounded_wait(
+        int(limit_us), _ptr(dev_err), _ptr(result), _stream(stream)))
+
+
 def msa_splitk_combine(partial_o, partial_lse, num_splits: int, total_q: int, num_q_heads: int,
                        out, stream=None):
     _check("msa_splitk_combine", load().msa_splitk_combine(
@@ -244,19 +288,27 @@ class Path:
         self.kv_dtype = MSA_KV_FP8_E4M3 if prob["kv_fp8"] else MSA_KV_BF16
         nc = msa_index_select_counters(self.rp, prob["H_idxk"])
         self.counters = torch.zeros((max(nc, 1),), dtype=torch.int32, device=dev)
+        self.idx_dtype = prob.get("idx_dtype", "bf16")
+        self.kidx = index_k(prob["k_idx"], prob.get("k_idx_scale"), prob["H_idxk"],
+                            self.idx_dtype)
+        self.index_flags = 0
 
     def index_scores(self, stream=None):
         p = self.p
-        msa_index_scores(self.rp, p["q_idx"], p["k_idx"], p["H_kv"], p["H_idxk"], self.max_blocks,
-                         self.scores, self.dev_err, stream)
+        if self.idx_dtype == "bf16" and not self.index_flags:
+            msa_index_scores(self.rp, p["q_idx"], p["k_idx"], p["H_kv"], p["H_idxk"],
+                             self.max_blocks, self.scores, self.dev_err, stream)
+        else:
+            msa_index_scores_k(self.rp, p["q_idx"], self.kidx, p["H_kv"], self.max_blocks,
+                               self.index_flags, self.scores, self.dev_err, stream)
 
     def index_select(self, stream=None):
         """Stages 1 and 2 in one call (one launch on the decode / speculative routes)."""
         p = self.p
-        msa_index_select(self.rp, p["q_idx"], p["k_idx"], p["H_kv"], p["H_idxk"],
-                         self.max_blocks, p["top_k"], p["init_blocks"], p["local_blocks"],
-                         self.scores, self.block_ids, self.num_selected, self.counters,
-                         self.dev_err, stream)
+        msa_index_select_k(self.rp, p["q_idx"], self.kidx, p["H_kv"], self.max_blocks,
+                           p["top_k"], p["init_blocks"], p["local_blocks"], self.index_flags,
+                           self.scores, self.block_ids, self.num_selected, self.counters,
+                           self.dev_err, stream)
 
     def select(self, scores=None, stream=None):
         p = self.p
@@ -275,15 +327,17 @@ class Path:
                               self.num_splits, self.workspace, self.out if combine else 0,
                               self.dev_err, stream, workspace_bytes=self.workspace_bytes)
 
-    def select_attend(self, stream=None):
-        """Stages 2 and 3 in one call (msa_select_sparse_attn_paged: one launch on decode)."""
+    def select_attend(self, stream=None, combine=True):
+        """Stages 2 and 3 in one call (msa_select_sparse_attn_paged: one launch on decode).
+        With combine=False on the decode / speculative routes only the split-K partials are
+        written; ``combine()`` then merges them."""
         p = self.p
         msa_select_sparse_attn_paged(self.rp, self.scores, p["top_k"], p["init_blocks"],
                                      p["local_blocks"], p["q"], p["k"], p["v"], self.kv_dtype,
                                      p["H_q"], p["H_kv"], self.max_blocks, p["scale"],
                                      self.num_splits, self.workspace, self.block_ids,
-                                     self.num_selected, self.out, self.dev_err, stream,
-                                     workspace_bytes=self.workspace_bytes)
+                                     self.num_selected, self.out if combine else 0,
+                                     self.dev_err, stream, workspace_bytes=self.workspace_bytes)
 
     def partials(self):
         n, o_off, l_off = msa_attn_partials(self.rp, self.p["S"], self.p["H_q"], self.p["H_kv"],

@@ -19,10 +19,13 @@
  *            BlockSparseConfig, block_sparse_select, positions_of_blocks.
  *   [latent] Mojo "Struct_latent_sparse_attention_ragged_paged": the ragged / paged argument
  *            set (input_row_offsets, cache_lengths, kv_lookup_table, scale).
+ *   [trtllm] TensorRT-LLM "DeepSeekSparseAttentionConfig": indexer_k_dtype (scaled FP8 / FP4
+ *            index-K caches).
  *
  * Conventions shared by every entry point
  *   - Head dim and page size are both 128 and fixed ([msa] summary; [ferrox] "The block size
- *     is an ABI").  Index-K is always BF16; main K/V is BF16 or scale-free FP8 e4m3 ([msa]).
+ *     is an ABI").  Index-K is BF16 ([msa]) or a scaled FP8 / FP4 format ([trtllm],
+ *     msa_index_scores_k); main K/V is BF16 or scale-free FP8 e4m3 ([msa]).
  *   - Every pointer argument named "device" must point to device memory owned by the caller.
  *     The library allocates no device memory, never synchronises, and never reads device
  *     memory from the host.  Every call only enqueues work on `stream` and returns.
@@ -163,6 +166,58 @@ MSA_API msa_status_t msa_index_select(const msa_ragged_paged_t *rp, const void *
                               int32_t *dev_err, struct CUstream_st *stream);
 
 /*
+ * Scaled index-K caches ([trtllm] TensorRT-LLM "DeepSeekSparseAttentionConfig", field
+ * indexer_k_dtype: fp8 stores one E4M3 byte per element with a per-128 float32 scale, 132 B per
+ * token; fp4 packs two E2M1 codes per byte with a per-32 UE8M0 exponent, 68 B per token).
+ *
+ * Element c of token `tok` of (page, head) tile r = page * num_heads + head is
+ *   MSA_IDX_BF16      codes bf16 [r][tok][c]
+ *   MSA_IDX_FP8_E4M3  e4m3(codes u8 [r][tok][c]) * scales f32 [r][tok]
+ *   MSA_IDX_FP4_E2M1  e2m1(nibble) * 2^(scales u8 [r][tok][c / 32] - 127), the nibble being the
+ *                     low half of codes u8 [r][tok][c / 2] for even c, the high half for odd c
+ * (e4m3: the "fn" variant, bias 7, no infinities; e2m1: bias 1, values 0 .. 6; UE8M0 0xFF is
+ * NaN).  The scales tensor of one tile is 512 contiguous bytes in both scaled formats.  Scores
+ * are the max over positions of sum_c q_idx[c] * element(c), accumulated in fp32; the scaled
+ * formats multiply q_idx (converted to f16 after a power-of-two prescale that keeps every row
+ * below 2^15 in magnitude, undone exactly) with the codes (converted to f16 exactly) and apply
+ * the scales to the fp32 products.  A q_idx element of magnitude below 2^-14 (after the
+ * prescale) is rounded to f16's subnormal grid (absolute error <= 2^-25).
+ */
+typedef enum {
+    MSA_IDX_BF16 = 0,
+    MSA_IDX_FP8_E4M3 = 1, /* e4m3 codes + one f32 scale per token */
+    MSA_IDX_FP4_E2M1 = 2  /* e2m1 code pairs + one UE8M0 exponent per 32 elements */
+} msa_idx_dtype_t;
+
+typedef struct {
+    msa_idx_dtype_t dtype;
+    const void *codes;  /* device, 16-byte aligned: bf16 [num_pages, num_heads, 128, 128] |
+                           u8 [num_pages, num_heads, 128, 128] | u8 [num_pages, num_heads, 128,
+                           64] */
+    const void *scales; /* device, 16-byte aligned: NULL (bf16) | f32 [num_pages, num_heads,
+                           128] | u8 [num_pages, num_heads, 128, 4] */
+    int32_t num_heads;  /* 1 or num_kv_heads (as num_idx_k_heads) */
+} msa_index_k_t;
+
+/*
+ * msa_index_scores_k / msa_index_select_k — msa_index_scores / msa_index_select over an index-K
+ * cache in any msa_idx_dtype_t (the BF16 entry points are these with MSA_IDX_BF16; their
+ * results are bit-identical).  `flags` must be 0 except as stated below.  Scaled formats run
+ * the warp-MMA indexer on every route (the prefill route's tcgen05 indexer takes BF16 only).
+ */
+MSA_API msa_status_t msa_index_scores_k(const msa_ragged_paged_t *rp, const void *q_idx,
+                                        const msa_index_k_t *k_idx, int32_t num_kv_heads,
+                                        int32_t max_blocks, uint32_t flags, float *scores,
+                                        int32_t *dev_err, struct CUstream_st *stream);
+MSA_API msa_status_t msa_index_select_k(const msa_ragged_paged_t *rp, const void *q_idx,
+                                        const msa_index_k_t *k_idx, int32_t num_kv_heads,
+                                        int32_t max_blocks, int32_t top_k, int32_t init_blocks,
+                                        int32_t local_blocks, uint32_t flags, float *scores,
+                                        int32_t *block_ids, int32_t *num_selected,
+                                        int32_t *counters, int32_t *dev_err,
+                                        struct CUstream_st *stream);
+
+/*
  * msa_sparse_attn_paged — stage 3 ([ferrox] positions_of_blocks: the selected blocks'
  * positions, ascending and causally clipped; "an ordinary masked pass over the positions
  * those blocks cover"; [msa] "Three attention routes").
@@ -240,11 +295,15 @@ MSA_API msa_status_t msa_select_sparse_attn_paged(
  * that scratch in a device array that is part of the library itself: MSA_NOALLOC_SCRATCH_BYTES
  * on every GPU the library is loaded on, held until the process exits.  It allocates nothing.
  *
+ *   - `out` is required (MSA_ERR_INVALID_ARG when NULL): the split-K partials stay in the
+ *     library's own array, which the caller cannot reach, so the combine always runs.
  *   - A shape whose msa_attn_workspace_bytes exceeds MSA_NOALLOC_SCRATCH_BYTES is rejected
  *     with MSA_ERR_UNSUPPORTED before anything is enqueued (use msa_sparse_attn_paged with a
  *     workspace of your own for it).
- *   - The first call on a device looks the array's device address up (once per device, with
- *     that device current); make that first call before any stream capture.
+ *   - The first call on a device looks the array's device address up (with that device
+ *     current) and keeps it for that device's current context; a call in a new context (after
+ *     cudaDeviceReset, for instance) looks it up again.  Make the first call on each device,
+ *     and the first after a reset, before any stream capture.
  *   - Every call on a device shares the one array and it keeps the last call's contents
  *     (nothing in it needs to start at zero).  Calls whose work overlaps on the GPU race on
  *     it: run them on one stream, or order them.
@@ -274,6 +333,25 @@ MSA_API msa_status_t msa_sparse_attn_paged_noalloc(
 MSA_API msa_status_t msa_splitk_combine(const float *partial_o, const float *partial_lse,
                                 int32_t num_splits, int32_t total_q, int32_t num_q_heads,
                                 void *out, struct CUstream_st *stream);
+
+/*
+ * msa_selftest_bounded_wait — a diagnostic (the pages have no counterpart): runs the bounded
+ * pipeline wait that every pipelined kernel of this library uses on barriers that nothing ever
+ * completes, so that its give-up path can be checked on a GPU without hanging it.
+ *
+ * One CTA: a first waiter gives up after `limit_us` microseconds, ORs MSA_DEVERR_TIMEOUT into
+ * *dev_err and raises the CTA's abort flag; a second waiter (limit 4 x limit_us) leaves as soon
+ * as it sees that flag; a last wait on a completed phase returns at once.  The kernel returns
+ * normally and the context stays usable.
+ *
+ *   limit_us  1 .. 1000000
+ *   dev_err   device int32 (nullable), as for the other entry points
+ *   result    device uint32 [5], 4-byte aligned (output): [0] first waiter (1 = the phase
+ *             completed, 2 = gave up), [1] its wait in microseconds, [2] / [3] the same for the
+ *             second waiter, [4] the wait on the completed phase (1 = returned true)
+ */
+MSA_API msa_status_t msa_selftest_bounded_wait(uint32_t limit_us, int32_t *dev_err,
+                                               uint32_t *result, struct CUstream_st *stream);
 
 /* Host-only helpers (no device work, no CUDA call). */
 

@@ -25,10 +25,29 @@ REL_GAP = 1e-3
 ATTN_TOL = {False: (2e-2, 2e-3), True: (6e-2, 6e-3)}
 
 
+def dequantized_index_k(prob) -> torch.Tensor:
+    """The index-K cache of ``prob`` as fp32 values [num_pages, H_idxk, 128, 128], decoded with
+    library routines (torch for bf16, e4m3 and e8m0, ml_dtypes for e2m1)."""
+    dt = prob.get("idx_dtype", "bf16")
+    codes = prob["k_idx"].cpu()
+    if dt == "bf16":
+        return codes.float()
+    sc = prob["k_idx_scale"].cpu()
+    if dt == "fp8":
+        return codes.view(torch.float8_e4m3fn).float() * sc[..., None]
+    import ml_dtypes
+    c = codes.numpy()
+    lo = (c & 15).view(ml_dtypes.float4_e2m1fn).astype(np.float32)
+    hi = (c >> 4).view(ml_dtypes.float4_e2m1fn).astype(np.float32)
+    v = torch.from_numpy(np.stack([lo, hi], axis=-1).reshape(c.shape[:3] + (128,)))
+    ex = sc.view(torch.float8_e8m0fnu).float()
+    return v * ex.repeat_interleave(32, dim=-1)
+
+
 def block_key_norms(prob) -> np.ndarray:
     """max over each block's positions of ||k_idx[pos]||: [batch, H_idxk, max_blocks]
     (positions >= L_b excluded)."""
-    kn = torch.nan_to_num(prob["k_idx"].float(), nan=0.0).norm(dim=-1)   # [pool, H_idxk, 128]
+    kn = torch.nan_to_num(dequantized_index_k(prob), nan=0.0).norm(dim=-1)  # [pool, H, 128]
     table = prob["table"].long().clamp(min=0)
     out = kn[table].amax(dim=-1)                                          # [batch, max_pages, H]
     return out.permute(0, 2, 1).cpu().numpy()
@@ -157,3 +176,100 @@ def fp32_exact(x):
     """fp64 copy of the fp32 rounding of x (the values a GPU select sees)."""
     return np.asarray(x, dtype=np.float32).astype(np.float64)
 
+
+
+# ------------------------------------------------------------------ planted large logits
+LOG2E = 1.4426950408889634
+
+
+def plant_large_keys(prob, every=4, phase=3, factor=16.0):
+    """A copy of ``prob`` whose main K rows of every block j with j % every == phase (in each
+    sequence's own block order) are multiplied by ``factor`` (a power of two: exact in bf16,
+    and in e4m3 for N(0,1) values).  Those blocks then hold logits about ``factor`` times
+    larger than the others, so that a row's running maximum jumps far up at a block that
+    comes after blocks it has already accumulated."""
+    p = dict(prob)
+    k = prob["k"].clone()
+    table = prob["table"].cpu()
+    pages = []
+    for b in range(prob["batch"]):
+        nb = int((table[b] >= 0).sum())
+        pages += [int(table[b, j]) for j in range(phase, nb, every)]
+    idx = torch.tensor(sorted(set(pages)), dtype=torch.long, device=k.device)
+    if idx.numel():
+        k[idx] = (k[idx].float() * factor).to(k.dtype)
+    p["k"] = k
+    return p
+
+
+def block_max_logits(prob, ids, cnt):
+    """[total_q, H_q, S] largest raw logit q . k over the causally visible positions of each
+    selected block (-inf for padding slots), computed densely per sequence in fp32 on the
+    problem's device (a check of how the inputs were built, not a reference)."""
+    dev = prob["q"].device
+    ro = prob["row_off"].cpu().tolist()
+    cl = prob["cache_len"].cpu().tolist()
+    table = prob["table"].cpu()
+    H_q, H_kv = prob["H_q"], prob["H_kv"]
+    G = H_q // H_kv
+    ids = np.asarray(ids)
+    cnt = np.asarray(cnt)
+    S = ids.shape[2]
+    out = np.full((prob["total_q"], H_q, S), -np.inf)
+    for b in range(prob["batch"]):
+        n = ro[b + 1] - ro[b]
+        if n == 0:
+            continue
+        L = cl[b] + n
+        nb = (L + BLOCK - 1) // BLOCK
+        pg = table[b, :nb].long().to(dev)
+        kb = prob["k"][pg].float().nan_to_num(0.0)            # [nb, H_kv, 128, 128]
+        kb = kb.permute(1, 0, 2, 3).reshape(H_kv, nb * BLOCK, -1)
+        q = prob["q"][ro[b]:ro[b + 1]].float().reshape(n, H_kv, G, -1)
+        lg = torch.einsum("tgjd,gpd->tgjp", q, kb)             # [n, H_kv, G, nb*128]
+        pos = torch.arange(nb * BLOCK, device=dev)
+        p_t = cl[b] + torch.arange(n, device=dev)
+        lg = lg.masked_fill(pos[None, None, None, :] > p_t[:, None, None, None], -float("inf"))
+        bm = lg.reshape(n, H_kv, G, nb, BLOCK).amax(-1).reshape(n, H_q, nb).cpu().numpy()
+        for i in range(n):
+            t = ro[b] + i
+            for h in range(H_q):
+                g = h // G
+                sel = ids[t, g, :cnt[t, g]]
+                out[t, h, :len(sel)] = bm[i, h, sel]
+    return out
+
+
+def lazy_rescale_events(prob, ids, cnt, bmax, tile_tokens, groups, threshold_log2=8.0):
+    """How often a row's running maximum moves up by more than 2^threshold_log2 (exp2 domain:
+    scale * log2(e) * logit) at a block after one the row has already accumulated, with the
+    blocks of each query tile's union of selections dealt out to ``groups`` alternating
+    groups (each keeping its own running maximum, moved only past the threshold).  With
+    tile_tokens = 1 and groups = 1 that is the row's own list of blocks."""
+    ro = prob["row_off"].cpu().tolist()
+    H_q, H_kv = prob["H_q"], prob["H_kv"]
+    G = H_q // H_kv
+    sl2 = prob["scale"] * LOG2E
+    ids = np.asarray(ids)
+    cnt = np.asarray(cnt)
+    events = 0
+    for b in range(prob["batch"]):
+        for t0 in range(ro[b], ro[b + 1], tile_tokens):
+            t1 = min(t0 + tile_tokens, ro[b + 1])
+            for g in range(H_kv):
+                union = sorted(set(int(j) for t in range(t0, t1)
+                                   for j in ids[t, g, :cnt[t, g]]))
+                for t in range(t0, t1):
+                    own = {int(j): s for s, j in enumerate(ids[t, g, :cnt[t, g]])}
+                    for h in range(g * G, (g + 1) * G):
+                        m = [-np.inf] * groups
+                        for i, j in enumerate(union):
+                            if j not in own:
+                                continue
+                            mb = bmax[t, h, own[j]] * sl2
+                            w = i % groups
+                            if mb > m[w] + threshold_log2:
+                                if np.isfinite(m[w]):
+                                    events += 1
+                                m[w] = mb
+    return events

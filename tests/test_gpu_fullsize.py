@@ -14,6 +14,7 @@ import numpy as np
 import pytest
 import torch
 
+import oracle
 from block_sparse_paged_scores_b200 import msa
 from block_sparse_paged_scores_b200 import workload as wl
 from parity_tools import (check_attention, check_scores, check_selection, head_rows_mask,
@@ -119,3 +120,9 @@ def test_full_size_workload(name):
         same = check_selection(ids[t:t + 1], cnt[t:t + 1], oids, ocnt, sc, sub)
         mask = head_rows_mask(same, G)
         check_attention(out[t:t + 1].float().cpu(), oout, prob["kv_fp8"], rows_mask=mask)
+        # every head of the row, near-ties included, against the oracle's attention over the
+        # GPU's own selection
+        gout = oracle.attention(sub["row_off"], sub["cache_len"], sub["table"], sub["q"],
+                                sub["k"], sub["v"], sub["kv_fp8"], ids[t:t + 1], cnt[t:t + 1],
+                                sub["scale"])
+        check_attention(out[t:t + 1].float().cpu(), gout, prob["kv_fp8"])

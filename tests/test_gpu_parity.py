@@ -11,8 +11,9 @@ import torch
 import oracle
 from block_sparse_paged_scores_b200 import msa
 from block_sparse_paged_scores_b200 import workload as wl
-from parity_tools import (check_attention, check_scores, check_selection, fp32_exact,
-                          head_rows_mask, oracle_forward)
+from parity_tools import (block_max_logits, check_attention, check_scores, check_selection,
+                          fp32_exact, head_rows_mask, lazy_rescale_events, oracle_forward,
+                          plant_large_keys)
 
 pytestmark = pytest.mark.gpu
 
@@ -106,11 +107,16 @@ def test_whole_path_matches_oracle(name):
     path.run()
     torch.cuda.synchronize()
     assert int(path.dev_err.item()) == 0
-    same = check_selection(path.block_ids.cpu().numpy(), path.num_selected.cpu().numpy(), ids,
-                           cnt, sc, p)
+    g_ids, g_cnt = path.block_ids.cpu().numpy(), path.num_selected.cpu().numpy()
+    same = check_selection(g_ids, g_cnt, ids, cnt, sc, p)
     assert same.mean() > 0.9
     mask = head_rows_mask(same, p["H_q"] // p["H_kv"])
     check_attention(path.out.float().cpu(), out, p["kv_fp8"], rows_mask=mask)
+    # every row, near-ties included, against the oracle's attention over the GPU's selection
+    # (a valid top-k under the oracle's scores, checked above)
+    out_g = oracle.attention(p["row_off"], p["cache_len"], p["table"], p["q"], p["k"], p["v"],
+                             p["kv_fp8"], g_ids, g_cnt, p["scale"])
+    check_attention(path.out.float().cpu(), out_g, p["kv_fp8"])
 
 
 @pytest.mark.parametrize("name,splits", [("bf16_decode", n) for n in (1, 2, 3, 7, 19, 148, 700)]
@@ -348,3 +354,155 @@ def test_indexer_for_many_short_sequences(kw):
                                     p["init_blocks"], p["local_blocks"])
     assert np.array_equal(path.num_selected.cpu().numpy(), cnt)
     assert np.array_equal(path.block_ids.cpu().numpy(), ids)
+
+
+# ------------------------------------------------------------------ large late logits
+# Every fourth block of each sequence has its keys scaled by 16 (exact), so that a row's
+# running maximum jumps up by far more than the prefill kernel's lazy-rescale threshold
+# (2^8 in the exp2 domain, about 63 in raw q . k at scale 1/sqrt(128)) at a block that comes
+# after blocks it has already accumulated: the rescale of the accumulated output must then
+# run, with a factor strictly between 0 and 1.  The opposite case (the largest keys first,
+# in block 0, which every row selects) is the "early" plant.
+PLANTED = {
+    "prefill": ("prefill", 16, 2),                   # tcgen05 route: 16-token tiles, 2 groups
+    "prefill_gqa4": ("prefill_gqa4", 32, 2),         # tcgen05, 32-token tiles
+    "prefill_fp8": ("prefill_fp8", 1, 1),            # FP8 KV prefill (tile kernel)
+    "bf16_decode": ("bf16_decode", 1, 1),
+    "decode_gqa16": ("decode_gqa16", 1, 1),
+    "spec_decode": ("spec_decode", 1, 1),
+    "fp8_decode": ("fp8_decode", 1, 1),
+    "fp8_spec": ("fp8_spec", 1, 1),
+}
+
+
+@pytest.mark.parametrize("plant", ["late", "early"])
+@pytest.mark.parametrize("name", sorted(PLANTED))
+def test_large_logits_after_accumulated_blocks(name, plant):
+    base, tile_tokens, groups = PLANTED[name]
+    p0 = _problem(base)
+    p = plant_large_keys(p0, every=4, phase=3) if plant == "late" else \
+        plant_large_keys(p0, every=1 << 30, phase=0)
+    sc, ids, cnt, out = oracle_forward(p)
+    # the inputs do what they are meant to: the running maximum moves up past the threshold
+    # after accumulated blocks (late), or never needs to (early: block 0 holds the largest)
+    bmax = block_max_logits(_gpu(p), ids, cnt)
+    ev = lazy_rescale_events(p, ids, cnt, bmax, tile_tokens, groups)
+    if plant == "late":
+        assert ev >= 20, ev
+    # the oracle's selection, then the whole path
+    path = msa.Path(_gpu(p))
+    path.attend(block_ids=torch.from_numpy(ids).cuda(), num_selected=torch.from_numpy(cnt).cuda())
+    torch.cuda.synchronize()
+    assert int(path.dev_err.item()) == 0
+    check_attention(path.out.float().cpu(), out, p["kv_fp8"])
+    full = msa.Path(_gpu(p))
+    full.run()
+    torch.cuda.synchronize()
+    assert int(full.dev_err.item()) == 0
+    g_ids, g_cnt = full.block_ids.cpu().numpy(), full.num_selected.cpu().numpy()
+    check_selection(g_ids, g_cnt, ids, cnt, sc, p)
+    out_g = oracle.attention(p["row_off"], p["cache_len"], p["table"], p["q"], p["k"], p["v"],
+                             p["kv_fp8"], g_ids, g_cnt, p["scale"])
+    check_attention(full.out.float().cpu(), out_g, p["kv_fp8"])
+
+
+# ------------------------------------------------------------------ scaled index-K caches
+SCALED = {
+    "fp8idx_decode": (W["bf16_decode"], dict(batch=4, kv_len=(2000, 9000), idx_dtype="fp8")),
+    "fp4idx_decode": (W["bf16_decode"], dict(batch=4, kv_len=(2000, 9000), idx_dtype="fp4")),
+    "fp8idx_spec": (W["spec_decode"], dict(batch=6, kv_len=(1500, 5000), idx_dtype="fp8")),
+    "fp4idx_spec_ragged": (W["spec_decode"], dict(batch=6, q_len=(2, 8), kv_len=(1000, 4000),
+                                                   idx_dtype="fp4")),
+    "fp8idx_per_head": (W["bf16_decode"], dict(batch=3, kv_len=(1000, 5000), H_idxk=8,
+                                               idx_dtype="fp8")),
+    "fp4idx_per_head": (W["bf16_decode"], dict(batch=3, kv_len=(1000, 5000), H_idxk=8,
+                                               idx_dtype="fp4")),
+    "fp4idx_short": (W["bf16_decode"], dict(batch=6, kv_len=(1, 300), idx_dtype="fp4")),
+    "fp8idx_fp8kv": (W["fp8_long_decode"], dict(batch=3, kv_len=(3000, 12000),
+                                                idx_dtype="fp8")),
+    "fp4idx_fp8kv": (W["fp8_long_decode"], dict(batch=3, kv_len=(3000, 12000),
+                                                idx_dtype="fp4")),
+    "fp8idx_prefill": (W["ragged_prefill"], dict(batch=2, q_len=(40, 200), prior_len=(0, 1500),
+                                                 idx_dtype="fp8")),
+    "fp4idx_prefill": (W["ragged_prefill"], dict(batch=2, q_len=(40, 200), prior_len=(0, 1500),
+                                                 idx_dtype="fp4")),
+}
+
+
+def _scaled_problem(name):
+    spec, kw = SCALED[name]
+    p = wl.generate(spec.scaled(**kw), seed=2000 + sorted(SCALED).index(name))
+    if name.endswith("_decode"):
+        # a few rows far beyond f16's range (exact powers of two in bf16): the kernel's
+        # per-row prescale must keep them finite
+        p["q_idx"] = p["q_idx"].clone()
+        p["q_idx"][1] = p["q_idx"][1] * 2.0 ** 17
+        p["q_idx"][2, :2] = p["q_idx"][2, :2] * 2.0 ** 40
+    return p
+
+
+_scaled_cache = {}
+
+
+def _scaled_oracle(name):
+    if name not in _scaled_cache:
+        p = _scaled_problem(name)
+        _scaled_cache[name] = (p, oracle_forward(p))
+    return _scaled_cache[name]
+
+
+@pytest.mark.parametrize("name", sorted(SCALED))
+def test_scaled_index_k_scores_match_oracle(name):
+    p, (sc, _, _, _) = _scaled_oracle(name)
+    path = msa.Path(_gpu(p))
+    path.index_scores()
+    torch.cuda.synchronize()
+    assert int(path.dev_err.item()) == 0
+    check_scores(path.scores.cpu().numpy(), sc, p, p["max_blocks"])
+
+
+@pytest.mark.parametrize("name", sorted(SCALED))
+def test_scaled_index_k_fused_selection_is_bit_exact(name):
+    """msa_index_select_k: the same scores as msa_index_scores_k, and the oracle's selection
+    on those scores, bit for bit."""
+    p = _gpu(_scaled_problem(name))
+    one, two = msa.Path(p), msa.Path(p)
+    for _ in range(2):
+        one.index_select()
+    two.index_scores()
+    torch.cuda.synchronize()
+    assert int(one.dev_err.item()) == 0 and int(two.dev_err.item()) == 0
+    assert torch.equal(one.scores, two.scores)
+    sc = one.scores.cpu().numpy().astype(np.float64)
+    ids, cnt = oracle.select_blocks(p["row_off"].cpu(), p["cache_len"].cpu(), sc, p["top_k"],
+                                    p["init_blocks"], p["local_blocks"])
+    assert np.array_equal(one.num_selected.cpu().numpy(), cnt)
+    assert np.array_equal(one.block_ids.cpu().numpy(), ids)
+    assert int(one.counters.abs().sum().item()) == 0
+
+
+@pytest.mark.parametrize("name", sorted(SCALED))
+def test_scaled_index_k_whole_path_matches_oracle(name):
+    p, (sc, ids, cnt, out) = _scaled_oracle(name)
+    path = msa.Path(_gpu(p))
+    path.run()
+    torch.cuda.synchronize()
+    assert int(path.dev_err.item()) == 0
+    g_ids, g_cnt = path.block_ids.cpu().numpy(), path.num_selected.cpu().numpy()
+    same = check_selection(g_ids, g_cnt, ids, cnt, sc, p)
+    assert same.mean() > 0.9
+    out_g = oracle.attention(p["row_off"], p["cache_len"], p["table"], p["q"], p["k"], p["v"],
+                             p["kv_fp8"], g_ids, g_cnt, p["scale"])
+    check_attention(path.out.float().cpu(), out_g, p["kv_fp8"])
+
+
+@pytest.mark.parametrize("name", ["bf16_decode", "spec_ragged_q", "bf16_decode_idxk_per_head",
+                                  "prefill"])
+def test_bf16_descriptor_entry_points_equal_the_bf16_ones(name):
+    p = _gpu(_problem(name))
+    a, b = msa.Path(p), msa.Path(p)
+    a.index_scores()
+    msa.msa_index_scores_k(b.rp, p["q_idx"], b.kidx, p["H_kv"], b.max_blocks, 0, b.scores,
+                           b.dev_err)
+    torch.cuda.synchronize()
+    assert torch.equal(a.scores, b.scores)

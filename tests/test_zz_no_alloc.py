@@ -3,17 +3,18 @@
 It exists for callers that cannot hand the library a workspace (a runtime whose device memory
 plan is fixed before serving starts, a plugin interface that passes only inputs and outputs):
 its scratch is a device array inside the library.  These tests call it through the C ABI and
-check it against msa_sparse_attn_paged with a caller-provided workspace, twice in a row (the
-array keeps the previous call's contents), and check that a shape needing more scratch than
-the array holds is refused before anything runs.  This file is collected last on purpose.
+check it against msa_sparse_attn_paged with a caller-provided workspace: the kernels and the
+split-K partitions are the same, so the outputs must be bit-identical, on two calls in a row
+(the array keeps the previous call's contents) and after a call of another shape with many
+partitions (its partials are still in the array and must never be read).  They also check
+that a shape needing more scratch than the array holds, and a NULL output, are refused before
+anything runs.  This file is collected last on purpose.
 """
-import numpy as np
 import pytest
 import torch
 
 from block_sparse_paged_scores_b200 import msa
 from block_sparse_paged_scores_b200 import workload as wl
-from parity_tools import check_attention
 
 pytestmark = pytest.mark.gpu
 
@@ -25,27 +26,58 @@ CASES = {
 }
 
 
-def _noalloc(path, out):
+def _noalloc(path, out, num_splits=None):
     p = path.p
     msa.msa_sparse_attn_paged_noalloc(path.rp, p["q"], p["k"], p["v"], path.kv_dtype,
                                       path.block_ids, path.num_selected, p["S"], p["H_q"],
-                                      p["H_kv"], path.max_blocks, p["scale"], path.num_splits,
+                                      p["H_kv"], path.max_blocks, p["scale"],
+                                      path.num_splits if num_splits is None else num_splits,
                                       out, path.dev_err)
+
+
+def _reference(prob, num_splits=0):
+    """Scores, selection and the workspace call's output for ``prob``."""
+    path = msa.Path(prob, num_splits=num_splits)
+    path.run()
+    torch.cuda.synchronize()
+    assert int(path.dev_err.item()) == 0
+    return path, path.out.clone()
 
 
 @pytest.mark.parametrize("name", sorted(CASES))
 def test_noalloc_matches_workspace_call_twice_in_a_row(name):
     prob = wl.generate(CASES[name], seed=4242, device="cuda")
-    path = msa.Path(prob)
-    path.run()                                     # scores, selection, reference output
-    torch.cuda.synchronize()
-    ref = path.out.clone()
+    path, ref = _reference(prob)
     for _ in range(2):
         out = torch.full_like(ref, float("nan"))
         _noalloc(path, out)
         torch.cuda.synchronize()
         assert int(path.dev_err.item()) == 0
-        check_attention(out.float().cpu(), ref.double().cpu().numpy(), prob["kv_fp8"])
+        assert torch.equal(out, ref)
+
+
+def test_noalloc_leftovers_of_a_larger_call_are_never_read():
+    """Many split-K partitions on one shape, then a single partition (the attention kernel
+    writes the output itself) and a few partitions on another: each equal to the workspace
+    call with the same partition count."""
+    first = wl.generate(CASES["bf16_decode"], seed=11, device="cuda")
+    second = wl.generate(wl.BF16_DECODE.scaled(batch=3, kv_len=(300, 2500)), seed=12,
+                         device="cuda")
+    for prob, splits in ((first, 61), (second, 1), (second, 3), (first, 2)):
+        path, ref = _reference(prob, num_splits=splits)
+        out = torch.full_like(ref, float("nan"))
+        _noalloc(path, out, num_splits=splits)
+        torch.cuda.synchronize()
+        assert int(path.dev_err.item()) == 0
+        assert torch.equal(out, ref), splits
+
+
+def test_noalloc_refuses_a_null_output():
+    prob = wl.generate(CASES["bf16_decode"], seed=7, device="cuda")
+    path, _ = _reference(prob)
+    with pytest.raises(msa.MSAError) as ei:
+        _noalloc(path, None)
+    assert ei.value.status == msa.MSA_ERR_INVALID_ARG
 
 
 def test_noalloc_refuses_a_shape_beyond_its_scratch():
