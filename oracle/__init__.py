@@ -59,6 +59,8 @@ def _load():
         lib.orc_index_scores.argtypes = [I, P, P, P, I, P, I, P, P, I, I, I, P]
         lib.orc_select_blocks.restype = None
         lib.orc_select_blocks.argtypes = [I, P, P, I, I, P, I, I, I, I, P, P]
+        lib.orc_select_blocks_shared.restype = None
+        lib.orc_select_blocks_shared.argtypes = [I, P, P, I, I, P, I, I, I, I, P, P]
         lib.orc_attention.restype = None
         lib.orc_attention.argtypes = [I, P, P, P, I, P, P, P, I, I, I, P, P, I,
                                       ctypes.c_double, P]
@@ -168,6 +170,25 @@ def select_blocks(row_off, cache_len, scores, top_k, init_blocks, local_blocks):
     return ids, counts
 
 
+def select_blocks_shared(row_off, cache_len, scores, top_k, init_blocks, local_blocks):
+    """The selection with the indexer top-k shared across a sequence's new tokens: the top-k
+    of the first new token's candidates, plus each token's own forced blocks, ascending.  Only
+    the first new token's row of ``scores`` is read."""
+    lib = _load()
+    row_off, p_off = _c(_ints(row_off), np.int32)
+    cache_len, p_cl = _c(_ints(cache_len), np.int32)
+    sc, p_sc = _c(np.asarray(scores, dtype=np.float64), np.float64)
+    total_q, H_kv, max_blocks = sc.shape
+    S = init_blocks + local_blocks + top_k
+    ids = np.empty((total_q, H_kv, S), dtype=np.int32)
+    counts = np.empty((total_q, H_kv), dtype=np.int32)
+    lib.orc_select_blocks_shared(row_off.shape[0] - 1, p_off, p_cl, H_kv, max_blocks, p_sc,
+                                 top_k, init_blocks, local_blocks, S,
+                                 ids.ctypes.data_as(ctypes.c_void_p),
+                                 counts.ctypes.data_as(ctypes.c_void_p))
+    return ids, counts
+
+
 def attention(row_off, cache_len, table, q, k_cache, v_cache, kv_fp8, ids, counts, scale):
     """Attention output [total_q, H_q, 128] in fp64 over the selected, causally clipped
     positions.  q bf16 [total_q, H_q, 128]; caches bf16 or e4m3 [num_pages, H_kv, 128, 128]."""
@@ -194,14 +215,15 @@ def attention(row_off, cache_len, table, q, k_cache, v_cache, kv_fp8, ids, count
     return out
 
 
-def forward(inp, top_k, init_blocks, local_blocks, scale, max_blocks):
+def forward(inp, top_k, init_blocks, local_blocks, scale, max_blocks, share=False):
     """The whole path: scores -> selection -> attention.  ``inp`` is a mapping with the
-    tensors named as in the C-ABI (row_off, cache_len, table, q, q_idx, k_idx, k, v, kv_fp8)."""
+    tensors named as in the C-ABI (row_off, cache_len, table, q, q_idx, k_idx, k, v, kv_fp8).
+    ``share``: the indexer top-k shared across each sequence's new tokens."""
     sc = index_scores(inp["row_off"], inp["cache_len"], inp["table"], inp["q_idx"],
                       inp["k_idx"], max_blocks, inp.get("k_idx_scale"),
                       inp.get("idx_dtype", "bf16"))
-    ids, counts = select_blocks(inp["row_off"], inp["cache_len"], sc, top_k, init_blocks,
-                                local_blocks)
+    sel = select_blocks_shared if share else select_blocks
+    ids, counts = sel(inp["row_off"], inp["cache_len"], sc, top_k, init_blocks, local_blocks)
     out = attention(inp["row_off"], inp["cache_len"], inp["table"], inp["q"], inp["k"],
                     inp["v"], inp["kv_fp8"], ids, counts, scale)
     return sc, ids, counts, out

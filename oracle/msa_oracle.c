@@ -244,6 +244,66 @@ void orc_select_blocks(int batch, const int32_t *row_off, const int32_t *cache_l
 }
 
 /* ---------------------------------------------------------------------------------------
+ * Stage 2 with the indexer top-k shared across draft tokens: TensorRT-LLM
+ * "DeepSeekSparseAttentionConfig", field index_share_for_mtp_iteration ("reuse the indexer
+ * Top-K across MTP draft steps instead of recomputing it each step").  Reading: the top-k is
+ * computed once per (sequence, KV head), for the sequence's first new token, over that
+ * token's candidates (its visible blocks minus its own forced blocks), from that token's
+ * scores; every new token of the sequence then selects its own forced blocks ([ferrox] "Four
+ * rules") together with that shared top-k, ascending.  The shared blocks lie below the first
+ * token's position, so every later token of the sequence can see them.
+ * ------------------------------------------------------------------------------------- */
+void orc_select_blocks_shared(int batch, const int32_t *row_off, const int32_t *cache_len,
+                              int H_kv, int max_blocks, const double *scores, int top_k,
+                              int init_blocks, int local_blocks, int S, int32_t *ids,
+                              int32_t *counts)
+{
+    for (int b = 0; b < batch; ++b) {
+        int q_len = row_off[b + 1] - row_off[b];
+        if (q_len <= 0)
+            continue;
+        int t0 = row_off[b];
+        int nb0 = visible_blocks(query_position(cache_len, b, 0));
+        int nb_last = visible_blocks(query_position(cache_len, b, q_len - 1));
+        for (int g = 0; g < H_kv; ++g) {
+            /* the shared top-k: the first token's candidates by its own scores */
+            const double *srow = scores + ((size_t)t0 * H_kv + g) * max_blocks;
+            char *shared = (char *)calloc((size_t)nb_last, 1);
+            orc_cand *cand = (orc_cand *)malloc(sizeof(orc_cand) * (size_t)nb0);
+            int nc = 0;
+            for (int j = 0; j < nb0; ++j) {
+                int forced0 = (j < init_blocks) || (j >= nb0 - local_blocks);
+                if (!forced0) {
+                    cand[nc].score = srow[j];
+                    cand[nc].id = j;
+                    ++nc;
+                }
+            }
+            qsort(cand, (size_t)nc, sizeof(orc_cand), cand_order);
+            for (int r = 0; r < nc && r < top_k; ++r)
+                shared[cand[r].id] = 1;
+            /* every token: its own forced blocks and the shared top-k */
+            for (int i = 0; i < q_len; ++i) {
+                int t = row_off[b] + i;
+                int nb = visible_blocks(query_position(cache_len, b, i));
+                int32_t *out = ids + ((size_t)t * H_kv + g) * S;
+                int n = 0;
+                for (int j = 0; j < nb; ++j) {
+                    int forced = (j < init_blocks) || (j >= nb - local_blocks);
+                    if (forced || shared[j])
+                        out[n++] = j;
+                }
+                counts[(size_t)t * H_kv + g] = n;
+                for (int r = n; r < S; ++r)
+                    out[r] = -1;
+            }
+            free(shared);
+            free(cand);
+        }
+    }
+}
+
+/* ---------------------------------------------------------------------------------------
  * Stage 3: attention over the positions the selected blocks cover, ascending and causally
  * clipped ([ferrox] positions_of_blocks), with softmax(scale * q . k) in fp64 ("an
  * ordinary masked pass over the positions those blocks cover").

@@ -227,6 +227,79 @@ def _brute_force_select(scores, nb, init, local, top_k):
     return sorted(forced | winners[0])
 
 
+def test_shared_select_hand_worked_cases():
+    cases = json.load(open(os.path.join(GOLDEN, "select_shared_worked_examples.json")))["cases"]
+    for c in cases:
+        n = c["q_len"]
+        mb = max(len(r) for r in c["scores"])
+        sc = np.full((n, 1, mb), -np.inf)
+        for i, r in enumerate(c["scores"]):
+            sc[i, 0, :len(r)] = r
+        ids, cnt = oracle.select_blocks_shared(np.array([0, n]), np.array([c["cache_len"]]), sc,
+                                               c["top_k"], c["init"], c["local"])
+        got = [ids[i, 0, :cnt[i, 0]].tolist() for i in range(n)]
+        assert got == c["expected"], c["name"]
+
+
+@pytest.mark.parametrize("seed", range(30))
+def test_shared_select_matches_exhaustive_search(seed):
+    """The shared part is the exhaustive top-k of the first token's candidates; each token adds
+    its own forced blocks; rows after the first are never read."""
+    rng = np.random.default_rng(100 + seed)
+    q_len = int(rng.integers(1, 9))
+    nb0 = int(rng.integers(1, 11))
+    cache_len = (nb0 - 1) * BLOCK + int(rng.integers(0, BLOCK))
+    init, local, top_k = (int(x) for x in rng.integers(0, 3, size=3))
+    top_k += int(rng.integers(0, 3))
+    if init + local + top_k == 0:
+        top_k = 1
+    nb_last = (cache_len + q_len - 1) // BLOCK + 1
+    sc = rng.integers(-3, 4, size=(q_len, 1, nb_last)).astype(np.float64)
+    ids, cnt = oracle.select_blocks_shared(np.array([0, q_len]), np.array([cache_len]), sc,
+                                           top_k, init, local)
+    forced0 = {j for j in range(nb0) if j < init or j >= nb0 - local}
+    shared = set(_brute_force_select(sc[0, 0], nb0, init, local, top_k)) - forced0
+    for i in range(q_len):
+        nb = (cache_len + i) // BLOCK + 1
+        forced = {j for j in range(nb) if j < init or j >= nb - local}
+        assert ids[i, 0, :cnt[i, 0]].tolist() == sorted(forced | shared)
+        assert all(x == -1 for x in ids[i, 0, cnt[i, 0]:])
+    # rows after the first do not matter
+    sc2 = sc.copy()
+    sc2[1:] = rng.normal(size=sc2[1:].shape)
+    ids2, cnt2 = oracle.select_blocks_shared(np.array([0, q_len]), np.array([cache_len]), sc2,
+                                             top_k, init, local)
+    assert np.array_equal(ids, ids2) and np.array_equal(cnt, cnt2)
+
+
+@pytest.mark.parametrize("name,kw", [("spec_decode", dict(batch=3, kv_len=(700, 1500))),
+                                     ("spec_decode", dict(batch=4, q_len=(1, 8),
+                                                          kv_len=(100, 900))),
+                                     ("bf16_decode", dict(batch=3, kv_len=(300, 2000)))])
+def test_shared_select_on_generated_problems(name, kw):
+    p = _small(name, **kw)
+    sc = oracle.index_scores(p["row_off"], p["cache_len"], p["table"], p["q_idx"], p["k_idx"],
+                             p["max_blocks"])
+    ids, cnt = oracle.select_blocks_shared(p["row_off"], p["cache_len"], sc, p["top_k"],
+                                           p["init_blocks"], p["local_blocks"])
+    own, own_cnt = oracle.select_blocks(p["row_off"], p["cache_len"], sc, p["top_k"],
+                                        p["init_blocks"], p["local_blocks"])
+    ro = p["row_off"].tolist()
+    for b in range(p["batch"]):
+        if ro[b + 1] == ro[b]:
+            continue
+        t0 = ro[b]
+        # the first token keeps its ordinary selection
+        assert np.array_equal(ids[t0], own[t0]) and np.array_equal(cnt[t0], own_cnt[t0])
+        for t in range(t0, ro[b + 1]):
+            for g in range(p["H_kv"]):
+                sel = ids[t, g, :cnt[t, g]].tolist()
+                assert sel == sorted(set(sel)) and len(sel) >= 1
+                assert cnt[t, g] <= p["S"]
+    if name == "bf16_decode":       # one token per sequence: sharing changes nothing
+        assert np.array_equal(ids, own) and np.array_equal(cnt, own_cnt)
+
+
 @pytest.mark.parametrize("seed", range(40))
 def test_select_matches_exhaustive_search(seed):
     rng = np.random.default_rng(seed)
