@@ -156,19 +156,27 @@ class ClockSampler:
 
 
 # ------------------------------------------------------------------ algorithmic work
-def algorithmic_bytes(prob, block_ids, num_selected):
+# index-K bytes per token and head: bf16; e4m3 + f32 scale; e2m1 pairs + 4 UE8M0 exponents
+INDEX_K_TOKEN_BYTES = {"bf16": 256, "fp8": 132, "fp4": 68}
+
+
+def algorithmic_bytes(prob, block_ids, num_selected, shared=False):
     """HBM bytes the method itself must move per step (implementation traffic excluded):
-    index: every visible index-K position of every sequence (+ q_idx); attention: K and V of
-    every valid position of each (sequence, KV head)'s union of selected blocks (+ q, out)."""
+    index: every visible index-K position of every sequence (only the first new token's, with
+    the top-k shared across draft tokens) (+ q_idx); attention: K and V of every valid
+    position of each (sequence, KV head)'s union of selected blocks (+ q, out)."""
     import numpy as np
     BLOCK, D = 128, 128
     kv_elem = 1 if prob["kv_fp8"] else 2
     ro = prob["row_off"].cpu().tolist()
+    cl = prob["cache_len"].cpu().tolist()
     L = prob["kv_lens"]
     ids = block_ids.cpu().numpy()
     cnt = num_selected.cpu().numpy()
-    idx_bytes = sum(L[b] for b in range(prob["batch"]) if ro[b + 1] > ro[b]) * \
-        prob["H_idxk"] * D * 2 + prob["total_q"] * prob["H_kv"] * D * 2
+    tok_bytes = INDEX_K_TOKEN_BYTES[prob.get("idx_dtype", "bf16")]
+    seen = [(cl[b] + 1 if shared else L[b]) for b in range(prob["batch"]) if ro[b + 1] > ro[b]]
+    idx_bytes = sum(seen) * prob["H_idxk"] * tok_bytes + \
+        (prob["batch"] if shared else prob["total_q"]) * prob["H_kv"] * D * 2
     kv_bytes = 0
     for b in range(prob["batch"]):
         if ro[b + 1] == ro[b]:
@@ -379,6 +387,17 @@ def run_reference(args):
     return 0
 
 
+# Variants of the five workloads with the options the pages add: the index-K cache in a scaled
+# format (TensorRT-LLM DeepSeekSparseAttentionConfig, indexer_k_dtype) and the indexer top-k
+# shared across draft tokens (index_share_for_mtp_iteration).  name -> (workload, spec
+# changes, Path options)
+VARIANTS = {
+    "fp8_long_decode_fp8_index_k": ("fp8_long_decode", dict(idx_dtype="fp8"), {}),
+    "fp8_long_decode_fp4_index_k": ("fp8_long_decode", dict(idx_dtype="fp4"), {}),
+    "spec_decode_shared_topk": ("spec_decode", {}, dict(share_selection=True)),
+}
+
+
 def bench_workload(name, args, ws, rank, dev, sampler, with_cpu):
     """Every measurement of one workload: the timed whole-path step (median of repeated
     K-step blocks), per-launch times of the same launches, the roofline of the dominant one,
@@ -386,11 +405,13 @@ def bench_workload(name, args, ws, rank, dev, sampler, with_cpu):
     from block_sparse_paged_scores_b200 import msa
     from block_sparse_paged_scores_b200 import workload as wl
 
-    spec = wl.WORKLOADS[name]
+    base, changes, path_kw = VARIANTS.get(name, (name, {}, {}))
+    spec = wl.WORKLOADS[base].scaled(**changes)
     if args.batch:
         spec = spec.scaled(batch=args.batch)
-    prob = wl.generate(spec, seed=wl.SEEDS[name] + 1000 * rank, device=dev)
-    path = msa.Path(prob, num_splits=args.splits)
+    prob = wl.generate(spec, seed=wl.SEEDS[base] + 1000 * rank, device=dev)
+    path = msa.Path(prob, num_splits=args.splits, **path_kw)
+    shared = bool(path_kw.get("share_selection"))
     stream = torch.cuda.current_stream(dev)
     fp8 = prob["kv_fp8"]
     G = prob["H_q"] // prob["H_kv"]
@@ -400,7 +421,9 @@ def bench_workload(name, args, ws, rank, dev, sampler, with_cpu):
     splits = msa.msa_attn_partials(path.rp, prob["S"], prob["H_q"], prob["H_kv"],
                                    path.max_blocks, args.splits)[0] if stream_route else 1
     combine = stream_route and splits > 1
-    if decode:          # index, attention with the selection inside, [combine]
+    if shared:          # index with the selection inside, plan, attention, [combine]
+        launches = 3 + int(combine)
+    elif decode:        # index, attention with the selection inside, [combine]
         launches = 2 + int(combine)
     elif stream_route:  # index, select, plan, attention, [combine]
         launches = 4 + int(combine)
@@ -413,7 +436,7 @@ def bench_workload(name, args, ws, rank, dev, sampler, with_cpu):
     torch.cuda.synchronize(dev)
     assert int(path.dev_err.item()) == 0, f"device error flag set during warm-up ({name})"
 
-    idx_bytes, attn_bytes = algorithmic_bytes(prob, path.block_ids, path.num_selected)
+    idx_bytes, attn_bytes = algorithmic_bytes(prob, path.block_ids, path.num_selected, shared)
     flush = idx_bytes + attn_bytes < L2_BYTES
     flush_buf = torch.empty(2 * L2_BYTES, dtype=torch.uint8, device=dev) if flush else None
 
@@ -432,7 +455,16 @@ def bench_workload(name, args, ws, rank, dev, sampler, with_cpu):
     assert int(path.dev_err.item()) == 0, f"device error flag set ({name})"
 
     # ---- the same launches, one group at a time (events between them)
-    if decode:
+    if shared:
+        groups = {"index_select_shared": lambda: path.index_select(stream)}
+        attn_key = "attention_incl_plan"
+        if combine:
+            groups[attn_key] = lambda: path.attend(stream=stream, combine=False)
+            groups["combine"] = lambda: path.combine(stream)
+        else:
+            groups[attn_key] = lambda: path.attend(stream=stream)
+        attn_src = ("attention_stream.cu", "attn_common.cuh", "select_row.cuh")
+    elif decode:
         groups = {"index_scores": lambda: path.index_scores(stream)}
         if combine:
             groups["attention_with_selection"] = lambda: path.select_attend(stream,
@@ -454,10 +486,11 @@ def bench_workload(name, args, ws, rank, dev, sampler, with_cpu):
         attn_src = (("attention_stream.cu", "attn_common.cuh", "select_row.cuh")
                     if stream_route else
                     (("attention_tile.cu", "attn_common.cuh") if fp8 else ("attention_tc.cu",)))
-    idx_src = ("indexer.cu", "select_row.cuh") if stream_route else ("indexer_tc.cu",)
+    idx_src = (("indexer.cu", "select_row.cuh")
+               if stream_route or prob["idx_dtype"] != "bf16" else ("indexer_tc.cu",))
     st = stage_times(list(groups.values()), args.steps, stream, args.stage_seconds)
     stages = dict(zip(groups, st))
-    if stream_route:
+    if stream_route and not shared:
         # for comparison: the first two stages as one msa_index_select launch
         stages["fused_index_select"] = stage_times([lambda: path.index_select(stream)],
                                                    args.steps, stream,
@@ -465,15 +498,15 @@ def bench_workload(name, args, ws, rank, dev, sampler, with_cpu):
 
     # ---- roofline of the dominant launch group of the step
     hbm, bf16, bf16_sus, peak_src = measured_peaks()
-    kinds = {"index_scores": (stages["index_scores"], idx_src),
-             attn_key: (stages[attn_key], attn_src)}
+    idx_key = "index_select_shared" if shared else "index_scores"
+    kinds = {idx_key: (stages[idx_key], idx_src), attn_key: (stages[attn_key], attn_src)}
     dom = max(kinds, key=lambda k: kinds[k][0])
     d_ms, d_src = kinds[dom]
-    traffic_kernel = "index_scores" if dom == "index_scores" else "attention"
+    traffic_kernel = "index_scores" if dom == idx_key else "attention"
     traffic = profiled_traffic(traffic_kernel, name, source_digest(*d_src))
     if tensor_route:
         idx_flops, attn_flops = algorithmic_flops(prob, path.block_ids, path.num_selected)
-        d_flops = idx_flops if dom == "index_scores" else attn_flops
+        d_flops = idx_flops if dom == idx_key else attn_flops
         achieved = d_flops / (d_ms * 1e-3) / 1e12
         roofline = {"bound": "tensor", "kernel": dom, "achieved": achieved, "peak": bf16,
                     "unit": "TFLOP/s", "frac": achieved / bf16, "peak_source": peak_src,
@@ -482,7 +515,7 @@ def bench_workload(name, args, ws, rank, dev, sampler, with_cpu):
                     "note": "algorithmic FLOPs (selected, causally clipped positions only) over "
                             "the launch group's median time, against the measured bf16 burst "
                             "peak"}
-        if dom != "index_scores" and not fp8:
+        if dom != idx_key and not fp8:
             ex = executed_flops_tiles(prob, path.block_ids, path.num_selected, 128 // G)
             roofline["executed_flops_per_launch"] = ex
             roofline["executed_tflops"] = ex / (d_ms * 1e-3) / 1e12
@@ -491,7 +524,7 @@ def bench_workload(name, args, ws, rank, dev, sampler, with_cpu):
                 "achieved_TFLOPs": (idx_flops + attn_flops) / (ms_block / args.steps * 1e-3)
                 / 1e12}
     else:
-        d_bytes = idx_bytes if dom == "index_scores" else attn_bytes
+        d_bytes = idx_bytes if dom == idx_key else attn_bytes
         achieved = d_bytes / (d_ms * 1e-3) / 1e9
         roofline = {"bound": "hbm", "kernel": dom, "achieved": achieved, "peak": hbm,
                     "unit": "GB/s", "frac": achieved / hbm, "peak_source": peak_src,
@@ -583,7 +616,8 @@ def bench_workload(name, args, ws, rank, dev, sampler, with_cpu):
                    "local_blocks": prob["local_blocks"],
                    "kv_lens": f"{spec.kv_len}" if spec.prior_len is None else
                    f"prior {spec.prior_len} + new {spec.q_len}",
-                   "kv_dtype": spec.kv_dtype, "index_k_dtype": "bf16",
+                   "kv_dtype": spec.kv_dtype, "index_k_dtype": spec.idx_dtype,
+                   "topk_shared_across_drafts": shared,
                    "split_k_partials": splits, "parallelism": f"replicas x{ws}", "l2": l2},
         "timing": {"blocks": n_blocks, "steps_per_block": args.steps,
                    "block_ms_min_median_max": [min(blocks), statistics.median(blocks),
@@ -623,8 +657,9 @@ def run_ours(args):
                           with_cpu=rank == 0 and ws == 1 and not args.no_cpu_baseline)
     others = {}
     if not args.only:
-        # the other workloads, each measured the same way (every rank takes the same steps)
-        for name in wl.WORKLOADS:
+        # the other workloads and the variants, each measured the same way (every rank takes
+        # the same steps)
+        for name in list(wl.WORKLOADS) + list(VARIANTS):
             if name != args.workload:
                 others[name] = bench_workload(name, args, ws, rank, dev, sampler, False)
     if sampler:

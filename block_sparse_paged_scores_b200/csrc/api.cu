@@ -279,13 +279,21 @@ bool index_k_ok(const msa_index_k_t *k, int32_t num_kv_heads) {
   return false;
 }
 
+// The flags msa_index_scores_k / msa_index_select_k accept for this batch.
+bool index_flags_ok(const msa_ragged_paged_t *rp, uint32_t flags) {
+  if (flags & ~static_cast<uint32_t>(MSA_SHARE_ACROSS_DRAFTS)) return false;
+  return !(flags & MSA_SHARE_ACROSS_DRAFTS) || rp->max_q_len <= MSA_MAX_SPEC_DRAFT;
+}
+
 msa_status_t index_scores_impl(const msa_ragged_paged_t *rp, const void *q_idx,
                                const msa_index_k_t *kidx, int32_t num_kv_heads,
-                               int32_t max_blocks, float *scores, int32_t *dev_err,
-                               cudaStream_t stream, const FusedSelect *fs) {
+                               int32_t max_blocks, uint32_t flags, float *scores,
+                               int32_t *dev_err, cudaStream_t stream, const FusedSelect *fs) {
   if (!ragged_ok(rp) || !q_idx || !scores || num_kv_heads < 1 || !index_k_ok(kidx, num_kv_heads) ||
-      max_blocks < 1 || max_blocks > rp->max_pages_per_seq || !aligned(q_idx, 16))
+      max_blocks < 1 || max_blocks > rp->max_pages_per_seq || !aligned(q_idx, 16) ||
+      !index_flags_ok(rp, flags))
     return MSA_ERR_INVALID_ARG;
+  const bool share = (flags & MSA_SHARE_ACROSS_DRAFTS) != 0;
   const void *k_idx_cache = kidx->codes;
   const int32_t num_idx_k_heads = kidx->num_heads;
   const int idx_fmt = static_cast<int>(kidx->dtype);
@@ -326,6 +334,11 @@ msa_status_t index_scores_impl(const msa_ragged_paged_t *rp, const void *q_idx,
   }
   a.qt = rp->max_q_len * Hg <= 32 ? rp->max_q_len : (32 / Hg > 0 ? 32 / Hg : 1);
   a.tiles = (rp->max_q_len + a.qt - 1) / a.qt;
+  if (share) {  // only each sequence's first new token is scored
+    a.qt = 1;
+    a.tiles = 1;
+    a.share = 1;
+  }
   const int mt = a.qt * Hg <= 16 ? 1 : 2;
   // pages per CTA: about eight CTAs per SM over the launch, at least 4 pages each
   const long long units = static_cast<long long>(rp->batch) * a.tiles * num_idx_k_heads;
@@ -374,9 +387,8 @@ msa_status_t msa_index_scores_k(const msa_ragged_paged_t *rp, const void *q_idx,
                                 const msa_index_k_t *k_idx, int32_t num_kv_heads,
                                 int32_t max_blocks, uint32_t flags, float *scores,
                                 int32_t *dev_err, struct CUstream_st *stream) {
-  if (flags != 0) return MSA_ERR_INVALID_ARG;
-  if (ragged_ok(rp) && rp->total_q == 0) return MSA_OK;  // nothing to score
-  return index_scores_impl(rp, q_idx, k_idx, num_kv_heads, max_blocks, scores, dev_err,
+  if (ragged_ok(rp) && rp->total_q == 0 && index_flags_ok(rp, flags)) return MSA_OK;
+  return index_scores_impl(rp, q_idx, k_idx, num_kv_heads, max_blocks, flags, scores, dev_err,
                            reinterpret_cast<cudaStream_t>(stream), nullptr);
 }
 
@@ -403,7 +415,7 @@ msa_status_t msa_index_select_k(const msa_ragged_paged_t *rp, const void *q_idx,
   const long long S = static_cast<long long>(top_k) + init_blocks + local_blocks;
   if (!ragged_ok(rp) || num_kv_heads < 1 || !k_idx || k_idx->num_heads < 1 || max_blocks < 1 ||
       top_k < 0 || init_blocks < 0 || local_blocks < 0 || S < 1 || S > (1 << 20) ||
-      flags != 0)
+      !index_flags_ok(rp, flags))
     return MSA_ERR_INVALID_ARG;
   if (rp->total_q == 0) return MSA_OK;
   if (!block_ids || !num_selected) return MSA_ERR_INVALID_ARG;
@@ -415,11 +427,12 @@ msa_status_t msa_index_select_k(const msa_ragged_paged_t *rp, const void *q_idx,
     if (!counters || !aligned(counters, 4)) return MSA_ERR_INVALID_ARG;
     const FusedSelect fs{counters, block_ids, num_selected, top_k, init_blocks, local_blocks,
                          static_cast<int>(S)};
-    return index_scores_impl(rp, q_idx, k_idx, num_kv_heads, max_blocks, scores, dev_err, st,
-                             &fs);
+    return index_scores_impl(rp, q_idx, k_idx, num_kv_heads, max_blocks, flags, scores, dev_err,
+                             st, &fs);
   }
-  const msa_status_t e =
-      index_scores_impl(rp, q_idx, k_idx, num_kv_heads, max_blocks, scores, dev_err, st, nullptr);
+  if (flags & MSA_SHARE_ACROSS_DRAFTS) return MSA_ERR_UNSUPPORTED;  // the fused route only
+  const msa_status_t e = index_scores_impl(rp, q_idx, k_idx, num_kv_heads, max_blocks, flags,
+                                           scores, dev_err, st, nullptr);
   if (e != MSA_OK) return e;
   return msa_select_blocks(rp, scores, num_kv_heads, max_blocks, top_k, init_blocks,
                            local_blocks, block_ids, num_selected, dev_err, stream);

@@ -81,10 +81,13 @@ __device__ __forceinline__ float ue8m0_to_float(uint32_t x) {
 
 // The consumer warps (threads 0..127) of every CTA of a unit call this once the CTA's scores
 // are written; the last CTA to arrive selects for the unit's rows.
+// With the top-k shared across draft tokens (a.share: the unit scored only the sequence's first
+// new token), the last CTA selects for every new token of the sequence (q_len of them) from the
+// first token's scores.
 template <int KPL>
 __device__ __forceinline__ void count_out_and_select(const IndexerArgs &a, int b, int tile,
                                                      int hk, int row0, int tok0, int ntok,
-                                                     int cl, volatile int *is_last) {
+                                                     int cl, int q_len, volatile int *is_last) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   named_bar_sync(2, kConsumerWarps * 32);  // every thread's scores written
   if (threadIdx.x == 0) {
@@ -100,14 +103,17 @@ __device__ __forceinline__ void count_out_and_select(const IndexerArgs &a, int b
   named_bar_sync(2, kConsumerWarps * 32);
   if (!*is_last) return;
   const int Hg = a.H_kv / a.H_idxk;
-  for (int r = warp; r < ntok * Hg; r += kConsumerWarps) {
+  const int n_out = a.share ? q_len : ntok;  // tokens selected for
+  for (int r = warp; r < n_out * Hg; r += kConsumerWarps) {
     const int tl = r / Hg, g = hk + (r % Hg) * a.H_idxk;
     const size_t item = static_cast<size_t>(row0 + tok0 + tl) * a.H_kv + g;
-    const int nb = min((cl + tok0 + tl) / kBlock + 1, a.max_blocks);
+    const size_t src = a.share ? static_cast<size_t>(row0) * a.H_kv + g : item;
+    const int nb_out = min((cl + tok0 + tl) / kBlock + 1, a.max_blocks);
+    const int nb = a.share ? min(cl / kBlock + 1, a.max_blocks) : nb_out;
     const int nsel =
-        select_row<(KPL > 0 ? KPL : 0), true>(a.scores + item * a.max_blocks, nb, a.top_k,
+        select_row<(KPL > 0 ? KPL : 0), true>(a.scores + src * a.max_blocks, nb, a.top_k,
                                               a.init_blocks, a.local_blocks, a.S,
-                                              a.block_ids + item * a.S, a.dev_err, lane);
+                                              a.block_ids + item * a.S, a.dev_err, lane, nb_out);
     if (lane == 0) a.num_selected[item] = nsel;
   }
 }
@@ -182,7 +188,7 @@ __global__ void __launch_bounds__(kThreads)
     if (KPL >= 0) {
       __syncthreads();  // every thread's -inf fills, before the count
       if (warp < kConsumerWarps)
-        count_out_and_select<KPL>(a, b, tile, hk, row0, tok0, ntok, cl, is_last);
+        count_out_and_select<KPL>(a, b, tile, hk, row0, tok0, ntok, cl, q_len, is_last);
     }
     return;
   }
@@ -437,7 +443,8 @@ __global__ void __launch_bounds__(kThreads)
       a.scores[(static_cast<size_t>(t) * a.H_kv + g) * a.max_blocks + j] = m;
     }
   }
-  if (KPL >= 0) count_out_and_select<KPL>(a, b, tile, hk, row0, tok0, ntok, cl, is_last);
+  if (KPL >= 0)
+    count_out_and_select<KPL>(a, b, tile, hk, row0, tok0, ntok, cl, q_len, is_last);
 }
 
 template <int MT, int KPL, int ST, int IF>

@@ -35,6 +35,9 @@ struct IndexerArgs {
   int32_t *counters;
   int32_t *block_ids, *num_selected;  // [total_q, H_kv, S], [total_q, H_kv]
   int top_k, init_blocks, local_blocks, S;
+  // Top-k shared across each sequence's new tokens: one tile of one token (the first) per
+  // sequence is scored, and the fused selection writes every token's row from it.
+  int share;
 };
 // mt = 16-row MMA tiles per CTA (1 or 2)
 cudaError_t launch_index_scores(const CUtensorMap &kidx_map, const IndexerArgs &a, int mt,

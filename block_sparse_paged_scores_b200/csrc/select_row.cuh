@@ -82,16 +82,25 @@ struct SelKeys {
 
 // One warp selects for one (row, KV head): srow = its nb visible scores (nb >= 1), out = its S
 // id slots; returns the number selected (lane-uniform).  S >= init + local + top_k.
+//
+// nb_out > nb (the indexer top-k shared across a sequence's draft tokens: TensorRT-LLM
+// "DeepSeekSparseAttentionConfig", index_share_for_mtp_iteration): srow and nb are the first
+// draft token's, whose candidates and top-k they give; the output is for a later token that
+// sees nb_out blocks: its own forced blocks of [0, nb_out) together with that top-k.
 template <int KPL, bool CG>
 __device__ __forceinline__ int select_row(const float *srow, int nb, int top_k, int init_blocks,
                                           int local_blocks, int S, int32_t *out,
-                                          int32_t *dev_err, int lane) {
+                                          int32_t *dev_err, int lane, int nb_out = 0) {
   const unsigned lt_mask = (1u << lane) - 1u;
+  if (nb_out < nb) nb_out = nb;
   // forced: [0, init_e) and [local_lo, nb); candidates: [init_e, local_lo)
   const int init_e = min(init_blocks, nb);
   const int local_lo = max(init_e, nb - local_blocks);
   const int n_cand = local_lo - init_e;
   const bool take_all = n_cand <= top_k;
+  // the output row's own forced blocks: [0, init_o) and [local_o, nb_out)
+  const int init_o = min(init_blocks, nb_out);
+  const int local_o = max(init_o, nb_out - local_blocks);
 
   SelKeys<KPL, CG> keys;
   uint32_t T = 0xffffffffu;  // top_k == 0: no candidate passes
@@ -120,18 +129,18 @@ __device__ __forceinline__ int select_row(const float *srow, int nb, int top_k, 
   int nsel = 0, eq_seen = 0;
   auto pass = [&](int i, uint32_t key_reg) {
     const int j = i * 32 + lane;
-    const bool in = j < nb;
-    const bool cand = in && j >= init_e && j < local_lo;
+    const bool cand = j < nb && j >= init_e && j < local_lo;
+    const bool forced = j < nb_out && (j < init_o || j >= local_o);
     bool take;
     if (take_all) {
-      take = in;
+      take = forced || cand;
     } else {
       const uint32_t key =
           KPL > 0 ? key_reg : (cand ? score_key(load_score<CG>(srow + j)) : 0u);
       const bool eq = cand && key == T;
       const unsigned eqm = __ballot_sync(0xffffffffu, eq);
       const int eq_rank = eq_seen + __popc(eqm & lt_mask);
-      take = (in && !cand) || (cand && key > T) || (eq && eq_rank < need_eq);
+      take = forced || (cand && key > T) || (eq && eq_rank < need_eq);
       eq_seen += __popc(eqm);
     }
     const unsigned tm = __ballot_sync(0xffffffffu, take);
@@ -141,7 +150,7 @@ __device__ __forceinline__ int select_row(const float *srow, int nb, int top_k, 
     }
     nsel += __popc(tm);
   };
-  const int passes = (nb + 31) / 32;
+  const int passes = (nb_out + 31) / 32;
   if (KPL > 0) {
 #pragma unroll
     for (int i = 0; i < (KPL > 0 ? KPL : 1); ++i)
@@ -149,7 +158,7 @@ __device__ __forceinline__ int select_row(const float *srow, int nb, int top_k, 
   } else {
     for (int i = 0; i < passes; ++i) pass(i, 0u);
   }
-  if (nsel > S) {  // cannot happen when S == init + local + top_k
+  if (nsel > S) {  // cannot happen when S >= init + local + top_k
     if (lane == 0) report(dev_err, MSA_DEVERR_NUM_SELECTED);
     nsel = S;
   }

@@ -21,6 +21,7 @@ MSA_IDX_BF16, MSA_IDX_FP8_E4M3, MSA_IDX_FP4_E2M1 = 0, 1, 2
 IDX_DTYPES = {"bf16": MSA_IDX_BF16, "fp8": MSA_IDX_FP8_E4M3, "fp4": MSA_IDX_FP4_E2M1}
 MSA_DEVERR_PAGE_ID, MSA_DEVERR_LENGTHS, MSA_DEVERR_BLOCK_ID = 1, 2, 4
 MSA_DEVERR_NUM_SELECTED, MSA_DEVERR_TIMEOUT = 8, 16
+MSA_SHARE_ACROSS_DRAFTS = 1
 BLOCK = 128
 HEAD_DIM = 128
 
@@ -264,12 +265,15 @@ class Path:
     enqueues index scores -> selection -> attention on the current stream: by default the
     last two as one msa_select_sparse_attn_paged call (``select_in_attention``); with
     ``fused_select`` the first two as one msa_index_select call; with neither, three separate
-    calls."""
+    calls.  ``share_selection``: the indexer top-k shared across each sequence's draft tokens
+    (MSA_SHARE_ACROSS_DRAFTS, through msa_index_select_k), then the attention."""
 
     def __init__(self, prob: dict, num_splits: int = 0, max_blocks: Optional[int] = None,
-                 fused_select: bool = False, select_in_attention: bool = True):
+                 fused_select: bool = False, select_in_attention: bool = True,
+                 share_selection: bool = False):
         self.p = prob
-        self.fused_select = fused_select
+        self.share_selection = share_selection
+        self.fused_select = fused_select or share_selection
         self.select_in_attention = select_in_attention
         dev = prob["q"].device
         self.max_blocks = int(max_blocks or prob["max_blocks"])
@@ -291,7 +295,7 @@ class Path:
         self.idx_dtype = prob.get("idx_dtype", "bf16")
         self.kidx = index_k(prob["k_idx"], prob.get("k_idx_scale"), prob["H_idxk"],
                             self.idx_dtype)
-        self.index_flags = 0
+        self.index_flags = MSA_SHARE_ACROSS_DRAFTS if share_selection else 0
 
     def index_scores(self, stream=None):
         p = self.p

@@ -201,10 +201,22 @@ typedef struct {
 
 /*
  * msa_index_scores_k / msa_index_select_k — msa_index_scores / msa_index_select over an index-K
- * cache in any msa_idx_dtype_t (the BF16 entry points are these with MSA_IDX_BF16; their
- * results are bit-identical).  `flags` must be 0 except as stated below.  Scaled formats run
- * the warp-MMA indexer on every route (the prefill route's tcgen05 indexer takes BF16 only).
+ * cache in any msa_idx_dtype_t (the BF16 entry points are these with MSA_IDX_BF16 and flags 0;
+ * their results are bit-identical).  Scaled formats run the warp-MMA indexer on every route
+ * (the prefill route's tcgen05 indexer takes BF16 only).
+ *
+ * flags: 0, or MSA_SHARE_ACROSS_DRAFTS ([trtllm] index_share_for_mtp_iteration: reuse the
+ * indexer top-k across draft tokens instead of recomputing it for each), accepted on the
+ * decode and speculative routes (max_q_len <= MSA_MAX_SPEC_DRAFT; MSA_ERR_INVALID_ARG
+ * otherwise).  Then only the first new token of each sequence is scored (the other rows of
+ * `scores` are not written), and msa_index_select_k selects for every new token t of the
+ * sequence its own forced blocks (init / local, for its own position) together with the top_k
+ * of the first token's candidates (its visible blocks minus its own forced blocks) by the
+ * first token's scores, ascending.  Those blocks lie below the first token's position, so every
+ * later token can read them.  num_selected[t] <= S as ever.
  */
+#define MSA_SHARE_ACROSS_DRAFTS 1u
+
 MSA_API msa_status_t msa_index_scores_k(const msa_ragged_paged_t *rp, const void *q_idx,
                                         const msa_index_k_t *k_idx, int32_t num_kv_heads,
                                         int32_t max_blocks, uint32_t flags, float *scores,

@@ -506,3 +506,72 @@ def test_bf16_descriptor_entry_points_equal_the_bf16_ones(name):
                            b.dev_err)
     torch.cuda.synchronize()
     assert torch.equal(a.scores, b.scores)
+
+
+# ------------------------------------------------------------------ top-k shared across drafts
+SHARED = {
+    "spec_decode": lambda: _problem("spec_decode"),
+    "spec_ragged_q": lambda: _problem("spec_ragged_q"),
+    "spec_gqa4": lambda: _problem("spec_gqa4"),
+    "fp8_spec": lambda: _problem("fp8_spec"),
+    "bf16_decode": lambda: _problem("bf16_decode"),
+    "short_contexts": lambda: wl.generate(W["spec_decode"].scaled(batch=8, q_len=(1, 8),
+                                                                  kv_len=(9, 400)), seed=31),
+    "fp4idx_spec": lambda: _scaled_problem("fp4idx_spec_ragged"),
+}
+
+
+@pytest.mark.parametrize("name", sorted(SHARED))
+def test_shared_selection_is_bit_exact(name):
+    """msa_index_select_k with MSA_SHARE_ACROSS_DRAFTS: the first tokens' scores against the
+    oracle's, every token's selection against the oracle's shared selection on the GPU's own
+    scores (bit for bit), twice in a row (counters back at zero)."""
+    p = SHARED[name]()
+    sc, _, _, _ = oracle_forward(p)
+    path = msa.Path(_gpu(p), share_selection=True)
+    path.scores.fill_(float("nan"))          # rows after the first must not be read
+    for _ in range(2):
+        path.index_select()
+    torch.cuda.synchronize()
+    assert int(path.dev_err.item()) == 0
+    assert int(path.counters.abs().sum().item()) == 0
+    ro = p["row_off"].tolist()
+    assert all(ro[b + 1] > ro[b] for b in range(p["batch"]))
+    first = ro[:-1]                          # each sequence's first new token
+    g_sc = path.scores.cpu().numpy()
+    firsts = dict(p, row_off=torch.arange(p["batch"] + 1, dtype=torch.int32),
+                  q_idx=p["q_idx"][first], total_q=p["batch"])
+    check_scores(g_sc[first], sc[first], firsts, p["max_blocks"])
+    ids, cnt = oracle.select_blocks_shared(p["row_off"], p["cache_len"],
+                                           g_sc.astype(np.float64), p["top_k"],
+                                           p["init_blocks"], p["local_blocks"])
+    assert np.array_equal(path.num_selected.cpu().numpy(), cnt)
+    assert np.array_equal(path.block_ids.cpu().numpy(), ids)
+
+
+@pytest.mark.parametrize("name", sorted(SHARED))
+def test_shared_selection_whole_path_matches_oracle(name):
+    p = SHARED[name]()
+    path = msa.Path(_gpu(p), share_selection=True)
+    path.run()
+    torch.cuda.synchronize()
+    assert int(path.dev_err.item()) == 0
+    g_ids, g_cnt = path.block_ids.cpu().numpy(), path.num_selected.cpu().numpy()
+    out = oracle.attention(p["row_off"], p["cache_len"], p["table"], p["q"], p["k"], p["v"],
+                           p["kv_fp8"], g_ids, g_cnt, p["scale"])
+    check_attention(path.out.float().cpu(), out, p["kv_fp8"])
+    # and against the oracle's own whole shared path wherever the first token's cut is clear
+    sc, o_ids, o_cnt, o_out = oracle.forward(p, p["top_k"], p["init_blocks"], p["local_blocks"],
+                                             p["scale"], p["max_blocks"], share=True)
+    same = np.all(g_ids == o_ids, axis=2) & (g_cnt == o_cnt)
+    assert same.mean() > 0.9
+    mask = head_rows_mask(same, p["H_q"] // p["H_kv"])
+    check_attention(path.out.float().cpu(), o_out, p["kv_fp8"], rows_mask=mask)
+
+
+def test_shared_selection_is_refused_on_the_prefill_route():
+    p = _gpu(_problem("prefill"))
+    path = msa.Path(p, share_selection=True)
+    with pytest.raises(msa.MSAError) as ei:
+        path.index_select()
+    assert ei.value.status == msa.MSA_ERR_INVALID_ARG
