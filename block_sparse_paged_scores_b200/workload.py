@@ -238,3 +238,97 @@ def to_device(prob: dict, device) -> dict:
     for k_, v_ in prob.items():
         out[k_] = v_.to(device) if isinstance(v_, torch.Tensor) else v_
     return out
+
+
+# ------------------------------------------------------------------ latent sparse attention
+@dataclasses.dataclass(frozen=True)
+class LatentSpec:
+    """A workload of the latent sparse attention op (Mojo
+    Struct_latent_sparse_attention_ragged_paged): a K = V latent (128 wide, shared by the H
+    query heads) in two paged leaves with a layer axis, a sliding window over one and a
+    per-query entry list into the other, a per-head sink."""
+    name: str
+    batch: int
+    q_len: IntOrRange
+    H: int
+    window: int
+    n_entries: int
+    swa_len: IntOrRange        # prior tokens of the sliding-window leaf (new ones follow)
+    comp_len: IntOrRange       # entries of the compressed leaf
+    layers: int = 2
+    layer: int = 1
+
+    def scaled(self, **kw) -> "LatentSpec":
+        return dataclasses.replace(self, **kw)
+
+
+LATENT_DECODE = LatentSpec("latent_decode", batch=64, q_len=1, H=64, window=128,
+                           n_entries=512, swa_len=(1024, 8192), comp_len=(2048, 8192))
+
+
+def _paged_leaf(lengths, first_needed, layers, gen_cpu, gdev, device, poison):
+    """A paged leaf holding positions [first_needed[b], lengths[b]) of every sequence (pages
+    below the first needed one are left out of the table, -1), N(0,1) bf16 values, the pool
+    shuffled; unused pool pages and positions past a sequence's end are NaN."""
+    batch = len(lengths)
+    nb = [(int(L) + BLOCK - 1) // BLOCK for L in lengths]
+    lo = [int(f) // BLOCK for f in first_needed]
+    total = sum(n - l for n, l in zip(nb, lo))
+    pool = max(total, 1)
+    perm = torch.randperm(pool, generator=gen_cpu)
+    max_pages = max(1, max(nb))
+    table = torch.full((batch, max_pages), -1, dtype=torch.int32)
+    cur = 0
+    for b in range(batch):
+        for j in range(lo[b], nb[b]):
+            table[b, j] = int(perm[cur])
+            cur += 1
+    kv = _normal_pages((pool, layers, BLOCK, HEAD_DIM), gdev, device, torch.bfloat16)
+    if poison:
+        unused = perm[total:].to(device)
+        if unused.numel():
+            kv[unused] = float("nan")
+        for b in range(batch):
+            tail = int(lengths[b]) % BLOCK
+            if tail:
+                kv[int(table[b, nb[b] - 1]), :, tail:] = float("nan")
+    return kv, table
+
+
+def generate_latent(spec: LatentSpec, seed: int, device="cpu", poison: bool = True) -> dict:
+    """One seeded latent problem.  Draw order: lengths (new tokens, window-leaf prior, compressed
+    leaf), the window leaf's page permutation, the compressed leaf's, each query's entry list
+    (a uniform random subset of its sequence's compressed entries, ascending, -1 padded when
+    the leaf is shorter than n_entries), then q, the window leaf, the compressed leaf and the
+    sinks as N(0,1)."""
+    gcpu = torch.Generator().manual_seed(seed)
+    q_lens = _draw(spec.q_len, spec.batch, gcpu)
+    swa_prior = _draw(spec.swa_len, spec.batch, gcpu)
+    comp_len = _draw(spec.comp_len, spec.batch, gcpu)
+    L_swa = swa_prior + q_lens
+    first = torch.clamp(swa_prior - spec.window + 1, min=0)
+    row_off = torch.zeros(spec.batch + 1, dtype=torch.int32)
+    row_off[1:] = torch.cumsum(q_lens, 0).to(torch.int32)
+    total_q = int(row_off[-1])
+    gdev = torch.Generator(device=device).manual_seed(seed)
+    swa_kv, swa_table = _paged_leaf(L_swa.tolist(), first.tolist(), spec.layers, gcpu, gdev,
+                                    device, poison)
+    comp_kv, comp_table = _paged_leaf(comp_len.tolist(), [0] * spec.batch, spec.layers, gcpu,
+                                      gdev, device, poison)
+    comp_idx = torch.full((total_q, spec.n_entries), -1, dtype=torch.int32)
+    for b in range(spec.batch):
+        n = min(spec.n_entries, int(comp_len[b]))
+        for t in range(int(row_off[b]), int(row_off[b + 1])):
+            comp_idx[t, :n] = torch.sort(torch.randperm(int(comp_len[b]), generator=gcpu)[:n])[0]
+    q = torch.randn((total_q, spec.H, HEAD_DIM), generator=gdev, device=device).to(torch.bfloat16)
+    sink = torch.randn((spec.H,), generator=gdev, device=device, dtype=torch.float32)
+    return dict(
+        name=spec.name, spec=spec, seed=seed, batch=spec.batch, total_q=total_q,
+        max_q_len=max(1, int(q_lens.max())), H=spec.H, window=spec.window,
+        n_entries=spec.n_entries, row_off=row_off.to(device), q=q,
+        swa_kv=swa_kv, swa_len=swa_prior.to(torch.int32).to(device),
+        swa_table=swa_table.to(device), swa_layer=spec.layer,
+        comp_kv=comp_kv, comp_len=comp_len.to(torch.int32).to(device),
+        comp_table=comp_table.to(device), comp_layer=spec.layer,
+        comp_idx=comp_idx.to(device), sink=sink, scale=1.0 / math.sqrt(HEAD_DIM),
+        q_lens=q_lens.tolist(), swa_lens=L_swa.tolist(), comp_lens=comp_len.tolist())

@@ -61,6 +61,9 @@ def _load():
         lib.orc_select_blocks.argtypes = [I, P, P, I, I, P, I, I, I, I, P, P]
         lib.orc_select_blocks_shared.restype = None
         lib.orc_select_blocks_shared.argtypes = [I, P, P, I, I, P, I, I, I, I, P, P]
+        lib.orc_latent_attention.restype = None
+        lib.orc_latent_attention.argtypes = [I, P, P, I, I, P, I, I, P, P, I, P, I, I, P, I, P,
+                                             I, P, ctypes.c_double, P]
         lib.orc_attention.restype = None
         lib.orc_attention.argtypes = [I, P, P, P, I, P, P, P, I, I, I, P, P, I,
                                       ctypes.c_double, P]
@@ -227,3 +230,31 @@ def forward(inp, top_k, init_blocks, local_blocks, scale, max_blocks, share=Fals
     out = attention(inp["row_off"], inp["cache_len"], inp["table"], inp["q"], inp["k"],
                     inp["v"], inp["kv_fp8"], ids, counts, scale)
     return sc, ids, counts, out
+
+
+def latent_attention(row_off, q, window, swa_kv, swa_layer, swa_len, swa_table, comp_kv,
+                     comp_layer, comp_table, comp_idx, sink, scale):
+    """Latent sparse attention [total_q, H, 128] in fp64: K = V latent rows from the
+    sliding-window leaf (the ``window`` positions ending at each query's position
+    swa_len[b] + i) and from the compressed leaf (comp_idx [total_q, n_entries], -1 padding),
+    with the per-head sink in the denominator.  Leaves bf16 [pages, layers, 128, 128]."""
+    lib = _load()
+    row_off, p_off = _c(_ints(row_off), np.int32)
+    qb, p_q = _c(_bits16(q), np.uint16)
+    sw, p_sw = _c(_bits16(swa_kv), np.uint16)
+    cp, p_cp = _c(_bits16(comp_kv), np.uint16)
+    sl, p_sl = _c(_ints(swa_len), np.int32)
+    st, p_st = _c(_ints(swa_table), np.int32)
+    ct, p_ct = _c(_ints(comp_table), np.int32)
+    ci, p_ci = _c(_ints(comp_idx), np.int32)
+    sk = np.asarray(sink.detach().cpu().numpy() if hasattr(sink, "detach") else sink,
+                    dtype=np.float32)
+    sk, p_sk = _c(sk, np.float32)
+    total_q, H, _ = qb.shape
+    out = np.empty((total_q, H, HEAD_DIM), dtype=np.float64)
+    lib.orc_latent_attention(row_off.shape[0] - 1, p_off, p_q, H, int(window), p_sw,
+                             sw.shape[1], int(swa_layer), p_sl, p_st, st.shape[1], p_cp,
+                             cp.shape[1], int(comp_layer), p_ct, ct.shape[1], p_ci,
+                             ci.shape[1], p_sk, float(scale),
+                             out.ctypes.data_as(ctypes.c_void_p))
+    return out

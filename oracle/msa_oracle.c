@@ -373,3 +373,87 @@ void orc_attention(int batch, const int32_t *row_off, const int32_t *cache_len,
         }
     }
 }
+
+/* ---------------------------------------------------------------------------------------
+ * Latent sparse attention: Mojo "Struct_latent_sparse_attention_ragged_paged" (the
+ * mo.latent_sparse_attention.ragged.paged op): sparse attention over a K = V latent shared by
+ * all query heads, read from two paged leaves, the sliding-window leaf by position range and
+ * the compressed leaf by an explicit per-query entry list, with a per-head attention sink in
+ * the softmax denominator.
+ *
+ * Readings where the page gives only the op's arguments:
+ *   - the latent is 128 wide, both leaves are paged like the main cache (128 tokens a page,
+ *     page(b, pos) = table[b][pos / 128]) with a layer axis: [pages][layers][128][128] bf16,
+ *     and `layer` picks the layer;
+ *   - the window of the query at position p = swa_cache_lengths[b] + i is the `window`
+ *     positions ending at p (inclusive), clipped at 0; the new tokens are already in that leaf;
+ *   - comp_indices [total_q][n_entries] lists logical positions of the sequence's compressed
+ *     leaf; -1 is padding; every listed entry counts (as listed);
+ *   - the sink of head h adds exp(sink[h]) to the denominator (natural-log domain, not scaled)
+ *     and contributes no value:
+ *       out = sum_x e^(z_x) v_x / (e^(sink) + sum_x e^(z_x)),  z_x = scale * q . v_x.
+ * ------------------------------------------------------------------------------------- */
+void orc_latent_attention(int batch, const int32_t *row_off, const uint16_t *q, int H,
+                          int window, const uint16_t *swa_kv, int swa_layers, int swa_layer,
+                          const int32_t *swa_len, const int32_t *swa_table, int swa_max_pages,
+                          const uint16_t *comp_kv, int comp_layers, int comp_layer,
+                          const int32_t *comp_table, int comp_max_pages,
+                          const int32_t *comp_idx, int n_entries, const float *sink,
+                          double scale, double *out)
+{
+    for (int b = 0; b < batch; ++b) {
+        int q_len = row_off[b + 1] - row_off[b];
+#pragma omp parallel for collapse(2) schedule(dynamic)
+        for (int i = 0; i < q_len; ++i) {
+            for (int h = 0; h < H; ++h) {
+                int t = row_off[b] + i;
+                int p = swa_len[b] + i;
+                int w0 = p - window + 1;
+                if (w0 < 0)
+                    w0 = 0;
+                int n = (p - w0 + 1) + n_entries;
+                const uint16_t **rows = (const uint16_t **)malloc(sizeof(*rows) * (size_t)n);
+                int np = 0;
+                for (int pos = w0; pos <= p; ++pos) {
+                    int page = swa_table[(size_t)b * swa_max_pages + pos / ORC_BLOCK];
+                    rows[np++] = swa_kv + (((size_t)page * swa_layers + swa_layer) * ORC_BLOCK +
+                                           (size_t)(pos % ORC_BLOCK)) * ORC_D;
+                }
+                for (int e = 0; e < n_entries; ++e) {
+                    int pos = comp_idx[(size_t)t * n_entries + e];
+                    if (pos < 0)
+                        continue;
+                    int page = comp_table[(size_t)b * comp_max_pages + pos / ORC_BLOCK];
+                    rows[np++] = comp_kv + (((size_t)page * comp_layers + comp_layer) *
+                                                ORC_BLOCK + (size_t)(pos % ORC_BLOCK)) * ORC_D;
+                }
+                const uint16_t *qv = q + ((size_t)t * H + h) * ORC_D;
+                double *z = (double *)malloc(sizeof(double) * (size_t)(np > 0 ? np : 1));
+                double m = (double)sink[h];
+                for (int x = 0; x < np; ++x) {
+                    double dot = 0.0;
+                    for (int c = 0; c < ORC_D; ++c)
+                        dot += orc_bf16_value(qv[c]) * orc_bf16_value(rows[x][c]);
+                    z[x] = scale * dot;
+                    if (z[x] > m)
+                        m = z[x];
+                }
+                double l = exp((double)sink[h] - m); /* the sink: denominator only */
+                double acc[ORC_D];
+                for (int c = 0; c < ORC_D; ++c)
+                    acc[c] = 0.0;
+                for (int x = 0; x < np; ++x) {
+                    double w = exp(z[x] - m);
+                    l += w;
+                    for (int c = 0; c < ORC_D; ++c)
+                        acc[c] += w * orc_bf16_value(rows[x][c]);
+                }
+                double *o = out + ((size_t)t * H + h) * ORC_D;
+                for (int c = 0; c < ORC_D; ++c)
+                    o[c] = acc[c] / l;
+                free(z);
+                free(rows);
+            }
+        }
+    }
+}

@@ -535,3 +535,104 @@ def test_attention_hand_worked_cases():
         exp = c.get("expected") or c.get("expected_token0")
         for key, formula in exp.items():
             assert out[0, 0, int(key[3:])] == pytest.approx(eval(formula, env), rel=1e-14), c["name"]
+
+
+# ----------------------------------------------------------------------------- latent attention
+def _latent(batch=3, q_len=(1, 4), swa_len=(100, 700), comp_len=(300, 900), n_entries=48, H=6,
+            window=128, seed=3):
+    spec = wl.LATENT_DECODE.scaled(batch=batch, q_len=q_len, swa_len=swa_len,
+                                   comp_len=comp_len, n_entries=n_entries, H=H, window=window)
+    return wl.generate_latent(spec, seed=seed)
+
+
+def _latent_oracle(p, **over):
+    d = dict(p, **over)
+    return oracle.latent_attention(d["row_off"], d["q"], d["window"], d["swa_kv"],
+                                   d["swa_layer"], d["swa_len"], d["swa_table"], d["comp_kv"],
+                                   d["comp_layer"], d["comp_table"], d["comp_idx"], d["sink"],
+                                   d["scale"])
+
+
+def _leaf_row(kv, table, layer, b, pos):
+    return kv[int(table[b, pos // BLOCK]), layer, pos % BLOCK].double()
+
+
+def _latent_rows(p, t):
+    """The K = V rows query t reads, gathered from the two leaves by the layouts' own rules."""
+    ro = p["row_off"].tolist()
+    b = max(i for i in range(p["batch"]) if ro[i] <= t)
+    pos = int(p["swa_len"][b]) + (t - ro[b])
+    rows = [_leaf_row(p["swa_kv"], p["swa_table"], p["swa_layer"], b, x)
+            for x in range(max(0, pos - p["window"] + 1), pos + 1)]
+    rows += [_leaf_row(p["comp_kv"], p["comp_table"], p["comp_layer"], b, int(e))
+             for e in p["comp_idx"][t].tolist() if e >= 0]
+    return torch.stack(rows)
+
+
+@pytest.mark.parametrize("seed", [3, 4])
+def test_latent_attention_equals_sdpa_with_a_sink_key(seed):
+    """torch's scaled_dot_product_attention in fp64 over the gathered rows plus one extra key
+    of zeros (value zero) whose additive mask bias is the head's sink."""
+    p = _latent(seed=seed)
+    got = _latent_oracle(p)
+    for t in range(p["total_q"]):
+        kv = _latent_rows(p, t)                                      # [n, 128]
+        n = kv.shape[0]
+        k_ext = torch.cat([kv, torch.zeros(1, 128, dtype=torch.float64)])
+        q = p["q"][t].double()[:, None, :]                           # [H, 1, 128]
+        bias = torch.zeros(p["H"], 1, n + 1, dtype=torch.float64)
+        bias[:, 0, n] = p["sink"].double()
+        ref = torch.nn.functional.scaled_dot_product_attention(
+            q, k_ext[None].expand(p["H"], -1, -1), k_ext[None].expand(p["H"], -1, -1),
+            attn_mask=bias, scale=p["scale"])[:, 0]
+        np.testing.assert_allclose(got[t], ref.numpy(), rtol=1e-12, atol=1e-13)
+
+
+def test_latent_attention_with_q_zero_is_the_mean_shrunk_by_the_sink():
+    p = _latent(seed=5)
+    p["q"] = torch.zeros_like(p["q"])
+    got = _latent_oracle(p)
+    for t in range(p["total_q"]):
+        kv = _latent_rows(p, t)
+        n = kv.shape[0]
+        ref = kv.sum(0)[None, :] / (torch.exp(p["sink"].double())[:, None] + n)
+        np.testing.assert_allclose(got[t], ref.numpy(), rtol=1e-12, atol=1e-14)
+
+
+def test_latent_attention_without_sink_and_window_is_dense_causal_attention():
+    """A window longer than every sequence, no compressed entries and a sink of -inf: ordinary
+    causal attention over the whole window leaf (K = V)."""
+    p = _latent(seed=6, window=100000)
+    p["comp_idx"] = torch.full_like(p["comp_idx"], -1)
+    p["sink"] = torch.full_like(p["sink"], -float("inf"))
+    got = _latent_oracle(p)
+    ro = p["row_off"].tolist()
+    for b in range(p["batch"]):
+        L = int(p["swa_len"][b]) + ro[b + 1] - ro[b]
+        kv = torch.stack([_leaf_row(p["swa_kv"], p["swa_table"], p["swa_layer"], b, x)
+                          for x in range(L)])
+        q = p["q"][ro[b]:ro[b + 1]].double().permute(1, 0, 2)       # [H, n, 128]
+        n = q.shape[1]
+        mask = torch.arange(L)[None, :] <= (L - n + torch.arange(n))[:, None]
+        ref = torch.nn.functional.scaled_dot_product_attention(
+            q, kv[None].expand(p["H"], -1, -1), kv[None].expand(p["H"], -1, -1),
+            attn_mask=mask, scale=p["scale"]).permute(1, 0, 2)
+        np.testing.assert_allclose(got[ro[b]:ro[b + 1]], ref.numpy(), rtol=1e-11, atol=1e-12)
+
+
+def test_latent_attention_window_one_is_a_sigmoid_gate():
+    p = _latent(seed=7, window=1)
+    p["comp_idx"] = torch.full_like(p["comp_idx"], -1)
+    got = _latent_oracle(p)
+    for t in range(p["total_q"]):
+        v = _latent_rows(p, t)[0]                                     # the query's own row
+        z = p["scale"] * (p["q"][t].double() @ v)                     # [H]
+        gate = 1.0 / (1.0 + torch.exp(p["sink"].double() - z))
+        np.testing.assert_allclose(got[t], (gate[:, None] * v[None]).numpy(), rtol=1e-12,
+                                   atol=1e-14)
+
+
+def test_latent_attention_huge_sink_takes_all_the_mass():
+    p = _latent(seed=8)
+    p["sink"] = torch.full_like(p["sink"], 1e4)
+    assert np.abs(_latent_oracle(p)).max() < 1e-100
