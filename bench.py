@@ -555,7 +555,7 @@ def bench_workload(name, args, ws, rank, dev, sampler, with_cpu):
             serial_step()
         serial_ms = statistics.median(time_block(serial_step, args.steps, stream)
                                       for _ in range(3))
-        pipe = msa.HostPipeline(prob, num_splits=args.splits)
+        pipe = msa.HostPipeline(prob, num_splits=args.splits, **path_kw)
         packed = pipe.pack(host)  # the step's inputs as one pinned buffer: one copy per step
         for i in range(max(2, args.warmup)):
             pipe.submit(packed, outs[i % 2])
@@ -637,6 +637,76 @@ def bench_workload(name, args, ws, rank, dev, sampler, with_cpu):
     return res
 
 
+def bench_latent(name, args, ws, rank, dev, sampler):
+    """The latent sparse attention op (Mojo Struct_latent_sparse_attention_ragged_paged) on
+    its decode workload: batch 64, 64 heads, a 128-position window, 512 compressed entries per
+    query; measured like the other workloads (median of repeated K-step blocks)."""
+    from block_sparse_paged_scores_b200 import msa
+    from block_sparse_paged_scores_b200 import workload as wl
+
+    spec = wl.LATENT_DECODE
+    if args.batch:
+        spec = spec.scaled(batch=args.batch)
+    prob = wl.generate_latent(spec, seed=11 + 1000 * rank, device=dev)
+    path = msa.LatentPath(prob)
+    stream = torch.cuda.current_stream(dev)
+    step = lambda: path.run(stream)
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(dev)
+    assert int(path.dev_err.item()) == 0, "device error flag set (latent)"
+    # algorithmic bytes: every latent row a query reads, once per query (K = V), + q and out
+    ci = prob["comp_idx"].cpu()
+    comp_len = prob["comp_len"].cpu()
+    ro = prob["row_off"].cpu().tolist()
+    rows = 0
+    for b in range(prob["batch"]):
+        for i in range(ro[b + 1] - ro[b]):
+            p_ = int(prob["swa_len"][b]) + i
+            rows += p_ - max(0, p_ - prob["window"] + 1) + 1
+            e = ci[ro[b] + i]
+            rows += int(((e >= 0) & (e < comp_len[b])).sum())
+    alg_bytes = rows * 256 + prob["total_q"] * prob["H"] * 256 * 2
+    flush = alg_bytes < L2_BYTES
+    flush_buf = torch.empty(2 * L2_BYTES, dtype=torch.uint8, device=dev) if flush else None
+    first = time_block(step, args.steps, stream, flush_buf)
+    n_blocks = blocks_for(first, args.min_seconds, ws, dev)
+    barrier(ws, dev)
+    t_wall0 = time.time()
+    blocks = [time_block(step, args.steps, stream, flush_buf) for _ in range(n_blocks)]
+    barrier(ws, dev)
+    t_wall1 = time.time()
+    ms_block = max_over_ranks(statistics.median(blocks), ws, dev)
+    tokens = sum_over_ranks(prob["total_q"], ws, dev)
+    hbm, _, _, peak_src = measured_peaks()
+    step_ms = ms_block / args.steps
+    achieved = alg_bytes / (step_ms * 1e-3) / 1e9
+    launches = 1 + int(path.num_splits > 1)
+    res = {
+        "value": tokens * args.steps / (ms_block * 1e-3), "ms_per_step": step_ms, "dtype": "bf16",
+        "config": {"workload": name, "batch": prob["batch"], "q_tokens_per_step": prob["total_q"],
+                   "heads": prob["H"], "latent_dim": 128, "window": prob["window"],
+                   "compressed_entries_per_query": prob["n_entries"],
+                   "splits": path.num_splits, "parallelism": f"replicas x{ws}",
+                   "l2": (f"{alg_bytes / 2**20:.1f} MiB touched per step: L2 flushed before "
+                          f"every step, time = sum of the steps' own intervals") if flush else
+                         "inputs larger than L2, no flush"},
+        "timing": {"blocks": n_blocks, "steps_per_block": args.steps,
+                   "block_ms_min_median_max": [min(blocks), statistics.median(blocks),
+                                               max(blocks)]},
+        "roofline": {"bound": "hbm", "kernel": "latent_attention (+ combine)",
+                     "achieved": achieved, "peak": hbm, "unit": "GB/s", "frac": achieved / hbm,
+                     "peak_source": peak_src, "traffic": None,
+                     "algorithmic_bytes_per_launch": alg_bytes,
+                     "note": "a few MiB per step: bound by latency, not by HBM bandwidth"},
+        "launches_per_step": launches, "gpu_launches": launches * args.steps * n_blocks,
+        "clocks": sampler.summary(t_wall0, t_wall1) if sampler else None, "e2e": None,
+    }
+    del path, prob, flush_buf
+    torch.cuda.empty_cache()
+    return res
+
+
 def run_ours(args):
     from block_sparse_paged_scores_b200 import build as msa_build
     from block_sparse_paged_scores_b200 import msa
@@ -662,6 +732,7 @@ def run_ours(args):
         for name in list(wl.WORKLOADS) + list(VARIANTS):
             if name != args.workload:
                 others[name] = bench_workload(name, args, ws, rank, dev, sampler, False)
+        others["latent_decode"] = bench_latent("latent_decode", args, ws, rank, dev, sampler)
     if sampler:
         sampler.stop()
     if rank != 0:

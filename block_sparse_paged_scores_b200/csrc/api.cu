@@ -679,3 +679,102 @@ msa_status_t msa_select_sparse_attn_paged(
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------- latent sparse attention
+namespace {
+
+constexpr int kLatMaxSplits = 64;
+
+bool leaf_ok(const msa_latent_leaf_t *l, int32_t batch) {
+  return l && l->kv && l->cache_lengths && l->lookup_table && l->max_pages_per_seq >= 1 &&
+         l->num_pages >= 1 && l->num_layers >= 1 && l->layer >= 0 && l->layer < l->num_layers &&
+         aligned(l->kv, 16) && batch >= 1;
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t msa_latent_workspace_bytes(int32_t total_q, int32_t num_heads, int32_t num_splits) {
+  if (total_q < 1 || num_heads < 1 || num_splits <= 1) return 0;
+  const size_t rows = static_cast<size_t>(num_splits) * total_q * num_heads;
+  return round_up(rows * kHeadDim * sizeof(float), 256) + round_up(rows * sizeof(float), 256);
+}
+
+int32_t msa_latent_default_splits(int32_t total_q, int32_t num_heads, int32_t window,
+                                  int32_t n_entries, int32_t num_sms) {
+  if (total_q < 1 || num_heads < 1 || window < 1 || n_entries < 0 || num_sms < 1) return 1;
+  const long long items =
+      static_cast<long long>(total_q) * ((num_heads + latent_rows_per_cta() - 1) /
+                                         latent_rows_per_cta());
+  const long long want = (2LL * num_sms + items - 1) / items;
+  const long long tiles = (static_cast<long long>(window) + n_entries +
+                           latent_tile_positions() - 1) / latent_tile_positions();
+  long long s = std::min<long long>(want, std::max<long long>(1, tiles / 2));
+  s = std::max<long long>(1, std::min<long long>(s, kLatMaxSplits));
+  return static_cast<int32_t>(s);
+}
+
+msa_status_t msa_latent_sparse_attn_paged(
+    const int32_t *input_row_offsets, int32_t batch, int32_t total_q, int32_t max_q_len,
+    const void *q, int32_t num_heads, const msa_latent_leaf_t *swa, int32_t window,
+    const msa_latent_leaf_t *comp, const int32_t *comp_indices, int32_t n_entries,
+    const float *attn_sink, float scale, int32_t num_splits, void *workspace,
+    size_t workspace_bytes, void *out, int32_t *dev_err, struct CUstream_st *stream) {
+  if (!input_row_offsets || batch < 1 || total_q < 0 || max_q_len < 1 || num_heads < 1 ||
+      !leaf_ok(swa, batch) || !leaf_ok(comp, batch) || window < 1 || n_entries < 0 ||
+      (n_entries > 0 && (!comp_indices || !aligned(comp_indices, 4))) || !attn_sink ||
+      !(scale > 0.f) || !isfinite(scale) || num_splits < 0 || num_splits > kLatMaxSplits)
+    return MSA_ERR_INVALID_ARG;
+  if (total_q == 0) return MSA_OK;
+  if (!q || !out || !aligned(q, 16) || !aligned(out, 16)) return MSA_ERR_INVALID_ARG;
+  if ((num_heads + latent_rows_per_cta() - 1) / latent_rows_per_cta() > 65535)
+    return MSA_ERR_UNSUPPORTED;
+  const int splits = num_splits > 0 ? num_splits
+                                    : msa_latent_default_splits(total_q, num_heads, window,
+                                                                n_entries,
+                                                                num_sms_of_current_device());
+  const size_t need = msa_latent_workspace_bytes(total_q, num_heads, splits);
+  if (need > 0 && (!workspace || workspace_bytes < need || !aligned(workspace, 256)))
+    return MSA_ERR_INVALID_ARG;
+  LatentArgs a;
+  a.row_off = input_row_offsets;
+  a.batch = batch;
+  a.total_q = total_q;
+  a.max_q_len = max_q_len;
+  a.q = static_cast<const uint16_t *>(q);
+  a.H = num_heads;
+  a.swa_kv = static_cast<const uint16_t *>(swa->kv);
+  a.swa_len = swa->cache_lengths;
+  a.swa_table = swa->lookup_table;
+  a.swa_pages = swa->num_pages;
+  a.swa_layers = swa->num_layers;
+  a.swa_layer = swa->layer;
+  a.swa_max_pages = swa->max_pages_per_seq;
+  a.window = window;
+  a.comp_kv = static_cast<const uint16_t *>(comp->kv);
+  a.comp_len = comp->cache_lengths;
+  a.comp_table = comp->lookup_table;
+  a.comp_pages = comp->num_pages;
+  a.comp_layers = comp->num_layers;
+  a.comp_layer = comp->layer;
+  a.comp_max_pages = comp->max_pages_per_seq;
+  a.comp_idx = comp_indices;
+  a.n_entries = n_entries;
+  a.sink = attn_sink;
+  a.scale_log2 = scale * 1.4426950408889634f;
+  a.splits = splits;
+  const size_t rows = static_cast<size_t>(splits) * total_q * num_heads;
+  uint8_t *ws = static_cast<uint8_t *>(workspace);
+  a.part_o = need ? reinterpret_cast<float *>(ws) : nullptr;
+  a.part_lse = need ? reinterpret_cast<float *>(ws + round_up(rows * kHeadDim * sizeof(float),
+                                                              256))
+                    : nullptr;
+  a.out = static_cast<uint16_t *>(out);
+  a.dev_err = dev_err;
+  return launch_latent_attention(a, reinterpret_cast<cudaStream_t>(stream)) == cudaSuccess
+             ? MSA_OK
+             : MSA_ERR_CUDA;
+}
+
+}  // extern "C"

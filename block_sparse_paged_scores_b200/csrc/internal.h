@@ -106,6 +106,34 @@ bool attention_tc_supported(int G, int qt);
 cudaError_t launch_attention_tc(const CUtensorMap &kmap, const CUtensorMap &vmap,
                                 const AttnArgs &a, cudaStream_t s);
 
+// ---- latent sparse attention (latent.cu)
+struct LatentArgs {
+  const int32_t *row_off;
+  int batch, total_q, max_q_len;
+  const uint16_t *q;  // bf16 bits [total_q, H, 128]
+  int H;
+  // sliding-window leaf: bf16 [swa_pages, swa_layers, 128, 128], swa_len = prior tokens
+  const uint16_t *swa_kv;
+  const int32_t *swa_len, *swa_table;
+  int swa_pages, swa_layers, swa_layer, swa_max_pages, window;
+  // compressed leaf: bf16 [comp_pages, comp_layers, 128, 128], comp_len = its entries
+  const uint16_t *comp_kv;
+  const int32_t *comp_len, *comp_table;
+  int comp_pages, comp_layers, comp_layer, comp_max_pages;
+  const int32_t *comp_idx;  // [total_q, n_entries], -1 = padding
+  int n_entries;
+  const float *sink;  // [H]
+  float scale_log2;
+  int splits;                // position-list splits (grid.z); 1: the kernel writes `out`
+  float *part_o, *part_lse;  // [splits][total_q][H][128], [splits][total_q][H]
+  uint16_t *out;             // bf16 bits [total_q, H, 128]
+  int32_t *dev_err;
+};
+int latent_rows_per_cta();
+int latent_tile_positions();
+// enqueues the attention and, with more than one split, the combine
+cudaError_t launch_latent_attention(const LatentArgs &a, cudaStream_t s);
+
 // ---- split-K combine (combine.cu)
 cudaError_t launch_combine(const float *part_o, const float *part_lse, int splits, int total_q,
                            int H_q, uint16_t *out, cudaStream_t s);

@@ -51,6 +51,21 @@ def index_k(codes, scales, num_heads: int, idx_dtype: str = "bf16") -> IndexK:
     return IndexK(IDX_DTYPES[idx_dtype], _ptr(codes), _ptr(scales), int(num_heads))
 
 
+class LatentLeaf(ctypes.Structure):
+    """msa_latent_leaf_t: one paged leaf of the latent sparse attention."""
+    _fields_ = [("kv", ctypes.c_void_p), ("cache_lengths", ctypes.c_void_p),
+                ("lookup_table", ctypes.c_void_p), ("max_pages_per_seq", ctypes.c_int32),
+                ("num_pages", ctypes.c_int32), ("num_layers", ctypes.c_int32),
+                ("layer", ctypes.c_int32)]
+
+
+def latent_leaf(kv, cache_lengths, lookup_table, layer: int) -> LatentLeaf:
+    """The msa_latent_leaf_t view of a leaf (kv bf16 [pages, layers, 128, 128]; no copies)."""
+    return LatentLeaf(_ptr(kv), _ptr(cache_lengths), _ptr(lookup_table),
+                      int(lookup_table.shape[-1]), int(kv.shape[0]), int(kv.shape[1]),
+                      int(layer))
+
+
 _lib: Optional[ctypes.CDLL] = None
 
 
@@ -97,6 +112,14 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.msa_attn_partials.restype = I
     lib.msa_attn_partials.argtypes = [RP, I, I, I, I, I, ctypes.POINTER(ctypes.c_size_t),
                                       ctypes.POINTER(ctypes.c_size_t)]
+    LL = ctypes.POINTER(LatentLeaf)
+    lib.msa_latent_sparse_attn_paged.restype = I
+    lib.msa_latent_sparse_attn_paged.argtypes = [P, I, I, I, P, I, LL, I, LL, P, I, P, F, I, P,
+                                                 ctypes.c_size_t, P, P, P]
+    lib.msa_latent_workspace_bytes.restype = ctypes.c_size_t
+    lib.msa_latent_workspace_bytes.argtypes = [I, I, I]
+    lib.msa_latent_default_splits.restype = I
+    lib.msa_latent_default_splits.argtypes = [I, I, I, I, I]
     lib.msa_selftest_bounded_wait.restype = I
     lib.msa_selftest_bounded_wait.argtypes = [ctypes.c_uint32, P, P, P]
     lib.msa_status_string.restype = ctypes.c_char_p
@@ -243,6 +266,61 @@ def msa_sparse_attn_paged_noalloc(rp: RaggedPaged, q, k_cache, v_cache, kv_dtype
         ctypes.byref(rp), _ptr(q), _ptr(k_cache), _ptr(v_cache), int(kv_dtype), _ptr(block_ids),
         _ptr(num_selected), S, num_q_heads, num_kv_heads, max_blocks, float(scale), num_splits,
         _ptr(out), _ptr(dev_err), _stream(stream)))
+
+
+def msa_latent_workspace_bytes(total_q: int, num_heads: int, num_splits: int) -> int:
+    return int(load().msa_latent_workspace_bytes(total_q, num_heads, num_splits))
+
+
+def msa_latent_default_splits(total_q: int, num_heads: int, window: int, n_entries: int,
+                              num_sms: int) -> int:
+    return int(load().msa_latent_default_splits(total_q, num_heads, window, n_entries, num_sms))
+
+
+def msa_latent_sparse_attn_paged(input_row_offsets, batch: int, total_q: int, max_q_len: int,
+                                 q, num_heads: int, swa: LatentLeaf, window: int,
+                                 comp: LatentLeaf, comp_indices, n_entries: int, attn_sink,
+                                 scale: float, num_splits: int, workspace, out, dev_err=None,
+                                 stream=None, workspace_bytes: Optional[int] = None):
+    if workspace_bytes is None:
+        workspace_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _check("msa_latent_sparse_attn_paged", load().msa_latent_sparse_attn_paged(
+        _ptr(input_row_offsets), batch, total_q, max_q_len, _ptr(q), num_heads,
+        ctypes.byref(swa), window, ctypes.byref(comp), _ptr(comp_indices), n_entries,
+        _ptr(attn_sink), float(scale), num_splits, _ptr(workspace), int(workspace_bytes),
+        _ptr(out), _ptr(dev_err), _stream(stream)))
+
+
+class LatentPath:
+    """One latent sparse attention problem (a dict laid out as workload.generate_latent
+    returns) with its output, workspace and error word allocated once; ``run()`` enqueues
+    msa_latent_sparse_attn_paged on the current stream."""
+
+    def __init__(self, prob: dict, num_splits: int = 0):
+        self.p = prob
+        dev = prob["q"].device
+        self.swa = latent_leaf(prob["swa_kv"], prob["swa_len"], prob["swa_table"],
+                               prob["swa_layer"])
+        self.comp = latent_leaf(prob["comp_kv"], prob["comp_len"], prob["comp_table"],
+                                prob["comp_layer"])
+        self.num_splits = num_splits or msa_latent_default_splits(
+            prob["total_q"], prob["H"], prob["window"], prob["n_entries"],
+            torch.cuda.get_device_properties(dev).multi_processor_count)
+        ws = msa_latent_workspace_bytes(prob["total_q"], prob["H"], self.num_splits)
+        self.workspace = torch.empty((max(ws, 1),), dtype=torch.uint8, device=dev)
+        self.workspace_bytes = ws
+        self.out = torch.empty((prob["total_q"], prob["H"], HEAD_DIM), dtype=torch.bfloat16,
+                               device=dev)
+        self.dev_err = torch.zeros((1,), dtype=torch.int32, device=dev)
+
+    def run(self, stream=None):
+        p = self.p
+        msa_latent_sparse_attn_paged(p["row_off"], p["batch"], p["total_q"], p["max_q_len"],
+                                     p["q"], p["H"], self.swa, p["window"], self.comp,
+                                     p["comp_idx"], p["n_entries"], p["sink"], p["scale"],
+                                     self.num_splits, self.workspace, self.out, self.dev_err,
+                                     stream, workspace_bytes=self.workspace_bytes)
+        return self.out
 
 
 def msa_selftest_bounded_wait(limit_us: int, dev_err, result, stream=None):

@@ -365,7 +365,62 @@ MSA_API msa_status_t msa_splitk_combine(const float *partial_o, const float *par
 MSA_API msa_status_t msa_selftest_bounded_wait(uint32_t limit_us, int32_t *dev_err,
                                                uint32_t *result, struct CUstream_st *stream);
 
+/*
+ * msa_latent_sparse_attn_paged — latent sparse attention ([latent] Mojo
+ * "Struct_latent_sparse_attention_ragged_paged": sparse attention over a shared K = V latent
+ * read from two paged leaves, the sliding-window leaf by position range and the compressed
+ * leaf by an explicit per-query entry list, with a per-head attention sink in the
+ * denominator).
+ *
+ *   For query row t = input_row_offsets[b] + i at position p = swa->cache_lengths[b] + i and
+ *   head h:  out[t, h] = sum_x e^(z_x) v_x / (e^(attn_sink[h]) + sum_x e^(z_x)),
+ *   z_x = scale * q[t, h] . v_x, over the latent rows v_x of
+ *     - the window leaf at positions max(0, p - window + 1) .. p (the new tokens' rows are
+ *       already in that leaf), and
+ *     - the compressed leaf at positions comp_indices[t, e] >= 0 (e < n_entries; -1 is
+ *       padding, every listed entry counts); an entry >= comp->cache_lengths[b] sets
+ *       MSA_DEVERR_BLOCK_ID and is skipped.
+ *   Position x of leaf L for sequence b is row x % 128 of page L->lookup_table[b *
+ *   L->max_pages_per_seq + x / 128], layer L->layer.  FP32 accumulation, BF16 output.
+ *
+ *   q            device bf16 [total_q, num_heads, 128], 16-byte aligned
+ *   leaves       msa_latent_leaf_t (below); kv 16-byte aligned
+ *   comp_indices device int32 [total_q, n_entries] (may be NULL when n_entries == 0)
+ *   attn_sink    device f32 [num_heads]
+ *   window >= 1; n_entries >= 0; scale > 0
+ *   num_splits   0 = a count that fills the GPU (msa_latent_default_splits), else 1 .. 64:
+ *                each query's list of rows (window, then entries) is cut into that many equal
+ *                shares; with more than one the partials live in `workspace` (at least
+ *                msa_latent_workspace_bytes bytes, 256-byte aligned) and a combine follows
+ *   out          device bf16 [total_q, num_heads, 128], 16-byte aligned
+ */
+typedef struct {
+    const void *kv;               /* device bf16 [num_pages, num_layers, 128 tokens, 128] */
+    const int32_t *cache_lengths; /* device [batch]: window leaf: prior tokens; compressed
+                                     leaf: its entries */
+    const int32_t *lookup_table;  /* device [batch * max_pages_per_seq], -1 = no page */
+    int32_t max_pages_per_seq;
+    int32_t num_pages;
+    int32_t num_layers;
+    int32_t layer;                /* 0 .. num_layers - 1 */
+} msa_latent_leaf_t;
+
+MSA_API msa_status_t msa_latent_sparse_attn_paged(
+    const int32_t *input_row_offsets, int32_t batch, int32_t total_q, int32_t max_q_len,
+    const void *q, int32_t num_heads, const msa_latent_leaf_t *swa, int32_t window,
+    const msa_latent_leaf_t *comp, const int32_t *comp_indices, int32_t n_entries,
+    const float *attn_sink, float scale, int32_t num_splits, void *workspace,
+    size_t workspace_bytes, void *out, int32_t *dev_err, struct CUstream_st *stream);
+
 /* Host-only helpers (no device work, no CUDA call). */
+
+/* Bytes of `workspace` msa_latent_sparse_attn_paged needs (0 for a single split). */
+MSA_API size_t msa_latent_workspace_bytes(int32_t total_q, int32_t num_heads,
+                                          int32_t num_splits);
+/* The split count msa_latent_sparse_attn_paged uses when num_splits == 0: enough CTAs for two
+ * per SM, at most one share per two 64-row tiles of the longest list and at most 64. */
+MSA_API int32_t msa_latent_default_splits(int32_t total_q, int32_t num_heads, int32_t window,
+                                          int32_t n_entries, int32_t num_sms);
 
 /* Bytes of `workspace` that msa_sparse_attn_paged needs for this shape (0 when none). */
 MSA_API size_t msa_attn_workspace_bytes(const msa_ragged_paged_t *rp, int32_t S,

@@ -39,15 +39,19 @@ def test_digest_ignores_comments_and_layout_but_not_code(bench, tmp_path, monkey
 
 def test_traffic_records_are_complete(bench):
     d = json.load(open(os.path.join(ROOT, "profiles", "traffic.json")))
+    known = set(bench.VARIANTS) | {"bf16_decode", "ragged_prefill", "spec_decode",
+                                   "fp8_long_decode", "tiny_decode"}
     for key, e in d.items():
         kernel, workload = key.split("/")
-        assert workload in ("bf16_decode", "ragged_prefill", "spec_decode", "fp8_long_decode",
-                            "tiny_decode")
+        assert kernel in ("index_scores", "attention") and workload in known
         assert e["dram_bytes_per_launch"] > 0 and e["captured_dram_bytes_per_launch"] > 0
         assert "captured_workload" in e and "source_digest" in e
-    # the bench's dominant kernel on the default workload has a capture of its current code
-    digest = bench.source_digest("attention_stream.cu", "attn_common.cuh", "select_row.cuh")
-    assert bench.profiled_traffic("attention", "bf16_decode", digest) is not None
+    # the committed captures of the attention kernels are of their current code
+    stream = bench.source_digest("attention_stream.cu", "attn_common.cuh", "select_row.cuh")
+    for w in ("bf16_decode", "spec_decode", "spec_decode_shared_topk"):
+        assert bench.profiled_traffic("attention", w, stream) is not None, w
+    assert bench.profiled_traffic("attention", "ragged_prefill",
+                                  bench.source_digest("attention_tc.cu")) is not None
     assert bench.profiled_traffic("attention", "bf16_decode", "0" * 16) is None
 
 
