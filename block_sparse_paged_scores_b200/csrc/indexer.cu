@@ -354,60 +354,94 @@ __global__ void __launch_bounds__(kThreads)
         }
       } else {
         const uint8_t *sc = scale_st + s * kScaleBytes;
+        const uint8_t *tile = stages + s * kTileBytes;
         const int j4 = lane & 3;
+        // the four n-tiles (8 positions each) are interleaved at every k-step so that their
+        // accumulator chains run side by side
+        if constexpr (IF == kIdxFp8) {
 #pragma unroll
-        for (int nt = 0; nt < 4; ++nt) {
-          const int pos = pbase + nt * 8 + (lane >> 2);         // this lane's B column
-          const int c0 = pbase + nt * 8 + 2 * j4;                // its two C columns
-          if constexpr (IF == kIdxFp8) {
+          for (int ks = 0; ks < 8; ++ks) {
+            uint32_t w[4];
 #pragma unroll
-            for (int ks = 0; ks < 8; ++ks) {
-              const uint32_t w = *reinterpret_cast<const uint32_t *>(
-                  stages + s * kTileBytes + sw128(pos, ks, kTileBytes) + 4 * j4);
-              const uint32_t b0 = e4m3x2_to_f16x2(static_cast<uint16_t>(w & 0xffffu));
-              const uint32_t b1 = e4m3x2_to_f16x2(static_cast<uint16_t>(w >> 16));
+            for (int nt = 0; nt < 4; ++nt)
+              w[nt] = *reinterpret_cast<const uint32_t *>(
+                  tile + sw128(pbase + nt * 8 + (lane >> 2), ks, kTileBytes) + 4 * j4);
+#pragma unroll
+            for (int nt = 0; nt < 4; ++nt) {
+              const uint32_t b0 = e4m3x2_to_f16x2(static_cast<uint16_t>(w[nt] & 0xffffu));
+              const uint32_t b1 = e4m3x2_to_f16x2(static_cast<uint16_t>(w[nt] >> 16));
 #pragma unroll
               for (int mt = 0; mt < MT; ++mt) mma_f16(acc[mt][nt], qa[mt][ks], b0, b1);
             }
-            const float2 ts = *reinterpret_cast<const float2 *>(sc + 4 * c0);  // token scales
+          }
+#pragma unroll
+          for (int nt = 0; nt < 4; ++nt) {
+            const float2 ts =
+                *reinterpret_cast<const float2 *>(sc + 4 * (pbase + nt * 8 + 2 * j4));
 #pragma unroll
             for (int mt = 0; mt < MT; ++mt)
 #pragma unroll
               for (int e = 0; e < 4; ++e)
                 acc[mt][nt][e] *= ((e & 1) ? ts.y : ts.x) * qinv[mt][e >> 1];
-          } else {
-            const uint32_t ex0 = *reinterpret_cast<const uint32_t *>(sc + 4 * c0);
-            const uint32_t ex1 = *reinterpret_cast<const uint32_t *>(sc + 4 * c0 + 4);
+          }
+        } else {
+          // exponents of the two C columns of every n-tile: 4 bytes (groups) per position
+          uint32_t ex[4][2];
+#pragma unroll
+          for (int nt = 0; nt < 4; ++nt) {
+            const uint2 e2 =
+                *reinterpret_cast<const uint2 *>(sc + 4 * (pbase + nt * 8 + 2 * j4));
+            ex[nt][0] = e2.x;
+            ex[nt][1] = e2.y;
+          }
+          // NP n-tiles at a time (all four with one 16-row tile, two with two: registers)
+          constexpr int NP = MT == 1 ? 4 : 2;
+#pragma unroll
+          for (int n0 = 0; n0 < 4; n0 += NP)
 #pragma unroll
             for (int gq = 0; gq < 4; ++gq) {
-              const uint32_t w = *reinterpret_cast<const uint32_t *>(
-                  stages + s * kTileBytes + sw128(pos >> 1, 4 * (pos & 1) + gq, kTileBytes) +
-                  4 * j4);
-              float cg[MT][4];
+              uint32_t w[NP];
 #pragma unroll
-              for (int mt = 0; mt < MT; ++mt)
-#pragma unroll
-                for (int e = 0; e < 4; ++e) cg[mt][e] = 0.f;
-#pragma unroll
-              for (int h = 0; h < 2; ++h) {
-                const uint32_t b0 = e2m1x2_to_f16x2((w >> (16 * h)) & 0xffu);
-                const uint32_t b1 = e2m1x2_to_f16x2((w >> (16 * h + 8)) & 0xffu);
-#pragma unroll
-                for (int mt = 0; mt < MT; ++mt) mma_f16(cg[mt], qa[mt][2 * gq + h], b0, b1);
+              for (int u = 0; u < NP; ++u) {
+                const int pos = pbase + (n0 + u) * 8 + (lane >> 2);
+                w[u] = *reinterpret_cast<const uint32_t *>(
+                    tile + sw128(pos >> 1, 4 * (pos & 1) + gq, kTileBytes) + 4 * j4);
               }
-              const float e0 = ue8m0_to_float((ex0 >> (8 * gq)) & 0xffu);
-              const float e1 = ue8m0_to_float((ex1 >> (8 * gq)) & 0xffu);
+              float cg[MT][NP][4];
 #pragma unroll
               for (int mt = 0; mt < MT; ++mt)
 #pragma unroll
-                for (int e = 0; e < 4; ++e)
-                  acc[mt][nt][e] = fmaf(cg[mt][e], (e & 1) ? e1 : e0, acc[mt][nt][e]);
+                for (int u = 0; u < NP; ++u)
+#pragma unroll
+                  for (int e = 0; e < 4; ++e) cg[mt][u][e] = 0.f;
+#pragma unroll
+              for (int h = 0; h < 2; ++h)
+#pragma unroll
+                for (int u = 0; u < NP; ++u) {
+                  const uint32_t b0 = e2m1x2_to_f16x2((w[u] >> (16 * h)) & 0xffu);
+                  const uint32_t b1 = e2m1x2_to_f16x2((w[u] >> (16 * h + 8)) & 0xffu);
+#pragma unroll
+                  for (int mt = 0; mt < MT; ++mt)
+                    mma_f16(cg[mt][u], qa[mt][2 * gq + h], b0, b1);
+                }
+#pragma unroll
+              for (int u = 0; u < NP; ++u) {
+                const int nt = n0 + u;
+                const float e0 = ue8m0_to_float((ex[nt][0] >> (8 * gq)) & 0xffu);
+                const float e1 = ue8m0_to_float((ex[nt][1] >> (8 * gq)) & 0xffu);
+#pragma unroll
+                for (int mt = 0; mt < MT; ++mt)
+#pragma unroll
+                  for (int e = 0; e < 4; ++e)
+                    acc[mt][nt][e] = fmaf(cg[mt][u][e], (e & 1) ? e1 : e0, acc[mt][nt][e]);
+              }
             }
 #pragma unroll
-            for (int mt = 0; mt < MT; ++mt)
+          for (int mt = 0; mt < MT; ++mt)
+#pragma unroll
+            for (int nt = 0; nt < 4; ++nt)
 #pragma unroll
               for (int e = 0; e < 4; ++e) acc[mt][nt][e] *= qinv[mt][e >> 1];
-          }
         }
       }
     }

@@ -46,7 +46,11 @@ def test_traffic_records_are_complete(bench):
         assert kernel in ("index_scores", "attention") and workload in known
         assert e["dram_bytes_per_launch"] > 0 and e["captured_dram_bytes_per_launch"] > 0
         assert "captured_workload" in e and "source_digest" in e
-    # the committed captures of the attention kernels are of their current code
+    # the headline's dominant kernel (the indexer on FP8 long-context decode) and the attention
+    # kernels have committed captures of their current code
+    index = bench.source_digest("indexer.cu", "select_row.cuh")
+    for w in ("fp8_long_decode", "fp8_long_decode_fp8_index_k", "fp8_long_decode_fp4_index_k"):
+        assert bench.profiled_traffic("index_scores", w, index) is not None, w
     stream = bench.source_digest("attention_stream.cu", "attn_common.cuh", "select_row.cuh")
     for w in ("bf16_decode", "spec_decode", "spec_decode_shared_topk"):
         assert bench.profiled_traffic("attention", w, stream) is not None, w
