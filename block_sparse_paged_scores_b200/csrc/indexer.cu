@@ -53,9 +53,11 @@ constexpr uint32_t tile_bytes() {
 }
 template <int IF>
 constexpr uint32_t scale_bytes() { return IF == kIdxBf16 ? 0u : 512u; }
-// The ring keeps the same bytes in flight for every format: smaller tiles, more stages.
+// Ring depth of the scaled formats: 3 fp8 / 6 fp4 stages (about 50 KiB), so that four CTAs fit
+// on an SM (their registers allow four): more consumer warps to hide the conversion chains'
+// latency, about the same bytes in flight as the bf16 ring.
 template <int ST, int IF>
-constexpr int ring_stages() { return ST * static_cast<int>(32768u / tile_bytes<IF>()); }
+constexpr int ring_stages() { return IF == kIdxBf16 ? ST : (IF == kIdxFp8 ? 3 : 6); }
 
 template <int kStages, int IF>
 constexpr size_t smem_bytes() {
@@ -120,8 +122,10 @@ __device__ __forceinline__ void count_out_and_select(const IndexerArgs &a, int b
 
 // KPL < 0: scores only; KPL >= 0: selection fused, KPL keys per lane in registers (0: any
 // number of blocks, read from L2 on every pass).
+// With one 16-row tile the scaled formats are bounded to four CTAs per SM (registers <= 102
+// per thread; two tiles would spill).
 template <int MT, int KPL, int kStages, int IF>
-__global__ void __launch_bounds__(kThreads)
+__global__ void __launch_bounds__(kThreads, (IF != kIdxBf16 && MT == 1) ? 4 : 1)
     index_scores_kernel(const __grid_constant__ CUtensorMap kmap, const IndexerArgs a) {
   constexpr uint32_t kTileBytes = tile_bytes<IF>();
   constexpr uint32_t kScaleBytes = scale_bytes<IF>();
@@ -368,8 +372,8 @@ __global__ void __launch_bounds__(kThreads)
                   tile + sw128(pbase + nt * 8 + (lane >> 2), ks, kTileBytes) + 4 * j4);
 #pragma unroll
             for (int nt = 0; nt < 4; ++nt) {
-              const uint32_t b0 = e4m3x2_to_f16x2(static_cast<uint16_t>(w[nt] & 0xffffu));
-              const uint32_t b1 = e4m3x2_to_f16x2(static_cast<uint16_t>(w[nt] >> 16));
+              uint32_t b0, b1;
+              e4m3x4_to_f16x2x2(w[nt], b0, b1);
 #pragma unroll
               for (int mt = 0; mt < MT; ++mt) mma_f16(acc[mt][nt], qa[mt][ks], b0, b1);
             }
@@ -414,16 +418,16 @@ __global__ void __launch_bounds__(kThreads)
                 for (int u = 0; u < NP; ++u)
 #pragma unroll
                   for (int e = 0; e < 4; ++e) cg[mt][u][e] = 0.f;
+              uint32_t bf[NP][4];
+#pragma unroll
+              for (int u = 0; u < NP; ++u) e2m1x8_to_f16x2x4(w[u], bf[u]);
 #pragma unroll
               for (int h = 0; h < 2; ++h)
 #pragma unroll
-                for (int u = 0; u < NP; ++u) {
-                  const uint32_t b0 = e2m1x2_to_f16x2((w[u] >> (16 * h)) & 0xffu);
-                  const uint32_t b1 = e2m1x2_to_f16x2((w[u] >> (16 * h + 8)) & 0xffu);
+                for (int u = 0; u < NP; ++u)
 #pragma unroll
                   for (int mt = 0; mt < MT; ++mt)
-                    mma_f16(cg[mt][u], qa[mt][2 * gq + h], b0, b1);
-                }
+                    mma_f16(cg[mt][u], qa[mt][2 * gq + h], bf[u][2 * h], bf[u][2 * h + 1]);
 #pragma unroll
               for (int u = 0; u < NP; ++u) {
                 const int nt = n0 + u;
