@@ -395,6 +395,11 @@ VARIANTS = {
     "fp8_long_decode_fp8_index_k": ("fp8_long_decode", dict(idx_dtype="fp8"), {}),
     "fp8_long_decode_fp4_index_k": ("fp8_long_decode", dict(idx_dtype="fp4"), {}),
     "spec_decode_shared_topk": ("spec_decode", {}, dict(share_selection=True)),
+    # ragged prefill whose index queries are coherent across neighbouring tokens (a 256-token
+    # moving average of N(0,1) draws, neighbour correlation about 0.996): the tokens of a tile
+    # select similar blocks, as the queries of a trained model do, instead of independent
+    # random sets
+    "ragged_prefill_coherent_queries": ("ragged_prefill", dict(q_idx_window=256), {}),
 }
 
 

@@ -57,6 +57,9 @@ class WorkloadSpec:
     pool_pages: int = 0        # minimum pool size (extra pages stay unused and poisoned)
     idx_dtype: str = "bf16"    # index-K cache: "bf16" | "fp8" (e4m3 + f32 scale per token)
                                # | "fp4" (e2m1 + ue8m0 exponent per 32 elements)
+    q_idx_window: int = 0      # > 1: each sequence's index queries are the moving average of
+                               # that many consecutive N(0,1) draws (times sqrt(window): unit
+                               # variance), so that neighbouring tokens' queries are coherent
 
     @property
     def H_q(self) -> int:
@@ -187,7 +190,20 @@ def generate(spec: WorkloadSpec, seed: int, device="cpu", poison: bool = True) -
     bf16 = torch.bfloat16
     kvt = torch.float8_e4m3fn if spec.kv_dtype == "fp8" else bf16
     q = torch.randn((total_q, spec.H_q, HEAD_DIM), generator=gdev, device=device).to(bf16)
-    q_idx = torch.randn((total_q, spec.H_kv, HEAD_DIM), generator=gdev, device=device).to(bf16)
+    q_idx = torch.randn((total_q, spec.H_kv, HEAD_DIM), generator=gdev, device=device)
+    if spec.q_idx_window > 1:
+        w = spec.q_idx_window
+        coh = torch.empty_like(q_idx)
+        for b in range(spec.batch):
+            r0, r1 = int(row_off[b]), int(row_off[b + 1])
+            if r1 == r0:
+                continue
+            e = torch.randn((r1 - r0 + w - 1, spec.H_kv, HEAD_DIM), generator=gdev,
+                            device=device, dtype=torch.float64)
+            c = torch.cat([torch.zeros_like(e[:1]), torch.cumsum(e, 0)])
+            coh[r0:r1] = ((c[w:] - c[:-w]) / math.sqrt(w)).float()
+        q_idx = coh
+    q_idx = q_idx.to(bf16)
     k_idx = _normal_pages((pool, spec.H_idxk, BLOCK, HEAD_DIM), gdev, device, bf16)
     k = _normal_pages((pool, spec.H_kv, BLOCK, HEAD_DIM), gdev, device, kvt)
     v = _normal_pages((pool, spec.H_kv, BLOCK, HEAD_DIM), gdev, device, kvt)
