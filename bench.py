@@ -400,6 +400,9 @@ VARIANTS = {
     # select similar blocks, as the queries of a trained model do, instead of independent
     # random sets
     "ragged_prefill_coherent_queries": ("ragged_prefill", dict(q_idx_window=256), {}),
+    # ragged prefill over a scale-free FP8 e4m3 KV cache (the tcgen05 kernel converts the tiles
+    # to f16 in shared memory)
+    "ragged_prefill_fp8_kv": ("ragged_prefill", dict(kv_dtype="fp8"), {}),
 }
 
 
@@ -489,8 +492,7 @@ def bench_workload(name, args, ws, rank, dev, sampler, with_cpu):
         else:
             groups[attn_key] = lambda: path.attend(stream=stream)
         attn_src = (("attention_stream.cu", "attn_common.cuh", "select_row.cuh")
-                    if stream_route else
-                    (("attention_tile.cu", "attn_common.cuh") if fp8 else ("attention_tc.cu",)))
+                    if stream_route else ("attention_tc.cu",))
     idx_src = (("indexer.cu", "select_row.cuh")
                if stream_route or prob["idx_dtype"] != "bf16" else ("indexer_tc.cu",))
     st = stage_times(list(groups.values()), args.steps, stream, args.stage_seconds)
@@ -520,7 +522,7 @@ def bench_workload(name, args, ws, rank, dev, sampler, with_cpu):
                     "note": "algorithmic FLOPs (selected, causally clipped positions only) over "
                             "the launch group's median time, against the measured bf16 burst "
                             "peak"}
-        if dom != idx_key and not fp8:
+        if dom != idx_key:
             ex = executed_flops_tiles(prob, path.block_ids, path.num_selected, 128 // G)
             roofline["executed_flops_per_launch"] = ex
             roofline["executed_tflops"] = ex / (d_ms * 1e-3) / 1e12

@@ -124,7 +124,7 @@ bool make_route(const msa_ragged_paged_t *rp, int S, int H_q, int H_kv, int max_
   const int G = H_q / H_kv;
   r->plan = rp->max_q_len > 1;
   r->stream = rp->max_q_len <= MSA_MAX_SPEC_DRAFT;
-  r->tc = !r->stream && !fp8 && G <= 128 && attention_tc_supported(G, std::max(1, 128 / G));
+  r->tc = !r->stream && G <= 128 && attention_tc_supported(G, std::max(1, 128 / G));
   if (!r->plan) {
     r->qt = 1;
   } else {
@@ -614,7 +614,7 @@ msa_status_t attn_impl(const msa_ragged_paged_t *rp, const void *q, const void *
   a.init_blocks = sel ? sel->init_blocks : 0;
   a.local_blocks = sel ? sel->local_blocks : 0;
   if (r.tc)
-    return launch_attention_tc(kmap, vmap, a, s) == cudaSuccess ? MSA_OK : MSA_ERR_CUDA;
+    return launch_attention_tc(kmap, vmap, a, fp8, s) == cudaSuccess ? MSA_OK : MSA_ERR_CUDA;
   if (!r.stream)
     return launch_attention_tiles(kmap, vmap, a, fp8, r.rg, s) == cudaSuccess ? MSA_OK
                                                                              : MSA_ERR_CUDA;

@@ -44,7 +44,10 @@ namespace {
 constexpr int kTcRows = 128;                     // MMA M: query rows of the tile
 constexpr uint32_t kTcTile = 32768;              // one (page, head) bf16 tile
 constexpr uint32_t kTcHalf = 16384;              // one swizzled [128][128 B] box
-constexpr int kKStages = 3;
+constexpr uint32_t kTc8Tile = 16384;             // one (page, head) e4m3 tile
+constexpr int k8Stages = 2;                       // e4m3 staging tiles per operand (FP8 KV)
+template <bool F8>
+constexpr int k_stages() { return F8 ? 2 : 3; }   // K ring (f16 tiles for FP8 KV)
 constexpr int kVStages = 2;
 constexpr uint32_t kTcQBytes = 2 * kTcHalf;      // Q: 128 rows x 128 dims bf16
 constexpr uint32_t kTcCols = 512;                // TMEM columns allocated
@@ -62,17 +65,47 @@ static_assert(128 * kRegsRoles + 256 * kRegsSoftmax <= kTcThreads * kRegsLaunch,
               "register split must fit in the launch's registers");
 constexpr float kLazyLog2 = 8.f;                 // rescale only when the max grows by > 2^8
 
+// FP8 KV adds the e4m3 staging tiles and keeps the epilogue's reduction buffers in the K
+// staging (free by then); 225 KiB.
+template <bool F8>
 constexpr size_t tc_smem_bytes() {
-  return 1024 + (kKStages + kVStages) * kTcTile + kTcQBytes +
-         (2 * kKStages + 2 * kVStages + 2 * 3 + 1) * sizeof(uint64_t) +
-         2 * 2 * kTcRows * sizeof(float) + 64;
+  return 1024 + (k_stages<F8>() + kVStages) * kTcTile + (F8 ? 2 * k8Stages * kTc8Tile : 0) +
+         kTcQBytes +
+         (2 * k_stages<F8>() + 2 * kVStages + (F8 ? 4 * k8Stages : 0) + 2 * 3 + 1) *
+             sizeof(uint64_t) +
+         (F8 ? 0 : 2 * 2 * kTcRows * sizeof(float)) + 64;
 }
+static_assert(tc_smem_bytes<true>() <= 232448 && tc_smem_bytes<false>() <= 232448,
+              "shared memory per CTA");
 
 // S = Q K^T: A = Q (K-major, 128 rows), B = K tile (K-major, 128 positions), K = 128 dims.
 // O += P V: A = P (TMEM), B = V tile (N-major: 128 dims contiguous in two 64-dim boxes 16 KiB
 // apart; 8-position groups 1 KiB apart).
-constexpr uint32_t kIdescQK = umma_idesc_bf16(128, 128, false);
-constexpr uint32_t kIdescPV = umma_idesc_bf16(128, 128, true);
+template <bool F8>
+constexpr uint32_t idesc_qk() { return F8 ? umma_idesc_f16(128, 128, false) : umma_idesc_bf16(128, 128, false); }
+template <bool F8>
+constexpr uint32_t idesc_pv() { return F8 ? umma_idesc_f16(128, 128, true) : umma_idesc_bf16(128, 128, true); }
+
+// Q rows (tok * G + head) as f16 in the MMA's K-major swizzled layout, dims in their natural
+// order (the FP8-KV tiles: f16 operands; a q value outside f16's range is rounded as cvt does).
+__device__ __forceinline__ void stage_q_f16(uint8_t *qs, const uint16_t *q, int t0, int rows,
+                                            int G, int H_q, int g, int tid, int nthreads) {
+  constexpr uint32_t sub = kTcRows * 128;
+  for (int idx = tid; idx < kTcRows * 16; idx += nthreads) {
+    const int r = idx >> 4, c = idx & 15;  // 8 dims (one 16-byte chunk) of row r
+    uint4 o = make_uint4(0, 0, 0, 0);
+    if (r < rows) {
+      const int t = t0 + r / G, h = g * G + r % G;
+      const uint4 x = *reinterpret_cast<const uint4 *>(
+          q + (static_cast<size_t>(t) * H_q + h) * kHeadDim + c * 8);
+      const float2 f0 = bf16x2_to_float2(x.x), f1 = bf16x2_to_float2(x.y);
+      const float2 f2 = bf16x2_to_float2(x.z), f3 = bf16x2_to_float2(x.w);
+      o = make_uint4(pack_f16x2(f0.x, f0.y), pack_f16x2(f1.x, f1.y), pack_f16x2(f2.x, f2.y),
+                     pack_f16x2(f3.x, f3.y));
+    }
+    *reinterpret_cast<uint4 *>(qs + sw128(r, c, sub)) = o;
+  }
+}
 
 __device__ __forceinline__ uint64_t kmajor_desc(uint32_t base, int kstep) {
   // 16 bf16 of K per step: steps 0-3 inside the first 64-column box, 4-7 in the second
@@ -85,9 +118,13 @@ __device__ __forceinline__ uint64_t nmajor_desc(uint32_t base, int kstep) {
 // TMEM column of P's 16-position K-slice `kstep` in group `w`'s S/P buffer
 __device__ __forceinline__ uint32_t p_col(int w, int kstep) { return w * 128 + kstep * 8; }
 
+template <bool F8>
 __global__ void __launch_bounds__(kTcThreads, 1)
     attn_tc_kernel(const __grid_constant__ CUtensorMap kmap,
                    const __grid_constant__ CUtensorMap vmap, const AttnArgs a) {
+  constexpr int kKStages = k_stages<F8>();
+  constexpr uint32_t kIdescQK = idesc_qk<F8>();
+  constexpr uint32_t kIdescPV = idesc_pv<F8>();
   pdl_wait();
   pdl_launch_dependents();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -132,18 +169,27 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                                               ~static_cast<uintptr_t>(1023));
   uint8_t *kst = smem;                                  // [3] K tiles
   uint8_t *vst = kst + kKStages * kTcTile;              // [2] V tiles
-  uint8_t *qs = vst + kVStages * kTcTile;               // Q, K-major SW128
+  uint8_t *k8st = vst + kVStages * kTcTile;             // FP8 KV: [2] e4m3 K tiles
+  uint8_t *v8st = k8st + (F8 ? k8Stages * kTc8Tile : 0);  // FP8 KV: [2] e4m3 V tiles
+  uint8_t *qs = v8st + (F8 ? k8Stages * kTc8Tile : 0);    // Q, K-major SW128
   uint64_t *k_full = reinterpret_cast<uint64_t *>(qs + kTcQBytes);
   uint64_t *k_empty = k_full + kKStages;
   uint64_t *v_full = k_empty + kKStages;
   uint64_t *v_empty = v_full + kVStages;
-  uint64_t *s_full = v_empty + kVStages;  // [2 groups] S of the group's block written
+  uint64_t *k8_full = v_empty + kVStages;  // FP8 KV: staging tile landed / converted
+  uint64_t *k8_empty = k8_full + (F8 ? k8Stages : 0);
+  uint64_t *v8_full = k8_empty + (F8 ? k8Stages : 0);
+  uint64_t *v8_empty = v8_full + (F8 ? k8Stages : 0);
+  uint64_t *s_full = v8_empty + (F8 ? k8Stages : 0);  // [2 groups] S of the group's block
   uint64_t *p_full = s_full + 2;          // [2 groups] P of the group's block written
   uint64_t *o_done = p_full + 2;          // [2 groups] the group's P V done
   uint64_t *mma_done = o_done + 2;
-  float *red_m = reinterpret_cast<float *>(mma_done + 1);  // [2 groups][128]
-  float *red_l = red_m + 2 * kTcRows;                      // [2 groups][128]
-  uint32_t *tmem_base_s = reinterpret_cast<uint32_t *>(red_l + 2 * kTcRows);
+  // [2 groups][128] each, for the epilogue (FP8 KV: in the K staging, free by then)
+  float *red_m = F8 ? reinterpret_cast<float *>(k8st) : reinterpret_cast<float *>(mma_done + 1);
+  float *red_l = red_m + 2 * kTcRows;
+  uint32_t *tmem_base_s =
+      reinterpret_cast<uint32_t *>(F8 ? reinterpret_cast<uint8_t *>(mma_done + 1)
+                                      : reinterpret_cast<uint8_t *>(red_l + 2 * kTcRows));
   volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_base_s + 1);
 
   if (threadIdx.x == 0) {
@@ -155,6 +201,13 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       mbar_init(&v_full[s], 1);
       mbar_init(&v_empty[s], 1);
     }
+    if (F8)
+      for (int s = 0; s < k8Stages; ++s) {
+        mbar_init(&k8_full[s], 1);
+        mbar_init(&k8_empty[s], 1);
+        mbar_init(&v8_full[s], 1);
+        mbar_init(&v8_empty[s], 1);
+      }
     for (int w = 0; w < 2; ++w) {
       mbar_init(&s_full[w], 1);
       mbar_init(&p_full[w], kSoftWarps / 2);
@@ -169,7 +222,10 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     tmem_relinquish();
   }
   // Q rows (tok * G + head) into shared memory in the MMA's K-major swizzled layout
-  stage_q<false, kTcRows>(qs, a.q, t0, rows, a.G, a.H_q, g, threadIdx.x, blockDim.x);
+  if constexpr (F8)
+    stage_q_f16(qs, a.q, t0, rows, a.G, a.H_q, g, threadIdx.x, blockDim.x);
+  else
+    stage_q<false, kTcRows>(qs, a.q, t0, rows, a.G, a.H_q, g, threadIdx.x, blockDim.x);
   fence_async_shared();
   tc_fence_before();
   __syncthreads();
@@ -179,7 +235,96 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   if (warp < 4) {
   // warpgroup 0: the roles, on few registers (each branch keeps its own budget to the end)
   asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegsRoles));
-  if (warp == 0 || warp == kVWarp) {
+  if (F8 && warp == 0) {
+    // ============================================================== e4m3 K and V producer
+    if (lane == 0) {
+      prefetch_tmap(&kmap);
+      prefetch_tmap(&vmap);
+    }
+    bool dead = false;
+    for (int base = 0; base < nblk && !dead; base += 32) {
+      int j = -1, page = -1;
+      if (base + lane < nblk) {
+        j = list[base + lane];
+        if (j >= 0 && j < a.max_blocks) page = a.table[static_cast<size_t>(b) * a.max_pages + j];
+      }
+      const int cnt = min(32, nblk - base);
+      for (int k = 0; k < cnt && !dead; ++k) {
+        const int jj = __shfl_sync(0xffffffffu, j, k);
+        const int pg = __shfl_sync(0xffffffffu, page, k);
+        if (lane == 0) {
+          const int i = base + k;
+          const int s8 = i % k8Stages;
+          const bool jok = jj >= 0 && jj < a.max_blocks;
+          const bool ok = jok && pg >= 0 && pg < a.num_pages;
+          if (!ok) report(a.dev_err, jok ? MSA_DEVERR_PAGE_ID : MSA_DEVERR_BLOCK_ID);
+          for (int op = 0; op < 2 && !dead; ++op) {  // K, then V
+            uint64_t *full8 = op ? v8_full : k8_full, *empty8 = op ? v8_empty : k8_empty;
+            uint8_t *dst = (op ? v8st : k8st) + s8 * kTc8Tile;
+            if (i >= k8Stages && !mbar_wait(&empty8[s8], ((i / k8Stages) - 1) & 1, abort_flag)) {
+              report(a.dev_err, MSA_DEVERR_TIMEOUT);
+              *abort_flag = 1;
+              dead = true;
+            } else if (ok) {
+              mbar_arrive_expect_tx(&full8[s8], kTc8Tile);
+              tma_load_3d(dst, op ? &vmap : &kmap, &full8[s8], 0, 0, pg * a.H_kv + g);
+            } else {
+              // an unusable page: zeros, so that its block adds nothing (scores masked too)
+              uint4 *z = reinterpret_cast<uint4 *>(dst);
+              for (uint32_t w = 0; w < kTc8Tile / 16; ++w) z[w] = make_uint4(0, 0, 0, 0);
+              fence_async_shared();
+              mbar_arrive(&full8[s8]);
+            }
+          }
+        }
+        dead = __shfl_sync(0xffffffffu, dead, 0);
+      }
+    }
+  } else if (F8 && (warp == 2 || warp == 3)) {
+    // ============================================================== e4m3 -> f16 converters
+    // warp 3 converts K tiles, warp 2 V tiles, from the staging ring into the f16 ring in the
+    // layout a TMA load of a bf16 tile gives (two 128-byte-swizzled 64-dim boxes); one cvt per
+    // two codes, exact.
+    const bool is_k = warp == 3;
+    uint8_t *stg = is_k ? k8st : v8st;
+    uint64_t *full8 = is_k ? k8_full : v8_full, *empty8 = is_k ? k8_empty : v8_empty;
+    uint8_t *ring = is_k ? kst : vst;
+    uint64_t *full = is_k ? k_full : v_full, *empty = is_k ? k_empty : v_empty;
+    const int nst = is_k ? kKStages : kVStages;
+    for (int i = 0; i < nblk; ++i) {
+      const int s8 = i % k8Stages, s = i % nst;
+      bool ok = mbar_wait(&full8[s8], (i / k8Stages) & 1, abort_flag);
+      if (ok && i >= nst) ok = mbar_wait(&empty[s], ((i / nst) - 1) & 1, abort_flag);
+      if (!__all_sync(0xffffffffu, ok)) {
+        if (lane == 0) {
+          report(a.dev_err, MSA_DEVERR_TIMEOUT);
+          *abort_flag = 1;
+        }
+        break;
+      }
+      tc_fence_after();
+      const uint8_t *src = stg + s8 * kTc8Tile;
+      uint8_t *dst = ring + s * kTcTile;
+#pragma unroll 4
+      for (int k = 0; k < 32; ++k) {
+        const int task = lane + 32 * k, r = task >> 3, c = task & 7;  // 16 codes: dims 16c ..
+        const uint4 x = *reinterpret_cast<const uint4 *>(src + sw128(r, c, kTc8Tile));
+        uint4 lo, hi;
+        e4m3x4_to_f16x2x2(x.x, lo.x, lo.y);
+        e4m3x4_to_f16x2x2(x.y, lo.z, lo.w);
+        e4m3x4_to_f16x2x2(x.z, hi.x, hi.y);
+        e4m3x4_to_f16x2x2(x.w, hi.z, hi.w);
+        *reinterpret_cast<uint4 *>(dst + sw128(r, 2 * c, kTcHalf)) = lo;
+        *reinterpret_cast<uint4 *>(dst + sw128(r, 2 * c + 1, kTcHalf)) = hi;
+      }
+      fence_async_shared();  // the f16 tile, before the MMA (async proxy) reads it
+      __syncwarp();
+      if (lane == 0) {
+        mbar_arrive(&full[s]);
+        mbar_arrive(&empty8[s8]);
+      }
+    }
+  } else if (!F8 && (warp == 0 || warp == kVWarp)) {
     // ============================================================== K or V producer
     const bool is_k = warp == 0;
     const CUtensorMap *map = is_k ? &kmap : &vmap;
@@ -415,9 +560,15 @@ __global__ void __launch_bounds__(kTcThreads, 1)
               const float2 x = fma2(make_float2(__uint_as_float(v[64 * h + e]),
                                                 __uint_as_float(v[64 * h + e + 1])),
                                     make_float2(sc, sc), make_float2(nb, nb));
-              const uint32_t pb = pack_bf16x2(fast_exp2(x.x), fast_exp2(x.y));
-              pk[e >> 1] = pb;
-              ps2[(e >> 1) & 3] = add2(ps2[(e >> 1) & 3], bf16x2_to_float2(pb));
+              if constexpr (F8) {  // f16 P; its rounding (2^-11) is left out of the sum
+                const float e0 = fast_exp2(x.x), e1 = fast_exp2(x.y);
+                pk[e >> 1] = pack_f16x2(e0, e1);
+                ps2[(e >> 1) & 3] = add2(ps2[(e >> 1) & 3], make_float2(e0, e1));
+              } else {
+                const uint32_t pb = pack_bf16x2(fast_exp2(x.x), fast_exp2(x.y));
+                pk[e >> 1] = pb;
+                ps2[(e >> 1) & 3] = add2(ps2[(e >> 1) & 3], bf16x2_to_float2(pb));
+              }
             }
           } else {
 #pragma unroll
@@ -428,9 +579,10 @@ __global__ void __launch_bounds__(kTcThreads, 1)
               const float x1 = (use && pe + 1 <= lim)
                                    ? fmaf(__uint_as_float(v[pe + 1]), sc, nb)
                                    : -INFINITY;
-              const uint32_t pb = pack_bf16x2(fast_exp2(x0), fast_exp2(x1));
+              const float e0 = fast_exp2(x0), e1 = fast_exp2(x1);
+              const uint32_t pb = F8 ? pack_f16x2(e0, e1) : pack_bf16x2(e0, e1);
               pk[e >> 1] = pb;
-              const float2 pf = bf16x2_to_float2(pb);
+              const float2 pf = F8 ? make_float2(e0, e1) : bf16x2_to_float2(pb);
               ps4[(e >> 1) & 3] += pf.x + pf.y;
             }
           }
@@ -535,12 +687,9 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   if (warp == 1) tmem_dealloc(tbase, kTcCols);
 }
 
-}  // namespace
-
-bool attention_tc_supported(int G, int qt) { return qt * G <= kTcRows && qt <= 32; }
-
-cudaError_t launch_attention_tc(const CUtensorMap &kmap, const CUtensorMap &vmap,
-                                const AttnArgs &a, cudaStream_t s) {
+template <bool F8>
+cudaError_t launch_tc(const CUtensorMap &kmap, const CUtensorMap &vmap, const AttnArgs &a,
+                      cudaStream_t s) {
   // The register split is only valid for a launch with exactly kRegsLaunch registers per
   // thread (a larger split than the launch holds would wait forever): checked once per device.
   static int checked[64] = {0};
@@ -548,18 +697,28 @@ cudaError_t launch_attention_tc(const CUtensorMap &kmap, const CUtensorMap &vmap
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
   if (!checked[dev]) {
     cudaFuncAttributes fa;
-    cudaError_t e = cudaFuncGetAttributes(&fa, reinterpret_cast<const void *>(&attn_tc_kernel));
+    cudaError_t e =
+        cudaFuncGetAttributes(&fa, reinterpret_cast<const void *>(&attn_tc_kernel<F8>));
     if (e != cudaSuccess) return e;
     if (fa.numRegs != kRegsLaunch || fa.maxThreadsPerBlock < kTcThreads)
       return cudaErrorInvalidConfiguration;
     checked[dev] = 1;
   }
-  const size_t smem = tc_smem_bytes();
-  cudaError_t e = ensure_smem_limit(reinterpret_cast<const void *>(&attn_tc_kernel),
+  const size_t smem = tc_smem_bytes<F8>();
+  cudaError_t e = ensure_smem_limit(reinterpret_cast<const void *>(&attn_tc_kernel<F8>),
                                     static_cast<int>(smem));
   if (e != cudaSuccess) return e;
   const dim3 grid(a.batch * a.tiles, a.H_kv);
-  return launch_pdl(attn_tc_kernel, grid, dim3(kTcThreads), smem, s, kmap, vmap, a);
+  return launch_pdl(attn_tc_kernel<F8>, grid, dim3(kTcThreads), smem, s, kmap, vmap, a);
+}
+
+}  // namespace
+
+bool attention_tc_supported(int G, int qt) { return qt * G <= kTcRows && qt <= 32; }
+
+cudaError_t launch_attention_tc(const CUtensorMap &kmap, const CUtensorMap &vmap,
+                                const AttnArgs &a, bool fp8, cudaStream_t s) {
+  return fp8 ? launch_tc<true>(kmap, vmap, a, s) : launch_tc<false>(kmap, vmap, a, s);
 }
 
 }  // namespace msa

@@ -101,10 +101,11 @@ cudaError_t launch_attention_stream(const CUtensorMap &kmap, const CUtensorMap &
                                     cudaStream_t s);
 cudaError_t launch_attention_tiles(const CUtensorMap &kmap, const CUtensorMap &vmap,
                                    const AttnArgs &a, bool fp8, int rg, cudaStream_t s);
-// prefill on tcgen05 (attention_tc.cu): BF16 KV, tiles of qt tokens x G heads <= 128 rows
+// prefill on tcgen05 (attention_tc.cu): tiles of qt tokens x G heads <= 128 rows; BF16 KV, or
+// e4m3 KV converted to f16 in shared memory (f16 MMAs)
 bool attention_tc_supported(int G, int qt);
 cudaError_t launch_attention_tc(const CUtensorMap &kmap, const CUtensorMap &vmap,
-                                const AttnArgs &a, cudaStream_t s);
+                                const AttnArgs &a, bool fp8, cudaStream_t s);
 
 // ---- latent sparse attention (latent.cu)
 struct LatentArgs {
