@@ -81,14 +81,22 @@ constexpr int slice_floats() {
   return 16 * MergeRow<FP8>::kStride + 32;
 }
 
-template <bool FP8, int RG>
+// Decode with the selection inside (SEL > 0): the selecting warps hand the producer each
+// selected block with its page id, for the CTA's first kSelSlots work-list slots, and the
+// number selected, for its first kSelItems items, through shared memory.  A CTA whose range is
+// longer reads them back from global memory instead.
+constexpr int kSelSlots = 1024;
+constexpr int kSelItems = 128;
+
+template <bool FP8, int RG, int SEL = -1>
 constexpr size_t stream_smem_bytes() {
   using C = StreamCfg<FP8, RG>;
   constexpr int W = stream_pq<FP8, RG>() * stream_teams<FP8, RG>();  // warps per row group
   return 1024 + C::kSlots * C::kTile + 2 * (RG * 16 * 256) +            // tiles, 2 Q buffers
          RG * (W / 2) * slice_floats<FP8>() * sizeof(float) +           // merge slices
          (2 * C::kSlots + 4) * sizeof(uint64_t) + C::kSlots * 3 * sizeof(int) +
-         2 * sizeof(SegMeta) + 16;
+         2 * sizeof(SegMeta) + 16 +
+         (SEL > 0 ? 16 + kSelSlots * sizeof(int2) + kSelItems * sizeof(int) : 0);
 }
 
 struct Item {
@@ -97,8 +105,10 @@ struct Item {
   const uint32_t *masks;
 };
 
+// u_known >= 0: the item's number selected, already known (the selection inside the kernel)
 template <bool PLAN>
-__device__ __forceinline__ Item load_item(const AttnArgs &a, int it, bool reporter) {
+__device__ __forceinline__ Item load_item(const AttnArgs &a, int it, bool reporter,
+                                          int u_known = -1) {
   Item m;
   const int y = it / a.H_kv;
   m.g = it % a.H_kv;
@@ -133,7 +143,7 @@ __device__ __forceinline__ Item load_item(const AttnArgs &a, int it, bool report
     } else {
       const size_t sel = static_cast<size_t>(m.t0) * a.H_kv + m.g;
       m.list = a.block_ids + sel * a.S;
-      int u = a.num_selected[sel];
+      int u = u_known >= 0 ? u_known : a.num_selected[sel];
       if (u < 0 || u > a.S) {
         if (reporter) report(a.dev_err, MSA_DEVERR_NUM_SELECTED);
         u = u < 0 ? 0 : a.S;
@@ -200,6 +210,12 @@ __global__ void __launch_bounds__(32 * (stream_consumer_warps<FP8, RG>() + 1))
   int *slot_ok = reinterpret_cast<int *>(slot_mask + NSLOT);
   SegMeta *meta = reinterpret_cast<SegMeta *>(slot_ok + NSLOT);  // [2], one per Q buffer
   volatile int *abort_flag = reinterpret_cast<volatile int *>(meta + 2);
+  int2 *sel_pairs = reinterpret_cast<int2 *>(
+      (reinterpret_cast<uintptr_t>(abort_flag + 4) + 15) & ~static_cast<uintptr_t>(15));
+  int *sel_u = reinterpret_cast<int *>(sel_pairs + kSelSlots);  // used when SEL > 0
+  const int n_items = it_last - it_first + 1;
+  // the selection hands its result over in shared memory (see kSelSlots)
+  const bool sel_smem = SEL > 0 && r1 - r0 <= kSelSlots && n_items <= kSelItems;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < NSLOT; ++s) {
@@ -214,55 +230,231 @@ __global__ void __launch_bounds__(32 * (stream_consumer_warps<FP8, RG>() + 1))
     fence_mbar_init();
   }
   __syncthreads();
+
+  // ---- producer state and helpers (warp NCW; declared here because, on decode with the
+  // selection inside, the producer hands the first segment over while the others select)
+  int q_staged = -1;  // item whose Q rows are in Q buffer 0 already
+  bool dead = false;
+  uint32_t nload0 = 0, nload1 = 0;  // tile loads issued into each team's ring
+  int n = 0;                        // non-empty segments handed over
+  int seg_k = 0;                    // blocks of the current segment issued so far
+  // waits (lane 0) until the consumers are done with Q buffer n & 1; false on timeout
+  auto claim_qbuf = [&](int n_) -> bool {
+    bool ok = true;
+    if (lane == 0 && n_ >= 2) ok = mbar_wait(&qempty[n_ & 1], ((n_ >> 1) - 1) & 1, abort_flag);
+    ok = __shfl_sync(0xffffffffu, ok, 0);
+    if (!ok && lane == 0) {
+      report(a.dev_err, MSA_DEVERR_TIMEOUT);
+      *abort_flag = 1;
+    }
+    return ok;
+  };
+  // hands segment n's Q rows (staged already when q_ready) and metadata to the consumers
+  auto hand_segment = [&](const Item &m, int v0, int v1, int piece, bool q_ready) -> bool {
+    if (!claim_qbuf(n)) return false;
+    const int buf = n & 1;
+    if (!q_ready)
+      stage_q<FP8, QR>(qbufs + buf * QBUF, a.q, m.t0, m.rows, a.G, a.H_q, m.g, lane, 32);
+    if (lane == 0) {
+      SegMeta md;
+      md.valid = 1;
+      md.t0 = m.t0;
+      md.rows = m.rows;
+      md.cl = m.cl;
+      md.tok0 = m.tok0;
+      md.g = m.g;
+      md.L = m.L;
+      md.v0 = v0;
+      md.v1 = v1;
+      md.piece = piece;
+      meta[buf] = md;
+    }
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&qfull[buf]);
+    ++n;
+    seg_k = 0;
+    return true;
+  };
+  // lane 0: K and V tile loads of block jj (page pg, token mask mm) of KV head g into the
+  // ring of the team that reads the segment's seg_k-th block; false on timeout
+  auto issue_block = [&](int jj, int pg, uint32_t mm, int g) -> bool {
+    const bool jok = jj >= 0 && jj < a.max_blocks;
+    const bool ok = jok && pg >= 0 && pg < a.num_pages;
+    if (!ok) report(a.dev_err, jok ? MSA_DEVERR_PAGE_ID : MSA_DEVERR_BLOCK_ID);
+    const int c2 = pg * a.H_kv + g;
+    const int tm = seg_k % NT;  // the team that reads this block
+    ++seg_k;
+#pragma unroll
+    for (int kv = 0; kv < 2; ++kv) {
+      const uint32_t nl = tm ? nload1 : nload0;
+      const int s = tm * NR + static_cast<int>(nl % NR);
+      if (nl >= static_cast<uint32_t>(NR) &&
+          !mbar_wait(&sempty[s], ((nl / NR) - 1) & 1, abort_flag)) {
+        report(a.dev_err, MSA_DEVERR_TIMEOUT);
+        *abort_flag = 1;
+        return false;
+      }
+      slot_j[s] = jj;
+      slot_mask[s] = mm;
+      slot_ok[s] = ok;
+      if (ok) {
+        const CUtensorMap *mp = kv ? &vmap : &kmap;
+        uint8_t *dst = slots + s * TILE;
+        mbar_arrive_expect_tx(&sfull[s], TILE);
+        tma_load_3d(dst, mp, &sfull[s], 0, 0, c2);
+        if (!FP8) tma_load_3d(dst + TILE / 2, mp, &sfull[s], 64, 0, c2);
+      } else {
+        mbar_arrive(&sfull[s]);
+      }
+      if (tm)
+        nload1 = nl + 1;
+      else
+        nload0 = nl + 1;
+    }
+    return true;
+  };
+  int pre_it = -1, pre_u = 0;  // item whose segment was handed over before the selection
+
+  if (warp == NCW && lane == 0) {  // kernel parameters: no earlier kernel writes them
+    prefetch_tmap(&kmap);
+    prefetch_tmap(&vmap);
+  }
   pdl_wait();  // block ids, selection counts and the plan (or the scores) come from earlier kernels
   pdl_launch_dependents();
 
+  if constexpr (SEL > 0) {
+    // The producer hands the first segment (Q rows and metadata) to the consumers before the
+    // selection is known: the number of blocks selected follows from the sequence length
+    // alone (the forced blocks and min(top_k, candidates)), and so does the segment.  After
+    // the selection it only issues the tile loads, in the list's order.
+    if (warp == NCW && sel_smem) {
+      const Item m0 = load_item<false>(a, it_first, false, 0);
+      if (m0.ntok > 0) {
+        int nb = m0.cl / kBlock + 1;
+        if (nb > a.max_blocks) nb = a.max_blocks;  // reported by the selecting warp
+        const int init_e = min(a.init_blocks, nb);
+        const int local_lo = max(init_e, nb - a.local_blocks);
+        const int u =
+            min(init_e + (nb - local_lo) + min(max(a.top_k, 0), local_lo - init_e), a.S);
+        int v0, v1;
+        segment(a, it_first, r0, r1, u, v0, v1);
+        const long long base = static_cast<long long>(it_first) * a.cap;
+        const int piece = static_cast<int>(blockIdx.x - base / a.R);
+        if (v1 > v0 && hand_segment(m0, v0, v1, piece, false)) {
+          q_staged = it_first;
+          pre_it = it_first;
+          pre_u = u;
+        }
+      }
+    }
+  }
+
+  // Decode with the selection inside: every warp of the CTA selects rows of the CTA's items
+  // (one query row per item; block_sparse_select as in select.cu), before any of them is
+  // streamed.  Items shared with a neighbouring CTA are selected by both, with identical
+  // results.  The loads that do not depend on one another are issued together, in one memory
+  // round trip: each selecting warp's row metadata, the scores of the row where the sequence's
+  // first query row lies when every sequence has the same number of rows (read again from the
+  // right row otherwise), and the page ids of its first item's blocks (held one per lane and
+  // block, so that the lane that takes a block also knows its page); the producer's first Q
+  // rows while the others select.
+  constexpr int KS = SEL > 0 ? SEL : 1;
   if constexpr (SEL >= 0) {
-    // Decode: every warp of the CTA selects rows of the CTA's items (one query row per item;
-    // block_sparse_select as in select.cu), before any of them is streamed.  Items shared
-    // with a neighbouring CTA are selected by both, with identical results.
-    const int n_items = it_last - it_first + 1;
+    const int rows_per_seq = a.total_q / max(a.batch, 1);
     for (int k = warp; k < n_items; k += NCW + 1) {
       const int it = it_first + k;
       const int g = it % a.H_kv, b = it / a.H_kv;  // one query tile per sequence
+      const bool keep = sel_smem && k == warp;    // hand the result over in shared memory
+      // page id of block 32 i + lane, loaded with the scores when a lane holds up to 16 blocks
+      // (more would spill registers: the producer then looks the pages up itself)
+      constexpr bool kPagesInRegs = KS <= 16;
+      uint32_t sel_page[kPagesInRegs ? KS : 1];
+      float sc[KS];           // score of block 32 i + lane (SEL > 0)
+      const int guess = b * rows_per_seq;
+      auto load_scores = [&](int row) {
+        const float *sr = a.scores + (static_cast<size_t>(row) * a.H_kv + g) * a.max_blocks;
+#pragma unroll
+        for (int i = 0; i < KS; ++i) {
+          const int j = 32 * i + lane;
+          sc[i] = j < a.max_blocks ? sr[j] : -INFINITY;
+        }
+      };
+      if constexpr (SEL > 0) load_scores(guess);
+      if (kPagesInRegs && keep) {
+#pragma unroll
+        for (int i = 0; i < KS; ++i) {
+          const int j = 32 * i + lane;
+          sel_page[i] =
+              j < a.max_blocks ? a.table[static_cast<size_t>(b) * a.max_pages + j] : 0xffffffffu;
+        }
+      }
       const int row0 = a.row_off[b];
-      if (a.row_off[b + 1] - row0 <= 0) continue;  // no query row
+      if (a.row_off[b + 1] - row0 <= 0) {  // no query row
+        if (sel_smem && lane == 0) sel_u[k] = -1;
+        continue;
+      }
       int nb = max(a.cache_len[b], 0) / kBlock + 1;
       if (nb > a.max_blocks) {
         if (lane == 0) report(a.dev_err, MSA_DEVERR_LENGTHS);
         nb = a.max_blocks;
       }
+      if constexpr (SEL > 0) {
+        if (row0 != guess) load_scores(row0);
+      }
       const size_t sel = static_cast<size_t>(row0) * a.H_kv + g;
-      const int nsel = select_row<(SEL > 0 ? SEL : 0), false>(
-          a.scores + sel * a.max_blocks, nb, a.top_k, a.init_blocks, a.local_blocks, a.S,
-          a.sel_ids + sel * a.S, a.dev_err, lane);
-      if (lane == 0) a.sel_counts[sel] = nsel;
+      const long long slot0 = static_cast<long long>(it) * a.cap - r0;
+      // the selected blocks of this CTA's range, with their pages, into shared memory
+      struct Emit {
+        const uint32_t *page;  // this lane's sel_page
+        int2 *pairs;
+        long long slot0, n;
+        bool keep;
+        __device__ __forceinline__ void put(int pos, int j, int pg) const {
+          const long long slot = slot0 + pos;
+          if (keep && slot >= 0 && slot < n) pairs[slot] = make_int2(j, pg);
+        }
+        __device__ __forceinline__ void taken(int pos, int j, int i) const {
+          put(pos, j, kPagesInRegs ? static_cast<int>(page[i < KS ? i : 0]) : -1);
+        }
+        __device__ __forceinline__ void gathered(int pos, int j, int i, int src,
+                                                 bool valid) const {
+          int pg = -1;
+          if constexpr (kPagesInRegs) {  // pass i's page of lane src, one shuffle per pass
+#pragma unroll
+            for (int t = 0; t < KS; ++t) {
+              const int v = __shfl_sync(0xffffffffu, static_cast<int>(page[t]), src);
+              if (t == i) pg = v;
+            }
+          }
+          if (valid) put(pos, j, pg);
+        }
+      };
+      const Emit emit{sel_page, sel_pairs, slot0, r1 - r0, keep};
+      auto score = [&](int i) { return sc[i < KS ? i : 0]; };
+      const int nsel = select_row_from<(SEL > 0 ? SEL : 0), false>(
+          score, a.scores + sel * a.max_blocks, nb, a.top_k, a.init_blocks, a.local_blocks, a.S,
+          a.sel_ids + sel * a.S, a.dev_err, lane, 0, emit);
+      if (lane == 0) {
+        a.sel_counts[sel] = nsel;
+        if (sel_smem) sel_u[k] = keep ? nsel : -1;
+      }
+    }
+    if (warp == NCW && NCW >= n_items && pre_it < 0) {  // the producer selected nothing: its first Q rows
+      const Item m0 = load_item<false>(a, it_first, false, 0);
+      if (m0.ntok > 0) {
+        stage_q<FP8, QR>(qbufs, a.q, m0.t0, m0.rows, a.G, a.H_q, m0.g, lane, 32);
+        q_staged = it_first;
+      }
     }
     __syncthreads();  // the producer reads the selection back
   }
 
   if (warp == NCW) {
     // ============================================================== producer warp
-    if (lane == 0) {
-      prefetch_tmap(&kmap);
-      prefetch_tmap(&vmap);
-    }
-    bool dead = false;
-    uint32_t nload0 = 0, nload1 = 0;  // tile loads issued into each team's ring
-    int n = 0;                        // non-empty segments handed over
-    // waits (lane 0) until the consumers are done with Q buffer n & 1; false on timeout
-    auto claim_qbuf = [&](int n_) -> bool {
-      bool ok = true;
-      if (lane == 0 && n_ >= 2) ok = mbar_wait(&qempty[n_ & 1], ((n_ >> 1) - 1) & 1, abort_flag);
-      ok = __shfl_sync(0xffffffffu, ok, 0);
-      if (!ok && lane == 0) {
-        report(a.dev_err, MSA_DEVERR_TIMEOUT);
-        *abort_flag = 1;
-      }
-      return ok;
-    };
     for (int it = it_first; it <= it_last && !dead; ++it) {
-      const Item m = load_item<PLAN>(a, it, lane == 0);
+      // >= 0: the item's selection is in sel_pairs / sel_u
+      const int u_sm = sel_smem ? sel_u[it - it_first] : -1;
+      const Item m = load_item<PLAN>(a, it, lane == 0, u_sm);
       if (m.ntok == 0) continue;  // a tile past its sequence's end: no rows
       int v0, v1;
       segment(a, it, r0, r1, m.U, v0, v1);
@@ -285,30 +477,13 @@ __global__ void __launch_bounds__(32 * (stream_consumer_warps<FP8, RG>() + 1))
       }
       if (v1 <= v0) continue;
 
-      // ---- Q rows and metadata of this segment
-      if (!claim_qbuf(n)) {
+      // ---- Q rows and metadata of this segment (handed over already for pre_it)
+      const bool pre = it == pre_it;
+      if (pre && m.U != pre_u && lane == 0) report(a.dev_err, MSA_DEVERR_NUM_SELECTED);
+      if (!pre && !hand_segment(m, v0, v1, piece, n == 0 && it == q_staged)) {
         dead = true;
         break;
       }
-      const int buf = n & 1;
-      stage_q<FP8, QR>(qbufs + buf * QBUF, a.q, m.t0, m.rows, a.G, a.H_q, m.g, lane, 32);
-      if (lane == 0) {
-        SegMeta md;
-        md.valid = 1;
-        md.t0 = m.t0;
-        md.rows = m.rows;
-        md.cl = m.cl;
-        md.tok0 = m.tok0;
-        md.g = m.g;
-        md.L = m.L;
-        md.v0 = v0;
-        md.v1 = v1;
-        md.piece = piece;
-        meta[buf] = md;
-      }
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&qfull[buf]);
-      ++n;
 
       // ---- K and V tiles.  The warp resolves 32 blocks' page ids at a time (one lane
       // each) so that lane 0 never waits on a dependent lookup between two TMAs.
@@ -317,51 +492,26 @@ __global__ void __launch_bounds__(32 * (stream_consumer_warps<FP8, RG>() + 1))
         int j = -1, page = -1;
         uint32_t msk = 0u;
         if (e < v1) {
-          j = m.list[e];
-          msk = PLAN ? m.masks[e] : 0xffffffffu;
-          if (j >= 0 && j < a.max_blocks)
-            page = a.table[static_cast<size_t>(m.b) * a.max_pages + j];
+          if (u_sm >= 0) {  // e lies in this CTA's range: its slot was written
+            const int2 pr = sel_pairs[static_cast<long long>(it) * a.cap + e - r0];
+            j = pr.x;
+            page = pr.y;
+            msk = 0xffffffffu;
+            if (page < 0 && j >= 0 && j < a.max_blocks)  // not resolved by the selecting warp
+              page = a.table[static_cast<size_t>(m.b) * a.max_pages + j];
+          } else {
+            j = m.list[e];
+            msk = PLAN ? m.masks[e] : 0xffffffffu;
+            if (j >= 0 && j < a.max_blocks)
+              page = a.table[static_cast<size_t>(m.b) * a.max_pages + j];
+          }
         }
         const int cnt = min(32, v1 - bbase);
         for (int i = 0; i < cnt; ++i) {
           const int jj = __shfl_sync(0xffffffffu, j, i);
           const int pg = __shfl_sync(0xffffffffu, page, i);
           const uint32_t mm = __shfl_sync(0xffffffffu, msk, i);
-          if (lane == 0) {
-            const bool jok = jj >= 0 && jj < a.max_blocks;
-            const bool ok = jok && pg >= 0 && pg < a.num_pages;
-            if (!ok) report(a.dev_err, jok ? MSA_DEVERR_PAGE_ID : MSA_DEVERR_BLOCK_ID);
-            const int c2 = pg * a.H_kv + m.g;
-            const int tm = (bbase + i - v0) % NT;  // the team that reads this block
-#pragma unroll
-            for (int kv = 0; kv < 2; ++kv) {
-              const uint32_t nl = tm ? nload1 : nload0;
-              const int s = tm * NR + static_cast<int>(nl % NR);
-              if (nl >= static_cast<uint32_t>(NR) &&
-                  !mbar_wait(&sempty[s], ((nl / NR) - 1) & 1, abort_flag)) {
-                report(a.dev_err, MSA_DEVERR_TIMEOUT);
-                *abort_flag = 1;
-                dead = true;
-                break;
-              }
-              slot_j[s] = jj;
-              slot_mask[s] = mm;
-              slot_ok[s] = ok;
-              if (ok) {
-                const CUtensorMap *mp = kv ? &vmap : &kmap;
-                uint8_t *dst = slots + s * TILE;
-                mbar_arrive_expect_tx(&sfull[s], TILE);
-                tma_load_3d(dst, mp, &sfull[s], 0, 0, c2);
-                if (!FP8) tma_load_3d(dst + TILE / 2, mp, &sfull[s], 64, 0, c2);
-              } else {
-                mbar_arrive(&sfull[s]);
-              }
-              if (tm)
-                nload1 = nl + 1;
-              else
-                nload0 = nl + 1;
-            }
-          }
+          if (lane == 0 && !issue_block(jj, pg, mm, m.g)) dead = true;
           dead = __shfl_sync(0xffffffffu, dead, 0);
           if (dead) break;
         }
@@ -530,7 +680,8 @@ __global__ void __launch_bounds__(32 * (stream_consumer_warps<FP8, RG>() + 1))
 template <bool FP8, int RG, bool PLAN, int SEL, bool SWAP = false>
 cudaError_t launch_stream_one(const CUtensorMap &kmap, const CUtensorMap &vmap,
                               const AttnArgs &a, int grid, cudaStream_t s) {
-  const size_t smem = stream_smem_bytes<FP8, RG>();
+  constexpr size_t smem = stream_smem_bytes<FP8, RG, SEL>();
+  static_assert(smem <= 227 * 1024, "shared memory of one CTA");
   auto fn = &attn_stream_kernel<FP8, RG, PLAN, SEL, SWAP>;
   cudaError_t e = ensure_smem_limit(reinterpret_cast<const void *>(fn), static_cast<int>(smem));
   if (e != cudaSuccess) return e;

@@ -6,10 +6,14 @@
 // blocks compete on score; equal scores go to the lower block id.
 //
 // The candidates' scores become order-preserving uint32 keys held in registers; the exact
-// top_k-th largest key is then built bit by bit from the top (32 rounds of "how many keys are
-// >= this prefix", one warp reduction each, no atomics).  One ascending pass over the block ids
-// keeps the forced blocks, every candidate above that threshold, and the lowest-id candidates
-// equal to it until top_k are taken, so the output comes out in ascending order with no sort.
+// top_k-th largest key is then built from the top, two bits a round (at most 16 rounds of "how
+// many keys are >= each of three prefixes", three warp reductions in flight, no atomics).  The
+// search stops early when a prefix has exactly top_k keys at or above it: those keys are then
+// the top_k, whatever the lower bits (with continuous scores this happens once the prefix
+// separates the top_k-th key from the next one, after about half the bits).  One ascending pass
+// over the block ids keeps the forced blocks, every candidate above the threshold, and the
+// lowest-id candidates equal to it until top_k are taken, so the output comes out in ascending
+// order with no sort.
 //
 // Used by the selection kernel (select.cu) and by the decode indexer's last CTA of each
 // (sequence, tile, index head) (indexer.cu), which reads scores other CTAs wrote in the same
@@ -35,12 +39,13 @@ __device__ __forceinline__ float load_score(const float *p) {
 template <int KPL, bool CG>
 struct SelKeys {
   uint32_t k[KPL > 0 ? KPL : 1];
-  __device__ __forceinline__ void load(const float *srow, int nb, int lane, int init_e,
-                                       int local_lo) {
+  // score(i): the score of block 32 i + lane
+  template <typename Score>
+  __device__ __forceinline__ void load(Score score, int nb, int lane, int init_e, int local_lo) {
 #pragma unroll
     for (int i = 0; i < KPL; ++i) {
       const int j = i * 32 + lane;
-      k[i] = (j < nb && j >= init_e && j < local_lo) ? score_key(load_score<CG>(srow + j)) : 0u;
+      k[i] = (j < nb && j >= init_e && j < local_lo) ? score_key(score(i)) : 0u;
     }
   }
   // number of candidate keys >= x (over the warp); four independent partial counts
@@ -57,6 +62,31 @@ struct SelKeys {
         c += score_key(load_score<CG>(srow + j)) >= x;
     }
     return __reduce_add_sync(0xffffffffu, c);
+  }
+  // numbers of candidate keys >= x1, >= x2 and >= x3 (three reductions in flight at once)
+  __device__ __forceinline__ void count_ge3(uint32_t x1, uint32_t x2, uint32_t x3,
+                                            const float *srow, int lane, int init_e,
+                                            int local_lo, uint32_t &c1, uint32_t &c2,
+                                            uint32_t &c3) const {
+    uint32_t a1 = 0, a2 = 0, a3 = 0;
+    if (KPL > 0) {
+#pragma unroll
+      for (int i = 0; i < KPL; ++i) {
+        a1 += k[i] >= x1;
+        a2 += k[i] >= x2;
+        a3 += k[i] >= x3;
+      }
+    } else {
+      for (int j = init_e + lane; j < local_lo; j += 32) {
+        const uint32_t key = score_key(load_score<CG>(srow + j));
+        a1 += key >= x1;
+        a2 += key >= x2;
+        a3 += key >= x3;
+      }
+    }
+    c1 = __reduce_add_sync(0xffffffffu, a1);
+    c2 = __reduce_add_sync(0xffffffffu, a2);
+    c3 = __reduce_add_sync(0xffffffffu, a3);
   }
   // largest and smallest candidate key over the warp
   __device__ __forceinline__ void range(const float *srow, int lane, int init_e, int local_lo,
@@ -87,10 +117,38 @@ struct SelKeys {
 // "DeepSeekSparseAttentionConfig", index_share_for_mtp_iteration): srow and nb are the first
 // draft token's, whose candidates and top-k they give; the output is for a later token that
 // sees nb_out blocks: its own forced blocks of [0, nb_out) together with that top-k.
-template <int KPL, bool CG>
-__device__ __forceinline__ int select_row(const float *srow, int nb, int top_k, int init_blocks,
-                                          int local_blocks, int S, int32_t *out,
-                                          int32_t *dev_err, int lane, int nb_out = 0) {
+//
+// For callers that keep more per selected block, emit is told of each one in one of two ways:
+// emit.taken(pos, j, i) by the lane that takes block j = 32 i + lane as the pos-th selected
+// block; or emit.gathered(pos, j, i, src, valid), called by every lane of the warp together,
+// where a valid lane writes the pos-th selected block j = 32 i + src (lane src holds it).
+struct NoEmit {
+  __device__ __forceinline__ void taken(int, int, int) const {}
+  __device__ __forceinline__ void gathered(int, int, int, int, bool) const {}
+};
+
+// Position of the set bit of rank r (0: the lowest) in m (r < popc(m)).
+__device__ __forceinline__ int nth_set_bit(uint32_t m, int r) {
+  int b = 0;
+#pragma unroll
+  for (int w = 16; w >= 1; w >>= 1) {
+    const int c = __popc(m & ((1u << w) - 1u));
+    if (r >= c) {
+      r -= c;
+      m >>= w;
+      b += w;
+    }
+  }
+  return b;
+}
+//
+// select_row_from takes the row's scores through score(i) (block 32 i + lane) when KPL > 0, for
+// callers that loaded them already; select_row reads them from srow.
+template <int KPL, bool CG, typename Emit, typename Score>
+__device__ __forceinline__ int select_row_from(Score score, const float *srow, int nb, int top_k,
+                                               int init_blocks, int local_blocks, int S,
+                                               int32_t *out, int32_t *dev_err, int lane,
+                                               int nb_out, Emit emit) {
   const unsigned lt_mask = (1u << lane) - 1u;
   if (nb_out < nb) nb_out = nb;
   // forced: [0, init_e) and [local_lo, nb); candidates: [init_e, local_lo)
@@ -106,7 +164,7 @@ __device__ __forceinline__ int select_row(const float *srow, int nb, int top_k, 
   uint32_t T = 0xffffffffu;  // top_k == 0: no candidate passes
   int need_eq = 0;
   if (!take_all && top_k > 0) {
-    keys.load(srow, nb, lane, init_e, local_lo);
+    keys.load(score, nb, lane, init_e, local_lo);
     // T = the top_k-th largest candidate key: the largest x with count(key >= x) >= top_k,
     // built one bit at a time from the top.  Every candidate key lies in [kmin, kmax], so T
     // shares their common leading bits and only the bits below can still be open.
@@ -116,13 +174,41 @@ __device__ __forceinline__ int select_row(const float *srow, int nb, int top_k, 
     const uint32_t diff = kmax ^ kmin;
     const int top = diff == 0u ? -1 : 31 - __clz(diff);  // highest bit where they differ
     T = top < 0 ? kmax : (kmax & ~((2u << top) - 1u));
-    for (int bit = top; bit >= 0; --bit) {
-      const uint32_t x = T | (1u << bit);
-      if (keys.count_ge(x, srow, lane, init_e, local_lo) >= k) T = x;
+    bool exact = false;  // exactly top_k keys are >= T
+    int bit = top;
+    // two bits a round: the largest of the digits 1..3 whose prefix keeps >= top_k keys
+    // (digit 0 keeps T, which has >= top_k keys by construction)
+    for (; bit >= 1; bit -= 2) {
+      const uint32_t x1 = T | (1u << (bit - 1)), x2 = T | (2u << (bit - 1)),
+                     x3 = T | (3u << (bit - 1));
+      uint32_t c1, c2, c3;
+      keys.count_ge3(x1, x2, x3, srow, lane, init_e, local_lo, c1, c2, c3);
+      const uint32_t c = c3 >= k ? c3 : (c2 >= k ? c2 : c1);
+      if (c >= k) {
+        T = c3 >= k ? x3 : (c2 >= k ? x2 : x1);
+        if (c == k) {
+          exact = true;
+          break;
+        }
+      }
     }
-    const uint32_t above =
-        T == 0xffffffffu ? 0u : keys.count_ge(T + 1u, srow, lane, init_e, local_lo);
-    need_eq = static_cast<int>(k - above);  // how many candidates equal to T are taken
+    if (!exact && bit == 0) {  // the last bit on its own
+      const uint32_t x = T | 1u;
+      const uint32_t c = keys.count_ge(x, srow, lane, init_e, local_lo);
+      if (c >= k) {
+        T = x;
+        exact = c == k;
+      }
+    }
+    if (exact) {
+      // take every key >= T (T > 0: it has a bit set): keys > T - 1, none by equality
+      T -= 1u;
+      need_eq = 0;
+    } else {
+      const uint32_t above =
+          T == 0xffffffffu ? 0u : keys.count_ge(T + 1u, srow, lane, init_e, local_lo);
+      need_eq = static_cast<int>(k - above);  // how many candidates equal to T are taken
+    }
   }
 
   // one ascending pass: forced, above T, and the lowest-id candidates equal to T
@@ -146,12 +232,56 @@ __device__ __forceinline__ int select_row(const float *srow, int nb, int top_k, 
     const unsigned tm = __ballot_sync(0xffffffffu, take);
     if (take) {
       const int pos = nsel + __popc(tm & lt_mask);
-      if (pos < S) out[pos] = j;
+      if (pos < S) {
+        out[pos] = j;
+        emit.taken(pos, j, i);
+      }
     }
     nsel += __popc(tm);
   };
   const int passes = (nb_out + 31) / 32;
-  if (KPL > 0) {
+  if (KPL > 0 && need_eq == 0) {
+    // No candidate is taken by equality (take_all, or the early exit, or no tie at T): every
+    // pass's take mask is independent of the others, so all ballots go out together; then
+    // lane q writes the q-th selected block (q = lane, lane + 32, ...), found from the prefix
+    // of the passes' counts and a rank search in its pass's mask: no divergent stores.
+    constexpr int KP = KPL > 0 ? KPL : 1;
+    unsigned tm[KP];
+    int first[KP];  // selected blocks before pass i
+#pragma unroll
+    for (int i = 0; i < KP; ++i) {
+      const int j = i * 32 + lane;
+      const bool cand = j < nb && j >= init_e && j < local_lo;
+      const bool forced = j < nb_out && (j < init_o || j >= local_o);
+      const bool take = i < passes && (forced || (cand && (take_all || keys.k[i] > T)));
+      tm[i] = __ballot_sync(0xffffffffu, take);
+    }
+#pragma unroll
+    for (int i = 0; i < KP; ++i) {
+      first[i] = nsel;
+      nsel += __popc(tm[i]);
+    }
+    const int nout = min(nsel, S);
+    for (int q0 = 0; q0 < nout; q0 += 32) {
+      const int q = q0 + lane;
+      int ii = 0;
+      uint32_t mi = tm[0];
+      int base = 0;
+#pragma unroll
+      for (int i = 1; i < KP; ++i) {
+        if (first[i] <= q) {
+          ii = i;
+          mi = tm[i];
+          base = first[i];
+        }
+      }
+      const bool valid = q < nout;
+      const int src = valid ? nth_set_bit(mi, q - base) : 0;
+      const int j = ii * 32 + src;
+      if (valid) out[q] = j;
+      emit.gathered(q, j, ii, src, valid);
+    }
+  } else if (KPL > 0) {
 #pragma unroll
     for (int i = 0; i < (KPL > 0 ? KPL : 1); ++i)
       if (i < passes) pass(i, keys.k[i]);
@@ -164,6 +294,16 @@ __device__ __forceinline__ int select_row(const float *srow, int nb, int top_k, 
   }
   for (int q = nsel + lane; q < S; q += 32) out[q] = -1;
   return nsel;
+}
+
+template <int KPL, bool CG, typename Emit = NoEmit>
+__device__ __forceinline__ int select_row(const float *srow, int nb, int top_k, int init_blocks,
+                                          int local_blocks, int S, int32_t *out,
+                                          int32_t *dev_err, int lane, int nb_out = 0,
+                                          Emit emit = Emit()) {
+  auto score = [&](int i) { return load_score<CG>(srow + i * 32 + lane); };
+  return select_row_from<KPL, CG>(score, srow, nb, top_k, init_blocks, local_blocks, S, out,
+                                  dev_err, lane, nb_out, emit);
 }
 
 }  // namespace msa
