@@ -505,93 +505,111 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       //   masked the diagonal blocks.
       const bool any_use = __any_sync(0xffffffffu, use);
       const bool plain = __all_sync(0xffffffffu, !use || lim >= kBlock - 1);
-      float m8[8];
-#pragma unroll
-      for (int k = 0; k < 8; ++k) m8[k] = -INFINITY;
+      // After its first block a row's unmasked blocks take their exponentials against the
+      // running max straight away: with the lazy rescale the block max matters only when it
+      // exceeds the running max by more than 2^8, which the block's sum then shows (a term
+      // above 2^8, or an infinite one); only then is the max computed and the block taken again.
+      // (BF16 KV only: the FP8 kernel's conversion warps leave no registers for it.)
+      const bool fast = !F8 && plain && __all_sync(0xffffffffu, !use || m_run > -INFINITY);
       uint32_t v[128];  // the row's 128 scores
       if (any_use) {
 #pragma unroll
         for (int c = 0; c < 4; ++c)
           tmem_ld32(s_addr + 32 * c, *reinterpret_cast<uint32_t(*)[32]>(v + 32 * c));
         tmem_wait_ld();
-        // row max (independent chains; three-input max where no position is masked)
-        if (plain) {
-#pragma unroll
-          for (int e = 0; e < 128; e += 8)
-#pragma unroll
-            for (int k = 0; k < 4; ++k)
-              m8[k] = fmax3(m8[k], __uint_as_float(v[e + 2 * k]),
-                            __uint_as_float(v[e + 2 * k + 1]));
-        } else {
-#pragma unroll
-          for (int e = 0; e < 128; ++e)
-            if (use && e <= lim) m8[e & 7] = fmaxf(m8[e & 7], __uint_as_float(v[e]));
-        }
-#pragma unroll
-        for (int k = 0; k < 4; ++k) m8[k] = fmaxf(m8[k], m8[k + 4]);
       }
-      const float mrow = fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3]));
-      const float mb = use ? mrow * a.scale_log2 : -INFINITY;
-      const float m_cand = fmaxf(m_run, mb);
       float alpha = 1.f;
-      if (m_cand > m_run + kLazyLog2) {  // also the first visible block (m_run = -inf)
-        alpha = fast_exp2(m_run - m_cand);
-        m_run = m_cand;
-      }
-      // x = s * sc + nb: P = 2^(scale log2e S - m) where the row uses the block, else 0
-      const float sc = use ? a.scale_log2 : 0.f;
-      const float nb = use ? -m_run : -INFINITY;
-      float ps4[4] = {0.f, 0.f, 0.f, 0.f};
-      float2 ps2[4] = {{0.f, 0.f}, {0.f, 0.f}, {0.f, 0.f}, {0.f, 0.f}};
-      if (!any_use) {
-        uint32_t z[32];
+      float lblk = 0.f;  // the block's sum of P
+#pragma unroll 1
+      for (int pass = fast ? 0 : 1; pass < 2; ++pass) {
+        if (pass == 1) {
+          if (fast) tmem_wait_st();  // the fast pass's P, before it is written again
+          float m8[8];
 #pragma unroll
-        for (int e = 0; e < 32; ++e) z[e] = 0u;
-        tmem_st32(s_addr, z);
-        tmem_st32(s_addr + 32, z);
-      } else {
-        // P as bf16 into TMEM over the first 64 columns of S (the scores were read already)
+          for (int k = 0; k < 8; ++k) m8[k] = -INFINITY;
+          if (any_use) {
+            // row max (independent chains; three-input max where no position is masked)
+            if (plain) {
 #pragma unroll
-        for (int h = 0; h < 2; ++h) {
-          uint32_t pk[32];
-          if (plain) {  // pairs on the packed fp32x2 pipe: one FMA and one add per pair
+              for (int e = 0; e < 128; e += 8)
 #pragma unroll
-            for (int e = 0; e < 64; e += 2) {
-              const float2 x = fma2(make_float2(__uint_as_float(v[64 * h + e]),
-                                                __uint_as_float(v[64 * h + e + 1])),
-                                    make_float2(sc, sc), make_float2(nb, nb));
-              if constexpr (F8) {  // f16 P; its rounding (2^-11) is left out of the sum
-                const float e0 = fast_exp2(x.x), e1 = fast_exp2(x.y);
-                pk[e >> 1] = pack_f16x2(e0, e1);
-                ps2[(e >> 1) & 3] = add2(ps2[(e >> 1) & 3], make_float2(e0, e1));
-              } else {
-                const uint32_t pb = pack_bf16x2(fast_exp2(x.x), fast_exp2(x.y));
+                for (int k = 0; k < 4; ++k)
+                  m8[k] = fmax3(m8[k], __uint_as_float(v[e + 2 * k]),
+                                __uint_as_float(v[e + 2 * k + 1]));
+            } else {
+#pragma unroll
+              for (int e = 0; e < 128; ++e)
+                if (use && e <= lim) m8[e & 7] = fmaxf(m8[e & 7], __uint_as_float(v[e]));
+            }
+#pragma unroll
+            for (int k = 0; k < 4; ++k) m8[k] = fmaxf(m8[k], m8[k + 4]);
+          }
+          const float mrow = fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3]));
+          const float mb = use ? mrow * a.scale_log2 : -INFINITY;
+          const float m_cand = fmaxf(m_run, mb);
+          if (m_cand > m_run + kLazyLog2) {  // also the first visible block (m_run = -inf)
+            alpha = fast_exp2(m_run - m_cand);
+            m_run = m_cand;
+          }
+        }
+        // x = s * sc + nb: P = 2^(scale log2e S - m) where the row uses the block, else 0
+        const float sc = use ? a.scale_log2 : 0.f;
+        const float nb = use ? -m_run : -INFINITY;
+        float ps4[4] = {0.f, 0.f, 0.f, 0.f};
+        float2 ps2[4] = {{0.f, 0.f}, {0.f, 0.f}, {0.f, 0.f}, {0.f, 0.f}};
+        if (!any_use) {
+          uint32_t z[32];
+#pragma unroll
+          for (int e = 0; e < 32; ++e) z[e] = 0u;
+          tmem_st32(s_addr, z);
+          tmem_st32(s_addr + 32, z);
+        } else {
+          // P as bf16 into TMEM over the first 64 columns of S (the scores were read already)
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            uint32_t pk[32];
+            if (plain) {  // pairs on the packed fp32x2 pipe: one FMA and one add per pair
+#pragma unroll
+              for (int e = 0; e < 64; e += 2) {
+                const float2 x = fma2(make_float2(__uint_as_float(v[64 * h + e]),
+                                                  __uint_as_float(v[64 * h + e + 1])),
+                                      make_float2(sc, sc), make_float2(nb, nb));
+                if constexpr (F8) {  // f16 P; its rounding (2^-11) is left out of the sum
+                  const float e0 = fast_exp2(x.x), e1 = fast_exp2(x.y);
+                  pk[e >> 1] = pack_f16x2(e0, e1);
+                  ps2[(e >> 1) & 3] = add2(ps2[(e >> 1) & 3], make_float2(e0, e1));
+                } else {
+                  const uint32_t pb = pack_bf16x2(fast_exp2(x.x), fast_exp2(x.y));
+                  pk[e >> 1] = pb;
+                  ps2[(e >> 1) & 3] = add2(ps2[(e >> 1) & 3], bf16x2_to_float2(pb));
+                }
+              }
+            } else {
+#pragma unroll
+              for (int e = 0; e < 64; e += 2) {
+                const int pe = 64 * h + e;
+                const float x0 = (use && pe <= lim) ? fmaf(__uint_as_float(v[pe]), sc, nb)
+                                                    : -INFINITY;
+                const float x1 = (use && pe + 1 <= lim)
+                                     ? fmaf(__uint_as_float(v[pe + 1]), sc, nb)
+                                     : -INFINITY;
+                const float e0 = fast_exp2(x0), e1 = fast_exp2(x1);
+                const uint32_t pb = F8 ? pack_f16x2(e0, e1) : pack_bf16x2(e0, e1);
                 pk[e >> 1] = pb;
-                ps2[(e >> 1) & 3] = add2(ps2[(e >> 1) & 3], bf16x2_to_float2(pb));
+                const float2 pf = F8 ? make_float2(e0, e1) : bf16x2_to_float2(pb);
+                ps4[(e >> 1) & 3] += pf.x + pf.y;
               }
             }
-          } else {
-#pragma unroll
-            for (int e = 0; e < 64; e += 2) {
-              const int pe = 64 * h + e;
-              const float x0 = (use && pe <= lim) ? fmaf(__uint_as_float(v[pe]), sc, nb)
-                                                  : -INFINITY;
-              const float x1 = (use && pe + 1 <= lim)
-                                   ? fmaf(__uint_as_float(v[pe + 1]), sc, nb)
-                                   : -INFINITY;
-              const float e0 = fast_exp2(x0), e1 = fast_exp2(x1);
-              const uint32_t pb = F8 ? pack_f16x2(e0, e1) : pack_bf16x2(e0, e1);
-              pk[e >> 1] = pb;
-              const float2 pf = F8 ? make_float2(e0, e1) : bf16x2_to_float2(pb);
-              ps4[(e >> 1) & 3] += pf.x + pf.y;
-            }
+            tmem_st32(s_addr + 32 * h, pk);
           }
-          tmem_st32(s_addr + 32 * h, pk);
         }
-      }
 #pragma unroll
-      for (int k = 0; k < 4; ++k) ps4[k] += ps2[k].x + ps2[k].y;
-      l_run = l_run * alpha + ((ps4[0] + ps4[1]) + (ps4[2] + ps4[3]));
+        for (int k = 0; k < 4; ++k) ps4[k] += ps2[k].x + ps2[k].y;
+        lblk = (ps4[0] + ps4[1]) + (ps4[2] + ps4[3]);
+        // every term <= 2^8 on the fast pass, or the rows concerned take the block again
+        if (pass == 0 && !__any_sync(0xffffffffu, use && !(lblk <= 256.f))) break;
+      }
+      l_run = l_run * alpha + lblk;
       // this group's previous P V (done before this block's S was written; waited here so
       // that every phase is observed in order) before its O is rescaled
       if (i >= 2 && !mbar_wait(&o_done[w], ((i >> 1) - 1) & 1, abort_flag)) {
