@@ -511,6 +511,19 @@ bool select_in_attention(const msa_ragged_paged_t *rp, int num_q_heads, int num_
   return rp->max_q_len == 1 && num_q_heads / num_kv_heads <= 16;
 }
 
+// Whether msa_select_sparse_attn_paged selects and plans in one launch for this shape: the
+// speculative route with tiles of at most kMaxSpecTileTokens tokens.
+bool select_with_plan(const msa_ragged_paged_t *rp, int S, int num_q_heads, int num_kv_heads,
+                      int max_blocks, int num_splits, msa_kv_dtype_t kv_dtype) {
+  if (rp->max_q_len <= 1 || rp->max_q_len > MSA_MAX_SPEC_DRAFT) return false;
+  Route r;
+  if (!make_route(rp, S, num_q_heads, num_kv_heads, max_blocks, num_splits,
+                  num_sms_of_current_device(), kv_dtype == MSA_KV_FP8_E4M3, &r))
+    return false;
+  return r.stream && r.plan && r.qt <= kMaxSpecTileTokens &&
+         select_plan_smem_bytes(max_blocks, r.cap, S) <= 200 * 1024;
+}
+
 // msa_sparse_attn_paged's body.  dry_run: validate only (nothing enqueued); sel: select inside
 // the decode attention kernel (block_ids / num_selected are then its outputs).
 msa_status_t attn_impl(const msa_ragged_paged_t *rp, const void *q, const void *k_cache,
@@ -541,14 +554,41 @@ msa_status_t attn_impl(const msa_ragged_paged_t *rp, const void *q, const void *
   if (static_cast<long long>(rp->batch) * r.tiles > 0x7fffffffLL) return MSA_ERR_UNSUPPORTED;
   if (r.bytes > 0 && (!workspace || workspace_bytes < r.bytes || !aligned(workspace, 256)))
     return MSA_ERR_INVALID_ARG;
-  if (sel && (!r.stream || r.plan || r.rg != 1)) return MSA_ERR_UNSUPPORTED;
+  // sel: on the decode route the attention kernel selects; on the speculative route one launch
+  // selects and plans (tiles of at most kMaxSpecTileTokens tokens)
+  if (sel && (!r.stream || (!r.plan && r.rg != 1) || (r.plan && r.qt > kMaxSpecTileTokens) ||
+              (r.plan && select_plan_smem_bytes(max_blocks, r.cap, S) > 200 * 1024)))
+    return MSA_ERR_UNSUPPORTED;
   if (dry_run) return MSA_OK;
 
   uint8_t *ws = static_cast<uint8_t *>(workspace);
   const cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   const bool fp8 = kv_dtype == MSA_KV_FP8_E4M3;
 
-  if (r.plan) {
+  if (r.plan && sel) {
+    SelectPlanArgs p;
+    p.row_off = rp->input_row_offsets;
+    p.cache_len = rp->cache_lengths;
+    p.scores = sel->scores;
+    p.block_ids = sel->block_ids;
+    p.num_selected = sel->num_selected;
+    p.list = reinterpret_cast<int32_t *>(ws + r.off_list);
+    p.masks = reinterpret_cast<uint32_t *>(ws + r.off_masks);
+    p.counts = reinterpret_cast<int32_t *>(ws + r.off_counts);
+    p.dev_err = dev_err;
+    p.batch = rp->batch;
+    p.max_q_len = rp->max_q_len;
+    p.H_kv = num_kv_heads;
+    p.S = S;
+    p.max_blocks = max_blocks;
+    p.qt = r.qt;
+    p.tiles = r.tiles;
+    p.cap = r.cap;
+    p.top_k = sel->top_k;
+    p.init_blocks = sel->init_blocks;
+    p.local_blocks = sel->local_blocks;
+    if (launch_select_plan(p, s) != cudaSuccess) return MSA_ERR_CUDA;
+  } else if (r.plan) {
     PlanArgs p;
     p.row_off = rp->input_row_offsets;
     p.cache_len = rp->cache_lengths;
@@ -607,12 +647,13 @@ msa_status_t attn_impl(const msa_ragged_paged_t *rp, const void *q, const void *
   // one partition: every item lies inside one CTA, which then writes the output itself
   a.direct = r.stream && r.splits == 1 && out != nullptr;
   a.dev_err = dev_err;
-  a.scores = sel ? sel->scores : nullptr;
-  a.sel_ids = sel ? sel->block_ids : nullptr;
-  a.sel_counts = sel ? sel->num_selected : nullptr;
-  a.top_k = sel ? sel->top_k : 0;
-  a.init_blocks = sel ? sel->init_blocks : 0;
-  a.local_blocks = sel ? sel->local_blocks : 0;
+  const AttnSelect *in_kernel = r.plan ? nullptr : sel;  // decode: the attention selects
+  a.scores = in_kernel ? in_kernel->scores : nullptr;
+  a.sel_ids = in_kernel ? in_kernel->block_ids : nullptr;
+  a.sel_counts = in_kernel ? in_kernel->num_selected : nullptr;
+  a.top_k = in_kernel ? in_kernel->top_k : 0;
+  a.init_blocks = in_kernel ? in_kernel->init_blocks : 0;
+  a.local_blocks = in_kernel ? in_kernel->local_blocks : 0;
   if (r.tc)
     return launch_attention_tc(kmap, vmap, a, fp8, s) == cudaSuccess ? MSA_OK : MSA_ERR_CUDA;
   if (!r.stream)
@@ -663,7 +704,8 @@ msa_status_t msa_select_sparse_attn_paged(
                                    workspace, workspace_bytes, out, dev_err, stream, true,
                                    nullptr);
   if (v != MSA_OK) return v;
-  if (select_in_attention(rp, num_q_heads, num_kv_heads)) {
+  if (select_in_attention(rp, num_q_heads, num_kv_heads) ||
+      select_with_plan(rp, Si, num_q_heads, num_kv_heads, max_blocks, num_splits, kv_dtype)) {
     const AttnSelect sel{scores, block_ids, num_selected, top_k, init_blocks, local_blocks};
     return attn_impl(rp, q, k_cache, v_cache, kv_dtype, block_ids, num_selected, Si,
                      num_q_heads, num_kv_heads, max_blocks, scale, num_splits, workspace,

@@ -67,6 +67,23 @@ struct PlanArgs {
 };
 cudaError_t launch_plan(const PlanArgs &a, cudaStream_t s);
 
+// ---- the speculative route's selection and plan in one launch (select_plan.cu): one CTA of qt
+// warps per (sequence, query tile, KV head); writes what select.cu and plan.cu write
+constexpr int kMaxSpecTileTokens = 8;  // tokens per speculative query tile (warps per CTA)
+struct SelectPlanArgs {
+  const int32_t *row_off, *cache_len;
+  const float *scores;
+  int32_t *block_ids, *num_selected;  // [total_q, H_kv, S], [total_q, H_kv]
+  int32_t *list;                      // [items, cap]
+  uint32_t *masks;                    // [items, cap]
+  int32_t *counts;                    // [items]
+  int32_t *dev_err;
+  int batch, max_q_len, H_kv, S, max_blocks, qt, tiles, cap;
+  int top_k, init_blocks, local_blocks;
+};
+size_t select_plan_smem_bytes(int max_blocks, int cap, int S);
+cudaError_t launch_select_plan(const SelectPlanArgs &a, cudaStream_t s);
+
 // ---- stage 3: sparse paged attention (attention_stream.cu: decode / speculative,
 //      attention_tile.cu: prefill)
 struct AttnArgs {

@@ -280,7 +280,9 @@ MSA_API msa_status_t msa_sparse_attn_paged(const msa_ragged_paged_t *rp, const v
  * On the decode route (max_q_len == 1) with a GQA group of at most 16 the selection runs inside
  * the attention launch: each CTA of the persistent kernel first selects the rows of the items in
  * its share of the work, then streams them, so the selection needs no launch of its own.  On the
- * other routes it enqueues the two stages one after the other.
+ * speculative route (tiles of at most 8 tokens) one launch selects every token's row and builds
+ * each query tile's union plan, which msa_sparse_attn_paged would otherwise build in a launch of
+ * its own.  On the prefill route it enqueues the two stages one after the other.
  *
  *   scores, top_k, init_blocks, local_blocks  as msa_select_blocks (S = init + local + top_k)
  *   block_ids, num_selected  device int32 [total_q, num_kv_heads, S] / [total_q, num_kv_heads]
