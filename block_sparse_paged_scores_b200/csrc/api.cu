@@ -257,10 +257,14 @@ int32_t msa_attn_partials(const msa_ragged_paged_t *rp, int32_t S, int32_t num_q
 
 namespace {
 
-// The selection to fuse into the decode indexer (nullptr: scores only).
+// The selection to fuse into the decode indexer (nullptr: scores only).  With publish set
+// instead (the one-call decode step), the indexer selects nothing: the last CTA of every unit
+// publishes publish[unit] = *epoch + 1.
 struct FusedSelect {
   int32_t *counters, *block_ids, *num_selected;
   int top_k, init_blocks, local_blocks, S;
+  int32_t *publish = nullptr;
+  const int32_t *epoch = nullptr;
 };
 
 // The prefill route scores BF16 index-K on tcgen05; the scaled formats take the warp-MMA
@@ -351,6 +355,8 @@ msa_status_t index_scores_impl(const msa_ragged_paged_t *rp, const void *q_idx,
   a.chunks = static_cast<int>(chunks);
   if (units * chunks > 0x7fffffffLL) return MSA_ERR_UNSUPPORTED;
   if (fs) {
+    a.publish = fs->publish;
+    a.epoch = fs->epoch;
     a.counters = fs->counters;
     a.block_ids = fs->block_ids;
     a.num_selected = fs->num_selected;
@@ -503,6 +509,10 @@ struct AttnSelect {
   const float *scores;
   int32_t *block_ids, *num_selected;
   int top_k, init_blocks, local_blocks;
+  // the one-call decode step's flags (ready == nullptr: wait for the whole earlier launch)
+  const int32_t *ready = nullptr;
+  int32_t *epoch = nullptr, *step_done = nullptr;
+  int H_idxk = 1;
 };
 
 // Whether msa_select_sparse_attn_paged selects inside the attention kernel for this shape: the
@@ -614,7 +624,7 @@ msa_status_t attn_impl(const msa_ragged_paged_t *rp, const void *q, const void *
   if (!page_tensor_map(&kmap, k_cache, tiles, fp8) || !page_tensor_map(&vmap, v_cache, tiles, fp8))
     return MSA_ERR_CUDA;
 
-  AttnArgs a;
+  AttnArgs a{};
   a.row_off = rp->input_row_offsets;
   a.cache_len = rp->cache_lengths;
   a.table = rp->kv_lookup_table;
@@ -654,6 +664,10 @@ msa_status_t attn_impl(const msa_ragged_paged_t *rp, const void *q, const void *
   a.top_k = in_kernel ? in_kernel->top_k : 0;
   a.init_blocks = in_kernel ? in_kernel->init_blocks : 0;
   a.local_blocks = in_kernel ? in_kernel->local_blocks : 0;
+  a.ready = in_kernel ? in_kernel->ready : nullptr;
+  a.epoch = in_kernel ? in_kernel->epoch : nullptr;
+  a.step_done = in_kernel ? in_kernel->step_done : nullptr;
+  a.H_idxk = in_kernel ? in_kernel->H_idxk : 1;
   if (r.tc)
     return launch_attention_tc(kmap, vmap, a, fp8, s) == cudaSuccess ? MSA_OK : MSA_ERR_CUDA;
   if (!r.stream)
@@ -718,6 +732,88 @@ msa_status_t msa_select_sparse_attn_paged(
   return attn_impl(rp, q, k_cache, v_cache, kv_dtype, block_ids, num_selected, Si, num_q_heads,
                    num_kv_heads, max_blocks, scale, num_splits, workspace, workspace_bytes, out,
                    dev_err, stream, false, nullptr);
+}
+
+// ---------------------------------------------------------------- one-call decode step
+// Words before the attention's workspace: the step epoch, the attention's done counter, the
+// indexer's per-unit counters and the per-unit ready flags.
+static size_t step_sync_bytes(const msa_ragged_paged_t *rp, int32_t num_idx_k_heads) {
+  const size_t units = static_cast<size_t>(rp->batch) * rp->max_q_len * num_idx_k_heads;
+  return (((2 + 2 * units) * sizeof(int32_t)) + 255) / 256 * 256;
+}
+
+size_t msa_decode_step_workspace_bytes(const msa_ragged_paged_t *rp, int32_t S,
+                                       int32_t num_q_heads, int32_t num_kv_heads,
+                                       int32_t num_idx_k_heads, int32_t max_blocks,
+                                       int32_t num_splits) {
+  if (!ragged_ok(rp) || num_idx_k_heads < 1) return 0;
+  return step_sync_bytes(rp, num_idx_k_heads) +
+         msa_attn_workspace_bytes(rp, S, num_q_heads, num_kv_heads, max_blocks, num_splits);
+}
+
+msa_status_t msa_decode_step(const msa_ragged_paged_t *rp, const void *q_idx,
+                             const msa_index_k_t *k_idx, int32_t top_k, int32_t init_blocks,
+                             int32_t local_blocks, const void *q, const void *k_cache,
+                             const void *v_cache, msa_kv_dtype_t kv_dtype, int32_t num_q_heads,
+                             int32_t num_kv_heads, int32_t max_blocks, float scale,
+                             int32_t num_splits, void *workspace, size_t workspace_bytes,
+                             float *scores, int32_t *block_ids, int32_t *num_selected, void *out,
+                             int32_t *dev_err, struct CUstream_st *stream) {
+  const long long S = static_cast<long long>(top_k) + init_blocks + local_blocks;
+  if (!ragged_ok(rp) || !k_idx || k_idx->num_heads < 1 || top_k < 0 || init_blocks < 0 ||
+      local_blocks < 0 || S < 1 || S > (1 << 20) || num_kv_heads < 1 ||
+      num_q_heads < num_kv_heads)
+    return MSA_ERR_INVALID_ARG;
+  if (rp->total_q == 0) return MSA_OK;
+  if (!scores || !block_ids || !num_selected || !workspace || !aligned(workspace, 256))
+    return MSA_ERR_INVALID_ARG;
+  const size_t sync = step_sync_bytes(rp, k_idx->num_heads);
+  if (workspace_bytes < sync) return MSA_ERR_INVALID_ARG;
+  uint8_t *ws = static_cast<uint8_t *>(workspace);
+  void *attn_ws = ws + sync;
+  const size_t attn_bytes = workspace_bytes - sync;
+  const int Si = static_cast<int>(S);
+  const bool fast = select_in_attention(rp, num_q_heads, num_kv_heads) &&
+                    num_kv_heads % k_idx->num_heads == 0 &&
+                    !index_uses_tc(rp, num_kv_heads / k_idx->num_heads,
+                                   static_cast<int>(k_idx->dtype));
+  if (!fast) {  // the two calls one after the other
+    const msa_status_t v = attn_impl(rp, q, k_cache, v_cache, kv_dtype, block_ids,
+                                     num_selected, Si, num_q_heads, num_kv_heads, max_blocks,
+                                     scale, num_splits, attn_ws, attn_bytes, out, dev_err,
+                                     stream, true, nullptr);
+    if (v != MSA_OK) return v;
+    const msa_status_t e = msa_index_scores_k(rp, q_idx, k_idx, num_kv_heads, max_blocks, 0u,
+                                              scores, dev_err, stream);
+    if (e != MSA_OK) return e;
+    return msa_select_sparse_attn_paged(rp, scores, top_k, init_blocks, local_blocks, q,
+                                        k_cache, v_cache, kv_dtype, num_q_heads, num_kv_heads,
+                                        max_blocks, scale, num_splits, attn_ws, attn_bytes,
+                                        block_ids, num_selected, out, dev_err, stream);
+  }
+  int32_t *words = reinterpret_cast<int32_t *>(ws);
+  const size_t units = static_cast<size_t>(rp->batch) * rp->max_q_len * k_idx->num_heads;
+  int32_t *epoch = words, *step_done = words + 1, *counters = words + 2;
+  int32_t *ready = counters + units;
+  AttnSelect sel{scores, block_ids, num_selected, top_k, init_blocks, local_blocks};
+  sel.ready = ready;
+  sel.epoch = epoch;
+  sel.step_done = step_done;
+  sel.H_idxk = k_idx->num_heads;
+  const msa_status_t v = attn_impl(rp, q, k_cache, v_cache, kv_dtype, block_ids, num_selected,
+                                   Si, num_q_heads, num_kv_heads, max_blocks, scale, num_splits,
+                                   attn_ws, attn_bytes, out, dev_err, stream, true, &sel);
+  if (v != MSA_OK) return v;
+  FusedSelect fs{counters, nullptr, nullptr, top_k, init_blocks, local_blocks, Si};
+  fs.publish = ready;
+  fs.epoch = epoch;
+  const msa_status_t e = index_scores_impl(rp, q_idx, k_idx, num_kv_heads, max_blocks, 0u,
+                                           scores, dev_err,
+                                           reinterpret_cast<cudaStream_t>(stream), &fs);
+  if (e != MSA_OK) return e;
+  return attn_impl(rp, q, k_cache, v_cache, kv_dtype, block_ids, num_selected, Si, num_q_heads,
+                   num_kv_heads, max_blocks, scale, num_splits, attn_ws, attn_bytes, out,
+                   dev_err, stream, false, &sel);
 }
 
 }  // extern "C"

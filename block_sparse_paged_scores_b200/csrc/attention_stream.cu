@@ -319,8 +319,12 @@ __global__ void __launch_bounds__(32 * (stream_consumer_warps<FP8, RG>() + 1))
     prefetch_tmap(&kmap);
     prefetch_tmap(&vmap);
   }
-  pdl_wait();  // block ids, selection counts and the plan (or the scores) come from earlier kernels
+  // With the flags of the one-call decode step the scores are waited for row by row below;
+  // nothing else this kernel reads comes from the launch before it.
+  const bool flagged = SEL >= 0 && a.ready != nullptr;
+  if (!flagged) pdl_wait();  // block ids, counts and the plan (or the scores): earlier kernels
   pdl_launch_dependents();
+  const int ready_value = flagged ? ld_acquire_gpu(a.epoch) + 1 : 0;
 
   if constexpr (SEL > 0) {
     // The producer hands the first segment (Q rows and metadata) to the consumers before the
@@ -379,7 +383,9 @@ __global__ void __launch_bounds__(32 * (stream_consumer_warps<FP8, RG>() + 1))
           sc[i] = j < a.max_blocks ? sr[j] : -INFINITY;
         }
       };
-      if constexpr (SEL > 0) load_scores(guess);
+      if constexpr (SEL > 0) {
+        if (!flagged) load_scores(guess);
+      }
       if (kPagesInRegs && keep) {
 #pragma unroll
         for (int i = 0; i < KS; ++i) {
@@ -398,7 +404,25 @@ __global__ void __launch_bounds__(32 * (stream_consumer_warps<FP8, RG>() + 1))
         if (lane == 0) report(a.dev_err, MSA_DEVERR_LENGTHS);
         nb = a.max_blocks;
       }
-      if constexpr (SEL > 0) {
+      if (flagged) {
+        // this row's index unit published by the indexer launch: every lane acquires the flag
+        // itself before reading the scores
+        const int32_t *f = a.ready + static_cast<size_t>(b) * a.H_idxk + g % a.H_idxk;
+        const uint64_t t0 = global_timer_ns();
+        bool timed_out = false;
+        while (!__all_sync(0xffffffffu, ld_acquire_gpu(f) == ready_value)) {
+          if (global_timer_ns() - t0 > kWaitTimeoutNs) {
+            timed_out = true;
+            break;
+          }
+          __nanosleep(128);
+        }
+        if (timed_out && lane == 0) {
+          report(a.dev_err, MSA_DEVERR_TIMEOUT);
+          *abort_flag = 1;
+        }
+        if constexpr (SEL > 0) load_scores(row0);
+      } else if constexpr (SEL > 0) {
         if (row0 != guess) load_scores(row0);
       }
       const size_t sel = static_cast<size_t>(row0) * a.H_kv + g;
@@ -521,6 +545,14 @@ __global__ void __launch_bounds__(32 * (stream_consumer_warps<FP8, RG>() + 1))
     if (!dead && claim_qbuf(n) && lane == 0) {
       meta[n & 1].valid = 0;
       mbar_arrive(&qfull[n & 1]);
+    }
+    // one-call decode step: every flag this CTA waits for was seen (the selection is done);
+    // the last CTA to get here advances the epoch for the next step
+    if (flagged && lane == 0) {
+      if (atomicAdd(a.step_done, 1) == static_cast<int>(gridDim.x) - 1) {
+        atomicExch(a.step_done, 0);
+        st_release_gpu(a.epoch, ready_value);
+      }
     }
     return;
   }

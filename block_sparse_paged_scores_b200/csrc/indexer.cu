@@ -120,7 +120,24 @@ __device__ __forceinline__ void count_out_and_select(const IndexerArgs &a, int b
   }
 }
 
-// KPL < 0: scores only; KPL >= 0: selection fused, KPL keys per lane in registers (0: any
+// The consumer warps of every CTA of a unit call this once the CTA's scores are written; the
+// last CTA to arrive publishes the unit (the one-call decode step).
+__device__ __forceinline__ void count_out_and_publish(const IndexerArgs &a, int b, int tile,
+                                                      int hk) {
+  named_bar_sync(2, kConsumerWarps * 32);  // every thread's scores written
+  if (threadIdx.x == 0) {
+    const size_t u = (static_cast<size_t>(b) * a.tiles + tile) * a.H_idxk + hk;
+    __threadfence();  // the CTA's scores (ordered before by the barrier), before the count
+    if (atomicAdd(a.counters + u, 1) == a.chunks - 1) {
+      __threadfence();  // every other CTA's scores, before the flag
+      atomicExch(a.counters + u, 0);
+      st_release_gpu(a.publish + u, ld_acquire_gpu(a.epoch) + 1);
+    }
+  }
+}
+
+// KPL == -2: scores, then the unit published (count_out_and_publish); KPL == -1: scores only;
+// KPL >= 0: selection fused, KPL keys per lane in registers (0: any
 // number of blocks, read from L2 on every pass).
 // With one 16-row tile the scaled formats are bounded to four CTAs per SM (registers <= 102
 // per thread; two tiles would spill).
@@ -189,10 +206,14 @@ __global__ void __launch_bounds__(kThreads, (IF != kIdxBf16 && MT == 1) ? 4 : 1)
   volatile int *is_last = abort_flag + 1;
 
   if (npages <= 0) {
-    if (KPL >= 0) {
+    if (KPL >= 0 || KPL == -2) {
       __syncthreads();  // every thread's -inf fills, before the count
-      if (warp < kConsumerWarps)
-        count_out_and_select<KPL>(a, b, tile, hk, row0, tok0, ntok, cl, q_len, is_last);
+      if (warp < kConsumerWarps) {
+        if constexpr (KPL == -2)
+          count_out_and_publish(a, b, tile, hk);
+        else
+          count_out_and_select<KPL>(a, b, tile, hk, row0, tok0, ntok, cl, q_len, is_last);
+      }
     }
     return;
   }
@@ -481,7 +502,9 @@ __global__ void __launch_bounds__(kThreads, (IF != kIdxBf16 && MT == 1) ? 4 : 1)
       a.scores[(static_cast<size_t>(t) * a.H_kv + g) * a.max_blocks + j] = m;
     }
   }
-  if (KPL >= 0)
+  if constexpr (KPL == -2)
+    count_out_and_publish(a, b, tile, hk);
+  else if constexpr (KPL >= 0)
     count_out_and_select<KPL>(a, b, tile, hk, row0, tok0, ntok, cl, q_len, is_last);
 }
 
@@ -509,6 +532,7 @@ template <int MT, int IF>
 cudaError_t launch_mt(const CUtensorMap &kidx_map, const IndexerArgs &a, int chunks,
                       cudaStream_t s) {
   if (!a.counters) return launch_st<MT, -1, IF>(kidx_map, a, chunks, s);
+  if (a.publish) return launch_st<MT, -2, IF>(kidx_map, a, chunks, s);
   if (a.max_blocks <= 4 * 32) return launch_st<MT, 4, IF>(kidx_map, a, chunks, s);
   if (a.max_blocks <= 16 * 32) return launch_st<MT, 16, IF>(kidx_map, a, chunks, s);
   if (a.max_blocks <= 32 * 32) return launch_st<MT, 32, IF>(kidx_map, a, chunks, s);

@@ -38,6 +38,11 @@ struct IndexerArgs {
   // Top-k shared across each sequence's new tokens: one tile of one token (the first) per
   // sequence is scored, and the fused selection writes every token's row from it.
   int share;
+  // One-call decode step (publish != nullptr, counters set, no fused selection): the last CTA
+  // of every unit publishes publish[unit] = *epoch + 1 (release) once the unit's scores are
+  // written, so that the attention launch, already running, can select that unit's rows.
+  int32_t *publish;
+  const int32_t *epoch;
 };
 // mt = 16-row MMA tiles per CTA (1 or 2)
 cudaError_t launch_index_scores(const CUtensorMap &kidx_map, const IndexerArgs &a, int mt,
@@ -110,6 +115,13 @@ struct AttnArgs {
   const float *scores;
   int32_t *sel_ids, *sel_counts;
   int top_k, init_blocks, local_blocks;
+  // One-call decode step (ready != nullptr, with the selection inside): the kernel does not
+  // wait for the whole indexer launch; each row's scores are read once its unit's flag
+  // ready[b * H_idxk + g % H_idxk] equals *epoch + 1 (acquire, bounded wait).  The last CTA
+  // to finish counting on *step_done sets it back to zero and advances *epoch.
+  const int32_t *ready;
+  int32_t *epoch, *step_done;
+  int H_idxk;
   int32_t *dev_err;
 };
 // rg = 16-row groups (1..4); plan = read the per-tile union instead of the selection

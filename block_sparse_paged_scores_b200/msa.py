@@ -100,6 +100,11 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.msa_select_sparse_attn_paged.restype = I
     lib.msa_select_sparse_attn_paged.argtypes = [RP, P, I, I, I, P, P, P, I, I, I, I, F, I, P,
                                                  ctypes.c_size_t, P, P, P, P, P]
+    lib.msa_decode_step_workspace_bytes.restype = ctypes.c_size_t
+    lib.msa_decode_step_workspace_bytes.argtypes = [RP, I, I, I, I, I, I]
+    lib.msa_decode_step.restype = I
+    lib.msa_decode_step.argtypes = [RP, P, IK, I, I, I, P, P, P, I, I, I, I, F, I, P,
+                                    ctypes.c_size_t, P, P, P, P, P, P]
     lib.msa_splitk_combine.restype = I
     lib.msa_splitk_combine.argtypes = [P, P, I, I, I, P, P]
     lib.msa_attn_workspace_bytes.restype = ctypes.c_size_t
@@ -256,6 +261,29 @@ def msa_select_sparse_attn_paged(rp: RaggedPaged, scores, top_k: int, init_block
         _ptr(out), _ptr(dev_err), _stream(stream)))
 
 
+def msa_decode_step_workspace_bytes(rp: RaggedPaged, S: int, num_q_heads: int,
+                                    num_kv_heads: int, num_idx_k_heads: int, max_blocks: int,
+                                    num_splits: int) -> int:
+    return int(load().msa_decode_step_workspace_bytes(ctypes.byref(rp), S, num_q_heads,
+                                                      num_kv_heads, num_idx_k_heads, max_blocks,
+                                                      num_splits))
+
+
+def msa_decode_step(rp: RaggedPaged, q_idx, k_idx: IndexK, top_k: int, init_blocks: int,
+                    local_blocks: int, q, k_cache, v_cache, kv_dtype: int, num_q_heads: int,
+                    num_kv_heads: int, max_blocks: int, scale: float, num_splits: int,
+                    workspace, scores, block_ids, num_selected, out, dev_err=None, stream=None,
+                    workspace_bytes: Optional[int] = None):
+    if workspace_bytes is None:
+        workspace_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _check("msa_decode_step", load().msa_decode_step(
+        ctypes.byref(rp), _ptr(q_idx), ctypes.byref(k_idx), top_k, init_blocks, local_blocks,
+        _ptr(q), _ptr(k_cache), _ptr(v_cache), int(kv_dtype), num_q_heads, num_kv_heads,
+        max_blocks, float(scale), num_splits, _ptr(workspace), int(workspace_bytes),
+        _ptr(scores), _ptr(block_ids), _ptr(num_selected), _ptr(out), _ptr(dev_err),
+        _stream(stream)))
+
+
 def msa_sparse_attn_paged_noalloc(rp: RaggedPaged, q, k_cache, v_cache, kv_dtype: int,
                                   block_ids, num_selected, S: int, num_q_heads: int,
                                   num_kv_heads: int, max_blocks: int, scale: float,
@@ -344,11 +372,13 @@ class Path:
     last two as one msa_select_sparse_attn_paged call (``select_in_attention``); with
     ``fused_select`` the first two as one msa_index_select call; with neither, three separate
     calls.  ``share_selection``: the indexer top-k shared across each sequence's draft tokens
-    (MSA_SHARE_ACROSS_DRAFTS, through msa_index_select_k), then the attention."""
+    (MSA_SHARE_ACROSS_DRAFTS, through msa_index_select_k), then the attention.  ``one_call``
+    (with ``select_in_attention``): the whole step as one msa_decode_step call, whose own
+    workspace (flags and counters first, zeroed once here) is ``step_workspace``."""
 
     def __init__(self, prob: dict, num_splits: int = 0, max_blocks: Optional[int] = None,
                  fused_select: bool = False, select_in_attention: bool = True,
-                 share_selection: bool = False):
+                 share_selection: bool = False, one_call: bool = True):
         self.p = prob
         self.share_selection = share_selection
         self.fused_select = fused_select or share_selection
@@ -374,6 +404,11 @@ class Path:
         self.kidx = index_k(prob["k_idx"], prob.get("k_idx_scale"), prob["H_idxk"],
                             self.idx_dtype)
         self.index_flags = MSA_SHARE_ACROSS_DRAFTS if share_selection else 0
+        self.one_call = one_call and select_in_attention and not self.fused_select
+        if self.one_call:
+            sb = msa_decode_step_workspace_bytes(self.rp, S, prob["H_q"], hkv, prob["H_idxk"],
+                                                 self.max_blocks, num_splits)
+            self.step_workspace = torch.zeros((max(sb, 256),), dtype=torch.uint8, device=dev)
 
     def index_scores(self, stream=None):
         p = self.p
@@ -430,7 +465,19 @@ class Path:
         n, o_ptr, l_ptr = self.partials()
         msa_splitk_combine(o_ptr, l_ptr, n, self.p["total_q"], self.p["H_q"], self.out, stream)
 
+    def step(self, stream=None):
+        """The whole step as one msa_decode_step call."""
+        p = self.p
+        msa_decode_step(self.rp, p["q_idx"], self.kidx, p["top_k"], p["init_blocks"],
+                        p["local_blocks"], p["q"], p["k"], p["v"], self.kv_dtype, p["H_q"],
+                        p["H_kv"], self.max_blocks, p["scale"], self.num_splits,
+                        self.step_workspace, self.scores, self.block_ids, self.num_selected,
+                        self.out, self.dev_err, stream)
+
     def run(self, stream=None):
+        if self.one_call:
+            self.step(stream)
+            return self.out
         if self.fused_select:
             self.index_select(stream)
         elif self.select_in_attention:

@@ -299,6 +299,40 @@ MSA_API msa_status_t msa_select_sparse_attn_paged(
     struct CUstream_st *stream);
 
 /*
+ * msa_decode_step — one step of the path in one call: msa_index_scores_k (no flags), then
+ * msa_select_sparse_attn_paged, with the same results (scores, block_ids, num_selected, out)
+ * ([msa] "Three attention routes", [ferrox] block_sparse_select, positions_of_blocks).
+ *
+ * On the decode route with the selection inside the attention (max_q_len == 1, a GQA group of
+ * at most 16), the attention launch does not wait for the whole indexer launch: the last CTA of
+ * each (sequence, index-K head) unit of the indexer publishes a flag once the unit's scores are
+ * written, and each attention CTA selects a row as soon as its unit's flag is up (a bounded
+ * wait), so the CTAs that start while the indexer's last units are still running begin early.
+ * On the other routes the two calls run one after the other.
+ *
+ *   q_idx, index_k, scores  as msa_index_scores_k (scores: output)
+ *   top_k .. out, dev_err, stream  as msa_select_sparse_attn_paged
+ *   workspace    device, >= msa_decode_step_workspace_bytes(...) bytes, 256-byte aligned.  Its
+ *                first msa_decode_step_workspace_bytes(...) - msa_attn_workspace_bytes(...)
+ *                bytes hold the step's flags and counters: zero them once before the first
+ *                call (every call leaves them ready for the next one) and again after a call
+ *                that reports a device error.  Calls sharing one workspace run on one stream.
+ */
+MSA_API size_t msa_decode_step_workspace_bytes(const msa_ragged_paged_t *rp, int32_t S,
+                                               int32_t num_q_heads, int32_t num_kv_heads,
+                                               int32_t num_idx_k_heads, int32_t max_blocks,
+                                               int32_t num_splits);
+MSA_API msa_status_t msa_decode_step(const msa_ragged_paged_t *rp, const void *q_idx,
+                                     const msa_index_k_t *index_k, int32_t top_k,
+                                     int32_t init_blocks, int32_t local_blocks, const void *q,
+                                     const void *k_cache, const void *v_cache,
+                                     msa_kv_dtype_t kv_dtype, int32_t num_q_heads,
+                                     int32_t num_kv_heads, int32_t max_blocks, float scale,
+                                     int32_t num_splits, void *workspace, size_t workspace_bytes,
+                                     float *scores, int32_t *block_ids, int32_t *num_selected,
+                                     void *out, int32_t *dev_err, struct CUstream_st *stream);
+
+/*
  * msa_sparse_attn_paged_noalloc — msa_sparse_attn_paged for callers that cannot provide a
  * workspace.  (This entry point has no counterpart on the pages: it is a deployment aid.)
  *
