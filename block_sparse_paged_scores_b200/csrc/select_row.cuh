@@ -15,7 +15,9 @@
 // lowest-id candidates equal to it until top_k are taken, so the output comes out in ascending
 // order with no sort.
 //
-// Used by the selection kernel (select.cu) and by the decode indexer's last CTA of each
+// Used by the selection kernel (select.cu), by the speculative selection-and-plan kernel
+// (select_plan.cu), by the decode attention's prologue (attention_stream.cu, which hands it the
+// scores it loaded already: select_row_from), and by the decode indexer's last CTA of each
 // (sequence, tile, index head) (indexer.cu), which reads scores other CTAs wrote in the same
 // launch and so loads them from L2 (CG = true).
 #pragma once
