@@ -177,3 +177,33 @@ def test_binding_raises_on_error_status(lib):
     with pytest.raises(msa.MSAError) as ei:
         msa.msa_select_blocks(rp, 0x10000, 8, 16, 0, 0, 0, 0x10000, 0x10000, stream=0)
     assert ei.value.status == msa.MSA_ERR_INVALID_ARG
+
+
+def test_decode_step_workspace_and_refusals(lib):
+    """msa_decode_step: its workspace is the step's flag and counter words (rounded to 256 bytes)
+    in front of the attention's; invalid arguments are refused before anything is enqueued."""
+    rp = _rp(batch=4, total_q=4, max_q_len=1)
+    attn = msa.msa_attn_workspace_bytes(rp, 19, 64, 8, 16, 2)
+    words = 2 + 2 * 4 * 1 * 1                      # epoch, done, counters, flags (1 index head)
+    assert msa.msa_decode_step_workspace_bytes(rp, 19, 64, 8, 1, 16, 2) == \
+        (words * 4 + 255) // 256 * 256 + attn
+    many = msa.msa_decode_step_workspace_bytes(_rp(batch=100, total_q=100), 19, 64, 8, 8, 16, 2)
+    assert many - msa.msa_attn_workspace_bytes(_rp(batch=100, total_q=100), 19, 64, 8, 16, 2) \
+        == ((2 + 2 * 100 * 8) * 4 + 255) // 256 * 256
+    assert msa.msa_decode_step_workspace_bytes(rp, 19, 64, 8, 0, 16, 2) == 0  # no index heads
+    P = 0x10000
+    k = msa.IndexK(msa.MSA_IDX_BF16, P, 0, 1)
+
+    def step(**kw):
+        return lib.msa_decode_step(
+            ctypes.byref(kw.get("rp", rp)), P, ctypes.byref(kw.get("k", k)), kw.get("top_k", 16),
+            1, 2, P, P, P, 0, 64, 8, 16, 0.1, 0, kw.get("ws", P), kw.get("ws_bytes", 1 << 20),
+            kw.get("scores", P), P, P, P, None, None)
+    assert step(top_k=-1) == msa.MSA_ERR_INVALID_ARG
+    assert step(scores=None) == msa.MSA_ERR_INVALID_ARG
+    assert step(ws=None) == msa.MSA_ERR_INVALID_ARG
+    assert step(ws=P + 64) == msa.MSA_ERR_INVALID_ARG               # 256-byte alignment
+    assert step(ws_bytes=8) == msa.MSA_ERR_INVALID_ARG              # no room for the flags
+    assert step(k=msa.IndexK(msa.MSA_IDX_BF16, P, 0, 0)) == msa.MSA_ERR_INVALID_ARG
+    empty = _rp(batch=4, total_q=0, max_q_len=1)
+    assert step(rp=empty, scores=None) == msa.MSA_OK                # nothing to do
