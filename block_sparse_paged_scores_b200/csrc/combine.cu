@@ -16,10 +16,13 @@ namespace msa {
 namespace {
 
 constexpr int kWarps = 8;
+constexpr int kPre = 2;  // partitions whose outputs are loaded with the log-sum-exps
 
 // One warp per (row, head).  All partitions' log-sum-exps are fetched at once (one lane
-// each), then every partition's output float4 is issued before any is used, so the warp
-// waits for about two memory latencies whatever the number of partitions.
+// each).  With at most kPre partitions their output float4s are fetched with them (one that
+// turns out empty is loaded but not used), so that the warp waits for one memory latency;
+// with more, every non-empty partition's output is issued before any is used (two latencies,
+// and no loads of empty partitions).
 __global__ void __launch_bounds__(32 * kWarps)
     combine_kernel(const float *__restrict__ part_o, const float *__restrict__ part_lse,
                    int splits, long long rows, uint16_t *__restrict__ out) {
@@ -30,6 +33,11 @@ __global__ void __launch_bounds__(32 * kWarps)
   if (row >= rows) return;
   float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
   float wsum = 0.f, M = -INFINITY;  // running max of the log-sum-exps seen so far
+  float4 pre[kPre];
+#pragma unroll
+  for (int s = 0; s < kPre; ++s)
+    if (splits <= kPre && s < splits)
+      pre[s] = reinterpret_cast<const float4 *>(part_o + (s * rows + row) * kHeadDim)[lane];
   for (int s0 = 0; s0 < splits; s0 += 32) {
     const int n = min(32, splits - s0);
     const float my_lse = lane < n ? part_lse[(s0 + lane) * rows + row] : -INFINITY;
@@ -50,8 +58,14 @@ __global__ void __launch_bounds__(32 * kWarps)
     for (int s = 0; s < n; ++s) {
       const float w = __shfl_sync(0xffffffffu, w_lane, s);
       if (w == 0.f) continue;
-      const float4 o =
-          reinterpret_cast<const float4 *>(part_o + ((s0 + s) * rows + row) * kHeadDim)[lane];
+      float4 o;
+      if (splits <= kPre) {
+#pragma unroll
+        for (int t = 0; t < kPre; ++t)
+          if (t == s) o = pre[t];
+      } else {
+        o = reinterpret_cast<const float4 *>(part_o + ((s0 + s) * rows + row) * kHeadDim)[lane];
+      }
       acc.x += w * o.x;
       acc.y += w * o.y;
       acc.z += w * o.z;
