@@ -324,7 +324,8 @@ __global__ void __launch_bounds__(32 * (stream_consumer_warps<FP8, RG>() + 1))
   const bool flagged = SEL >= 0 && a.ready != nullptr;
   if (!flagged) pdl_wait();  // block ids, counts and the plan (or the scores): earlier kernels
   pdl_launch_dependents();
-  const int ready_value = flagged ? ld_acquire_gpu(a.epoch) + 1 : 0;
+  const int ready_value =  // the step counter + 1 (wrapping)
+      flagged ? static_cast<int>(static_cast<uint32_t>(ld_acquire_gpu(a.epoch)) + 1u) : 0;
 
   if constexpr (SEL > 0) {
     // The producer hands the first segment (Q rows and metadata) to the consumers before the

@@ -131,7 +131,8 @@ __device__ __forceinline__ void count_out_and_publish(const IndexerArgs &a, int 
     if (atomicAdd(a.counters + u, 1) == a.chunks - 1) {
       __threadfence();  // every other CTA's scores, before the flag
       atomicExch(a.counters + u, 0);
-      st_release_gpu(a.publish + u, ld_acquire_gpu(a.epoch) + 1);
+      const uint32_t step = static_cast<uint32_t>(ld_acquire_gpu(a.epoch));
+      st_release_gpu(a.publish + u, static_cast<int>(step + 1u));  // wrapping
     }
   }
 }
