@@ -555,6 +555,12 @@ __global__ void __launch_bounds__(32 * (stream_consumer_warps<FP8, RG>() + 1))
         st_release_gpu(a.epoch, ready_value);
       }
     }
+    // every tile load it issued (lane 0 did) has landed before this warp exits
+    if (lane == 0) {
+      const bool landed =
+          drain_ring(sfull, NR, nload0) && (NT < 2 || drain_ring(sfull + NR, NR, nload1));
+      if (!landed) report(a.dev_err, MSA_DEVERR_TIMEOUT);
+    }
     return;
   }
 

@@ -242,6 +242,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       prefetch_tmap(&vmap);
     }
     bool dead = false;
+    uint32_t issued8[2] = {0u, 0u};  // K and V tiles given to the staging rings (lane 0)
     for (int base = 0; base < nblk && !dead; base += 32) {
       int j = -1, page = -1;
       if (base + lane < nblk) {
@@ -268,18 +269,24 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             } else if (ok) {
               mbar_arrive_expect_tx(&full8[s8], kTc8Tile);
               tma_load_3d(dst, op ? &vmap : &kmap, &full8[s8], 0, 0, pg * a.H_kv + g);
+              ++issued8[op];
             } else {
               // an unusable page: zeros, so that its block adds nothing (scores masked too)
               uint4 *z = reinterpret_cast<uint4 *>(dst);
               for (uint32_t w = 0; w < kTc8Tile / 16; ++w) z[w] = make_uint4(0, 0, 0, 0);
               fence_async_shared();
               mbar_arrive(&full8[s8]);
+              ++issued8[op];
             }
           }
         }
         dead = __shfl_sync(0xffffffffu, dead, 0);
       }
     }
+    // every tile load issued has landed before this warp exits
+    if (lane == 0 && !(drain_ring(k8_full, k8Stages, issued8[0]) &&
+                       drain_ring(v8_full, k8Stages, issued8[1])))
+      report(a.dev_err, MSA_DEVERR_TIMEOUT);
   } else if (F8 && (warp == 2 || warp == 3)) {
     // ============================================================== e4m3 -> f16 converters
     // warp 3 converts K tiles, warp 2 V tiles, from the staging ring into the f16 ring in the
@@ -334,6 +341,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     uint64_t *empty = is_k ? k_empty : v_empty;
     if (lane == 0) prefetch_tmap(map);
     bool dead = false;
+    uint32_t issued = 0;  // tiles given to the ring (lane 0)
     for (int base = 0; base < nblk && !dead; base += 32) {
       int j = -1, page = -1;
       if (base + lane < nblk) {
@@ -368,12 +376,15 @@ __global__ void __launch_bounds__(kTcThreads, 1)
               fence_async_shared();
               mbar_arrive(&full[s]);
             }
+            ++issued;
           }
         }
         dead = __shfl_sync(0xffffffffu, dead, 0);
         if (dead) break;
       }
     }
+    // every tile load issued has landed before this warp exits
+    if (lane == 0 && !drain_ring(full, nst, issued)) report(a.dev_err, MSA_DEVERR_TIMEOUT);
   } else if (warp == 1) {
     // ============================================================== MMA issuer
     if (lane == 0) {
@@ -442,9 +453,10 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         }
       }
       if (!alive) fail();
-      // every tcgen05 operation of this thread done before the TMEM is released
+      // every tcgen05 operation of this thread done before the TMEM is released (waited for
+      // even after an abort: bounded in time only)
       umma_commit(mma_done);
-      if (!mbar_wait(mma_done, 0, abort_flag)) report(a.dev_err, MSA_DEVERR_TIMEOUT);
+      if (!mbar_wait(mma_done, 0, nullptr)) report(a.dev_err, MSA_DEVERR_TIMEOUT);
     }
     __syncwarp();
   }

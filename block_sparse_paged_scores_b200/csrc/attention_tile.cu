@@ -120,6 +120,7 @@ __global__ void __launch_bounds__(32 * (RG * tile_pq<RG>() + 1))
       prefetch_tmap(&vmap);
     }
     bool dead = false;
+    uint32_t issued = 0;  // stages given K and V (lane 0)
     // 32 blocks' page ids resolved at a time, one lane each, then issued by lane 0
     for (int base = 0; base < nblk && !dead; base += 32) {
       int j = -1, page = -1;
@@ -164,12 +165,15 @@ __global__ void __launch_bounds__(32 * (RG * tile_pq<RG>() + 1))
               report(a.dev_err, jok ? MSA_DEVERR_PAGE_ID : MSA_DEVERR_BLOCK_ID);
               mbar_arrive(&full[s]);
             }
+            ++issued;
           }
         }
         dead = __shfl_sync(0xffffffffu, dead, 0);
         if (dead) break;
       }
     }
+    // every tile load issued has landed before this warp exits
+    if (lane == 0 && !drain_ring(full, NS, issued)) report(a.dev_err, MSA_DEVERR_TIMEOUT);
     return;
   }
 

@@ -233,6 +233,7 @@ __global__ void __launch_bounds__(kThreads, (IF != kIdxBf16 && MT == 1) ? 4 : 1)
     // ------------------------------------------------------------ producer: TMA page ring
     if (lane == 0) prefetch_tmap(&kmap);
     bool dead = false;
+    uint32_t issued = 0;  // pages given to the ring (lane 0)
     // 32 page ids fetched at a time, one lane each, then issued by lane 0
     for (int base = 0; base < npages && !dead; base += 32) {
       const int pg_l = base + lane < npages
@@ -269,12 +270,15 @@ __global__ void __launch_bounds__(kThreads, (IF != kIdxBf16 && MT == 1) ? 4 : 1)
               report(a.dev_err, MSA_DEVERR_PAGE_ID);
               mbar_arrive(&full[s]);
             }
+            ++issued;
           }
         }
         dead = __shfl_sync(0xffffffffu, dead, 0);
         if (dead) break;
       }
     }
+    // every tile load issued has landed before this warp exits
+    if (lane == 0 && !drain_ring(full, kStages, issued)) report(a.dev_err, MSA_DEVERR_TIMEOUT);
     return;
   }
 

@@ -130,6 +130,7 @@ __global__ void __launch_bounds__(kIxThreads, 1)
     // ============================================================== producer
     if (lane == 0) prefetch_tmap(&kmap);
     bool dead = false;
+    uint32_t issued = 0;  // pages given to the ring (lane 0)
     for (int base = 0; base < npages && !dead; base += 32) {
       const int pg_l = base + lane < npages
                            ? a.table[static_cast<size_t>(b) * a.max_pages + base + lane]
@@ -157,12 +158,16 @@ __global__ void __launch_bounds__(kIxThreads, 1)
               report(a.dev_err, MSA_DEVERR_PAGE_ID);
               mbar_arrive(&st_full[s]);
             }
+            ++issued;
           }
         }
         dead = __shfl_sync(0xffffffffu, dead, 0);
         if (dead) break;
       }
     }
+    // every tile load issued has landed before this warp exits
+    if (lane == 0 && !drain_ring(st_full, kIxStages, issued))
+      report(a.dev_err, MSA_DEVERR_TIMEOUT);
   } else if (warp == 1) {
     // ============================================================== MMA issuer
     if (lane == 0) {
@@ -183,8 +188,9 @@ __global__ void __launch_bounds__(kIxThreads, 1)
                        ks > 0 ? 1u : 0u);
         umma_commit(&s_full[sb]);
       }
+      // every MMA done before the TMEM is released (even after an abort: bounded in time only)
       umma_commit(mma_done);
-      if (!mbar_wait(mma_done, 0, abort_flag)) report(a.dev_err, MSA_DEVERR_TIMEOUT);
+      if (!mbar_wait(mma_done, 0, nullptr)) report(a.dev_err, MSA_DEVERR_TIMEOUT);
     }
     __syncwarp();
   } else {

@@ -75,9 +75,9 @@ __device__ __forceinline__ uint64_t global_timer_ns() {
   return t;
 }
 // Waits for the phase with the given parity to complete.  Gives up after kWaitTimeoutNs or
-// as soon as *abort is set, and then returns false (the caller reports and unwinds).  After
-// the first test the thread sleeps in the barrier between tests (at most 0.5 ms each), so
-// waiting warps take no issue slots from the working ones.
+// as soon as *abort is set (abort may be null: time only), and then returns false (the caller
+// reports and unwinds).  After the first test the thread sleeps in the barrier between tests
+// (at most 0.5 ms each), so waiting warps take no issue slots from the working ones.
 __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volatile int *abort,
                                           uint64_t limit_ns = kWaitTimeoutNs) {
   if (mbar_try_wait(bar, parity)) return true;
@@ -85,9 +85,20 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volati
   const uint32_t hint = limit_ns < 1000000ull ? static_cast<uint32_t>(limit_ns / 2) : 500000u;
   for (;;) {
     if (mbar_try_wait_sleep(bar, parity, hint)) return true;
-    if (*abort) return false;
+    if (abort != nullptr && *abort) return false;
     if (global_timer_ns() - t0 > limit_ns) return false;
   }
+}
+// A load role's last act: waits until every bulk copy it issued into a ring has landed, so
+// that none still writes into this CTA's shared memory after the CTA exits (after an abort
+// the consumers leave loads unread).  Load i of the ring completed phase i / stages of barrier
+// i % stages; the wait is on the last phase each barrier was given, bounded in time and deaf
+// to the abort flag.  Returns false if a wait gave up.
+__device__ __forceinline__ bool drain_ring(uint64_t *full, uint32_t stages, uint32_t issued) {
+  bool ok = true;
+  for (uint32_t s = 0; s < stages && s < issued; ++s)
+    ok = mbar_wait(&full[s], ((issued - 1u - s) / stages) & 1u, nullptr) && ok;
+  return ok;
 }
 
 // ------------------------------------------------------------------------------ TMA

@@ -75,3 +75,32 @@ def test_one_call_refuses_a_workspace_without_room_for_the_flags():
                             p["H_kv"], one.max_blocks, p["scale"], 0, one.step_workspace,
                             one.scores, one.block_ids, one.num_selected, one.out, one.dev_err,
                             workspace_bytes=8)
+
+
+def test_a_unit_never_published_times_out_and_the_next_call_is_exact():
+    """The attention's wait for a unit's flag is bounded.  With the indexer's per-unit counts
+    offset so that no CTA of a unit finds itself the last one, no flag goes up: every selecting
+    warp gives up after its limit, MSA_DEVERR_TIMEOUT is reported, the launches return (their
+    tile loads drained), and once the step's words are zeroed again the next call is exact."""
+    import time
+    prob, one, two = _pair("bf16_decode_small")
+    two.run()
+    one.run()
+    torch.cuda.synchronize()
+    assert int(one.dev_err.item()) == 0
+    units = prob["batch"] * prob["max_q_len"] * prob["H_idxk"]
+    counters = one.step_workspace[8:8 + 4 * units].view(torch.int32)
+    counters.fill_(1 << 20)
+    t0 = time.monotonic()
+    one.run()
+    torch.cuda.synchronize()
+    assert time.monotonic() - t0 < 60
+    assert int(one.dev_err.item()) & msa.MSA_DEVERR_TIMEOUT
+    one.step_workspace[:8 + 8 * units].zero_()
+    one.dev_err.zero_()
+    one.out.fill_(0)
+    one.run()
+    torch.cuda.synchronize()
+    assert int(one.dev_err.item()) == 0
+    assert torch.equal(one.block_ids, two.block_ids)
+    assert torch.equal(one.out, two.out)
