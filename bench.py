@@ -260,12 +260,15 @@ def profiled_traffic(kernel: str, workload: str, digest: str):
 
 # ------------------------------------------------------------------ CPU oracle sample
 def oracle_sample(workload: str, n_seq: int, seed: int):
-    """A bounded sample of a workload for the CPU oracle, and its description.  Decode-like
-    workloads: n_seq of their sequences (same distributions).  Prefill: one sequence with 16-64
-    new tokens over a prior cache drawn as in the workload (a whole prefill sequence is minutes
-    of fp64 work per pass)."""
+    """A bounded sample of a workload (or of a variant: its workload with the variant's
+    changes) for the CPU oracle, its description, and whether the indexer top-k is shared
+    across draft tokens.  Decode-like workloads: n_seq of their sequences (same
+    distributions).  Prefill: one sequence with 16-64 new tokens over a prior cache drawn as in
+    the workload (a whole prefill sequence is minutes of fp64 work per pass)."""
     from block_sparse_paged_scores_b200 import workload as wl
-    spec = wl.WORKLOADS[workload]
+    base, changes, path_kw = VARIANTS.get(workload, (workload, {}, {}))
+    spec = wl.WORKLOADS[base].scaled(**changes)
+    share = bool(path_kw.get("share_selection"))
     q_hi = spec.q_len[1] if isinstance(spec.q_len, tuple) else spec.q_len
     if q_hi > 8:
         p = wl.generate(spec.scaled(batch=1, q_len=(16, 64)), seed=seed)
@@ -274,16 +277,16 @@ def oracle_sample(workload: str, n_seq: int, seed: int):
     else:
         p = wl.generate(spec.scaled(batch=min(n_seq, spec.batch)), seed=seed)
         desc = f"{p['batch']} of {spec.batch} sequences of {workload} (same distributions)"
-    return p, desc
+    return p, desc, share
 
 
-def time_oracle(prob, min_seconds: float, max_seconds: float):
+def time_oracle(prob, min_seconds: float, max_seconds: float, share: bool = False):
     import oracle
     oracle.build()
     tokens, t0, reps = 0, time.perf_counter(), 0
     while True:
         oracle.forward(prob, prob["top_k"], prob["init_blocks"], prob["local_blocks"],
-                       prob["scale"], prob["max_blocks"])
+                       prob["scale"], prob["max_blocks"], share=share)
         tokens += prob["total_q"]
         reps += 1
         el = time.perf_counter() - t0
@@ -360,11 +363,11 @@ def run_reference(args):
     ws, rank, _ = dist_env()
     if rank != 0:
         return 0
-    prob, desc = oracle_sample(args.workload, args.cpu_sample_seqs, seed=7)
+    prob, desc, share = oracle_sample(args.workload, args.cpu_sample_seqs, seed=7)
     import oracle
     oracle.build()
     fwd = lambda: oracle.forward(prob, prob["top_k"], prob["init_blocks"], prob["local_blocks"],
-                                 prob["scale"], prob["max_blocks"])
+                                 prob["scale"], prob["max_blocks"], share=share)
     for _ in range(args.warmup):
         fwd()
     t0 = time.perf_counter()
@@ -601,8 +604,8 @@ def bench_workload(name, args, ws, rank, dev, sampler, with_cpu):
 
     cpu = None
     if with_cpu:
-        sample, desc = oracle_sample(name, args.cpu_sample_seqs, seed=7)
-        v, el, reps = time_oracle(sample, args.cpu_min_s, args.cpu_max_s)
+        sample, desc, share = oracle_sample(name, args.cpu_sample_seqs, seed=7)
+        v, el, reps = time_oracle(sample, args.cpu_min_s, args.cpu_max_s, share)
         cpu = {"value": v, "unit": UNIT, "cores": cpu_threads(), "kind": "oracle",
                "sample": f"{desc}, seed 7, {reps} pass(es), {el:.1f} s"}
 
@@ -766,7 +769,8 @@ def main(argv=None):
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="fp8_long_decode",
-                    help="the headline workload (the largest single-GPU configuration)")
+                    help="the headline workload (the largest single-GPU configuration), or "
+                    "another workload or variant to measure on its own (with --only)")
     ap.add_argument("--only", action="store_true",
                     help="measure the headline workload only (not the other four)")
     ap.add_argument("--splits", type=int, default=0, help="split-K partitions (0 = heuristic)")
@@ -783,6 +787,9 @@ def main(argv=None):
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
+    from block_sparse_paged_scores_b200 import workload as wl
+    if args.workload not in list(wl.WORKLOADS) + list(VARIANTS):
+        ap.error(f"--workload: one of {', '.join(list(wl.WORKLOADS) + list(VARIANTS))}")
     if args.impl == "reference":
         return run_reference(args)
     rc = run_ours(args)

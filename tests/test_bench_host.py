@@ -60,9 +60,17 @@ def test_traffic_records_are_complete(bench):
 
 
 @pytest.mark.parametrize("workload", ["tiny_decode", "bf16_decode", "spec_decode",
-                                      "fp8_long_decode", "ragged_prefill"])
+                                      "fp8_long_decode", "ragged_prefill",
+                                      "spec_decode_shared_topk", "fp8_long_decode_fp4_index_k",
+                                      "ragged_prefill_fp8_kv"])
 def test_oracle_samples_are_bounded(bench, workload):
-    p, desc = bench.oracle_sample(workload, 4, seed=7)
+    p, desc, share = bench.oracle_sample(workload, 4, seed=7)
+    assert share == (workload == "spec_decode_shared_topk")
+    base, changes, _ = bench.VARIANTS.get(workload, (workload, {}, {}))
+    if "idx_dtype" in changes:
+        assert p["idx_dtype"] == changes["idx_dtype"]
+    if "kv_dtype" in changes:
+        assert p["kv_fp8"]
     assert p["batch"] <= 4
     if p["max_q_len"] > 8:           # prefill: one sequence with 16-64 new tokens
         assert p["batch"] == 1 and 16 <= p["total_q"] <= 64
