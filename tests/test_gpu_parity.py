@@ -575,3 +575,33 @@ def test_shared_selection_is_refused_on_the_prefill_route():
     with pytest.raises(msa.MSAError) as ei:
         path.index_select()
     assert ei.value.status == msa.MSA_ERR_INVALID_ARG
+
+
+# ------------------------------------------------------------------ speculative indexer, 16 columns
+# The speculative route scores BF16 index-K on tcgen05 with a page's positions as M and a
+# unit's rows as N, padded to 16 or 32 columns.  The cases above reach 32 (4 draft tokens x 8
+# index-query heads); these reach 16 (two drafts x 8 heads; one index-K head per KV head, up to
+# 8 tokens x 1 head) and 32 with a padded quarter (three drafts x 8 heads).
+SPEC_TC = {
+    "two_drafts": dict(batch=5, q_len=2, kv_len=(700, 5000)),
+    "idxk_per_head": dict(batch=4, q_len=(2, 8), kv_len=(900, 4000), H_idxk=8),
+    "three_drafts": dict(batch=4, q_len=3, kv_len=(300, 3000)),
+}
+
+
+@pytest.mark.parametrize("name", sorted(SPEC_TC))
+def test_speculative_indexer_columns_match_oracle(name):
+    p = wl.generate(W["spec_decode"].scaled(**SPEC_TC[name]),
+                    seed=3100 + sorted(SPEC_TC).index(name))
+    sc, ids, cnt, out = oracle_forward(p)
+    path = msa.Path(_gpu(p))
+    path.run()
+    torch.cuda.synchronize()
+    assert int(path.dev_err.item()) == 0
+    check_scores(path.scores.cpu().numpy(), sc, p, p["max_blocks"])
+    g_ids, g_cnt = path.block_ids.cpu().numpy(), path.num_selected.cpu().numpy()
+    same = check_selection(g_ids, g_cnt, ids, cnt, sc, p)
+    assert same.mean() > 0.9
+    out_g = oracle.attention(p["row_off"], p["cache_len"], p["table"], p["q"], p["k"], p["v"],
+                             p["kv_fp8"], g_ids, g_cnt, p["scale"])
+    check_attention(path.out.float().cpu(), out_g, p["kv_fp8"])
