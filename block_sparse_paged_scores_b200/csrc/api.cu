@@ -268,15 +268,19 @@ struct FusedSelect {
 };
 
 // The prefill route scores BF16 index-K on tcgen05 (query rows as M); the speculative route
-// too, with a page's positions as M (its per-token top-k; the top-k shared across drafts
-// scores one token and stays on the warp-MMA kernel, which selects in the same launch); the
-// scaled formats take the warp-MMA kernel on every route.
+// too when its units hold more than 16 rows, with a page's positions as M and the rows as 32
+// columns (the per-token top-k; the top-k shared across drafts scores one token and stays on
+// the warp-MMA kernel, which selects in the same launch); the scaled formats take the warp-MMA
+// kernel on every route.
 bool index_uses_tc(const msa_ragged_paged_t *rp, int Hg, int idx_fmt) {
   return idx_fmt == kIdxBf16 && rp->max_q_len > MSA_MAX_SPEC_DRAFT && Hg <= 128;
 }
-bool index_uses_tc_pos(const msa_ragged_paged_t *rp, int idx_fmt, uint32_t flags) {
-  return idx_fmt == kIdxBf16 && rp->max_q_len >= 2 && rp->max_q_len <= MSA_MAX_SPEC_DRAFT &&
-         !(flags & MSA_SHARE_ACROSS_DRAFTS);
+bool index_uses_tc_pos(const msa_ragged_paged_t *rp, int Hg, int idx_fmt, uint32_t flags) {
+  if (idx_fmt != kIdxBf16 || rp->max_q_len < 2 || rp->max_q_len > MSA_MAX_SPEC_DRAFT ||
+      (flags & MSA_SHARE_ACROSS_DRAFTS) || Hg < 1 || Hg > 32)
+    return false;
+  const int qt = rp->max_q_len * Hg <= 32 ? rp->max_q_len : 32 / Hg;  // as index_scores_impl
+  return qt * Hg > 16;
 }
 
 bool index_k_ok(const msa_index_k_t *k, int32_t num_kv_heads) {
@@ -360,7 +364,7 @@ msa_status_t index_scores_impl(const msa_ragged_paged_t *rp, const void *q_idx,
   a.chunk = static_cast<int>(chunk);
   a.chunks = static_cast<int>(chunks);
   if (units * chunks > 0x7fffffffLL) return MSA_ERR_UNSUPPORTED;
-  const bool tc_pos = index_uses_tc_pos(rp, idx_fmt, flags);
+  const bool tc_pos = index_uses_tc_pos(rp, Hg, idx_fmt, flags);
   if (tc_pos && fs) return MSA_ERR_UNSUPPORTED;  // the caller selects with a separate launch
   if (fs) {
     a.publish = fs->publish;
@@ -441,7 +445,8 @@ msa_status_t msa_index_select_k(const msa_ragged_paged_t *rp, const void *q_idx,
   const bool fused =
       num_kv_heads % k_idx->num_heads == 0 &&
       !index_uses_tc(rp, num_kv_heads / k_idx->num_heads, static_cast<int>(k_idx->dtype)) &&
-      !index_uses_tc_pos(rp, static_cast<int>(k_idx->dtype), flags);
+      !index_uses_tc_pos(rp, num_kv_heads / k_idx->num_heads, static_cast<int>(k_idx->dtype),
+                         flags);
   if (fused) {
     if (!counters || !aligned(counters, 4)) return MSA_ERR_INVALID_ARG;
     const FusedSelect fs{counters, block_ids, num_selected, top_k, init_blocks, local_blocks,

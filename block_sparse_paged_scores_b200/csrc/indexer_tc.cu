@@ -259,8 +259,8 @@ __global__ void __launch_bounds__(kIxThreads, 1)
 // With a few draft tokens per sequence a unit has at most 32 rows (tokens x the index-query
 // heads of one index-K head), too few for M, and the row-major form above would be three
 // quarters padding.  Here the operands are swapped: S^T = K_page Q_idx^T with M = the page's
-// 128 positions, N = the unit's rows padded to NR (16 or 32), K = 128 dims, so no MMA works on
-// padding.  Each thread of the four epilogue warps holds one position (its TMEM lane) and the
+// 128 positions, N = the unit's rows padded to NR = 32 (the route takes units of more than 16
+// rows), K = 128 dims, so the MMAs work on little or no padding.  Each thread of the four epilogue warps holds one position (its TMEM lane) and the
 // NR row values of it; the max over the page's positions is one warp reduction per row on
 // order-preserving keys, then a max of the four warps' results through shared memory.  The
 // grid is the warp-MMA kernel's: one CTA per (chunk of pages, unit), a unit's chunks launched
@@ -530,8 +530,7 @@ cudaError_t launch_index_scores_tc_pos(const CUtensorMap &kidx_map, const Indexe
     const dim3 grid(a.batch * a.tiles * a.H_idxk * chunks);
     return launch_pdl(kernel, grid, dim3(kIxThreads), smem, s, kidx_map, a);
   };
-  const int rows = a.qt * (a.H_kv / a.H_idxk);
-  if (rows <= 16) return go(&index_scores_pos_kernel<16>, pos_smem_bytes<16>());
+  if (a.qt * (a.H_kv / a.H_idxk) > 32) return cudaErrorInvalidValue;
   return go(&index_scores_pos_kernel<32>, pos_smem_bytes<32>());
 }
 

@@ -52,7 +52,7 @@ cudaError_t launch_index_scores(const CUtensorMap &kidx_map, const IndexerArgs &
 cudaError_t launch_index_scores_tc(const CUtensorMap &kidx_map, const IndexerArgs &a,
                                    cudaStream_t s);
 // speculative route on tcgen05 (indexer_tc.cu): a page's 128 positions as M and the unit's
-// qt x (H_kv / H_idxk) <= 32 rows as N; the warp-MMA kernel's grid of chunks
+// qt x (H_kv / H_idxk) <= 32 rows as N = 32; the warp-MMA kernel's grid of chunks
 cudaError_t launch_index_scores_tc_pos(const CUtensorMap &kidx_map, const IndexerArgs &a,
                                        int chunks, cudaStream_t s);
 

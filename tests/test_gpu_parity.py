@@ -577,11 +577,12 @@ def test_shared_selection_is_refused_on_the_prefill_route():
     assert ei.value.status == msa.MSA_ERR_INVALID_ARG
 
 
-# ------------------------------------------------------------------ speculative indexer, 16 columns
+# ------------------------------------------------------------------ speculative indexer routes
 # The speculative route scores BF16 index-K on tcgen05 with a page's positions as M and a
-# unit's rows as N, padded to 16 or 32 columns.  The cases above reach 32 (4 draft tokens x 8
-# index-query heads); these reach 16 (two drafts x 8 heads; one index-K head per KV head, up to
-# 8 tokens x 1 head) and 32 with a padded quarter (three drafts x 8 heads).
+# unit's rows as 32 columns when a unit holds more than 16 rows (the cases above: 4 draft
+# tokens x 8 index-query heads), on the warp-MMA kernel otherwise.  Here: 16 rows (two drafts x
+# 8 heads) and 8 (one index-K head per KV head, up to 8 tokens x 1 head) on the warp-MMA
+# kernel, and 24 (three drafts x 8 heads: a quarter of the columns padding) on tcgen05.
 SPEC_TC = {
     "two_drafts": dict(batch=5, q_len=2, kv_len=(700, 5000)),
     "idxk_per_head": dict(batch=4, q_len=(2, 8), kv_len=(900, 4000), H_idxk=8),
@@ -590,7 +591,7 @@ SPEC_TC = {
 
 
 @pytest.mark.parametrize("name", sorted(SPEC_TC))
-def test_speculative_indexer_columns_match_oracle(name):
+def test_speculative_indexer_routes_match_oracle(name):
     p = wl.generate(W["spec_decode"].scaled(**SPEC_TC[name]),
                     seed=3100 + sorted(SPEC_TC).index(name))
     sc, ids, cnt, out = oracle_forward(p)
