@@ -447,8 +447,10 @@ msa_status_t msa_index_select_k(const msa_ragged_paged_t *rp, const void *q_idx,
       !index_uses_tc(rp, num_kv_heads / k_idx->num_heads, static_cast<int>(k_idx->dtype)) &&
       !index_uses_tc_pos(rp, num_kv_heads / k_idx->num_heads, static_cast<int>(k_idx->dtype),
                          flags);
+  // counters: required on the decode and speculative routes, whether or not this shape uses them
+  if (rp->max_q_len <= MSA_MAX_SPEC_DRAFT && (!counters || !aligned(counters, 4)))
+    return MSA_ERR_INVALID_ARG;
   if (fused) {
-    if (!counters || !aligned(counters, 4)) return MSA_ERR_INVALID_ARG;
     const FusedSelect fs{counters, block_ids, num_selected, top_k, init_blocks, local_blocks,
                          static_cast<int>(S)};
     return index_scores_impl(rp, q_idx, k_idx, num_kv_heads, max_blocks, flags, scores, dev_err,

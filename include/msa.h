@@ -144,8 +144,10 @@ MSA_API msa_status_t msa_select_blocks(const msa_ragged_paged_t *rp, const float
  * On the decode and speculative routes (max_q_len <= MSA_MAX_SPEC_DRAFT) it is one launch: the
  * CTAs that score one (sequence, tile of query tokens, index-K head) count themselves out on
  * `counters`, and the last one selects for that unit's rows, so the selection needs no launch
- * of its own.  On the prefill route it enqueues the two stages one after the other and does not
- * touch `counters`.
+ * of its own.  Two cases enqueue the two stages one after the other instead and do not touch
+ * `counters`: the prefill route, and the speculative route with a BF16 index-K cache, the
+ * top-k per token and units of more than 16 rows (tokens of a tile x index-query heads of one
+ * index-K head), which score on the tensor cores.
  *
  *   scores, block_ids, num_selected  as msa_index_scores / msa_select_blocks (all outputs;
  *                  `scores` stays valid after the call, as the selection's input)
