@@ -205,7 +205,8 @@ typedef struct {
  * msa_index_scores_k / msa_index_select_k — msa_index_scores / msa_index_select over an index-K
  * cache in any msa_idx_dtype_t (the BF16 entry points are these with MSA_IDX_BF16 and flags 0;
  * their results are bit-identical).  Scaled formats run the warp-MMA indexer on every route
- * (the prefill route's tcgen05 indexer takes BF16 only).
+ * (the tensor-core indexers, of the prefill route and of speculative units of more than 16
+ * rows, take BF16 only).
  *
  * flags: 0, or MSA_SHARE_ACROSS_DRAFTS ([trtllm] index_share_for_mtp_iteration: reuse the
  * indexer top-k across draft tokens instead of recomputing it for each), accepted on the
