@@ -420,7 +420,8 @@ class Path:
                                self.index_flags, self.scores, self.dev_err, stream)
 
     def index_select(self, stream=None):
-        """Stages 1 and 2 in one call (one launch on the decode / speculative routes)."""
+        """Stages 1 and 2 in one call (one launch on the decode route and on most speculative
+        shapes; two where the scores run on the tensor cores)."""
         p = self.p
         msa_index_select_k(self.rp, p["q_idx"], self.kidx, p["H_kv"], self.max_blocks,
                            p["top_k"], p["init_blocks"], p["local_blocks"], self.index_flags,
